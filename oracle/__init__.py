@@ -1,0 +1,17 @@
+"""CPU oracle (test infrastructure only; see ``tp_oracle``)."""
+
+from .tp_oracle import (  # noqa: F401
+    ACTIVATIONS,
+    apply_activation,
+    column_parallel_linear,
+    gelu_tanh,
+    mlp_sharded,
+    mlp_unsharded,
+    reduce_partials_fixed_order,
+    rel_err,
+    relu,
+    round_to_bf16,
+    row_parallel_partials,
+    shard_width,
+    silu,
+)

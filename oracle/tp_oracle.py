@@ -1,0 +1,245 @@
+"""CPU oracle for the Megatron tensor-parallel MLP block.
+
+TEST INFRASTRUCTURE ONLY.  Nothing in the product path may import, call or
+execute this module: only the tests, the smoke check and the bench's CPU
+baseline arm use it.  It shares no code with the CUDA library.
+
+What it computes, and where the pages state it:
+
+* Column-parallel linear -- W [d, k] is cut by output columns into p slices
+  W_i = W[:, i*s:(i+1)*s], s = k/p; every shard sees the whole X and forms
+  Y_i = act(X W_i + b_i) with no communication.  (skandtandon.pages.dev day-41
+  post, "Simulating column parallel linear"; "Tensor parallel math",
+  "Column-parallel: split the weight by output columns"; "Tensor Parallelism
+  Explained", section 1.A.)
+* Row-parallel linear -- W' [k, d] is cut by input rows into W'_i =
+  W'[i*s:(i+1)*s, :]; shard i consumes Y_i and emits a full-shape partial
+  Z_i = Y_i W'_i [T, d].  (day-41 post, "Simulating row parallel linear";
+  "Tensor parallel math", "Row-parallel: split the weight by input rows";
+  "Tensor Parallelism Explained", section 1.B.)
+* The all-reduce -- Z = sum_i Z_i; the output bias is added once, after the
+  sum.  On one device this is a fixed-order fp32 fold (day-41 post,
+  ``sum(partial_sums) + bias``; "Building GPT from Scratch -- Part 9",
+  "Implementation Sketch", RowParallelLinear.forward).
+* The Megatron MLP pairing -- column-parallel first layer, element-wise
+  activation applied per shard, row-parallel second layer, one reduction
+  ("Tensor parallel math", "The MLP block: column then row, one all-reduce";
+  day-41 post, "Pairing them: the Megatron-LM MLP").  SwiGLU variant:
+  Swish(X W_gate,i) * (X W_up,i) per shard, W_down row-parallel
+  ("Tensor Parallelism Explained", section 2.B).
+
+Readings taken where the pages are silent (each also listed in the design
+notes): GELU is the tanh form 0.5 h (1 + tanh(sqrt(2/pi) (h + 0.044715 h^3)))
+(Hendrycks & Gimpel); Swish is SiLU, h / (1 + e^-h); weights are stored
+[in, out] row-major (Y = X W); the fixed-order reduction is a left fold that
+starts from Z_0 (not from 0.0) and adds the bias last.
+
+Precision: every product and sum is taken in float64 from the exact input
+values; partials are rounded once to float32; the fold is float32
+round-to-nearest-even, one addition at a time.  A library matmul (numpy's
+float64 ``@``) serves as the dot-product step.
+"""
+
+from __future__ import annotations
+
+import math
+from typing import List, Optional, Sequence
+
+import numpy as np
+
+ACTIVATIONS = ("gelu_tanh", "swiglu", "identity", "relu")
+
+_SQRT_2_OVER_PI = math.sqrt(2.0 / math.pi)
+
+
+# --------------------------------------------------------------------------
+# element-wise activations (applied locally on each shard)
+# --------------------------------------------------------------------------
+
+def gelu_tanh(h: np.ndarray) -> np.ndarray:
+    """GELU, tanh form, in float64."""
+    h = np.asarray(h, dtype=np.float64)
+    return 0.5 * h * (1.0 + np.tanh(_SQRT_2_OVER_PI * (h + 0.044715 * h * h * h)))
+
+
+def silu(h: np.ndarray) -> np.ndarray:
+    """Swish with beta = 1 (SiLU), h / (1 + e^-h), in float64."""
+    h = np.asarray(h, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return h / (1.0 + np.exp(-h))
+
+
+def relu(h: np.ndarray) -> np.ndarray:
+    """max(0, h): the day-41 walkthrough's activation 'for simplicity'."""
+    return np.maximum(0.0, np.asarray(h, dtype=np.float64))
+
+
+def apply_activation(act: str, h: np.ndarray, up: Optional[np.ndarray] = None) -> np.ndarray:
+    """act(h); for SwiGLU ``h`` is the gate pre-activation X W_gate and ``up``
+    is X W_up."""
+    if act == "gelu_tanh":
+        return gelu_tanh(h)
+    if act == "relu":
+        return relu(h)
+    if act == "identity":
+        return np.asarray(h, dtype=np.float64)
+    if act == "swiglu":
+        if up is None:
+            raise ValueError("swiglu needs the up projection")
+        return silu(h) * np.asarray(up, dtype=np.float64)
+    raise ValueError(f"unknown activation {act!r}")
+
+
+# --------------------------------------------------------------------------
+# the plain (unsharded) block: the definition the sharded method must reach
+# --------------------------------------------------------------------------
+
+def _f64(a):
+    return None if a is None else np.asarray(a, dtype=np.float64)
+
+
+def mlp_unsharded(X, W1, b1, W2, b2, act: str, W_up=None) -> np.ndarray:
+    """Z = act(X W1 + b1) W2 + b2 in float64, no sharding at all.
+
+    For SwiGLU, W1 is W_gate and Z = (SiLU(X W_gate) * (X W_up)) W_down.
+    Returns the unrounded float64 result."""
+    X, W1, W2 = _f64(X), _f64(W1), _f64(W2)
+    H = X @ W1
+    if b1 is not None:
+        H = H + _f64(b1)[None, :]
+    U = None
+    if act == "swiglu":
+        U = X @ _f64(W_up)
+    Y = apply_activation(act, H, U)
+    Z = Y @ W2
+    if b2 is not None:
+        Z = Z + _f64(b2)[None, :]
+    return Z
+
+
+# --------------------------------------------------------------------------
+# the sharded method, written separately, one shard at a time
+# --------------------------------------------------------------------------
+
+def shard_width(k: int, p: int) -> int:
+    """s = k/p; the walkthrough asserts divisibility before slicing."""
+    if p < 1:
+        raise ValueError("p must be >= 1")
+    if k % p != 0:
+        raise ValueError(f"{k} features cannot be split evenly over {p} shards")
+    return k // p
+
+
+def _column_slice(W: np.ndarray, i: int, s: int) -> np.ndarray:
+    """Shard i's column block of an [in, out] weight: W[:, i*s:(i+1)*s]."""
+    return W[:, i * s:(i + 1) * s]
+
+
+def _vector_slice(b: np.ndarray, i: int, s: int) -> np.ndarray:
+    return b[i * s:(i + 1) * s]
+
+
+def _row_slice(W: np.ndarray, i: int, s: int) -> np.ndarray:
+    """Shard i's row block of a [k, d] weight: W[i*s:(i+1)*s, :]."""
+    return W[i * s:(i + 1) * s, :]
+
+
+def column_parallel_linear(X, W1, b1, p: int, act: str, W_up=None) -> List[np.ndarray]:
+    """Per-shard Y_i = act(X W1_i + b1_i), i = 0..p-1, each [T, s], float64.
+
+    The activation runs on each shard's slice alone, as the pairing allows
+    (it is element-wise)."""
+    k = np.shape(W1)[1]
+    s = shard_width(k, p)
+    X64 = _f64(X)
+    out = []
+    for i in range(p):
+        Wi = np.asarray(_column_slice(W1, i, s), dtype=np.float64)
+        Hi = X64 @ Wi
+        if b1 is not None:
+            Hi = Hi + np.asarray(_vector_slice(b1, i, s), dtype=np.float64)[None, :]
+        Ui = None
+        if act == "swiglu":
+            Ui = X64 @ np.asarray(_column_slice(W_up, i, s), dtype=np.float64)
+        out.append(apply_activation(act, Hi, Ui))
+    return out
+
+
+def row_parallel_partials(Y_shards: Sequence[np.ndarray], W2, p: int) -> List[np.ndarray]:
+    """Per-shard full-shape partials Z_i = Y_i W2_i, each [T, d], float64."""
+    if len(Y_shards) != p:
+        raise ValueError("need one hidden shard per partition")
+    k = np.shape(W2)[0]
+    s = shard_width(k, p)
+    out = []
+    for i in range(p):
+        W2i = np.asarray(_row_slice(W2, i, s), dtype=np.float64)
+        out.append(np.asarray(Y_shards[i], dtype=np.float64) @ W2i)
+    return out
+
+
+def reduce_partials_fixed_order(P: np.ndarray, b2: Optional[np.ndarray] = None) -> np.ndarray:
+    """Z = ((P_0 + P_1) + ...) + P_{p-1}  [+ b2], every addition a single
+    float32 round-to-nearest-even operation, shard index ascending.
+
+    ``P`` is float32 [p][T][d] (or a sequence of [T][d] float32 arrays);
+    ``b2`` is float32 [d] or None.  Returns float32 [T][d]."""
+    parts = [np.asarray(x) for x in P]
+    for x in parts:
+        if x.dtype != np.float32:
+            raise TypeError("partials must be float32")
+    acc = parts[0].copy()
+    for x in parts[1:]:
+        acc = np.add(acc, x, dtype=np.float32)
+    if b2 is not None:
+        b = np.asarray(b2)
+        if b.dtype != np.float32:
+            raise TypeError("b2 must be float32")
+        acc = np.add(acc, b[None, :], dtype=np.float32)
+    return acc
+
+
+def round_to_bf16(x: np.ndarray) -> np.ndarray:
+    """Round float64 values to the nearest bf16 value (8 significant bits,
+    ties to even), returned as float64.  Used for the device-faithful mode,
+    where the hidden shards are stored as bf16 between the two layers."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)                      # x = m * 2**e, 0.5 <= |m| < 1
+    return np.ldexp(np.rint(m * 256.0), e - 8)
+
+
+def mlp_sharded(X, W1, b1, W2, b2, p: int, act: str, W_up=None,
+                hidden_round: Optional[str] = None) -> dict:
+    """The whole method on p simulated shards.
+
+    Returns a dict with
+      ``Y``  -- list of p float64 hidden shards [T, s] (after the optional
+                storage rounding),
+      ``P``  -- float32 partials [p, T, d] (each rounded once from float64),
+      ``Z``  -- float32 result of the fixed-order fold (+ b2 last).
+
+    ``hidden_round`` = None keeps Y unrounded; "bf16" or "f32" rounds each
+    hidden shard to that storage type before the row-parallel layer."""
+    Y = column_parallel_linear(X, W1, b1, p, act, W_up)
+    if hidden_round == "bf16":
+        Y = [round_to_bf16(y) for y in Y]
+    elif hidden_round == "f32":
+        Y = [y.astype(np.float32).astype(np.float64) for y in Y]
+    elif hidden_round is not None:
+        raise ValueError(hidden_round)
+    P64 = row_parallel_partials(Y, W2, p)
+    P = np.stack([x.astype(np.float32) for x in P64])
+    b2_32 = None if b2 is None else np.asarray(b2, dtype=np.float32)
+    Z = reduce_partials_fixed_order(P, b2_32)
+    return {"Y": Y, "P": P, "Z": Z}
+
+
+def rel_err(got: np.ndarray, want: np.ndarray) -> float:
+    """max|got - want| / max|want| (the parity measure for float results)."""
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    den = float(np.max(np.abs(want))) if want.size else 0.0
+    num = float(np.max(np.abs(got - want))) if want.size else 0.0
+    if den == 0.0:
+        return num
+    return num / den
