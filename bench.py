@@ -1,0 +1,451 @@
+"""Benchmark of the sharded Megatron MLP block on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gpt2|toy|wide|decode|llama]
+                    [--mode partials|splitk] [--impl tp|reference]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+column-parallel GEMM + activation (all p shards), row-parallel GEMM to p fp32
+partials, fixed-order partial-sum reduction.  Each of the three C-ABI calls is
+bracketed by CUDA events on the launching stream, so the per-kernel durations
+(for the roofline figure) and the step time come from the same timed steps.
+L2 is flushed (a 256 MiB write) before every step, outside the events.
+
+With N > 1 (torchrun) every rank runs an independent replica on its own GPU:
+the block is single-GPU by design (the p shards are simulated on one device),
+so there is no data-path collective; the step time is the max over ranks and
+`value` counts the work of all ranks ("scaling": "weak").
+
+`--impl reference` times the CPU oracle (float64 numpy) on the host cores on a
+bounded token-row sample of the same workload, in the same metric.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads as WL  # noqa: E402
+
+METRIC = "sharded-MLP TFLOP/s & % BF16 tensor peak; partial-sum reduce HBM GB/s"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def whole_job_value(units_per_step_per_rank: float, n_ranks: int, ms_per_step_max: float) -> float:
+    """Aggregate throughput: the work of all ranks over the slowest rank's time."""
+    return units_per_step_per_rank * n_ranks / (ms_per_step_max * 1e-3)
+
+
+def reduce_max(values, dist=None, device=None):
+    """Element-wise max of a list of floats over all ranks (identity without a group)."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return list(values)
+    import torch
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.cpu().tolist()
+
+
+def reduce_bytes(w: WL.Workload) -> int:
+    """Algorithmic HBM bytes of the reduction: read p partials, write Z (+ b2)."""
+    return (w.p + 1) * w.T * w.d * 4 + (w.d * 4 if w.has_b2 else 0)
+
+
+def column_flops(w: WL.Workload) -> int:
+    return 2 * w.T * w.d * w.k * (2 if w.act == "swiglu" else 1)
+
+
+def row_flops(w: WL.Workload) -> int:
+    return 2 * w.T * w.k * w.d
+
+
+def column_bytes(w: WL.Workload) -> int:
+    e = 2 if w.dtype == "bf16" else 4
+    nw = 2 if w.act == "swiglu" else 1
+    return e * (w.T * w.d + nw * w.d * w.k + w.T * w.k + (w.k if w.has_b1 else 0))
+
+
+def row_bytes(w: WL.Workload) -> int:
+    e = 2 if w.dtype == "bf16" else 4
+    return e * (w.T * w.k + w.k * w.d) + 4 * w.p * w.T * w.d
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]) if parts[3] not in ("[N/A]", "N/A") else 0.0, parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
+        loaded = [r for r in rows if r[2] > 0.5 * max(x[2] for x in rows)] or rows
+        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def ncu_traffic(kernel_key: str):
+    """dram bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            table = json.load(f)
+    except Exception:
+        return None
+    ent = table.get(kernel_key)
+    if not ent:
+        return None
+    src = os.path.join(ROOT, "megatron_tensor_sharded_b200", "csrc", ent["source"])
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    if sha != ent.get("source_sha"):
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- CPU oracle arm
+
+def oracle_sample_rows(w: WL.Workload, target_flops: float = 4e10) -> int:
+    per_row = w.gemm_flops() / w.T
+    return int(max(1, min(w.T, target_flops // per_row)))
+
+
+def time_oracle(w: WL.Workload, inp: WL.Inputs, rows: int, min_seconds: float, max_reps: int):
+    """Time the oracle (as it stands) on the first `rows` token rows; returns
+    (seconds per rep, reps)."""
+    from oracle import tp_oracle as O
+    X = inp.values("X")[:rows]
+    args = (inp.values("W1"), inp.values("b1"), inp.values("W2"), inp.values("b2"))
+    Wu = inp.values("W_up")
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        O.mlp_sharded(X, args[0], args[1], args[2], args[3], w.p, w.act, W_up=Wu)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or reps >= max_reps:
+            return el / reps, reps
+
+
+def run_reference(a, w: WL.Workload, rank: int, world: int):
+    if rank != 0:
+        return 0
+    inp = WL.make_inputs(w)
+    rows = oracle_sample_rows(w)
+    flops = w.gemm_flops() * rows / w.T
+    for _ in range(a.warmup):
+        time_oracle(w, inp, rows, 0.0, 1)
+    times = []
+    for _ in range(a.steps):
+        t, _ = time_oracle(w, inp, rows, 0.0, 1)
+        times.append(t)
+    ms = 1e3 * sum(times) / len(times)
+    value = flops / (ms * 1e-3) / 1e12
+    sample = f"first {rows} of {w.T} token rows per step, full weights, p={w.p}"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "d": w.d, "k": w.k, "p": w.p, "act": w.act,
+                   "sample_rows": rows, "parallelism": "replicas" if world > 1 else "single"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    import megatron_tensor_sharded_b200 as tp
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    inp = WL.make_inputs(w)
+
+    def dev(x):
+        if x is None:
+            return None
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(x).to(device)
+
+    X, W1, Wu, b1, W2 = dev(inp.X), dev(inp.W1), dev(inp.W_up), dev(inp.b1), dev(inp.W2)
+    b2 = dev(inp.b2)
+    dtype = tp.DTYPE[w.dtype]
+    act = tp.ACT[w.act]
+    hdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    Y = torch.empty((w.p, w.T, w.s), dtype=hdt, device=device)
+    P = torch.empty((w.p, w.T, w.d), dtype=torch.float32, device=device)
+    Z = torch.empty((w.T, w.d), dtype=torch.float32, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    splitk = a.mode == "splitk"
+    stream = torch.cuda.current_stream(device)
+
+    if splitk:
+        # split-K over shards: the row layer accumulates every shard in TMEM
+        # and writes Z directly; it is reached through the block call
+        nbytes = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, w.p, dtype, act,
+                                                tp.TP_FLAG_SPLITK_FUSED)
+        ws_split = torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+        def step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            tp.tp_mlp_block(X, W1, Wu, b1, W2, b2, Z, ws_split, nbytes, w.T, w.d, w.k, w.p, dtype,
+                            act, tp.TP_FLAG_SPLITK_FUSED, stream=stream)
+            if ev is not None:
+                for e in ev[1:]:
+                    e.record(stream)
+    else:
+        def step(ev=None):
+            if ev is not None:
+                ev[0].record(stream)
+            tp.tp_column_linear(X, W1, Wu, b1, Y, w.T, w.d, w.k, w.p, dtype, act, stream=stream)
+            if ev is not None:
+                ev[1].record(stream)
+            tp.tp_row_linear(Y, W2, P, w.T, w.k, w.d, w.p, dtype, stream=stream)
+            if ev is not None:
+                ev[2].record(stream)
+            tp.tp_reduce_partials(P, b2, Z, w.T, w.d, w.p, stream=stream)
+            if ev is not None:
+                ev[3].record(stream)
+
+    for _ in range(a.warmup):
+        flush.zero_()
+        step()
+    tp.tp_sync_status(stream)
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        torch.cuda.synchronize(device)
+        n0 = tp.tp_kernel_launch_count()
+        t_wall = time.perf_counter()
+        for i in range(a.steps):
+            flush.zero_()
+            step(evs[i])
+        torch.cuda.synchronize(device)
+        t_wall = time.perf_counter() - t_wall
+        launches = tp.tp_kernel_launch_count() - n0
+        barrier()
+    tp.tp_sync_status(stream)
+    col_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    row_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    red_ms = [e[2].elapsed_time(e[3]) for e in evs]
+    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
+    local = [statistics.mean(step_ms), statistics.mean(col_ms), statistics.mean(row_ms),
+             statistics.mean(red_ms), float(launches)]
+    ms_step, ms_col, ms_row, ms_red, launches = reduce_max(local, dist if world > 1 else None, device)
+
+    # ---- end to end through the public block call, inputs from pinned host memory
+    e2e = None
+    if not a.no_e2e:
+        Xh = X.cpu().pin_memory()
+        Zh = torch.empty(Z.shape, dtype=Z.dtype).pin_memory()
+        flags = tp.TP_FLAG_SPLITK_FUSED if splitk else tp.TP_FLAG_NONE
+        nbytes = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, w.p, dtype, act, flags)
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        Xd = torch.empty_like(X)
+
+        def e2e_step():
+            Xd.copy_(Xh, non_blocking=True)
+            tp.tp_mlp_block(Xd, W1, Wu, b1, W2, b2, Z, ws, nbytes, w.T, w.d, w.k, w.p, dtype, act,
+                            flags, stream=stream)
+            Zh.copy_(Z, non_blocking=True)
+
+        for _ in range(a.warmup):
+            flush.zero_()
+            e2e_step()
+        torch.cuda.synchronize(device)
+        barrier()
+        eev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(a.steps)]
+        for i in range(a.steps):
+            flush.zero_()
+            eev[i][0].record(stream)
+            e2e_step()
+            eev[i][1].record(stream)
+        torch.cuda.synchronize(device)
+        barrier()
+        tp.tp_sync_status(stream)
+        e_ms = reduce_max([statistics.mean(x[0].elapsed_time(x[1]) for x in eev)],
+                          dist if world > 1 else None, device)[0]
+        e2e = {"value": whole_job_value(w.gemm_flops(), world, e_ms) / 1e12, "unit": UNIT,
+               "ms_per_step": e_ms, "h2d_bytes_per_step": Xh.numel() * Xh.element_size(),
+               "d2h_bytes_per_step": Zh.numel() * Zh.element_size(),
+               "call": "tp_mlp_block"}
+
+    peaks, peak_src = load_peaks()
+    value = whole_job_value(w.gemm_flops(), world, ms_step) / 1e12
+    if splitk:
+        dom_name, dom_ms, dom_flops = "tp_mlp_block(split-K)", ms_col, w.gemm_flops()
+    elif ms_col >= ms_row:
+        dom_name, dom_ms, dom_flops = "tc_gemm column (tp_column_linear)", ms_col, column_flops(w)
+    else:
+        dom_name, dom_ms, dom_flops = "tc_gemm row partials (tp_row_linear)", ms_row, row_flops(w)
+    if w.dtype == "bf16":
+        achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+        peak = peaks["bf16_tflops"]
+        key = f"{w.name}/{'column' if 'column' in dom_name else 'row'}"
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": ncu_traffic(key), "kernel": dom_name,
+                "peak_source": f"{peak_src} bf16 burst"}
+    else:
+        # fp32 path: latency bound; report its HBM rate
+        byts = column_bytes(w) if "column" in dom_name else row_bytes(w)
+        achieved = byts / (dom_ms * 1e-3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": None, "kernel": dom_name,
+                "peak_source": f"{peak_src} hbm copy"}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "T": w.T, "d": w.d, "k": w.k, "p": w.p, "act": w.act,
+                   "mode": a.mode, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "flushed before every step (256 MiB write, outside the timed events)"},
+        "pct_bf16_peak": 100.0 * value / (peaks["bf16_tflops"] * world) if w.dtype == "bf16" else None,
+        "reduce": None if splitk else {"GB/s": reduce_bytes(w) / (ms_red * 1e-3) / 1e9,
+                                       "ms": ms_red, "frac_hbm": reduce_bytes(w) / (ms_red * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                                       "bytes": reduce_bytes(w)},
+        "kernels_ms": {"column": ms_col, "row": ms_row, "reduce": ms_red},
+        "roofline": roof,
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "wall_s_timed_region": t_wall,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        rows = min(w.T, oracle_sample_rows(w))
+        sec, reps = time_oracle(w, inp, rows, min_seconds=10.0, max_reps=1000)
+        line["cpu_baseline"] = {"value": w.gemm_flops() * rows / w.T / sec / 1e12, "unit": UNIT,
+                                "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"first {rows} of {w.T} token rows, {reps} reps, float64"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["tp", "reference"], default="tp")
+    ap.add_argument("--workload", choices=sorted(WL.WORKLOADS), default="gpt2")
+    ap.add_argument("--mode", choices=["partials", "splitk"], default="partials")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    a = ap.parse_args(argv)
+    if a.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != a.gpus:
+        ap.error(f"--gpus {a.gpus} but WORLD_SIZE={world}")
+    w = WL.WORKLOADS[a.workload]
+    if a.impl == "reference":
+        return run_reference(a, w, rank, world)
+    return run_tp(a, w, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,188 @@
+/*
+ * tp_mlp.h -- C ABI of libtpmlp: the Megatron tensor-parallel MLP block run
+ * as p simulated shards on one NVIDIA B200 (sm_100a).
+ *
+ * The method (column-parallel first layer, per-shard activation, row-parallel
+ * second layer, one sum of partials) is the one set out on the pages:
+ *   - "Simulating column parallel linear", "Simulating row parallel linear"
+ *     and "Pairing them: the Megatron-LM MLP" (skandtandon.pages.dev, day-41
+ *     post on tensor parallelism);
+ *   - "Column-parallel: split the weight by output columns", "Row-parallel:
+ *     split the weight by input rows", "The MLP block: column then row, one
+ *     all-reduce" (aicassindra.com, "Tensor parallel math");
+ *   - sections 1.A, 1.B and 2.B of "Tensor Parallelism Explained: Splitting
+ *     Attention and FFN Weights Across GPUs" (initnode.dev), 2.B being the
+ *     SwiGLU variant.
+ *
+ * Notation: T tokens, d model width, k FFN width, p shards, s = k/p.
+ * All matrices are dense and row-major.  Weights are stored [in, out]
+ * (Y = X W), as on the day-41 post and "Tensor parallel math".
+ *
+ * Conventions shared by every call:
+ *   - Every pointer is a DEVICE pointer owned by the caller.  The library
+ *     never allocates device memory and never frees caller memory.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *     default stream).  Argument errors are returned synchronously before
+ *     anything is launched; a CUDA launch error returns TP_ERR_CUDA.
+ *   - Every wait inside the tensor-core kernels is bounded (default 2 s,
+ *     see tp_set_wait_timeout_ns).  A wait that runs out makes the kernel
+ *     record TP_ERR_DEVICE_TIMEOUT in a per-device status word and return;
+ *     tp_sync_status() reports and clears it.  Nothing traps or spins forever.
+ *   - dtype TP_BF16: X, weights, b1 and the hidden shards are bf16; products
+ *     accumulate in fp32 (tcgen05 tensor cores, TMEM accumulators); partials,
+ *     b2 and Z are fp32.  Requires d % 8 == 0, s % 8 == 0 and 16-byte aligned
+ *     X, W1, W_up, Y, W2, partials and Z (TMA row pitches), else
+ *     TP_ERR_ALIGNMENT.
+ *   - dtype TP_F32: everything fp32, plain fp32 FMA (no TF32); any sizes,
+ *     4-byte alignment.
+ *   - T == 0 (no tokens) is valid: nothing is launched, TP_OK is returned.
+ */
+#ifndef TP_MLP_H
+#define TP_MLP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TP_OK = 0,
+  TP_ERR_INVALID_ARG = 1,     /* null pointer, p < 1, negative size, bad enum   */
+  TP_ERR_INDIVISIBLE = 2,     /* k % p != 0: the walkthrough asserts
+                                 out_features % num_gpus == 0 before slicing
+                                 ("Simulating column parallel linear") and
+                                 in_features % num_gpus == 0 for the row split */
+  TP_ERR_ALIGNMENT = 3,       /* bf16 path: pitch or pointer not 16-byte aligned */
+  TP_ERR_UNSUPPORTED = 4,     /* combination not provided (see each call)       */
+  TP_ERR_CUDA = 5,            /* a CUDA runtime call failed                      */
+  TP_ERR_DEVICE_TIMEOUT = 6,  /* a bounded device-side wait gave up              */
+  TP_ERR_WORKSPACE = 7        /* tp_mlp_block: workspace missing or too small    */
+} tp_status;
+
+typedef enum { TP_F32 = 0, TP_BF16 = 1 } tp_dtype;
+
+typedef enum {
+  TP_ACT_GELU_TANH = 0,  /* 0.5 h (1 + tanh(sqrt(2/pi) (h + 0.044715 h^3)))     */
+  TP_ACT_SWIGLU = 1,     /* SiLU(X W_gate,i) * (X W_up,i), "Tensor Parallelism
+                            Explained" 2.B; SiLU(h) = h / (1 + e^-h)            */
+  TP_ACT_IDENTITY = 2,   /* h (exact-arithmetic tests)                          */
+  TP_ACT_RELU = 3        /* max(0, h), the day-41 walkthrough's activation      */
+} tp_act;
+
+/* tp_mlp_block flags */
+#define TP_FLAG_NONE 0
+/* Accumulate all p shards of the row-parallel layer in one tensor-core
+ * accumulator (split-K over shards) and write Z once, instead of writing p
+ * partials and folding them.  Same result up to fp32 summation order (not
+ * bit-identical to the fixed-order fold).  bf16 requires s % 64 == 0. */
+#define TP_FLAG_SPLITK_FUSED 1
+
+/*
+ * Column-parallel linear + activation, all p shards in one launch.
+ *   Y_i = act(X W1_i + b1_i),  W1_i = W1[:, i*s:(i+1)*s],  i = 0..p-1
+ * ("Simulating column parallel linear"; "Column-parallel: split the weight
+ * by output columns").  The activation is applied on each shard alone, which
+ * the pairing allows because it is element-wise ("The MLP block").
+ *
+ *   X     [T][d]        dtype
+ *   W1    [d][k]        dtype   (W_gate for SwiGLU)
+ *   W_up  [d][k]        dtype   SwiGLU only (must be non-NULL), else ignored
+ *   b1    [k]           dtype   nullable (no bias); with SwiGLU, b1 is added
+ *                               to the gate pre-activation
+ *   Y     [p][T][s]     dtype   output: shard i is a dense [T][s] matrix
+ *   returns TP_ERR_INDIVISIBLE when k % p != 0.
+ */
+tp_status tp_column_linear(const void* X, const void* W1, const void* W_up, const void* b1,
+                           void* Y, int64_t T, int64_t d, int64_t k, int p,
+                           tp_dtype dtype, tp_act act, void* stream);
+
+/*
+ * Row-parallel linear: full-shape partials, one per shard.
+ *   P_i = Y_i W2_i,  W2_i = W2[i*s:(i+1)*s, :]
+ * ("Simulating row parallel linear"; "Row-parallel: split the weight by
+ * input rows": every shard emits a [T, d] partial whose sum is the answer).
+ *
+ *   Y        [p][T][s]  dtype
+ *   W2       [k][d]     dtype
+ *   partials [p][T][d]  fp32 output
+ */
+tp_status tp_row_linear(const void* Y, const void* W2, float* partials,
+                        int64_t T, int64_t k, int64_t d, int p,
+                        tp_dtype dtype, void* stream);
+
+/*
+ * The sum that replaces the all-reduce, in a fixed order:
+ *   Z = ((P_0 + P_1) + ...) + P_{p-1}  [+ b2]
+ * every addition one fp32 round-to-nearest-even operation, shard index
+ * ascending, the output bias added once after the sum (day-41 post:
+ * sum(partial_sums) + bias).  Bit-reproducible: the same inputs always give
+ * the same bits, on any grid.
+ *
+ *   partials [p][T][d]  fp32
+ *   b2       [d]        fp32, nullable
+ *   Z        [T][d]     fp32 output (must not alias partials)
+ */
+tp_status tp_reduce_partials(const float* partials, const float* b2, float* Z,
+                             int64_t T, int64_t d, int p, void* stream);
+
+/*
+ * The whole block, Z = sum_i act(X W1_i + b1_i) W2_i  [+ b2]
+ * ("Pairing them: the Megatron-LM MLP"; "The MLP block: column then row,
+ * one all-reduce").  Default: tp_column_linear -> tp_row_linear ->
+ * tp_reduce_partials on `stream`, with the hidden shards and the partials
+ * in the caller's workspace.  With TP_FLAG_SPLITK_FUSED the second layer
+ * accumulates over all shards and writes Z directly (no partials).
+ *
+ *   workspace        device memory of at least
+ *                    tp_mlp_block_workspace_size(...) bytes, 256-byte aligned;
+ *                    contents on return: hidden shards [p][T][s] at offset 0,
+ *                    then (default mode) the partials [p][T][d] fp32 at the
+ *                    next 256-byte boundary.
+ *   other arguments  as for the three calls above.
+ */
+tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const void* b1,
+                       const void* W2, const float* b2, float* Z,
+                       void* workspace, size_t workspace_bytes,
+                       int64_t T, int64_t d, int64_t k, int p,
+                       tp_dtype dtype, tp_act act, int flags, void* stream);
+
+/* Workspace bytes tp_mlp_block needs for these arguments (0 if invalid). */
+size_t tp_mlp_block_workspace_size(int64_t T, int64_t d, int64_t k, int p,
+                                   tp_dtype dtype, tp_act act, int flags);
+
+/* Synchronise `stream`, then report (and clear) the device status word of
+ * the current device: TP_ERR_DEVICE_TIMEOUT if a bounded wait ran out since
+ * the last call, TP_ERR_CUDA if the stream reported an error, else TP_OK. */
+tp_status tp_sync_status(void* stream);
+
+/* Limit for every bounded device-side wait, in nanoseconds (default 2e9).
+ * Applies to launches made after the call. 0 restores the default. */
+void tp_set_wait_timeout_ns(uint64_t ns);
+
+/* Fault injection for tests of the bounded waits: when `stage_index` >= 0,
+ * the next tensor-core launch's producer skips the load of that pipeline
+ * slot (counted from 0 in issue order), so its consumer's wait must run
+ * out.  -1 (default) disables it.  Applies to the next launch only. */
+void tp_debug_drop_load(int64_t stage_index);
+
+/* Human-readable name of a status code. */
+const char* tp_status_string(int status);
+
+/* Detail of the last argument or CUDA error seen by this thread ("" if none). */
+const char* tp_last_error_detail(void);
+
+/* Number of GPU kernels this library has launched in this process. */
+uint64_t tp_kernel_launch_count(void);
+
+/* ABI version of this header (bumped on any signature change). */
+int tp_abi_version(void);
+
+#define TP_ABI_VERSION 1
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TP_MLP_H */

@@ -1,0 +1,163 @@
+"""Python binding of libtpmlp, the B200 (sm_100a) Megatron tensor-parallel
+MLP block on p simulated shards.
+
+Argument marshalling only: every call below forwards to the C ABI of the
+same name (``include/tp_mlp.h``); all arithmetic runs in the library's CUDA
+kernels.  Arguments that are device buffers accept a ``torch.Tensor`` (its
+``data_ptr()`` is passed), a raw integer address, or ``None`` (NULL).
+``stream=None`` means torch's current CUDA stream.
+
+Importing this package fails loudly when the shared library has not been
+built (``python -m megatron_tensor_sharded_b200.build``): there is no CPU or
+PyTorch fallback.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+__all__ = [
+    "TPError", "TP_F32", "TP_BF16", "TP_ACT_GELU_TANH", "TP_ACT_SWIGLU", "TP_ACT_IDENTITY",
+    "TP_ACT_RELU", "TP_FLAG_NONE", "TP_FLAG_SPLITK_FUSED", "STATUS", "ACT", "DTYPE",
+    "tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
+    "tp_mlp_block_workspace_size", "tp_sync_status", "tp_set_wait_timeout_ns",
+    "tp_debug_drop_load", "tp_status_string", "tp_last_error_detail",
+    "tp_kernel_launch_count", "tp_abi_version", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtpmlp.so")
+
+TP_F32, TP_BF16 = 0, 1
+TP_ACT_GELU_TANH, TP_ACT_SWIGLU, TP_ACT_IDENTITY, TP_ACT_RELU = 0, 1, 2, 3
+TP_FLAG_NONE, TP_FLAG_SPLITK_FUSED = 0, 1
+DTYPE = {"f32": TP_F32, "bf16": TP_BF16}
+ACT = {"gelu_tanh": TP_ACT_GELU_TANH, "swiglu": TP_ACT_SWIGLU, "identity": TP_ACT_IDENTITY,
+       "relu": TP_ACT_RELU}
+STATUS = {0: "TP_OK", 1: "TP_ERR_INVALID_ARG", 2: "TP_ERR_INDIVISIBLE", 3: "TP_ERR_ALIGNMENT",
+          4: "TP_ERR_UNSUPPORTED", 5: "TP_ERR_CUDA", 6: "TP_ERR_DEVICE_TIMEOUT",
+          7: "TP_ERR_WORKSPACE"}
+
+
+class TPError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+        super().__init__(f"{self.name}: {detail}")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run "
+                          "`python -m megatron_tensor_sharded_b200.build` (nvcc, sm_100a)")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, u64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
+    lib.tp_column_linear.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, vp]
+    lib.tp_row_linear.argtypes = [vp, vp, vp, i64, i64, i64, i32, i32, vp]
+    lib.tp_reduce_partials.argtypes = [vp, vp, vp, i64, i64, i32, vp]
+    lib.tp_mlp_block.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sz, i64, i64, i64, i32, i32, i32,
+                                 i32, vp]
+    lib.tp_mlp_block_workspace_size.argtypes = [i64, i64, i64, i32, i32, i32, i32]
+    lib.tp_mlp_block_workspace_size.restype = sz
+    lib.tp_sync_status.argtypes = [vp]
+    lib.tp_set_wait_timeout_ns.argtypes = [u64]
+    lib.tp_set_wait_timeout_ns.restype = None
+    lib.tp_debug_drop_load.argtypes = [i64]
+    lib.tp_debug_drop_load.restype = None
+    lib.tp_status_string.argtypes = [i32]
+    lib.tp_status_string.restype = ctypes.c_char_p
+    lib.tp_last_error_detail.argtypes = []
+    lib.tp_last_error_detail.restype = ctypes.c_char_p
+    lib.tp_kernel_launch_count.argtypes = []
+    lib.tp_kernel_launch_count.restype = u64
+    lib.tp_abi_version.argtypes = []
+    for f in ("tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
+              "tp_sync_status", "tp_abi_version"):
+        getattr(lib, f).restype = i32
+    return lib
+
+
+_lib = _load()
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        if torch.cuda.is_available() and torch.cuda.is_initialized():
+            return torch.cuda.current_stream().cuda_stream
+        return None
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, check: bool) -> int:
+    if check and status != 0:
+        raise TPError(status, tp_last_error_detail())
+    return status
+
+
+def tp_column_linear(X, W1, W_up, b1, Y, T, d, k, p, dtype, act, stream=None, check=True):
+    """Y_i = act(X W1_i + b1_i) for all p shards; Y is [p][T][k/p]."""
+    return _check(_lib.tp_column_linear(_ptr(X), _ptr(W1), _ptr(W_up), _ptr(b1), _ptr(Y), T, d, k,
+                                        p, dtype, act, _stream(stream)), check)
+
+
+def tp_row_linear(Y, W2, partials, T, k, d, p, dtype, stream=None, check=True):
+    """P_i = Y_i W2_i, fp32 partials [p][T][d]."""
+    return _check(_lib.tp_row_linear(_ptr(Y), _ptr(W2), _ptr(partials), T, k, d, p, dtype,
+                                     _stream(stream)), check)
+
+
+def tp_reduce_partials(partials, b2, Z, T, d, p, stream=None, check=True):
+    """Z = ((P_0 + P_1) + ...) + P_{p-1} [+ b2], fixed order, fp32."""
+    return _check(_lib.tp_reduce_partials(_ptr(partials), _ptr(b2), _ptr(Z), T, d, p,
+                                          _stream(stream)), check)
+
+
+def tp_mlp_block(X, W1, W_up, b1, W2, b2, Z, workspace, workspace_bytes, T, d, k, p, dtype, act,
+                 flags=TP_FLAG_NONE, stream=None, check=True):
+    """The whole block, Z = sum_i act(X W1_i + b1_i) W2_i [+ b2]."""
+    return _check(_lib.tp_mlp_block(_ptr(X), _ptr(W1), _ptr(W_up), _ptr(b1), _ptr(W2), _ptr(b2),
+                                    _ptr(Z), _ptr(workspace), workspace_bytes, T, d, k, p, dtype,
+                                    act, flags, _stream(stream)), check)
+
+
+def tp_mlp_block_workspace_size(T, d, k, p, dtype, act, flags=TP_FLAG_NONE) -> int:
+    return int(_lib.tp_mlp_block_workspace_size(T, d, k, p, dtype, act, flags))
+
+
+def tp_sync_status(stream=None, check=True):
+    return _check(_lib.tp_sync_status(_stream(stream)), check)
+
+
+def tp_set_wait_timeout_ns(ns: int) -> None:
+    _lib.tp_set_wait_timeout_ns(ns)
+
+
+def tp_debug_drop_load(stage_index: int) -> None:
+    _lib.tp_debug_drop_load(stage_index)
+
+
+def tp_status_string(status: int) -> str:
+    return _lib.tp_status_string(status).decode()
+
+
+def tp_last_error_detail() -> str:
+    return _lib.tp_last_error_detail().decode()
+
+
+def tp_kernel_launch_count() -> int:
+    return int(_lib.tp_kernel_launch_count())
+
+
+def tp_abi_version() -> int:
+    return int(_lib.tp_abi_version())

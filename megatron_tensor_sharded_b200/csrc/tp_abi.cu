@@ -1,0 +1,323 @@
+// C ABI of libtpmlp (declared in include/tp_mlp.h): argument validation,
+// per-device state, and dispatch to the kernels.  No device memory is
+// allocated here; the caller owns every buffer.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "tp_internal.h"
+#include "tp_mlp.h"
+
+// Per-device status word written by the bounded device-side waits.
+__device__ unsigned int g_tp_status_word = 0;
+
+namespace tpk {
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+std::atomic<uint64_t> g_timeout_ns{2000000000ull};
+std::atomic<int64_t> g_debug_drop{-1};
+thread_local char g_detail[512] = "";
+
+constexpr int kMaxDevices = 64;
+int g_num_sms[kMaxDevices] = {};
+int g_cc_major[kMaxDevices] = {};
+unsigned* g_status_addr[kMaxDevices] = {};
+std::mutex g_dev_mu;
+
+tp_status fail(tp_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+// Per-device properties and the device address of the status word, looked
+// up once per device with that device current.
+tp_status device_state(int* dev_out, int* sms, int* cc_major, unsigned** status) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(TP_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(TP_ERR_UNSUPPORTED, "device index %d", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  if (g_status_addr[dev] == nullptr) {
+    int n = 0, major = 0;
+    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    void* addr = nullptr;
+    if (e == cudaSuccess) e = cudaGetSymbolAddress(&addr, g_tp_status_word);
+    if (e != cudaSuccess)
+      return fail(TP_ERR_CUDA, "device set-up: %s", cudaGetErrorString(e));
+    g_num_sms[dev] = n;
+    g_cc_major[dev] = major;
+    g_status_addr[dev] = static_cast<unsigned*>(addr);
+  }
+  *dev_out = dev;
+  *sms = g_num_sms[dev];
+  *cc_major = g_cc_major[dev];
+  *status = g_status_addr[dev];
+  return TP_OK;
+}
+
+tp_status make_ctx(void* stream, bool tensor_core, LaunchCtx* c) {
+  int cc = 0;
+  tp_status st = device_state(&c->device, &c->num_sms, &cc, &c->err_word);
+  if (st != TP_OK) return st;
+  if (tensor_core && cc != 10)
+    return fail(TP_ERR_UNSUPPORTED, "bf16 path needs an sm_100 device (found sm_%d.x)", cc);
+  c->stream = static_cast<cudaStream_t>(stream);
+  c->timeout_ns = g_timeout_ns.load();
+  c->debug_drop = tensor_core ? g_debug_drop.exchange(-1) : -1;
+  return TP_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+tp_status check_shape(int64_t T, int64_t d, int64_t k, int p, int dtype) {
+  if (p < 1) return fail(TP_ERR_INVALID_ARG, "p = %d, must be >= 1", p);
+  if (T < 0 || d < 1 || k < 1)
+    return fail(TP_ERR_INVALID_ARG, "sizes T=%lld d=%lld k=%lld", (long long)T, (long long)d,
+                (long long)k);
+  if (dtype != TP_F32 && dtype != TP_BF16) return fail(TP_ERR_INVALID_ARG, "dtype %d", dtype);
+  if (k % p != 0)
+    return fail(TP_ERR_INDIVISIBLE, "%lld features cannot be split evenly over %d shards",
+                (long long)k, p);
+  if (T > INT32_MAX || d > INT32_MAX || k > INT32_MAX || T * d > (int64_t(1) << 46) ||
+      T * k > (int64_t(1) << 46) || d * k > (int64_t(1) << 46))
+    return fail(TP_ERR_UNSUPPORTED, "sizes too large");
+  if (dtype == TP_BF16 && (d % 8 != 0 || (k / p) % 8 != 0))
+    return fail(TP_ERR_ALIGNMENT, "bf16 needs d %% 8 == 0 and k/p %% 8 == 0 (d=%lld, s=%lld)",
+                (long long)d, (long long)(k / p));
+  return TP_OK;
+}
+
+tp_status check_ptr(const void* ptr, const char* name, int dtype, bool tma) {
+  if (ptr == nullptr) return fail(TP_ERR_INVALID_ARG, "%s is NULL", name);
+  if (dtype == TP_BF16 && tma && !aligned16(ptr))
+    return fail(TP_ERR_ALIGNMENT, "%s must be 16-byte aligned", name);
+  if (dtype == TP_F32 && !aligned4(ptr)) return fail(TP_ERR_ALIGNMENT, "%s must be 4-byte aligned", name);
+  return TP_OK;
+}
+
+tp_status check_act(int act, const void* W_up) {
+  if (act < TP_ACT_GELU_TANH || act > TP_ACT_RELU) return fail(TP_ERR_INVALID_ARG, "act %d", act);
+  if (act == TP_ACT_SWIGLU && W_up == nullptr)
+    return fail(TP_ERR_INVALID_ARG, "SwiGLU needs W_up");
+  return TP_OK;
+}
+
+tp_status cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return TP_OK;
+  return fail(TP_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define TP_TRY(expr)               \
+  do {                             \
+    const tp_status st_ = (expr);  \
+    if (st_ != TP_OK) return st_;  \
+  } while (0)
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+size_t workspace_bytes(int64_t T, int64_t d, int64_t k, int p, int dtype, int flags) {
+  const size_t esize = dtype == TP_BF16 ? 2 : 4;
+  size_t bytes = align256(static_cast<size_t>(T) * static_cast<size_t>(k) * esize);
+  if (!(flags & TP_FLAG_SPLITK_FUSED))
+    bytes += align256(static_cast<size_t>(p) * static_cast<size_t>(T) * static_cast<size_t>(d) * 4);
+  return bytes;
+}
+
+tp_status column_impl(const void* X, const void* W1, const void* W_up, const void* b1, void* Y,
+                      int64_t T, int64_t d, int64_t k, int p, int dtype, int act, void* stream) {
+  TP_TRY(check_shape(T, d, k, p, dtype));
+  TP_TRY(check_act(act, W_up));
+  if (T == 0) return TP_OK;
+  TP_TRY(check_ptr(X, "X", dtype, true));
+  TP_TRY(check_ptr(W1, "W1", dtype, true));
+  if (act == TP_ACT_SWIGLU) TP_TRY(check_ptr(W_up, "W_up", dtype, true));
+  TP_TRY(check_ptr(Y, "Y", dtype, true));
+  if (b1 != nullptr) TP_TRY(check_ptr(b1, "b1", dtype, false));
+  LaunchCtx c{};
+  TP_TRY(make_ctx(stream, dtype == TP_BF16, &c));
+  if (dtype == TP_BF16) return launch_tc_column(c, X, W1, W_up, b1, Y, T, d, k, p, act);
+  return cuda_status(launch_simt_column(c, static_cast<const float*>(X),
+                                        static_cast<const float*>(W1),
+                                        static_cast<const float*>(W_up),
+                                        static_cast<const float*>(b1), static_cast<float*>(Y), T,
+                                        d, k, p, act),
+                     "fp32 column launch");
+}
+
+tp_status row_impl(const void* Y, const void* W2, float* partials, int64_t T, int64_t k,
+                   int64_t d, int p, int dtype, void* stream) {
+  TP_TRY(check_shape(T, d, k, p, dtype));
+  if (T == 0) return TP_OK;
+  TP_TRY(check_ptr(Y, "Y", dtype, true));
+  TP_TRY(check_ptr(W2, "W2", dtype, true));
+  if (partials == nullptr) return fail(TP_ERR_INVALID_ARG, "partials is NULL");
+  if (!aligned16(partials) && dtype == TP_BF16)
+    return fail(TP_ERR_ALIGNMENT, "partials must be 16-byte aligned");
+  if (!aligned4(partials)) return fail(TP_ERR_ALIGNMENT, "partials must be 4-byte aligned");
+  LaunchCtx c{};
+  TP_TRY(make_ctx(stream, dtype == TP_BF16, &c));
+  if (dtype == TP_BF16) return launch_tc_row(c, Y, W2, partials, T, k, d, p);
+  return cuda_status(launch_simt_row(c, static_cast<const float*>(Y),
+                                     static_cast<const float*>(W2), partials, T, k, d, p),
+                     "fp32 row launch");
+}
+
+tp_status reduce_impl(const float* partials, const float* b2, float* Z, int64_t T, int64_t d,
+                      int p, void* stream) {
+  if (p < 1) return fail(TP_ERR_INVALID_ARG, "p = %d, must be >= 1", p);
+  if (T < 0 || d < 1) return fail(TP_ERR_INVALID_ARG, "sizes T=%lld d=%lld", (long long)T, (long long)d);
+  if (T == 0) return TP_OK;
+  if (partials == nullptr || Z == nullptr) return fail(TP_ERR_INVALID_ARG, "partials/Z is NULL");
+  if (!aligned4(partials) || !aligned4(Z) || (b2 != nullptr && !aligned4(b2)))
+    return fail(TP_ERR_ALIGNMENT, "fp32 buffers must be 4-byte aligned");
+  const uintptr_t p0 = reinterpret_cast<uintptr_t>(partials);
+  const uintptr_t p1 = p0 + static_cast<uintptr_t>(p) * T * d * 4;
+  const uintptr_t z0 = reinterpret_cast<uintptr_t>(Z);
+  const uintptr_t z1 = z0 + static_cast<uintptr_t>(T) * d * 4;
+  if (z0 < p1 && p0 < z1) return fail(TP_ERR_INVALID_ARG, "Z overlaps the partials");
+  LaunchCtx c{};
+  TP_TRY(make_ctx(stream, false, &c));
+  return cuda_status(launch_reduce(c, partials, b2, Z, T, d, p), "reduce launch");
+}
+
+}  // namespace
+
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+void set_error_detail(const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_detail, sizeof(g_detail), fmt, ap);
+  va_end(ap);
+}
+
+}  // namespace tpk
+
+using namespace tpk;
+
+extern "C" {
+
+tp_status tp_column_linear(const void* X, const void* W1, const void* W_up, const void* b1,
+                           void* Y, int64_t T, int64_t d, int64_t k, int p, tp_dtype dtype,
+                           tp_act act, void* stream) {
+  g_detail[0] = 0;
+  return column_impl(X, W1, W_up, b1, Y, T, d, k, p, dtype, act, stream);
+}
+
+tp_status tp_row_linear(const void* Y, const void* W2, float* partials, int64_t T, int64_t k,
+                        int64_t d, int p, tp_dtype dtype, void* stream) {
+  g_detail[0] = 0;
+  return row_impl(Y, W2, partials, T, k, d, p, dtype, stream);
+}
+
+tp_status tp_reduce_partials(const float* partials, const float* b2, float* Z, int64_t T,
+                             int64_t d, int p, void* stream) {
+  g_detail[0] = 0;
+  return reduce_impl(partials, b2, Z, T, d, p, stream);
+}
+
+size_t tp_mlp_block_workspace_size(int64_t T, int64_t d, int64_t k, int p, tp_dtype dtype,
+                                   tp_act act, int flags) {
+  if (check_shape(T, d, k, p, dtype) != TP_OK) return 0;
+  if (act < TP_ACT_GELU_TANH || act > TP_ACT_RELU) return 0;
+  return workspace_bytes(T, d, k, p, dtype, flags);
+}
+
+tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const void* b1,
+                       const void* W2, const float* b2, float* Z, void* workspace,
+                       size_t workspace_size, int64_t T, int64_t d, int64_t k, int p,
+                       tp_dtype dtype, tp_act act, int flags, void* stream) {
+  g_detail[0] = 0;
+  TP_TRY(check_shape(T, d, k, p, dtype));
+  TP_TRY(check_act(act, W_up));
+  if (flags & ~TP_FLAG_SPLITK_FUSED) return fail(TP_ERR_INVALID_ARG, "flags 0x%x", flags);
+  const bool splitk = (flags & TP_FLAG_SPLITK_FUSED) != 0;
+  if (splitk && dtype == TP_BF16 && (k / p) % 64 != 0)
+    return fail(TP_ERR_UNSUPPORTED, "split-K over shards needs k/p %% 64 == 0 for bf16");
+  if (T == 0) return TP_OK;
+  TP_TRY(check_ptr(X, "X", dtype, true));
+  TP_TRY(check_ptr(W1, "W1", dtype, true));
+  if (act == TP_ACT_SWIGLU) TP_TRY(check_ptr(W_up, "W_up", dtype, true));
+  TP_TRY(check_ptr(W2, "W2", dtype, true));
+  if (b1 != nullptr) TP_TRY(check_ptr(b1, "b1", dtype, false));
+  if (Z == nullptr) return fail(TP_ERR_INVALID_ARG, "Z is NULL");
+  if (!aligned16(Z)) return fail(TP_ERR_ALIGNMENT, "Z must be 16-byte aligned");
+  if (b2 != nullptr && !aligned4(b2)) return fail(TP_ERR_ALIGNMENT, "b2 must be 4-byte aligned");
+  const size_t need = workspace_bytes(T, d, k, p, dtype, flags);
+  if (workspace == nullptr || workspace_size < need)
+    return fail(TP_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need,
+                workspace == nullptr ? size_t(0) : workspace_size);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(TP_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* Y = ws;
+  TP_TRY(column_impl(X, W1, W_up, b1, Y, T, d, k, p, dtype, act, stream));
+  if (splitk) {
+    LaunchCtx c{};
+    TP_TRY(make_ctx(stream, dtype == TP_BF16, &c));
+    if (dtype == TP_BF16) return launch_tc_row_splitk(c, Y, W2, b2, Z, T, k, d, p);
+    return cuda_status(launch_simt_row_splitk(c, static_cast<const float*>(Y),
+                                              static_cast<const float*>(W2), b2, Z, T, k, d, p),
+                       "fp32 split-K launch");
+  }
+  const size_t esize = dtype == TP_BF16 ? 2 : 4;
+  float* P = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(T) * k * esize));
+  TP_TRY(row_impl(Y, W2, P, T, k, d, p, dtype, stream));
+  return reduce_impl(P, b2, Z, T, d, p, stream);
+}
+
+tp_status tp_sync_status(void* stream) {
+  g_detail[0] = 0;
+  int dev = 0, sms = 0, cc = 0;
+  unsigned* addr = nullptr;
+  TP_TRY(device_state(&dev, &sms, &cc, &addr));
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(TP_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
+  unsigned word = 0;
+  e = cudaMemcpyFromSymbol(&word, g_tp_status_word, sizeof(word));
+  if (e != cudaSuccess) return fail(TP_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+  if (word != 0) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_tp_status_word, &zero, sizeof(zero));
+    if (e != cudaSuccess) return fail(TP_ERR_CUDA, "status clear: %s", cudaGetErrorString(e));
+    return fail(TP_ERR_DEVICE_TIMEOUT, "device wait gave up (status bits 0x%x)", word);
+  }
+  return TP_OK;
+}
+
+void tp_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns == 0 ? 2000000000ull : ns); }
+
+void tp_debug_drop_load(int64_t stage_index) { g_debug_drop.store(stage_index < 0 ? -1 : stage_index); }
+
+const char* tp_status_string(int status) {
+  switch (status) {
+    case TP_OK: return "TP_OK";
+    case TP_ERR_INVALID_ARG: return "TP_ERR_INVALID_ARG: invalid argument";
+    case TP_ERR_INDIVISIBLE: return "TP_ERR_INDIVISIBLE: k is not divisible by p";
+    case TP_ERR_ALIGNMENT: return "TP_ERR_ALIGNMENT: pointer or pitch not aligned";
+    case TP_ERR_UNSUPPORTED: return "TP_ERR_UNSUPPORTED: unsupported combination";
+    case TP_ERR_CUDA: return "TP_ERR_CUDA: CUDA runtime error";
+    case TP_ERR_DEVICE_TIMEOUT: return "TP_ERR_DEVICE_TIMEOUT: a bounded device wait gave up";
+    case TP_ERR_WORKSPACE: return "TP_ERR_WORKSPACE: workspace missing or too small";
+    default: return "unknown tp_status";
+  }
+}
+
+const char* tp_last_error_detail(void) { return g_detail; }
+
+uint64_t tp_kernel_launch_count(void) { return g_launches.load(); }
+
+int tp_abi_version(void) { return TP_ABI_VERSION; }
+
+}  // extern "C"

@@ -1,0 +1,29 @@
+// Element-wise activations applied to each shard's slice of the hidden
+// layer.  The pairing lets them run locally because they are element-wise
+// ("Tensor parallel math", "The MLP block: column then row, one
+// all-reduce").  GELU is the tanh form; Swish is SiLU (beta = 1),
+// "Tensor Parallelism Explained" section 2.B.
+#pragma once
+
+#include <cmath>
+
+namespace tpk {
+
+enum ActKind : int { kActGeluTanh = 0, kActSwiglu = 1, kActIdentity = 2, kActRelu = 3 };
+
+__device__ __forceinline__ float gelu_tanh_f32(float h) {
+  const float kSqrt2OverPi = 0.7978845608028654f;
+  const float u = kSqrt2OverPi * (h + 0.044715f * h * h * h);
+  return 0.5f * h * (1.0f + tanhf(u));
+}
+
+__device__ __forceinline__ float silu_f32(float h) { return h / (1.0f + expf(-h)); }
+
+// Single-input activations (GELU / identity / ReLU).
+__device__ __forceinline__ float act_unary(int act, float h) {
+  if (act == kActGeluTanh) return gelu_tanh_f32(h);
+  if (act == kActRelu) return fmaxf(h, 0.0f);
+  return h;
+}
+
+}  // namespace tpk

@@ -1,0 +1,51 @@
+// Internal launchers shared by the C ABI translation unit and the kernel
+// translation units.  Not part of the public interface.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "tp_mlp.h"
+
+namespace tpk {
+
+struct LaunchCtx {
+  cudaStream_t stream;
+  int device;
+  int num_sms;
+  unsigned* err_word;    // device address of the per-device status word
+  uint64_t timeout_ns;   // limit of each bounded device wait
+  int64_t debug_drop;    // fault injection: pipeline slot whose load is skipped (-1: none)
+};
+
+// Counts one kernel launch (process-wide, thread-safe).
+void note_launch();
+
+// ---- fixed-order partial-sum reduction (tp_reduce.cu)
+cudaError_t launch_reduce(const LaunchCtx& c, const float* P, const float* b2, float* Z, int64_t T,
+                          int64_t d, int p);
+
+// ---- fp32 path, plain FMA, no TF32 (tp_simt_f32.cu)
+cudaError_t launch_simt_column(const LaunchCtx& c, const float* X, const float* W1,
+                               const float* Wup, const float* b1, float* Y, int64_t T, int64_t d,
+                               int64_t k, int p, int act);
+cudaError_t launch_simt_row(const LaunchCtx& c, const float* Y, const float* W2, float* P,
+                            int64_t T, int64_t k, int64_t d, int p);
+cudaError_t launch_simt_row_splitk(const LaunchCtx& c, const float* Y, const float* W2,
+                                   const float* b2, float* Z, int64_t T, int64_t k, int64_t d,
+                                   int p);
+
+// ---- bf16 tensor-core path, tcgen05 + TMEM + TMA (tp_gemm_sm100.cu)
+tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, const void* Wup,
+                           const void* b1, void* Y, int64_t T, int64_t d, int64_t k, int p,
+                           int act);
+tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float* P, int64_t T,
+                        int64_t k, int64_t d, int p);
+tp_status launch_tc_row_splitk(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
+                               float* Z, int64_t T, int64_t k, int64_t d, int p);
+
+// Records a human-readable detail for tp_last_error_detail().
+void set_error_detail(const char* fmt, ...);
+
+}  // namespace tpk

@@ -1,0 +1,137 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every function the header declares, and rejects bad arguments with the
+documented status codes before touching the device."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import megatron_tensor_sharded_b200 as tp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tp_mlp.h")
+
+FAKE = 0x10000      # never dereferenced: every case below fails validation first
+FAKE2 = 0x20000
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(tp_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary_calls():
+    names = declared_functions()
+    for required in ("tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(tp.LIB_PATH)
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_abi_version_matches_header():
+    m = re.search(r"#define TP_ABI_VERSION (\d+)", open(HEADER).read())
+    assert tp.tp_abi_version() == int(m.group(1))
+
+
+def test_status_strings():
+    for code, name in tp.STATUS.items():
+        assert tp.tp_status_string(code).startswith(name)
+    assert "unknown" in tp.tp_status_string(99)
+
+
+def _col(**kw):
+    a = dict(X=FAKE, W1=FAKE, W_up=None, b1=None, Y=FAKE2, T=4, d=64, k=256, p=4,
+             dtype=tp.TP_BF16, act=tp.TP_ACT_GELU_TANH)
+    a.update(kw)
+    return tp.tp_column_linear(a["X"], a["W1"], a["W_up"], a["b1"], a["Y"], a["T"], a["d"], a["k"],
+                               a["p"], a["dtype"], a["act"], stream=0, check=False)
+
+
+def test_column_validation():
+    assert _col(p=0) == 1
+    assert _col(p=-3) == 1
+    assert _col(k=10, p=4) == 2                          # indivisible (k % p != 0)
+    assert _col(k=64, p=5) == 2
+    assert _col(d=12) == 3                               # bf16 pitch not 16-byte multiple
+    assert _col(k=4 * 12, p=4) == 3                      # s = 12
+    assert _col(X=FAKE + 2) == 3                         # misaligned pointer
+    assert _col(X=None) == 1
+    assert _col(act=tp.TP_ACT_SWIGLU, W_up=None) == 1    # SwiGLU needs W_up
+    assert _col(act=7) == 1
+    assert _col(dtype=5) == 1
+    assert _col(d=0) == 1
+    assert _col(T=-1) == 1
+    assert _col(dtype=tp.TP_F32, X=FAKE + 2) == 3        # fp32 needs 4-byte alignment
+
+
+def test_empty_input_is_a_no_op():
+    n0 = tp.tp_kernel_launch_count()
+    assert _col(T=0, X=None, Y=None) == 0
+    assert tp.tp_row_linear(None, None, None, 0, 256, 64, 4, tp.TP_BF16, stream=0, check=False) == 0
+    assert tp.tp_reduce_partials(None, None, None, 0, 64, 4, stream=0, check=False) == 0
+    assert tp.tp_mlp_block(None, None, None, None, None, None, None, None, 0, 0, 64, 256, 4,
+                           tp.TP_BF16, tp.TP_ACT_GELU_TANH, stream=0, check=False) == 0
+    assert tp.tp_kernel_launch_count() == n0
+
+
+def test_row_and_reduce_validation():
+    assert tp.tp_row_linear(FAKE, FAKE, FAKE2, 4, 250, 64, 4, tp.TP_BF16, stream=0, check=False) == 2
+    assert tp.tp_row_linear(FAKE, FAKE, None, 4, 256, 64, 4, tp.TP_BF16, stream=0, check=False) == 1
+    assert tp.tp_row_linear(FAKE, FAKE, FAKE2 + 4, 4, 256, 64, 4, tp.TP_BF16, stream=0, check=False) == 3
+    assert tp.tp_reduce_partials(FAKE, None, FAKE2, 4, 64, 0, stream=0, check=False) == 1
+    assert tp.tp_reduce_partials(None, None, FAKE2, 4, 64, 2, stream=0, check=False) == 1
+    # Z inside the partials range
+    assert tp.tp_reduce_partials(FAKE, None, FAKE + 64, 4, 64, 2, stream=0, check=False) == 1
+    assert tp.tp_reduce_partials(FAKE + 2, None, FAKE2, 4, 64, 2, stream=0, check=False) == 3
+
+
+def test_workspace_size_formula():
+    # bf16: hidden shards T*k*2 bytes, then p*T*d*4 bytes of partials, each
+    # rounded up to 256 bytes
+    T, d, k, p = 1000, 768, 3072, 2
+    ys = -(-T * k * 2 // 256) * 256
+    ps = -(-p * T * d * 4 // 256) * 256
+    assert tp.tp_mlp_block_workspace_size(T, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH) == ys + ps
+    assert tp.tp_mlp_block_workspace_size(T, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH,
+                                          tp.TP_FLAG_SPLITK_FUSED) == ys
+    assert tp.tp_mlp_block_workspace_size(4, 512, 2048, 4, tp.TP_F32, tp.TP_ACT_GELU_TANH) == \
+        -(-4 * 2048 * 4 // 256) * 256 + -(-4 * 4 * 512 * 4 // 256) * 256
+    assert tp.tp_mlp_block_workspace_size(4, 512, 2047, 4, tp.TP_F32, tp.TP_ACT_GELU_TANH) == 0
+
+
+def test_block_validation():
+    def blk(**kw):
+        a = dict(X=FAKE, W1=FAKE, W_up=None, b1=None, W2=FAKE, b2=None, Z=FAKE2, ws=0x40000,
+                 wsb=1 << 30, T=4, d=64, k=256, p=4, dtype=tp.TP_BF16, act=tp.TP_ACT_GELU_TANH,
+                 flags=0)
+        a.update(kw)
+        return tp.tp_mlp_block(a["X"], a["W1"], a["W_up"], a["b1"], a["W2"], a["b2"], a["Z"],
+                               a["ws"], a["wsb"], a["T"], a["d"], a["k"], a["p"], a["dtype"],
+                               a["act"], a["flags"], stream=0, check=False)
+    assert blk(wsb=16) == 7
+    assert blk(ws=None) == 7
+    assert blk(ws=0x40000 + 16) == 3
+    assert blk(k=255) == 2
+    assert blk(flags=8) == 1
+    assert blk(k=4 * 72, flags=tp.TP_FLAG_SPLITK_FUSED) == 4   # s = 72, not a multiple of 64
+    assert blk(Z=None) == 1
+
+
+def test_valid_call_without_gpu_fails_loudly():
+    """With no CUDA device the library reports a CUDA error; it never falls
+    back to a host computation."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st = _col()
+    assert st == 5
+    with pytest.raises(tp.TPError):
+        tp.tp_column_linear(FAKE, FAKE, None, None, FAKE2, 4, 64, 256, 4, tp.TP_BF16,
+                            tp.TP_ACT_GELU_TANH, stream=0)

@@ -1,0 +1,152 @@
+"""GPU parity of the bf16 tensor-core path (tcgen05 + TMEM + TMA) against
+the oracle: bit-exact on small-integer inputs (every intermediate an exact
+integer), max|gpu - oracle| / max|oracle| <= 1e-2 on the workloads, which at
+full size are checked on sampled token rows (each output row depends only on
+its own input row, so the oracle can compute any row on its own)."""
+
+import numpy as np
+import pytest
+import torch
+
+import megatron_tensor_sharded_b200 as tp
+from oracle import tp_oracle as O
+import workloads as W
+from gpu_util import DeviceBlock, bits, host_f32
+
+pytestmark = pytest.mark.gpu
+
+TOL_BF16 = 1e-2
+
+
+def _oracle(inp, p, act, rows=None):
+    X = inp.values("X")
+    if rows is not None:
+        X = X[rows]
+    return O.mlp_sharded(X, inp.values("W1"), inp.values("b1"), inp.values("W2"),
+                         inp.values("b2"), p, act, W_up=inp.values("W_up"))
+
+
+@pytest.mark.parametrize("T,d,s,p", [(1, 64, 64, 1), (3, 64, 8, 4), (130, 200, 40, 4),
+                                     (257, 128, 72, 2), (128, 64, 256, 1), (129, 192, 128, 3),
+                                     (300, 136, 320, 2)])
+@pytest.mark.parametrize("act", ["identity", "relu"])
+def test_small_integer_inputs_bit_exact(T, d, s, p, act):
+    """Ragged token counts (not multiples of 128), K tails (d, s not
+    multiples of 64), N tails (k, d not multiples of 256), shards narrower
+    than a tile: all exact."""
+    k = s * p
+    inp = W.small_integer_inputs(T, d, k, seed=T + 7 * d + s, lo=-1, hi=1, act=act, dtype="bf16")
+    ref = _oracle(inp, p, act)
+    blk = DeviceBlock(inp, T, d, k, p, act)
+    blk.column()
+    blk.row()
+    blk.reduce()
+    blk.sync()
+    Y = host_f32(blk.Y)
+    for i in range(p):
+        assert np.array_equal(Y[i], ref["Y"][i].astype(np.float32)), i
+    assert np.array_equal(bits(host_f32(blk.P)), bits(ref["P"]))
+    assert np.array_equal(bits(host_f32(blk.Z)), bits(ref["Z"]))
+    blk.Z.fill_(float("nan"))
+    blk.block()
+    blk.sync()
+    assert np.array_equal(bits(host_f32(blk.Z)), bits(ref["Z"]))
+    if s % 64 == 0:
+        blk.Z.fill_(float("nan"))
+        blk.block(tp.TP_FLAG_SPLITK_FUSED)
+        blk.sync()
+        assert np.array_equal(bits(host_f32(blk.Z)), bits(ref["Z"]))
+
+
+def _random_bf16(T, d, k, act, with_bias, seed):
+    rng = np.random.default_rng(seed)
+    c = W.f32_to_bf16_bits
+    X = c(rng.standard_normal((T, d), dtype=np.float32))
+    W1 = c(rng.standard_normal((d, k), dtype=np.float32) * 0.05)
+    Wu = c(rng.standard_normal((d, k), dtype=np.float32) * 0.05) if act == "swiglu" else None
+    b1 = c(rng.standard_normal(k, dtype=np.float32) * 0.05) if with_bias else None
+    W2 = c(rng.standard_normal((k, d), dtype=np.float32) * 0.05)
+    b2 = rng.standard_normal(d, dtype=np.float32) * 0.05 if with_bias else None
+    return W.Inputs(X, W1, Wu, b1, W2, b2, "bf16")
+
+
+@pytest.mark.parametrize("act,with_bias", [("gelu_tanh", True), ("gelu_tanh", False),
+                                           ("swiglu", False), ("swiglu", True)])
+@pytest.mark.parametrize("T,d,k,p", [(200, 256, 1024, 4), (77, 192, 768, 2), (513, 512, 1536, 3)])
+def test_random_inputs(act, with_bias, T, d, k, p):
+    inp = _random_bf16(T, d, k, act, with_bias, seed=T + d + k + p)
+    ref = _oracle(inp, p, act)
+    blk = DeviceBlock(inp, T, d, k, p, act)
+    blk.column()
+    blk.row()
+    blk.reduce()
+    blk.sync()
+    Y = host_f32(blk.Y)
+    for i in range(p):
+        assert O.rel_err(Y[i], ref["Y"][i]) <= TOL_BF16, i
+    assert O.rel_err(host_f32(blk.P), ref["P"]) <= TOL_BF16
+    assert O.rel_err(host_f32(blk.Z), ref["Z"]) <= TOL_BF16
+    for flags in (tp.TP_FLAG_NONE, tp.TP_FLAG_SPLITK_FUSED):
+        if flags and (k // p) % 64:
+            continue
+        blk.Z.fill_(float("nan"))
+        blk.block(flags)
+        blk.sync()
+        assert O.rel_err(host_f32(blk.Z), ref["Z"]) <= TOL_BF16, flags
+
+
+def test_gpt2_config_full():
+    """GPT-2-small MLP, T=1024 d=768 k=3072 p=2, GELU(tanh), b1 and b2: every
+    output element against the oracle."""
+    w = W.WORKLOADS["gpt2"]
+    inp = W.make_inputs(w)
+    ref = _oracle(inp, w.p, w.act)
+    blk = DeviceBlock(inp, w.T, w.d, w.k, w.p, w.act)
+    blk.column()
+    blk.row()
+    blk.reduce()
+    blk.sync()
+    Y = host_f32(blk.Y)
+    for i in range(w.p):
+        assert O.rel_err(Y[i], ref["Y"][i]) <= TOL_BF16
+    assert O.rel_err(host_f32(blk.P), ref["P"]) <= TOL_BF16
+    assert O.rel_err(host_f32(blk.Z), ref["Z"]) <= TOL_BF16
+    for flags in (tp.TP_FLAG_NONE, tp.TP_FLAG_SPLITK_FUSED):
+        blk.Z.fill_(float("nan"))
+        blk.block(flags)
+        blk.sync()
+        assert O.rel_err(host_f32(blk.Z), ref["Z"]) <= TOL_BF16
+
+
+def _sample_rows(T):
+    cand = [0, 1, 127, 128, 129, 255, 1000, 2047, 2048, 3071, T - 129, T - 2, T - 1]
+    return sorted({r for r in cand if 0 <= r < T})
+
+
+@pytest.mark.parametrize("name", ["wide", "decode", "llama"])
+def test_full_size_configs_sampled_rows(name):
+    """Full-size workloads, launched exactly as the bench launches them;
+    the oracle recomputes sampled token rows (all rows for decode)."""
+    w = W.WORKLOADS[name]
+    inp = W.make_inputs(w)
+    rows = list(range(w.T)) if w.T <= 32 else _sample_rows(w.T)
+    ref = _oracle(inp, w.p, w.act, rows=rows)
+    blk = DeviceBlock(inp, w.T, w.d, w.k, w.p, w.act)
+    blk.column()
+    blk.row()
+    blk.reduce()
+    blk.sync()
+    idx = torch.tensor(rows, device="cuda")
+    Y = host_f32(blk.Y.index_select(1, idx))
+    for i in range(w.p):
+        assert O.rel_err(Y[i], ref["Y"][i]) <= TOL_BF16, i
+    assert O.rel_err(host_f32(blk.P.index_select(1, idx)), ref["P"]) <= TOL_BF16
+    assert O.rel_err(host_f32(blk.Z.index_select(0, idx)), ref["Z"]) <= TOL_BF16
+    assert not torch.isnan(blk.Z).any().item()
+    for flags in (tp.TP_FLAG_NONE, tp.TP_FLAG_SPLITK_FUSED):
+        Z2 = torch.full_like(blk.Z, float("nan"))
+        ws = blk.block(flags, Z=Z2)
+        blk.sync()
+        del ws
+        assert O.rel_err(host_f32(Z2.index_select(0, idx)), ref["Z"]) <= TOL_BF16, flags
+        assert not torch.isnan(Z2).any().item()
