@@ -282,34 +282,53 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
                                                 tp.TP_FLAG_SPLITK_FUSED)
         ws_split = torch.empty(nbytes, dtype=torch.uint8, device=device)
 
-        def step(ev=None):
+        def step(ev=None, st=None):
+            st = stream if st is None else st
             if ev is not None:
-                ev[0].record(stream)
+                ev[0].record(st)
             tp.tp_mlp_block(X, W1, Wu, b1, W2, b2, Z, ws_split, nbytes, w.T, w.d, w.k, w.p, dtype,
-                            act, tp.TP_FLAG_SPLITK_FUSED, stream=stream)
+                            act, tp.TP_FLAG_SPLITK_FUSED, stream=st)
             if ev is not None:
                 for e in ev[1:]:
-                    e.record(stream)
+                    e.record(st)
     else:
-        def step(ev=None):
+        def step(ev=None, st=None):
+            st = stream if st is None else st
             if ev is not None:
-                ev[0].record(stream)
-            tp.tp_column_linear(X, W1, Wu, b1, Y, w.T, w.d, w.k, w.p, dtype, act, stream=stream)
+                ev[0].record(st)
+            tp.tp_column_linear(X, W1, Wu, b1, Y, w.T, w.d, w.k, w.p, dtype, act, stream=st)
             if ev is not None:
-                ev[1].record(stream)
-            tp.tp_row_linear(Y, W2, P, w.T, w.k, w.d, w.p, dtype, stream=stream)
+                ev[1].record(st)
+            tp.tp_row_linear(Y, W2, P, w.T, w.k, w.d, w.p, dtype, stream=st)
             if ev is not None:
-                ev[2].record(stream)
-            tp.tp_reduce_partials(P, b2, Z, w.T, w.d, w.p, stream=stream)
+                ev[2].record(st)
+            tp.tp_reduce_partials(P, b2, Z, w.T, w.d, w.p, stream=st)
             if ev is not None:
-                ev[3].record(stream)
+                ev[3].record(st)
 
     for _ in range(a.warmup):
         flush.zero_()
         step()
     tp.tp_sync_status(stream)
 
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(a.steps)]
+    # The step is captured once as a CUDA graph (timing events between the
+    # three calls become event-record nodes) and replayed: no host work per
+    # step.  Kernels captured per step = launch-counter delta during capture.
+    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
+    graph = None
+    per_step_kernels = None
+    if not a.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        n_cap = tp.tp_kernel_launch_count()
+        with torch.cuda.graph(graph):
+            cap = torch.cuda.current_stream()
+            step(evs, cap)
+        per_step_kernels = tp.tp_kernel_launch_count() - n_cap
+        for _ in range(a.warmup):
+            flush.zero_()
+            graph.replay()
+        torch.cuda.synchronize(device)
+    col_ms, row_ms, red_ms, step_ms = [], [], [], []
     with ClockSampler(local_rank) as clocks:
         barrier()
         torch.cuda.synchronize(device)
@@ -317,16 +336,22 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
         t_wall = time.perf_counter()
         for i in range(a.steps):
             flush.zero_()
-            step(evs[i])
+            if graph is not None:
+                graph.replay()
+            else:
+                step(evs, stream)
+            torch.cuda.synchronize(device)
+            col_ms.append(evs[0].elapsed_time(evs[1]))
+            row_ms.append(evs[1].elapsed_time(evs[2]))
+            red_ms.append(evs[2].elapsed_time(evs[3]))
+            step_ms.append(evs[0].elapsed_time(evs[3]))
         torch.cuda.synchronize(device)
         t_wall = time.perf_counter() - t_wall
         launches = tp.tp_kernel_launch_count() - n0
+        if graph is not None:
+            launches = per_step_kernels * a.steps
         barrier()
     tp.tp_sync_status(stream)
-    col_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    row_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    red_ms = [e[2].elapsed_time(e[3]) for e in evs]
-    step_ms = [e[0].elapsed_time(e[3]) for e in evs]
     local = [statistics.mean(step_ms), statistics.mean(col_ms), statistics.mean(row_ms),
              statistics.mean(red_ms), float(launches)]
     ms_step, ms_col, ms_row, ms_red, launches = reduce_max(local, dist if world > 1 else None, device)
@@ -398,6 +423,7 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "T": w.T, "d": w.d, "k": w.k, "p": w.p, "act": w.act,
                    "mode": a.mode, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "launch": "eager" if graph is None else "cuda-graph replay of the three C-ABI calls",
                    "l2": "flushed before every step (256 MiB write, outside the timed events)"},
         "pct_bf16_peak": 100.0 * value / (peaks["bf16_tflops"] * world) if w.dtype == "bf16" else None,
         "reduce": None if splitk else {"GB/s": reduce_bytes(w) / (ms_red * 1e-3) / 1e9,
@@ -432,6 +458,7 @@ def main(argv=None):
     ap.add_argument("--workload", choices=sorted(WL.WORKLOADS), default="gpt2")
     ap.add_argument("--mode", choices=["partials", "splitk"], default="partials")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the three calls eagerly")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args(argv)
     if a.warmup < 3:

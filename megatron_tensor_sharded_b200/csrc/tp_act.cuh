@@ -19,6 +19,30 @@ __device__ __forceinline__ float gelu_tanh_f32(float h) {
 
 __device__ __forceinline__ float silu_f32(float h) { return h / (1.0f + expf(-h)); }
 
+// Hardware tanh (PTX tanh.approx.f32, one MUFU operation, relative error
+// about 2^-11): used where the result is stored as bf16 (8 significant bits),
+// so its error stays well below the storage rounding.
+__device__ __forceinline__ float tanh_mufu(float x) {
+  float y;
+  asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float gelu_tanh_mufu(float h) {
+  const float kSqrt2OverPi = 0.7978845608028654f;
+  const float u = kSqrt2OverPi * (h + 0.044715f * h * h * h);
+  return 0.5f * h * (1.0f + tanh_mufu(u));
+}
+
+// SiLU(h) = h * sigmoid(h), with sigmoid(h) = (1 + tanh(h / 2)) / 2.
+__device__ __forceinline__ float silu_mufu(float h) { return h * (0.5f + 0.5f * tanh_mufu(0.5f * h)); }
+
+__device__ __forceinline__ float act_unary_mufu(int act, float h) {
+  if (act == kActGeluTanh) return gelu_tanh_mufu(h);
+  if (act == kActRelu) return fmaxf(h, 0.0f);
+  return h;
+}
+
 // Single-input activations (GELU / identity / ReLU).
 __device__ __forceinline__ float act_unary(int act, float h) {
   if (act == kActGeluTanh) return gelu_tanh_f32(h);

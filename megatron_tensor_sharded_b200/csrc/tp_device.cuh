@@ -99,6 +99,16 @@ __device__ __forceinline__ bool wait_teardown(uint32_t bar, uint32_t parity, con
   }
 }
 
+// ------------------------------------------------- programmatic dependent launch
+// Wait until every grid this one depends on has completed and its memory is
+// visible (a no-op when the launch has no programmatic dependency).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Allow the next grid in the stream to be scheduled (it still runs its own
+// pdl_wait before touching memory this grid produces or consumes).
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // -------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_map(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

@@ -1,0 +1,38 @@
+// Kernel launch with programmatic dependent launch allowed: the kernel may
+// start while the previous kernel in the stream finishes; every kernel of
+// this library calls griddepcontrol.wait before its first global memory
+// access, so the overlap only covers launch latency and prologues.
+// Setting TP_DISABLE_PDL=1 in the environment launches them plainly.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include <cstdlib>
+
+namespace tpk {
+
+inline bool pdl_allowed() {
+  static const bool on = [] {
+    const char* e = std::getenv("TP_DISABLE_PDL");
+    return !(e != nullptr && e[0] == '1');
+  }();
+  return on;
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_allowed() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
+}  // namespace tpk

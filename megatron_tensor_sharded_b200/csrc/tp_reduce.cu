@@ -9,7 +9,9 @@
 
 #include <cstdint>
 
+#include "tp_device.cuh"
 #include "tp_internal.h"
+#include "tp_launch.cuh"
 
 namespace tpk {
 namespace {
@@ -28,6 +30,8 @@ __global__ void __launch_bounds__(256) reduce_vec_kernel(const float4* __restric
                                                          const float* __restrict__ b2,
                                                          float4* __restrict__ Z, int64_t n4,
                                                          int64_t d4, int p_runtime) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n4;
        i += stride) {
@@ -56,6 +60,8 @@ __global__ void __launch_bounds__(256) reduce_scalar_kernel(const float* __restr
                                                             const float* __restrict__ b2,
                                                             float* __restrict__ Z, int64_t n,
                                                             int64_t d, int p) {
+  pdl_wait();
+  pdl_launch_dependents();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += stride) {
@@ -76,6 +82,7 @@ cudaError_t launch_reduce(const LaunchCtx& c, const float* P, const float* b2, f
                        (reinterpret_cast<uintptr_t>(Z) % 16 == 0) &&
                        (b2 == nullptr || reinterpret_cast<uintptr_t>(b2) % 16 == 0);
   const int threads = 256;
+  cudaError_t e = cudaSuccess;
   if (aligned && d % 4 == 0) {
     const int64_t n4 = n / 4;
     // Enough resident threads to keep ~p loads in flight per thread on every
@@ -88,22 +95,22 @@ cudaError_t launch_reduce(const LaunchCtx& c, const float* P, const float* b2, f
     const int64_t d4 = d / 4;
     dim3 g(static_cast<unsigned>(blocks));
     switch (p) {
-      case 1: reduce_vec_kernel<1><<<g, threads, 0, c.stream>>>(P4, b2, Z4, n4, d4, p); break;
-      case 2: reduce_vec_kernel<2><<<g, threads, 0, c.stream>>>(P4, b2, Z4, n4, d4, p); break;
-      case 3: reduce_vec_kernel<3><<<g, threads, 0, c.stream>>>(P4, b2, Z4, n4, d4, p); break;
-      case 4: reduce_vec_kernel<4><<<g, threads, 0, c.stream>>>(P4, b2, Z4, n4, d4, p); break;
-      case 8: reduce_vec_kernel<8><<<g, threads, 0, c.stream>>>(P4, b2, Z4, n4, d4, p); break;
-      default: reduce_vec_kernel<0><<<g, threads, 0, c.stream>>>(P4, b2, Z4, n4, d4, p); break;
+      case 1: e = launch_pdl(reduce_vec_kernel<1>, g, dim3(threads), 0, c.stream, P4, b2, Z4, n4, d4, p); break;
+      case 2: e = launch_pdl(reduce_vec_kernel<2>, g, dim3(threads), 0, c.stream, P4, b2, Z4, n4, d4, p); break;
+      case 3: e = launch_pdl(reduce_vec_kernel<3>, g, dim3(threads), 0, c.stream, P4, b2, Z4, n4, d4, p); break;
+      case 4: e = launch_pdl(reduce_vec_kernel<4>, g, dim3(threads), 0, c.stream, P4, b2, Z4, n4, d4, p); break;
+      case 8: e = launch_pdl(reduce_vec_kernel<8>, g, dim3(threads), 0, c.stream, P4, b2, Z4, n4, d4, p); break;
+      default: e = launch_pdl(reduce_vec_kernel<0>, g, dim3(threads), 0, c.stream, P4, b2, Z4, n4, d4, p); break;
     }
   } else {
     int64_t blocks = (n + threads - 1) / threads;
     const int64_t cap = static_cast<int64_t>(c.num_sms) * 8;
     if (blocks > cap) blocks = cap;
-    reduce_scalar_kernel<<<static_cast<unsigned>(blocks), threads, 0, c.stream>>>(P, b2, Z, n, d,
-                                                                                  p);
+    e = launch_pdl(reduce_scalar_kernel, dim3(static_cast<unsigned>(blocks)), dim3(threads), 0,
+                   c.stream, P, b2, Z, n, d, p);
   }
   note_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace tpk

@@ -11,7 +11,9 @@
 #include <cstdint>
 
 #include "tp_act.cuh"
+#include "tp_device.cuh"
 #include "tp_internal.h"
+#include "tp_launch.cuh"
 
 namespace tpk {
 namespace {
@@ -69,6 +71,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtArgs a) {
   const int64_t m0 = static_cast<int64_t>(blockIdx.y) * TM;
   const int64_t n0 = static_cast<int64_t>(blockIdx.x) * TN;
   const int64_t batch = blockIdx.z;
+  pdl_wait();
+  pdl_launch_dependents();
 
   float acc[4][4], accu[4][4];
 #pragma unroll
@@ -142,9 +146,9 @@ template <int KIND>
 cudaError_t run(const LaunchCtx& c, const SimtArgs& a, int64_t batches) {
   dim3 grid(static_cast<unsigned>((a.N + TN - 1) / TN), static_cast<unsigned>((a.M + TM - 1) / TM),
             static_cast<unsigned>(batches));
-  simt_gemm_kernel<KIND><<<grid, 256, 0, c.stream>>>(a);
+  const cudaError_t e = launch_pdl(simt_gemm_kernel<KIND>, grid, dim3(256), 0, c.stream, a);
   note_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace
