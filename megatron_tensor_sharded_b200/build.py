@@ -1,6 +1,9 @@
 """Build libtpmlp.so in-tree with nvcc for sm_100a.
 
-    python -m megatron_tensor_sharded_b200.build [--force] [--verbose]
+    python megatron_tensor_sharded_b200/build.py [--force] [--verbose] [--ptxas-verbose]
+
+(Run it as a script, not through the package: importing the package loads the
+library this script builds.)
 
 Objects go to ``_build/`` at the repository root; the shared library is
 written next to this file so that the binding finds it without installation.
