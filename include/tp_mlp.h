@@ -148,6 +148,30 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
                        int64_t T, int64_t d, int64_t k, int p,
                        tp_dtype dtype, tp_act act, int flags, void* stream);
 
+/*
+ * tp_mlp_block without a caller workspace, for callers that cannot allocate
+ * device memory (a plugin inside a host framework that owns the whole device
+ * memory pool, or a latency-critical loop that cannot afford cudaMalloc's
+ * implicit device synchronisation).  The pages have no counterpart: this is
+ * a deployment convenience, not part of the method.
+ *
+ * Same arguments and result as tp_mlp_block, minus the workspace: the hidden
+ * shards and the partials live in one 16 MiB array of device memory inside
+ * the library (held by every GPU that loads the library until the process
+ * exits).  Nothing is allocated by the call.
+ *   - Problems whose scratch, tp_mlp_block_workspace_size(...), exceeds
+ *     16 MiB are rejected with TP_ERR_WORKSPACE.
+ *   - All calls share that array.  Calls whose kernels overlap on one GPU
+ *     (different streams or host threads) overwrite each other's scratch:
+ *     issue them on one stream, one after another.
+ *   - The first call on each device looks up the array's device address;
+ *     make that first call before any stream capture begins.
+ */
+tp_status tp_mlp_block_noalloc(const void* X, const void* W1, const void* W_up, const void* b1,
+                               const void* W2, const float* b2, float* Z,
+                               int64_t T, int64_t d, int64_t k, int p,
+                               tp_dtype dtype, tp_act act, int flags, void* stream);
+
 /* Workspace bytes tp_mlp_block needs for these arguments (0 if invalid). */
 size_t tp_mlp_block_workspace_size(int64_t T, int64_t d, int64_t k, int p,
                                    tp_dtype dtype, tp_act act, int flags);

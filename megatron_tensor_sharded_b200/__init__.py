@@ -8,7 +8,7 @@ kernels.  Arguments that are device buffers accept a ``torch.Tensor`` (its
 ``stream=None`` means torch's current CUDA stream.
 
 Importing this package fails loudly when the shared library has not been
-built (``python -m megatron_tensor_sharded_b200.build``): there is no CPU or
+built (``python megatron_tensor_sharded_b200/build.py``): there is no CPU or
 PyTorch fallback.
 """
 
@@ -21,6 +21,7 @@ __all__ = [
     "TPError", "TP_F32", "TP_BF16", "TP_ACT_GELU_TANH", "TP_ACT_SWIGLU", "TP_ACT_IDENTITY",
     "TP_ACT_RELU", "TP_FLAG_NONE", "TP_FLAG_SPLITK_FUSED", "STATUS", "ACT", "DTYPE",
     "tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
+    "tp_mlp_block_noalloc",
     "tp_mlp_block_workspace_size", "tp_sync_status", "tp_set_wait_timeout_ns",
     "tp_debug_drop_load", "tp_status_string", "tp_last_error_detail",
     "tp_kernel_launch_count", "tp_abi_version", "LIB_PATH",
@@ -49,7 +50,7 @@ class TPError(RuntimeError):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is not built; run "
-                          "`python -m megatron_tensor_sharded_b200.build` (nvcc, sm_100a)")
+                          "`python megatron_tensor_sharded_b200/build.py` (nvcc, sm_100a)")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i64, i32, u64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_uint64, ctypes.c_size_t
     lib.tp_column_linear.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32, vp]
@@ -57,6 +58,8 @@ def _load() -> ctypes.CDLL:
     lib.tp_reduce_partials.argtypes = [vp, vp, vp, i64, i64, i32, vp]
     lib.tp_mlp_block.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sz, i64, i64, i64, i32, i32, i32,
                                  i32, vp]
+    lib.tp_mlp_block_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32,
+                                         i32, vp]
     lib.tp_mlp_block_workspace_size.argtypes = [i64, i64, i64, i32, i32, i32, i32]
     lib.tp_mlp_block_workspace_size.restype = sz
     lib.tp_sync_status.argtypes = [vp]
@@ -72,6 +75,7 @@ def _load() -> ctypes.CDLL:
     lib.tp_kernel_launch_count.restype = u64
     lib.tp_abi_version.argtypes = []
     for f in ("tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
+              "tp_mlp_block_noalloc",
               "tp_sync_status", "tp_abi_version"):
         getattr(lib, f).restype = i32
     return lib
@@ -129,6 +133,16 @@ def tp_mlp_block(X, W1, W_up, b1, W2, b2, Z, workspace, workspace_bytes, T, d, k
     return _check(_lib.tp_mlp_block(_ptr(X), _ptr(W1), _ptr(W_up), _ptr(b1), _ptr(W2), _ptr(b2),
                                     _ptr(Z), _ptr(workspace), workspace_bytes, T, d, k, p, dtype,
                                     act, flags, _stream(stream)), check)
+
+
+def tp_mlp_block_noalloc(X, W1, W_up, b1, W2, b2, Z, T, d, k, p, dtype, act,
+                         flags=TP_FLAG_NONE, stream=None, check=True):
+    """The whole block without a caller workspace (for callers that cannot
+    allocate device memory): scratch comes from a fixed 16 MiB array inside
+    the library, shared by all calls, so calls must not overlap on the GPU."""
+    return _check(_lib.tp_mlp_block_noalloc(_ptr(X), _ptr(W1), _ptr(W_up), _ptr(b1), _ptr(W2),
+                                            _ptr(b2), _ptr(Z), T, d, k, p, dtype, act, flags,
+                                            _stream(stream)), check)
 
 
 def tp_mlp_block_workspace_size(T, d, k, p, dtype, act, flags=TP_FLAG_NONE) -> int:
