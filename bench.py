@@ -4,11 +4,14 @@
                     [--mode partials|splitk] [--impl tp|reference]
 
 One step = one pass of the whole hot path over one batch of synthetic input:
-column-parallel GEMM + activation (all p shards), row-parallel GEMM to p fp32
-partials, fixed-order partial-sum reduction.  Each of the three C-ABI calls is
-bracketed by CUDA events on the launching stream, so the per-kernel durations
-(for the roofline figure) and the step time come from the same timed steps.
-L2 is flushed (a 256 MiB write) before every step, outside the events.
+tp_mlp_block, i.e. the column-parallel GEMM + activation (all p shards), the
+row-parallel GEMM to p fp32 partials and the fixed-order partial-sum
+reduction (one persistent launch on the bf16 path).  The step is captured
+once as a CUDA graph and replayed; CUDA events on the launching stream
+bracket each replay.  A second loop times the same block as the three
+separate C-ABI calls, with events between them, for the per-kernel
+breakdown (column GEMM, row GEMM, reduction GB/s).  L2 is flushed (a 256 MiB
+write) before every step, outside the events.
 
 With N > 1 (torchrun) every rank runs an independent replica on its own GPU:
 the block is single-GPU by design (the p shards are simulated on one device),
@@ -272,98 +275,104 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
     P = torch.empty((w.p, w.T, w.d), dtype=torch.float32, device=device)
     Z = torch.empty((w.T, w.d), dtype=torch.float32, device=device)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
-    splitk = a.mode == "splitk"
     stream = torch.cuda.current_stream(device)
+    flags = tp.TP_FLAG_SPLITK_FUSED if a.mode == "splitk" else tp.TP_FLAG_NONE
+    if a.mode == "unfused":
+        flags = tp.TP_FLAG_UNFUSED
+    nbytes = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, w.p, dtype, act, flags)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
 
-    if splitk:
-        # split-K over shards: the row layer accumulates every shard in TMEM
-        # and writes Z directly; it is reached through the block call
-        nbytes = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, w.p, dtype, act,
-                                                tp.TP_FLAG_SPLITK_FUSED)
-        ws_split = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    def block_step(st):
+        tp.tp_mlp_block(X, W1, Wu, b1, W2, b2, Z, ws, nbytes, w.T, w.d, w.k, w.p, dtype, act,
+                        flags, stream=st)
 
-        def step(ev=None, st=None):
-            st = stream if st is None else st
-            if ev is not None:
-                ev[0].record(st)
-            tp.tp_mlp_block(X, W1, Wu, b1, W2, b2, Z, ws_split, nbytes, w.T, w.d, w.k, w.p, dtype,
-                            act, tp.TP_FLAG_SPLITK_FUSED, stream=st)
-            if ev is not None:
-                for e in ev[1:]:
-                    e.record(st)
-    else:
-        def step(ev=None, st=None):
-            st = stream if st is None else st
-            if ev is not None:
-                ev[0].record(st)
-            tp.tp_column_linear(X, W1, Wu, b1, Y, w.T, w.d, w.k, w.p, dtype, act, stream=st)
-            if ev is not None:
-                ev[1].record(st)
-            tp.tp_row_linear(Y, W2, P, w.T, w.k, w.d, w.p, dtype, stream=st)
-            if ev is not None:
-                ev[2].record(st)
-            tp.tp_reduce_partials(P, b2, Z, w.T, w.d, w.p, stream=st)
-            if ev is not None:
-                ev[3].record(st)
+    def calls_step(st, ev):
+        ev[0].record(st)
+        tp.tp_column_linear(X, W1, Wu, b1, Y, w.T, w.d, w.k, w.p, dtype, act, stream=st)
+        ev[1].record(st)
+        tp.tp_row_linear(Y, W2, P, w.T, w.k, w.d, w.p, dtype, stream=st)
+        ev[2].record(st)
+        tp.tp_reduce_partials(P, b2, Z, w.T, w.d, w.p, stream=st)
+        ev[3].record(st)
 
-    for _ in range(a.warmup):
-        flush.zero_()
-        step()
-    tp.tp_sync_status(stream)
-
-    # The step is captured once as a CUDA graph (timing events between the
-    # three calls become event-record nodes) and replayed: no host work per
-    # step.  Kernels captured per step = launch-counter delta during capture.
-    evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(4)]
-    graph = None
-    per_step_kernels = None
-    if not a.no_graph:
-        graph = torch.cuda.CUDAGraph()
-        n_cap = tp.tp_kernel_launch_count()
-        with torch.cuda.graph(graph):
-            cap = torch.cuda.current_stream()
-            step(evs, cap)
-        per_step_kernels = tp.tp_kernel_launch_count() - n_cap
+    def capture(fn):
+        """Warm up eagerly, then capture one step as a CUDA graph; returns
+        (graph, kernels of this library per step)."""
         for _ in range(a.warmup):
             flush.zero_()
-            graph.replay()
+            fn(stream)
+        tp.tp_sync_status(stream)
+        if a.no_graph:
+            return None, None
+        g = torch.cuda.CUDAGraph()
+        n0 = tp.tp_kernel_launch_count()
+        with torch.cuda.graph(g):
+            fn(torch.cuda.current_stream())
+        per_step = tp.tp_kernel_launch_count() - n0
+        for _ in range(a.warmup):
+            flush.zero_()
+            g.replay()
         torch.cuda.synchronize(device)
-    col_ms, row_ms, red_ms, step_ms = [], [], [], []
+        return g, per_step
+
+    # ---- the timed region: K steps of the block, one graph replay each
+    g_block, k_block = capture(block_step)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    step_ms = []
     with ClockSampler(local_rank) as clocks:
         barrier()
         torch.cuda.synchronize(device)
         n0 = tp.tp_kernel_launch_count()
         t_wall = time.perf_counter()
-        for i in range(a.steps):
+        for _ in range(a.steps):
             flush.zero_()
-            if graph is not None:
-                graph.replay()
+            e0.record(stream)
+            if g_block is not None:
+                g_block.replay()
             else:
-                step(evs, stream)
+                block_step(stream)
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            step_ms.append(e0.elapsed_time(e1))
+        t_wall = time.perf_counter() - t_wall
+        launches = tp.tp_kernel_launch_count() - n0
+        if g_block is not None:
+            launches = k_block * a.steps
+        barrier()
+    tp.tp_sync_status(stream)
+    ms_step, launches = reduce_max([statistics.mean(step_ms), float(launches)],
+                                   dist if world > 1 else None, device)
+
+    # ---- per-kernel breakdown of the same block as three separate calls
+    kernels = None
+    if a.mode != "splitk" and not a.no_breakdown:
+        evs = [torch.cuda.Event(enable_timing=True, external=not a.no_graph) for _ in range(4)]
+        g_calls, _ = capture(lambda st: calls_step(st, evs))
+        col_ms, row_ms, red_ms, sum_ms = [], [], [], []
+        barrier()
+        for _ in range(a.steps):
+            flush.zero_()
+            if g_calls is not None:
+                g_calls.replay()
+            else:
+                calls_step(stream, evs)
             torch.cuda.synchronize(device)
             col_ms.append(evs[0].elapsed_time(evs[1]))
             row_ms.append(evs[1].elapsed_time(evs[2]))
             red_ms.append(evs[2].elapsed_time(evs[3]))
-            step_ms.append(evs[0].elapsed_time(evs[3]))
-        torch.cuda.synchronize(device)
-        t_wall = time.perf_counter() - t_wall
-        launches = tp.tp_kernel_launch_count() - n0
-        if graph is not None:
-            launches = per_step_kernels * a.steps
+            sum_ms.append(evs[0].elapsed_time(evs[3]))
         barrier()
-    tp.tp_sync_status(stream)
-    local = [statistics.mean(step_ms), statistics.mean(col_ms), statistics.mean(row_ms),
-             statistics.mean(red_ms), float(launches)]
-    ms_step, ms_col, ms_row, ms_red, launches = reduce_max(local, dist if world > 1 else None, device)
+        tp.tp_sync_status(stream)
+        kernels = dict(zip(["column", "row", "reduce", "sum"],
+                           reduce_max([statistics.mean(x) for x in (col_ms, row_ms, red_ms, sum_ms)],
+                                      dist if world > 1 else None, device)))
 
     # ---- end to end through the public block call, inputs from pinned host memory
     e2e = None
     if not a.no_e2e:
         Xh = X.cpu().pin_memory()
         Zh = torch.empty(Z.shape, dtype=Z.dtype).pin_memory()
-        flags = tp.TP_FLAG_SPLITK_FUSED if splitk else tp.TP_FLAG_NONE
-        nbytes = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, w.p, dtype, act, flags)
-        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
         Xd = torch.empty_like(X)
 
         def e2e_step():
@@ -377,45 +386,58 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
             e2e_step()
         torch.cuda.synchronize(device)
         barrier()
-        eev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(a.steps)]
-        for i in range(a.steps):
+        t_e2e = []
+        for _ in range(a.steps):
             flush.zero_()
-            eev[i][0].record(stream)
+            e0.record(stream)
             e2e_step()
-            eev[i][1].record(stream)
-        torch.cuda.synchronize(device)
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            t_e2e.append(e0.elapsed_time(e1))
         barrier()
         tp.tp_sync_status(stream)
-        e_ms = reduce_max([statistics.mean(x[0].elapsed_time(x[1]) for x in eev)],
-                          dist if world > 1 else None, device)[0]
+        e_ms = reduce_max([statistics.mean(t_e2e)], dist if world > 1 else None, device)[0]
         e2e = {"value": whole_job_value(w.gemm_flops(), world, e_ms) / 1e12, "unit": UNIT,
                "ms_per_step": e_ms, "h2d_bytes_per_step": Xh.numel() * Xh.element_size(),
                "d2h_bytes_per_step": Zh.numel() * Zh.element_size(),
-               "call": "tp_mlp_block"}
+               "call": "tp_mlp_block, X host->device and Z device->host inside the timed step"}
 
     peaks, peak_src = load_peaks()
     value = whole_job_value(w.gemm_flops(), world, ms_step) / 1e12
-    if splitk:
-        dom_name, dom_ms, dom_flops = "tp_mlp_block(split-K)", ms_col, w.gemm_flops()
-    elif ms_col >= ms_row:
-        dom_name, dom_ms, dom_flops = "tc_gemm column (tp_column_linear)", ms_col, column_flops(w)
-    else:
-        dom_name, dom_ms, dom_flops = "tc_gemm row partials (tp_row_linear)", ms_row, row_flops(w)
+    kernel_name = {"partials": "tc_block_kernel (fused block: column GEMM, row GEMM, fixed-order fold)",
+                   "splitk": "tc_block_kernel (fused block, split-K over shards)",
+                   "unfused": "column GEMM + row GEMM + fold (separate launches)"}[a.mode]
     if w.dtype == "bf16":
-        achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+        achieved = w.gemm_flops() / (ms_step * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
-        key = f"{w.name}/{'column' if 'column' in dom_name else 'row'}"
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": ncu_traffic(key), "kernel": dom_name,
-                "peak_source": f"{peak_src} bf16 burst"}
+                "frac": achieved / peak, "traffic": ncu_traffic(f"{w.name}/{a.mode}"),
+                "kernel": kernel_name,
+                "duration": "block step time (graph replay, CUDA events on the launching stream)",
+                "peak_source": f"{peak_src} bf16 dense (burst)"}
     else:
-        # fp32 path: latency bound; report its HBM rate
-        byts = column_bytes(w) if "column" in dom_name else row_bytes(w)
-        achieved = byts / (dom_ms * 1e-3) / 1e9
+        byts = column_bytes(w) + row_bytes(w) + reduce_bytes(w)
+        achieved = byts / (ms_step * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None, "kernel": dom_name,
+                "frac": achieved / peak, "traffic": None, "kernel": kernel_name,
                 "peak_source": f"{peak_src} hbm copy"}
+
+    breakdown = None
+    if kernels is not None:
+        def tfl(f, ms):
+            return f / (ms * 1e-3) / 1e12
+        breakdown = {
+            "column": {"ms": kernels["column"], "TFLOP/s": tfl(column_flops(w), kernels["column"]),
+                       "frac_bf16_peak": tfl(column_flops(w), kernels["column"]) / peaks["bf16_tflops"]},
+            "row": {"ms": kernels["row"], "TFLOP/s": tfl(row_flops(w), kernels["row"]),
+                    "frac_bf16_peak": tfl(row_flops(w), kernels["row"]) / peaks["bf16_tflops"]},
+            "reduce": {"ms": kernels["reduce"], "GB/s": reduce_bytes(w) / (kernels["reduce"] * 1e-3) / 1e9,
+                       "frac_hbm": reduce_bytes(w) / (kernels["reduce"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                       "bytes": reduce_bytes(w)},
+            "step_ms": kernels["sum"],
+            "how": "the three C-ABI calls as one graph, external timing events between them",
+        }
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
@@ -423,13 +445,11 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "T": w.T, "d": w.d, "k": w.k, "p": w.p, "act": w.act,
                    "mode": a.mode, "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "launch": "eager" if graph is None else "cuda-graph replay of the three C-ABI calls",
+                   "launch": "eager" if g_block is None else "cuda-graph replay of tp_mlp_block",
                    "l2": "flushed before every step (256 MiB write, outside the timed events)"},
         "pct_bf16_peak": 100.0 * value / (peaks["bf16_tflops"] * world) if w.dtype == "bf16" else None,
-        "reduce": None if splitk else {"GB/s": reduce_bytes(w) / (ms_red * 1e-3) / 1e9,
-                                       "ms": ms_red, "frac_hbm": reduce_bytes(w) / (ms_red * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                                       "bytes": reduce_bytes(w)},
-        "kernels_ms": {"column": ms_col, "row": ms_row, "reduce": ms_red},
+        "reduce": None if breakdown is None else breakdown["reduce"],
+        "unfused_breakdown": breakdown,
         "roofline": roof,
         "gpu_launches": int(launches),
         "clocks": clocks.summary(),
@@ -456,9 +476,10 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tp", "reference"], default="tp")
     ap.add_argument("--workload", choices=sorted(WL.WORKLOADS), default="gpt2")
-    ap.add_argument("--mode", choices=["partials", "splitk"], default="partials")
+    ap.add_argument("--mode", choices=["partials", "splitk", "unfused"], default="partials")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-graph", action="store_true", help="launch the three calls eagerly")
+    ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of graph replay")
+    ap.add_argument("--no-breakdown", action="store_true", help="skip the per-kernel loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     a = ap.parse_args(argv)
     if a.warmup < 3:

@@ -78,6 +78,10 @@ typedef enum {
  * partials and folding them.  Same result up to fp32 summation order (not
  * bit-identical to the fixed-order fold).  bf16 requires s % 64 == 0. */
 #define TP_FLAG_SPLITK_FUSED 1
+/* Launch the block as separate kernels (column, row, fold) instead of the
+ * default single persistent launch of the bf16 path.  Same bits either way;
+ * for comparisons and diagnostics. */
+#define TP_FLAG_UNFUSED 2
 
 /*
  * Column-parallel linear + activation, all p shards in one launch.
@@ -130,16 +134,20 @@ tp_status tp_reduce_partials(const float* partials, const float* b2, float* Z,
 /*
  * The whole block, Z = sum_i act(X W1_i + b1_i) W2_i  [+ b2]
  * ("Pairing them: the Megatron-LM MLP"; "The MLP block: column then row,
- * one all-reduce").  Default: tp_column_linear -> tp_row_linear ->
- * tp_reduce_partials on `stream`, with the hidden shards and the partials
- * in the caller's workspace.  With TP_FLAG_SPLITK_FUSED the second layer
- * accumulates over all shards and writes Z directly (no partials).
+ * one all-reduce").  Computes exactly what tp_column_linear ->
+ * tp_row_linear -> tp_reduce_partials compute (bit for bit), with the hidden
+ * shards and the partials in the caller's workspace.  bf16 runs both GEMM
+ * layers as one persistent launch (row-parallel tiles start as soon as the
+ * hidden rows they read are complete), then the fixed-order fold.  With
+ * TP_FLAG_SPLITK_FUSED the second layer accumulates over all shards and
+ * writes Z directly (no partials).
  *
  *   workspace        device memory of at least
  *                    tp_mlp_block_workspace_size(...) bytes, 256-byte aligned;
  *                    contents on return: hidden shards [p][T][s] at offset 0,
  *                    then (default mode) the partials [p][T][d] fp32 at the
- *                    next 256-byte boundary.
+ *                    next 256-byte boundary, then tile counters (reset on
+ *                    every call).
  *   other arguments  as for the three calls above.
  */
 tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const void* b1,

@@ -125,12 +125,14 @@ tp_status cuda_status(cudaError_t e, const char* what) {
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
+// Workspace layout: hidden shards Y, then (default mode) the fp32 partials,
+// then the fused kernel's tile counters, each at a 256-byte boundary.
 size_t workspace_bytes(int64_t T, int64_t d, int64_t k, int p, int dtype, int flags) {
   const size_t esize = dtype == TP_BF16 ? 2 : 4;
   size_t bytes = align256(static_cast<size_t>(T) * static_cast<size_t>(k) * esize);
   if (!(flags & TP_FLAG_SPLITK_FUSED))
     bytes += align256(static_cast<size_t>(p) * static_cast<size_t>(T) * static_cast<size_t>(d) * 4);
-  return bytes;
+  return bytes + block_counter_bytes(T, d);
 }
 
 tp_status column_impl(const void* X, const void* W1, const void* W_up, const void* b1, void* Y,
@@ -240,7 +242,8 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
   g_detail[0] = 0;
   TP_TRY(check_shape(T, d, k, p, dtype));
   TP_TRY(check_act(act, W_up));
-  if (flags & ~TP_FLAG_SPLITK_FUSED) return fail(TP_ERR_INVALID_ARG, "flags 0x%x", flags);
+  if (flags & ~(TP_FLAG_SPLITK_FUSED | TP_FLAG_UNFUSED))
+    return fail(TP_ERR_INVALID_ARG, "flags 0x%x", flags);
   const bool splitk = (flags & TP_FLAG_SPLITK_FUSED) != 0;
   if (splitk && dtype == TP_BF16 && (k / p) % 64 != 0)
     return fail(TP_ERR_UNSUPPORTED, "split-K over shards needs k/p %% 64 == 0 for bf16");
@@ -262,6 +265,22 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* Y = ws;
+  const size_t esize = dtype == TP_BF16 ? 2 : 4;
+  const size_t y_bytes = align256(static_cast<size_t>(T) * k * esize);
+  float* P = splitk ? nullptr : reinterpret_cast<float*>(ws + y_bytes);
+  if (dtype == TP_BF16 && !(flags & TP_FLAG_UNFUSED)) {
+    // Both GEMM layers in one persistent launch (its tile counters start at
+    // 0), then the fixed-order fold of the partials.
+    int* counters = reinterpret_cast<int*>(ws + need - block_counter_bytes(T, d));
+    const cudaError_t e = cudaMemsetAsync(counters, 0, block_counter_bytes(T, d),
+                                          static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return fail(TP_ERR_CUDA, "counter reset: %s", cudaGetErrorString(e));
+    LaunchCtx c{};
+    TP_TRY(make_ctx(stream, true, &c));
+    TP_TRY(launch_tc_block(c, X, W1, W_up, b1, W2, b2, Y, P, Z, counters, T, d, k, p, act, splitk));
+    if (splitk) return TP_OK;
+    return reduce_impl(P, b2, Z, T, d, p, stream);
+  }
   TP_TRY(column_impl(X, W1, W_up, b1, Y, T, d, k, p, dtype, act, stream));
   if (splitk) {
     LaunchCtx c{};
@@ -271,8 +290,6 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
                                               static_cast<const float*>(W2), b2, Z, T, k, d, p),
                        "fp32 split-K launch");
   }
-  const size_t esize = dtype == TP_BF16 ? 2 : 4;
-  float* P = reinterpret_cast<float*>(ws + align256(static_cast<size_t>(T) * k * esize));
   TP_TRY(row_impl(Y, W2, P, T, k, d, p, dtype, stream));
   return reduce_impl(P, b2, Z, T, d, p, stream);
 }

@@ -41,218 +41,14 @@
 #include <cstring>
 #include <mutex>
 
-#include "tp_act.cuh"
-#include "tp_device.cuh"
+#include "tp_gemm_parts.cuh"
 #include "tp_internal.h"
 #include "tp_launch.cuh"
 
 namespace tpk {
 namespace {
 
-constexpr int BM = 128;                     // tile rows = UMMA M
-constexpr int BK = 64;                      // k per slot: 64 bf16 = one 128-byte swizzle row
-constexpr int UK = 16;                      // k per tcgen05.mma (16-bit inputs)
-constexpr int A_BYTES = BM * BK * 2;        // 16 KiB
-constexpr int B_BOX_COLS = 64;              // one swizzle atom wide
-constexpr int B_CHUNK_BYTES = BK * B_BOX_COLS * 2;  // 8 KiB
-constexpr int NUM_EPI_WARPS = 8;
-constexpr int NUM_THREADS = 128 + 32 * NUM_EPI_WARPS;
-constexpr int CTRL_BYTES = 256;
-constexpr int SMEM_LIMIT = 232448;          // max dynamic shared memory per block
-
-template <int BN_>
-struct Cfg {
-  static constexpr int BN = BN_;
-  static constexpr int B_CHUNKS = BN / B_BOX_COLS;
-  static constexpr int B_BYTES = B_CHUNKS * B_CHUNK_BYTES;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - CTRL_BYTES) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr int TMEM_COLS = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTRL_BYTES;
-  static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
-  static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "tile width");
-  static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
-  static_assert(8 * (2 * STAGES + 5) + 16 <= CTRL_BYTES, "control block");
-};
-
-enum Mode : int { kModeColumn = 0, kModeColumnSwiglu = 1, kModeRowPartial = 2, kModeRowSplitK = 3 };
-
-struct TcParams {
-  int32_t T;             // tokens
-  int32_t n_total;       // valid output columns: k (column) or d (row)
-  int32_t s;             // shard width k/p
-  int32_t p;
-  int32_t m_tiles, n_tiles, batches, num_tiles;
-  int32_t k_blocks;      // pipeline slots per tile
-  int32_t kb_per_shard;  // split-K: slots per shard (s / 64)
-  int32_t act;
-  const void* bias;      // b1 (bf16, column) or b2 (fp32, split-K row); may be null
-  void* out;             // Y bf16 [p][T][s] | P fp32 [p][T][d] | Z fp32 [T][d]
-  WaitCtl wait;
-  int64_t debug_drop;    // slot (in issue order) whose load is skipped; -1 none
-};
-
-struct TileCoord {
-  int32_t batch, m, n;
-};
-
-__device__ __forceinline__ TileCoord decode_tile(const TcParams& P, int32_t t) {
-  const int32_t per_batch = P.m_tiles * P.n_tiles;
-  TileCoord c;
-  c.batch = t / per_batch;
-  const int32_t r = t - c.batch * per_batch;
-  c.n = r / P.m_tiles;   // m fastest: neighbouring CTAs share the weight panel
-  c.m = r - c.n * P.m_tiles;
-  return c;
-}
-
-template <int MODE, int BN>
-__device__ __forceinline__ void issue_slot(const TcParams& P, const CUtensorMap* mA,
-                                           const CUtensorMap* mB0, const CUtensorMap* mB1,
-                                           const TileCoord& tc, int32_t kb, uint32_t sa,
-                                           uint32_t sb, uint32_t bar) {
-  constexpr int NCH = BN / B_BOX_COLS;
-  const int32_t row0 = tc.m * BM;
-  if constexpr (MODE == kModeColumn) {
-    tma_load_3d(sa, mA, bar, kb * BK, row0, 0);
-#pragma unroll
-    for (int c = 0; c < NCH; ++c)
-      tma_load_2d(sb + c * B_CHUNK_BYTES, mB0, bar, tc.n * BN + c * B_BOX_COLS, kb * BK);
-  } else if constexpr (MODE == kModeColumnSwiglu) {
-    tma_load_3d(sa, mA, bar, kb * BK, row0, 0);
-    const int32_t col0 = tc.n * (BN / 2);
-#pragma unroll
-    for (int c = 0; c < NCH / 2; ++c) {
-      tma_load_2d(sb + c * B_CHUNK_BYTES, mB0, bar, col0 + c * B_BOX_COLS, kb * BK);
-      tma_load_2d(sb + (c + NCH / 2) * B_CHUNK_BYTES, mB1, bar, col0 + c * B_BOX_COLS, kb * BK);
-    }
-  } else if constexpr (MODE == kModeRowPartial) {
-    tma_load_3d(sa, mA, bar, kb * BK, row0, tc.batch);
-#pragma unroll
-    for (int c = 0; c < NCH; ++c)
-      tma_load_2d(sb + c * B_CHUNK_BYTES, mB0, bar, tc.n * BN + c * B_BOX_COLS,
-                  tc.batch * P.s + kb * BK);
-  } else {  // split-K over shards: slot kb covers hidden columns [kb*64, kb*64+64)
-    const int32_t shard = kb / P.kb_per_shard;
-    const int32_t kin = kb - shard * P.kb_per_shard;
-    tma_load_3d(sa, mA, bar, kin * BK, row0, shard);
-#pragma unroll
-    for (int c = 0; c < NCH; ++c)
-      tma_load_2d(sb + c * B_CHUNK_BYTES, mB0, bar, tc.n * BN + c * B_BOX_COLS, kb * BK);
-  }
-}
-
-__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
-  return __uint_as_float(static_cast<uint32_t>(b) << 16);
-}
-
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  uint32_t u;
-  memcpy(&u, &v, 4);
-  return u;
-}
-
-// 8 consecutive output columns j..j+7 of one row, bf16, into shard storage.
-__device__ __forceinline__ void store_bf16x8(const TcParams& P, int row, int32_t j,
-                                             const float (&y)[8]) {
-  const int32_t shard = j / P.s;
-  const int32_t jj = j - shard * P.s;
-  const uint4 pk = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
-                              pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
-  __nv_bfloat16* Y = static_cast<__nv_bfloat16*>(P.out);
-  *reinterpret_cast<uint4*>(Y + (static_cast<int64_t>(shard) * P.T + row) * P.s + jj) = pk;
-}
-
-// Epilogue of one tile for one warp: TMEM lanes tacc's quadrant, accumulator
-// columns [c0, c0 + ncols) (ncols a multiple of 32).
-template <int MODE, int BN>
-__device__ __forceinline__ void epilogue_tile(const TcParams& P, const TileCoord& tc,
-                                              uint32_t tacc, int row, int half) {
-  const bool row_ok = row < P.T;
-  if constexpr (MODE == kModeColumn) {
-    const uint16_t* bias = static_cast<const uint16_t*>(P.bias);
-    constexpr int NQ = BN / 64;  // 32-column chunks per half
-#pragma unroll 1
-    for (int q = 0; q < NQ; ++q) {
-      const int c0 = half * (BN / 2) + q * 32;
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tacc + c0, v);
-      tmem_ld_wait();
-      if (!row_ok) continue;
-      const int32_t j0 = tc.n * BN + c0;
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int32_t j = j0 + g * 8;
-        if (j >= P.n_total) break;
-        float h[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          h[e] = __uint_as_float(v[g * 8 + e]);
-          if (bias != nullptr) h[e] += bf16_bits_to_float(__ldg(bias + j + e));
-          h[e] = act_unary_mufu(P.act, h[e]);
-        }
-        store_bf16x8(P, row, j, h);
-      }
-    }
-  } else if constexpr (MODE == kModeColumnSwiglu) {
-    const uint16_t* bias = static_cast<const uint16_t*>(P.bias);
-    constexpr int NQ = BN / 128;  // 32-column output chunks per half
-#pragma unroll 1
-    for (int q = 0; q < NQ; ++q) {
-      const int c0 = half * (BN / 4) + q * 32;   // gate column inside the accumulator
-      uint32_t g32[32], u32[32];
-      tmem_ld_32x32b_x32(tacc + c0, g32);
-      tmem_ld_32x32b_x32(tacc + BN / 2 + c0, u32);
-      tmem_ld_wait();
-      if (!row_ok) continue;
-      const int32_t j0 = tc.n * (BN / 2) + c0;
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int32_t j = j0 + g * 8;
-        if (j >= P.n_total) break;
-        float y[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float gate = __uint_as_float(g32[g * 8 + e]);
-          if (bias != nullptr) gate += bf16_bits_to_float(__ldg(bias + j + e));
-          y[e] = silu_mufu(gate) * __uint_as_float(u32[g * 8 + e]);
-        }
-        store_bf16x8(P, row, j, y);
-      }
-    }
-  } else {
-    const float* bias = static_cast<const float*>(P.bias);
-    float* out = static_cast<float*>(P.out);
-    const int64_t plane = (MODE == kModeRowPartial) ? static_cast<int64_t>(tc.batch) * P.T : 0;
-    constexpr int NQ = BN / 64;
-#pragma unroll 1
-    for (int q = 0; q < NQ; ++q) {
-      const int c0 = half * (BN / 2) + q * 32;
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tacc + c0, v);
-      tmem_ld_wait();
-      if (!row_ok) continue;
-      const int32_t j0 = tc.n * BN + c0;
-      float* dst = out + (plane + row) * static_cast<int64_t>(P.n_total);
-#pragma unroll
-      for (int g = 0; g < 8; ++g) {
-        const int32_t j = j0 + g * 4;
-        if (j >= P.n_total) break;
-        float4 o = make_float4(__uint_as_float(v[g * 4 + 0]), __uint_as_float(v[g * 4 + 1]),
-                               __uint_as_float(v[g * 4 + 2]), __uint_as_float(v[g * 4 + 3]));
-        if (MODE == kModeRowSplitK && bias != nullptr) {
-          o.x = __fadd_rn(o.x, bias[j + 0]);
-          o.y = __fadd_rn(o.y, bias[j + 1]);
-          o.z = __fadd_rn(o.z, bias[j + 2]);
-          o.w = __fadd_rn(o.w, bias[j + 3]);
-        }
-        *reinterpret_cast<float4*>(dst + j) = o;
-      }
-    }
-  }
-}
+using namespace gemm;
 
 template <int MODE, int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -399,13 +195,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int32_t lt = 0;
     for (int32_t t = blockIdx.x; t < P.num_tiles; t += gridDim.x, ++lt) {
       const uint32_t b = lt & 1, ap = (lt >> 1) & 1;
+      const TileCoord tc = decode_tile(P, t);
+      EpiBias<MODE, BN> eb;
+      load_epi_bias<MODE, BN>(P, tc, half, eb);
       bool ok = wait_bounded(accf_bar(b), ap, abort_flag, P.wait, kErrWaitAccFull);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
-      const TileCoord tc = decode_tile(P, t);
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * BN;
-      epilogue_tile<MODE, BN>(P, tc, tacc, tc.m * BM + quad * 32 + lane, half);
+      epilogue_tile<MODE, BN>(P, tc, tacc, tc.m * BM + quad * 32 + lane, half, eb);
       tc_fence_before();
       mbar_arrive(acce_bar(b));
     }
@@ -419,107 +217,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 }
 
 // ------------------------------------------------------------------ host side
-
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
-// Small cache of encoded tensor maps: the same buffers are used call after
-// call, and an encode is pure host work.
-struct MapKey {
-  const void* g;
-  uint64_t dims[3], strides[2];
-  uint32_t box[3];
-  int rank;
-  bool operator==(const MapKey& o) const { return memcmp(this, &o, sizeof(MapKey)) == 0; }
-};
-struct MapEntry {
-  MapKey key;
-  CUtensorMap map;
-  bool used;
-};
-constexpr int kMapCache = 32;
-MapEntry g_maps[kMapCache];
-int g_map_next = 0;
-std::mutex g_map_mu;
-
-// bf16 tensor map, 128-byte swizzle, zero fill outside the tensor.
-bool make_map(CUtensorMap* m, const void* gaddr, int rank, const uint64_t* dims,
-              const uint64_t* strides_bytes, const uint32_t* box) {
-  MapKey key;
-  memset(&key, 0, sizeof(key));
-  key.g = gaddr;
-  key.rank = rank;
-  for (int i = 0; i < rank; ++i) {
-    key.dims[i] = dims[i];
-    key.box[i] = box[i];
-  }
-  for (int i = 0; i < rank - 1; ++i) key.strides[i] = strides_bytes[i];
-  {
-    std::lock_guard<std::mutex> lk(g_map_mu);
-    for (auto& e : g_maps)
-      if (e.used && e.key == key) {
-        *m = e.map;
-        return true;
-      }
-  }
-  auto fn = encode_fn();
-  if (fn == nullptr) {
-    set_error_detail("cuTensorMapEncodeTiled unavailable");
-    return false;
-  }
-  cuuint64_t d[3], st[2];
-  cuuint32_t bx[3], es[3] = {1, 1, 1};
-  for (int i = 0; i < rank; ++i) {
-    d[i] = dims[i];
-    bx[i] = box[i];
-  }
-  for (int i = 0; i < rank - 1; ++i) st[i] = strides_bytes[i];
-  const CUresult r =
-      fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
-         const_cast<void*>(gaddr), d, st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) {
-    set_error_detail("cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
-    return false;
-  }
-  std::lock_guard<std::mutex> lk(g_map_mu);
-  MapEntry& e = g_maps[g_map_next];
-  g_map_next = (g_map_next + 1) % kMapCache;
-  e.key = key;
-  e.map = *m;
-  e.used = true;
-  return true;
-}
-
-// [rows][inner] bf16 matrices stacked `batches` times, boxes of 128 x 64.
-bool make_map_a(CUtensorMap* m, const void* g, int64_t inner, int64_t rows, int64_t batches) {
-  const uint64_t dims[3] = {static_cast<uint64_t>(inner), static_cast<uint64_t>(rows),
-                            static_cast<uint64_t>(batches)};
-  const uint64_t strides[2] = {static_cast<uint64_t>(inner) * 2,
-                               static_cast<uint64_t>(inner) * rows * 2};
-  const uint32_t box[3] = {BK, BM, 1};
-  return make_map(m, g, 3, dims, strides, box);
-}
-
-// [rows = k][cols = n] bf16 weight, N-contiguous, boxes of 64 k-rows x 64 cols.
-bool make_map_b(CUtensorMap* m, const void* g, int64_t cols, int64_t rows) {
-  const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
-  const uint64_t strides[1] = {static_cast<uint64_t>(cols) * 2};
-  const uint32_t box[2] = {B_BOX_COLS, BK};
-  return make_map(m, g, 2, dims, strides, box);
-}
 
 template <int MODE, int BN>
 tp_status launch_mode(const LaunchCtx& c, const CUtensorMap& a, const CUtensorMap& b0,
@@ -552,32 +249,6 @@ tp_status launch_mode(const LaunchCtx& c, const CUtensorMap& a, const CUtensorMa
     return TP_ERR_CUDA;
   }
   return TP_OK;
-}
-
-int32_t ceil_div(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
-
-// Tile width: minimise (waves of tiles over the SMs) x (per-tile cost), the
-// per-tile cost taken as BN plus a fixed 64-column overhead (pipeline fill,
-// epilogue).  Wide problems keep BN = 256, the most efficient per FLOP.
-int pick_bn(int64_t m_tiles, int64_t n_total, int64_t batches, int num_sms, bool swiglu) {
-  static const int cand_all[4] = {256, 192, 128, 64};
-  static const int cand_swiglu[2] = {256, 128};
-  const int* cand = swiglu ? cand_swiglu : cand_all;
-  const int n = swiglu ? 2 : 4;
-  int best = 256;
-  int64_t best_cost = INT64_MAX;
-  for (int i = 0; i < n; ++i) {
-    const int bn = cand[i];
-    const int64_t out_cols = swiglu ? bn / 2 : bn;
-    const int64_t tiles = m_tiles * ((n_total + out_cols - 1) / out_cols) * batches;
-    const int64_t waves = (tiles + num_sms - 1) / num_sms;
-    const int64_t cost = waves * (bn + 64);
-    if (cost < best_cost) {
-      best_cost = cost;
-      best = bn;
-    }
-  }
-  return best;
 }
 
 template <int MODE>

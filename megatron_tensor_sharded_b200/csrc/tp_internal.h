@@ -2,6 +2,7 @@
 // translation units.  Not part of the public interface.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -44,6 +45,29 @@ tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float
                         int64_t k, int64_t d, int p);
 tp_status launch_tc_row_splitk(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
                                float* Z, int64_t T, int64_t k, int64_t d, int p);
+
+// ---- tensor-core path host helpers (tp_tmap.cu)
+// bf16 tensor map with 128-byte swizzle and zero fill outside the tensor
+// (cached by address, sizes and box).
+bool make_map(CUtensorMap* m, const void* gaddr, int rank, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box);
+// [batches][rows][inner] bf16, boxes of 128 rows x 64 inner elements (K-major A tiles).
+bool make_map_a(CUtensorMap* m, const void* g, int64_t inner, int64_t rows, int64_t batches);
+// [rows][cols] bf16 weight, N-contiguous, boxes of 64 rows x 64 columns (N-major B tiles).
+bool make_map_b(CUtensorMap* m, const void* g, int64_t cols, int64_t rows);
+// Tile width (accumulator columns) for a GEMM with this tile space.
+int pick_bn(int64_t m_tiles, int64_t n_total, int64_t batches, int num_sms, bool swiglu);
+
+inline int32_t ceil_div(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
+
+// ---- fused block (tp_block_sm100.cu): column GEMM + row GEMM (+ fixed-order
+// fold of the partials, or split-K over shards) in one persistent launch.
+// `counters` is zeroed device scratch of block_counter_bytes() bytes.
+size_t block_counter_bytes(int64_t T, int64_t d);
+tp_status launch_tc_block(const LaunchCtx& c, const void* X, const void* W1, const void* Wup,
+                          const void* b1, const void* W2, const float* b2, void* Y, float* P,
+                          float* Z, int* counters, int64_t T, int64_t d, int64_t k, int p, int act,
+                          bool splitk);
 
 // Records a human-readable detail for tp_last_error_detail().
 void set_error_detail(const char* fmt, ...);

@@ -1,0 +1,151 @@
+// Host-side helpers of the tensor-core path: TMA tensor maps (with a small
+// cache, since the same buffers come back call after call) and the choice of
+// tile width.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "tp_internal.h"
+
+namespace tpk {
+namespace {
+
+constexpr uint32_t kBoxK = 64;      // k per pipeline slot (one 128-byte swizzle row of bf16)
+constexpr uint32_t kBoxRows = 128;  // A-tile rows
+constexpr uint32_t kBoxCols = 64;   // B box width (one swizzle atom)
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Small cache of encoded tensor maps: the same buffers are used call after
+// call, and an encode is pure host work.
+struct MapKey {
+  const void* g;
+  uint64_t dims[3], strides[2];
+  uint32_t box[3];
+  int rank;
+  bool operator==(const MapKey& o) const { return memcmp(this, &o, sizeof(MapKey)) == 0; }
+};
+struct MapEntry {
+  MapKey key;
+  CUtensorMap map;
+  bool used;
+};
+constexpr int kMapCache = 32;
+MapEntry g_maps[kMapCache];
+int g_map_next = 0;
+std::mutex g_map_mu;
+
+}  // namespace
+
+// bf16 tensor map, 128-byte swizzle, zero fill outside the tensor.
+bool make_map(CUtensorMap* m, const void* gaddr, int rank, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box) {
+  MapKey key;
+  memset(&key, 0, sizeof(key));
+  key.g = gaddr;
+  key.rank = rank;
+  for (int i = 0; i < rank; ++i) {
+    key.dims[i] = dims[i];
+    key.box[i] = box[i];
+  }
+  for (int i = 0; i < rank - 1; ++i) key.strides[i] = strides_bytes[i];
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    for (auto& e : g_maps)
+      if (e.used && e.key == key) {
+        *m = e.map;
+        return true;
+      }
+  }
+  auto fn = encode_fn();
+  if (fn == nullptr) {
+    set_error_detail("cuTensorMapEncodeTiled unavailable");
+    return false;
+  }
+  cuuint64_t d[3], st[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i < rank - 1; ++i) st[i] = strides_bytes[i];
+  const CUresult r =
+      fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+         const_cast<void*>(gaddr), d, st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    set_error_detail("cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
+    return false;
+  }
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  MapEntry& e = g_maps[g_map_next];
+  g_map_next = (g_map_next + 1) % kMapCache;
+  e.key = key;
+  e.map = *m;
+  e.used = true;
+  return true;
+}
+
+// [rows][inner] bf16 matrices stacked `batches` times, boxes of 128 x 64.
+bool make_map_a(CUtensorMap* m, const void* g, int64_t inner, int64_t rows, int64_t batches) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(inner), static_cast<uint64_t>(rows),
+                            static_cast<uint64_t>(batches)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(inner) * 2,
+                               static_cast<uint64_t>(inner) * rows * 2};
+  const uint32_t box[3] = {kBoxK, kBoxRows, 1};
+  return make_map(m, g, 3, dims, strides, box);
+}
+
+// [rows = k][cols = n] bf16 weight, N-contiguous, boxes of 64 k-rows x 64 cols.
+bool make_map_b(CUtensorMap* m, const void* g, int64_t cols, int64_t rows) {
+  const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(cols) * 2};
+  const uint32_t box[2] = {kBoxCols, kBoxK};
+  return make_map(m, g, 2, dims, strides, box);
+}
+
+
+// Tile width: minimise (waves of tiles over the SMs) x (per-tile cost), the
+// per-tile cost taken as BN plus a fixed 64-column overhead (pipeline fill,
+// epilogue).  Wide problems keep BN = 256, the most efficient per FLOP.
+int pick_bn(int64_t m_tiles, int64_t n_total, int64_t batches, int num_sms, bool swiglu) {
+  static const int cand_all[4] = {256, 192, 128, 64};
+  static const int cand_swiglu[2] = {256, 128};
+  const int* cand = swiglu ? cand_swiglu : cand_all;
+  const int n = swiglu ? 2 : 4;
+  int best = 256;
+  int64_t best_cost = INT64_MAX;
+  for (int i = 0; i < n; ++i) {
+    const int bn = cand[i];
+    const int64_t out_cols = swiglu ? bn / 2 : bn;
+    const int64_t tiles = m_tiles * ((n_total + out_cols - 1) / out_cols) * batches;
+    const int64_t waves = (tiles + num_sms - 1) / num_sms;
+    const int64_t cost = waves * (bn + 64);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = bn;
+    }
+  }
+  return best;
+}
+
+
+}  // namespace tpk

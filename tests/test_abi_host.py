@@ -94,15 +94,22 @@ def test_row_and_reduce_validation():
 
 def test_workspace_size_formula():
     # bf16: hidden shards T*k*2 bytes, then p*T*d*4 bytes of partials, each
-    # rounded up to 256 bytes
+    # rounded up to 256 bytes, then one int per 128-row m-tile of tile counters
+    def r256(n):
+        return -(-n // 256) * 256
+
+    def counters(T, d):
+        return r256(4 * (-(-T // 128)))
+
     T, d, k, p = 1000, 768, 3072, 2
-    ys = -(-T * k * 2 // 256) * 256
-    ps = -(-p * T * d * 4 // 256) * 256
-    assert tp.tp_mlp_block_workspace_size(T, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH) == ys + ps
+    ys = r256(T * k * 2)
+    ps = r256(p * T * d * 4)
+    assert tp.tp_mlp_block_workspace_size(T, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH) == \
+        ys + ps + counters(T, d)
     assert tp.tp_mlp_block_workspace_size(T, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH,
-                                          tp.TP_FLAG_SPLITK_FUSED) == ys
+                                          tp.TP_FLAG_SPLITK_FUSED) == ys + counters(T, d)
     assert tp.tp_mlp_block_workspace_size(4, 512, 2048, 4, tp.TP_F32, tp.TP_ACT_GELU_TANH) == \
-        -(-4 * 2048 * 4 // 256) * 256 + -(-4 * 4 * 512 * 4 // 256) * 256
+        r256(4 * 2048 * 4) + r256(4 * 4 * 512 * 4) + counters(4, 512)
     assert tp.tp_mlp_block_workspace_size(4, 512, 2047, 4, tp.TP_F32, tp.TP_ACT_GELU_TANH) == 0
 
 
@@ -120,6 +127,7 @@ def test_block_validation():
     assert blk(ws=0x40000 + 16) == 3
     assert blk(k=255) == 2
     assert blk(flags=8) == 1
+    assert blk(flags=4) == 1
     assert blk(k=4 * 72, flags=tp.TP_FLAG_SPLITK_FUSED) == 4   # s = 72, not a multiple of 64
     assert blk(Z=None) == 1
 

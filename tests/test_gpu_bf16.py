@@ -150,3 +150,47 @@ def test_full_size_configs_sampled_rows(name):
         del ws
         assert O.rel_err(host_f32(Z2.index_select(0, idx)), ref["Z"]) <= TOL_BF16, flags
         assert not torch.isnan(Z2).any().item()
+
+
+@pytest.mark.parametrize("T,d,s,p,act", [(1, 64, 64, 1, "gelu_tanh"), (130, 200, 40, 4, "relu"),
+                                         (257, 128, 72, 2, "gelu_tanh"), (300, 192, 128, 3, "swiglu"),
+                                         (1024, 768, 1536, 2, "gelu_tanh"), (16, 512, 448, 8, "swiglu"),
+                                         (700, 256, 256, 4, "swiglu")])
+def test_fused_block_matches_separate_kernels(T, d, s, p, act):
+    """tp_mlp_block's fused launch of both GEMM layers gives the same bits as
+    the separate column and row launches (both then take the same fixed-order
+    fold); split-K agrees with the oracle within tolerance."""
+    k = s * p
+    inp = _random_bf16(T, d, k, act, with_bias=(act != "swiglu"), seed=T + s)
+    blk = DeviceBlock(inp, T, d, k, p, act)
+    Zf = torch.full_like(blk.Z, float("nan"))
+    Zu = torch.full_like(blk.Z, float("nan"))
+    blk.block(tp.TP_FLAG_NONE, Z=Zf)
+    blk.block(tp.TP_FLAG_UNFUSED, Z=Zu)
+    blk.sync()
+    assert np.array_equal(bits(host_f32(Zf)), bits(host_f32(Zu)))
+    ref = _oracle(inp, p, act)
+    assert O.rel_err(host_f32(Zf), ref["Z"]) <= TOL_BF16
+    if s % 64 == 0:
+        Zs = torch.full_like(blk.Z, float("nan"))
+        blk.block(tp.TP_FLAG_SPLITK_FUSED, Z=Zs)
+        blk.sync()
+        assert O.rel_err(host_f32(Zs), ref["Z"]) <= TOL_BF16
+
+
+def test_fused_block_repeated_calls_reuse_counters():
+    """The tile counters live in the workspace and are reset by every call:
+    back-to-back calls on the same workspace give identical results."""
+    w = W.WORKLOADS["gpt2"]
+    blk = DeviceBlock(W.make_inputs(w), w.T, w.d, w.k, w.p, w.act)
+    n = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, w.p, blk.dtype, blk.act)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(3):
+        Z = torch.full_like(blk.Z, float("nan"))
+        tp.tp_mlp_block(blk.X, blk.W1, blk.Wu, blk.b1, blk.W2, blk.b2, Z, ws, n, w.T, w.d, w.k,
+                        w.p, blk.dtype, blk.act)
+        outs.append(Z)
+    blk.sync()
+    for Z in outs[1:]:
+        assert torch.equal(Z, outs[0])
