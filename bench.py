@@ -99,6 +99,16 @@ def row_bytes(w: WL.Workload) -> int:
     return e * (w.T * w.k + w.k * w.d) + 4 * w.p * w.T * w.d
 
 
+def block_bytes(w: WL.Workload) -> int:
+    """Minimum HBM bytes of one block step: read X, the weights and biases
+    once, write Z.  (The hidden shards and partials of this design add
+    2*T*k*e + 2*p*T*d*4 bytes on top when they leave L2.)"""
+    e = 2 if w.dtype == "bf16" else 4
+    nw = 2 if w.act == "swiglu" else 1
+    return (e * (w.T * w.d + nw * w.d * w.k + w.k * w.d + (w.k if w.has_b1 else 0))
+            + 4 * w.T * w.d + (4 * w.d if w.has_b2 else 0))
+
+
 def blas_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
@@ -167,8 +177,8 @@ class ClockSampler:
 
 
 def ncu_traffic(kernel_key: str):
-    """dram bytes per launch from a committed ncu summary, if it was taken on
-    the current kernel source (else None)."""
+    """dram bytes per launch from the committed ncu summary table, if it was
+    taken on the current kernel sources (else None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
@@ -178,12 +188,14 @@ def ncu_traffic(kernel_key: str):
     ent = table.get(kernel_key)
     if not ent:
         return None
-    src = os.path.join(ROOT, "megatron_tensor_sharded_b200", "csrc", ent["source"])
+    h = hashlib.sha256()
     try:
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
-    except OSError:
+        for src in ent["sources"]:
+            with open(os.path.join(ROOT, "megatron_tensor_sharded_b200", "csrc", src), "rb") as f:
+                h.update(f.read())
+    except (OSError, KeyError):
         return None
-    if sha != ent.get("source_sha"):
+    if h.hexdigest()[:16] != ent.get("source_sha"):
         return None
     return ent.get("dram_bytes_per_launch")
 
@@ -407,7 +419,11 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
     kernel_name = {"partials": "tc_block_kernel (fused block: column GEMM, row GEMM, fixed-order fold)",
                    "splitk": "tc_block_kernel (fused block, split-K over shards)",
                    "unfused": "column GEMM + row GEMM + fold (separate launches)"}[a.mode]
-    if w.dtype == "bf16":
+    # Roofline side: tensor peak unless the step's arithmetic intensity
+    # (FLOPs per minimum HBM byte) is below the measured ridge point.
+    intensity = w.gemm_flops() / block_bytes(w)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if w.dtype == "bf16" and intensity >= ridge:
         achieved = w.gemm_flops() / (ms_step * 1e-3) / 1e12
         peak = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -416,12 +432,15 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
                 "duration": "block step time (graph replay, CUDA events on the launching stream)",
                 "peak_source": f"{peak_src} bf16 dense (burst)"}
     else:
-        byts = column_bytes(w) + row_bytes(w) + reduce_bytes(w)
-        achieved = byts / (ms_step * 1e-3) / 1e9
+        achieved = block_bytes(w) / (ms_step * 1e-3) / 1e9
         peak = peaks["hbm_gbs"]
         roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": None, "kernel": kernel_name,
+                "frac": achieved / peak, "traffic": ncu_traffic(f"{w.name}/{a.mode}"),
+                "kernel": kernel_name, "bytes_per_step": block_bytes(w),
+                "duration": "block step time (graph replay, CUDA events on the launching stream)",
                 "peak_source": f"{peak_src} hbm copy"}
+    roof["intensity_flop_per_byte"] = intensity
+    roof["ridge_flop_per_byte"] = ridge
 
     breakdown = None
     if kernels is not None:
