@@ -289,8 +289,8 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
     flags = tp.TP_FLAG_SPLITK_FUSED if a.mode == "splitk" else tp.TP_FLAG_NONE
-    if a.mode == "unfused":
-        flags = tp.TP_FLAG_UNFUSED
+    if a.mode == "fused":
+        flags = tp.TP_FLAG_FUSED_LAUNCH
     nbytes = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, w.p, dtype, act, flags)
     ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
 
@@ -358,7 +358,7 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
 
     # ---- per-kernel breakdown of the same block as three separate calls
     kernels = None
-    if a.mode != "splitk" and not a.no_breakdown:
+    if a.mode == "partials" and not a.no_breakdown:
         evs = [torch.cuda.Event(enable_timing=True, external=not a.no_graph) for _ in range(4)]
         g_calls, _ = capture(lambda st: calls_step(st, evs))
         col_ms, row_ms, red_ms, sum_ms = [], [], [], []
@@ -416,9 +416,9 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
 
     peaks, peak_src = load_peaks()
     value = whole_job_value(w.gemm_flops(), world, ms_step) / 1e12
-    kernel_name = {"partials": "tc_block_kernel (fused block: column GEMM, row GEMM, fixed-order fold)",
-                   "splitk": "tc_block_kernel (fused block, split-K over shards)",
-                   "unfused": "column GEMM + row GEMM + fold (separate launches)"}[a.mode]
+    kernel_name = {"partials": "tp_mlp_block: column GEMM -> row GEMM -> fixed-order fold (PDL-chained)",
+                   "splitk": "tp_mlp_block split-K: column GEMM -> row GEMM accumulating all shards",
+                   "fused": "tc_block_kernel (both GEMM layers, one launch) -> fold"}[a.mode]
     # Roofline side: tensor peak unless the step's arithmetic intensity
     # (FLOPs per minimum HBM byte) is below the measured ridge point.
     intensity = w.gemm_flops() / block_bytes(w)
@@ -495,7 +495,7 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tp", "reference"], default="tp")
     ap.add_argument("--workload", choices=sorted(WL.WORKLOADS), default="gpt2")
-    ap.add_argument("--mode", choices=["partials", "splitk", "unfused"], default="partials")
+    ap.add_argument("--mode", choices=["partials", "splitk", "fused"], default="partials")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of graph replay")
     ap.add_argument("--no-breakdown", action="store_true", help="skip the per-kernel loop")

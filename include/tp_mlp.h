@@ -78,10 +78,11 @@ typedef enum {
  * partials and folding them.  Same result up to fp32 summation order (not
  * bit-identical to the fixed-order fold).  bf16 requires s % 64 == 0. */
 #define TP_FLAG_SPLITK_FUSED 1
-/* Launch the block as separate kernels (column, row, fold) instead of the
- * default single persistent launch of the bf16 path.  Same bits either way;
- * for comparisons and diagnostics. */
-#define TP_FLAG_UNFUSED 2
+/* bf16: run both GEMM layers in one persistent launch (row-parallel tiles
+ * start as soon as the hidden rows they read are complete) instead of one
+ * launch per layer.  Same bits either way; the default per-layer launches
+ * were faster on every measured shape (they use CTA-pair tiles). */
+#define TP_FLAG_FUSED_LAUNCH 2
 
 /*
  * Column-parallel linear + activation, all p shards in one launch.
@@ -136,9 +137,8 @@ tp_status tp_reduce_partials(const float* partials, const float* b2, float* Z,
  * ("Pairing them: the Megatron-LM MLP"; "The MLP block: column then row,
  * one all-reduce").  Computes exactly what tp_column_linear ->
  * tp_row_linear -> tp_reduce_partials compute (bit for bit), with the hidden
- * shards and the partials in the caller's workspace.  bf16 runs both GEMM
- * layers as one persistent launch (row-parallel tiles start as soon as the
- * hidden rows they read are complete), then the fixed-order fold.  With
+ * shards and the partials in the caller's workspace; the kernels are chained
+ * with programmatic dependent launch.  With
  * TP_FLAG_SPLITK_FUSED the second layer accumulates over all shards and
  * writes Z directly (no partials).
  *

@@ -19,7 +19,7 @@ import os
 
 __all__ = [
     "TPError", "TP_F32", "TP_BF16", "TP_ACT_GELU_TANH", "TP_ACT_SWIGLU", "TP_ACT_IDENTITY",
-    "TP_ACT_RELU", "TP_FLAG_NONE", "TP_FLAG_SPLITK_FUSED", "TP_FLAG_UNFUSED", "STATUS", "ACT", "DTYPE",
+    "TP_ACT_RELU", "TP_FLAG_NONE", "TP_FLAG_SPLITK_FUSED", "TP_FLAG_FUSED_LAUNCH", "STATUS", "ACT", "DTYPE",
     "tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
     "tp_mlp_block_noalloc",
     "tp_mlp_block_workspace_size", "tp_sync_status", "tp_set_wait_timeout_ns",
@@ -31,7 +31,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtpmlp.so
 
 TP_F32, TP_BF16 = 0, 1
 TP_ACT_GELU_TANH, TP_ACT_SWIGLU, TP_ACT_IDENTITY, TP_ACT_RELU = 0, 1, 2, 3
-TP_FLAG_NONE, TP_FLAG_SPLITK_FUSED, TP_FLAG_UNFUSED = 0, 1, 2
+TP_FLAG_NONE, TP_FLAG_SPLITK_FUSED, TP_FLAG_FUSED_LAUNCH = 0, 1, 2
 DTYPE = {"f32": TP_F32, "bf16": TP_BF16}
 ACT = {"gelu_tanh": TP_ACT_GELU_TANH, "swiglu": TP_ACT_SWIGLU, "identity": TP_ACT_IDENTITY,
        "relu": TP_ACT_RELU}

@@ -242,7 +242,7 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
   g_detail[0] = 0;
   TP_TRY(check_shape(T, d, k, p, dtype));
   TP_TRY(check_act(act, W_up));
-  if (flags & ~(TP_FLAG_SPLITK_FUSED | TP_FLAG_UNFUSED))
+  if (flags & ~(TP_FLAG_SPLITK_FUSED | TP_FLAG_FUSED_LAUNCH))
     return fail(TP_ERR_INVALID_ARG, "flags 0x%x", flags);
   const bool splitk = (flags & TP_FLAG_SPLITK_FUSED) != 0;
   if (splitk && dtype == TP_BF16 && (k / p) % 64 != 0)
@@ -268,7 +268,7 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
   const size_t esize = dtype == TP_BF16 ? 2 : 4;
   const size_t y_bytes = align256(static_cast<size_t>(T) * k * esize);
   float* P = splitk ? nullptr : reinterpret_cast<float*>(ws + y_bytes);
-  if (dtype == TP_BF16 && !(flags & TP_FLAG_UNFUSED)) {
+  if (dtype == TP_BF16 && (flags & TP_FLAG_FUSED_LAUNCH)) {
     // Both GEMM layers in one persistent launch (its tile counters start at
     // 0), then the fixed-order fold of the partials.
     int* counters = reinterpret_cast<int*>(ws + need - block_counter_bytes(T, d));

@@ -1,0 +1,333 @@
+// Per-layer bf16 GEMM on CTA pairs (tcgen05 cta_group::2), sm_100a.
+//
+// Same layers and epilogues as tp_gemm_sm100.cu (column-parallel + bias +
+// GELU/SwiGLU into the hidden shards, row-parallel fp32 partials, split-K
+// over shards): a cluster of two CTAs computes a 256 x PBN tile (PBN 128 or
+// 256).  Each CTA loads its own 128 rows of A and one half (PBN/2 columns) of
+// B, and the even CTA's single MMA thread issues tcgen05.mma.cta_group::2
+// M=256 N=PBN, which reads both CTAs' shared memory and writes each CTA's 128
+// accumulator rows into that CTA's TMEM.  Per SM this halves the B operand
+// bytes per MMA cycle (64 instead of 96 bytes per cycle at width 256).
+//
+// Synchronisation (all barrier waits bounded):
+//   full[s]   on the even CTA: its expect_tx of both CTAs' bytes, completed by
+//             both CTAs' TMA loads (cta_group::2 loads count on the even
+//             CTA's barrier);
+//   empty[s]  in each CTA: the MMA's commit multicast to both;
+//   accf[b]   in each CTA: the MMA's commit multicast to both;
+//   acce[b]   on the even CTA: one arrival per epilogue warp of both CTAs.
+// No load uses cluster multicast: every CTA reads its own tiles.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <mutex>
+
+#include "tp_gemm_parts.cuh"
+#include "tp_internal.h"
+#include "tp_launch.cuh"
+
+namespace tpk {
+namespace {
+
+using namespace gemm;
+
+constexpr int PBM = 2 * BM;  // rows of a pair tile
+
+// Pair tile of PBN accumulator columns: each CTA holds PBN/2 columns of B.
+template <int PBN>
+struct PCfg {
+  static constexpr int B_CHUNKS = PBN / 2 / B_BOX_COLS;
+  static constexpr int STAGE_BYTES = A_BYTES + B_CHUNKS * B_CHUNK_BYTES;
+  static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - CTRL_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTRL_BYTES;
+  static constexpr int TMEM_COLS = 2 * PBN <= 256 ? 256 : 512;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(PBM, PBN, /*a_mn=*/0, /*b_mn=*/1);
+  static_assert(PBN == 128 || PBN == 256, "pair tile width");
+  static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
+  static_assert(8 * (2 * STAGES + 5) + 16 <= CTRL_BYTES, "control block");
+};
+
+// Loads of one slot for this CTA: A rows [m*256 + rank*128, +128), B columns
+// [n*256 + rank*128, +128) of the layer's weight (SwiGLU: the even CTA loads
+// the gate columns, the odd CTA the matching up columns).
+template <int MODE, int PBN>
+__device__ __forceinline__ void issue_slot_pair(const TcParams& P, const CUtensorMap* mA,
+                                                const CUtensorMap* mB0, const CUtensorMap* mB1,
+                                                const TileCoord& tc, int32_t kb, uint32_t rank,
+                                                uint32_t sa, uint32_t sb, uint32_t bar) {
+  constexpr int PB_CHUNKS = PCfg<PBN>::B_CHUNKS;
+  const int32_t row0 = tc.m * PBM + static_cast<int32_t>(rank) * BM;
+  if constexpr (MODE == kModeColumn) {
+    tma_load_3d_pair(sa, mA, bar, kb * BK, row0, 0);
+    const int32_t col0 = tc.n * PBN + static_cast<int32_t>(rank) * (PBN / 2);
+#pragma unroll
+    for (int c = 0; c < PB_CHUNKS; ++c)
+      tma_load_2d_pair(sb + c * B_CHUNK_BYTES, mB0, bar, col0 + c * B_BOX_COLS, kb * BK);
+  } else if constexpr (MODE == kModeColumnSwiglu) {
+    tma_load_3d_pair(sa, mA, bar, kb * BK, row0, 0);
+    const CUtensorMap* mB = rank == 0 ? mB0 : mB1;
+    const int32_t col0 = tc.n * (PBN / 2);
+#pragma unroll
+    for (int c = 0; c < PB_CHUNKS; ++c)
+      tma_load_2d_pair(sb + c * B_CHUNK_BYTES, mB, bar, col0 + c * B_BOX_COLS, kb * BK);
+  } else if constexpr (MODE == kModeRowPartial) {
+    tma_load_3d_pair(sa, mA, bar, kb * BK, row0, tc.batch);
+    const int32_t col0 = tc.n * PBN + static_cast<int32_t>(rank) * (PBN / 2);
+#pragma unroll
+    for (int c = 0; c < PB_CHUNKS; ++c)
+      tma_load_2d_pair(sb + c * B_CHUNK_BYTES, mB0, bar, col0 + c * B_BOX_COLS,
+                       tc.batch * P.s + kb * BK);
+  } else {
+    const int32_t shard = kb / P.kb_per_shard;
+    const int32_t kin = kb - shard * P.kb_per_shard;
+    tma_load_3d_pair(sa, mA, bar, kin * BK, row0, shard);
+    const int32_t col0 = tc.n * PBN + static_cast<int32_t>(rank) * (PBN / 2);
+#pragma unroll
+    for (int c = 0; c < PB_CHUNKS; ++c)
+      tma_load_2d_pair(sb + c * B_CHUNK_BYTES, mB0, bar, col0 + c * B_BOX_COLS, kb * BK);
+  }
+}
+
+template <int MODE, int PBN>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA,
+                        const __grid_constant__ CUtensorMap mapB0,
+                        const __grid_constant__ CUtensorMap mapB1, const TcParams P) {
+  using C = PCfg<PBN>;
+  constexpr int PSTAGES = C::STAGES;
+  constexpr int PSTAGE_BYTES = C::STAGE_BYTES;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const ctrl = smem_raw + (base - raw) + PSTAGES * PSTAGE_BYTES;
+  uint64_t* const bars = reinterpret_cast<uint64_t*>(ctrl);
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * (2 * PSTAGES + 5));
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  auto full_bar = [&](uint32_t s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](uint32_t s) { return smem_u32(&bars[PSTAGES + s]); };
+  auto accf_bar = [&](uint32_t b) { return smem_u32(&bars[2 * PSTAGES + b]); };
+  auto acce_bar = [&](uint32_t b) { return smem_u32(&bars[2 * PSTAGES + 2 + b]); };
+  const uint32_t drain_bar = smem_u32(&bars[2 * PSTAGES + 4]);
+  auto slot_a = [&](uint32_t s) { return base + s * PSTAGE_BYTES; };
+  auto slot_b = [&](uint32_t s) { return base + s * PSTAGE_BYTES + A_BYTES; };
+
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const int32_t cluster = blockIdx.x / 2;
+  const int32_t nclusters = gridDim.x / 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < PSTAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), 2 * NUM_EPI_WARPS);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&mapA);
+    tma_prefetch_map(&mapB0);
+    if (MODE == kModeColumnSwiglu) tma_prefetch_map(&mapB1);
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  pdl_wait();
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      uint32_t stage = 0, phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int32_t t = cluster; ok && t < P.num_tiles; t += nclusters) {
+        const TileCoord tc = decode_tile(P, t);
+        for (int32_t kb = 0; kb < P.k_blocks; ++kb) {
+          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, P.wait, kErrWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          if (issued != P.debug_drop) {
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * PSTAGE_BYTES);
+            issue_slot_pair<MODE, PBN>(P, &mapA, &mapB0, &mapB1, tc, kb, rank, slot_a(stage),
+                                  slot_b(stage), mapa_shared(full_bar(stage), 0));
+          }
+          ++issued;
+          if (++stage == PSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // Teardown: our last loads must have landed before this CTA's shared
+      // memory is released.  The even CTA sees that on its full barriers; the
+      // odd CTA on its empty barriers (the MMA consumed the slot).
+      const int64_t first = issued > PSTAGES ? issued - PSTAGES : 0;
+      for (int64_t q = first; q < issued; ++q) {
+        if (q == P.debug_drop) continue;
+        const uint32_t s = static_cast<uint32_t>(q % PSTAGES);
+        const uint32_t ph = static_cast<uint32_t>((q / PSTAGES) & 1);
+        wait_teardown(rank == 0 ? full_bar(s) : empty_bar(s), ph, P.wait);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------------------------------------------- MMA issuer (pair)
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      int32_t lt = 0;
+      for (int32_t t = cluster; ok && t < P.num_tiles; t += nclusters, ++lt) {
+        const uint32_t b = lt & 1, ap = (lt >> 1) & 1;
+        if (!wait_bounded(acce_bar(b), ap ^ 1u, abort_flag, P.wait, kErrWaitAccEmpty)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + b * PBN;
+        for (int32_t kb = 0; kb < P.k_blocks; ++kb) {
+          if (!wait_bounded(full_bar(stage), phase, abort_flag, P.wait, kErrWaitFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = slot_a(stage), sb = slot_b(stage);
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk) {
+            const uint64_t adesc = smem_desc_sw128(sa + kk * UK * 2, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(sb + kk * UK * 128, B_CHUNK_BYTES, 1024);
+            tc_mma_f16_pair(d_tmem, adesc, bdesc, C::IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit_pair_mc(empty_bar(stage), 0x3);
+          if (++stage == PSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(accf_bar(b), 0x3);
+      }
+      tc_commit_pair_mc(drain_bar, 0x1);
+      wait_teardown(drain_bar, 0, P.wait);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    // -------------------------------------------------------------- epilogue
+    const int quad = warp & 3;
+    const int half = (warp - 4) >> 2;
+    int32_t lt = 0;
+    for (int32_t t = cluster; t < P.num_tiles; t += nclusters, ++lt) {
+      const uint32_t b = lt & 1, ap = (lt >> 1) & 1;
+      const TileCoord tc = decode_tile(P, t);
+      EpiBias<MODE, PBN> eb;
+      load_epi_bias<MODE, PBN>(P, tc, half, eb);
+      bool ok = wait_bounded(accf_bar(b), ap, abort_flag, P.wait, kErrWaitAccFull);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * PBN;
+      const int row = tc.m * PBM + static_cast<int>(rank) * BM + quad * 32 + lane;
+      epilogue_tile<MODE, PBN>(P, tc, tacc, row, half, eb);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(b), 0));
+    }
+  }
+
+  tc_fence_before();
+  cluster_sync();  // the pair's MMAs, commits and arrivals are done with both CTAs
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+}  // namespace
+
+template <int MODE, int PBN>
+tp_status launch_pair_mode(const LaunchCtx& c, const CUtensorMap& a, const CUtensorMap& b0,
+                           const CUtensorMap& b1, TcParams prm) {
+  constexpr int PSMEM_BYTES = PCfg<PBN>::SMEM_BYTES;
+  static bool attr_done[64] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    const int dev = c.device & 63;
+    if (!attr_done[dev]) {
+      if (cudaFuncSetAttribute(tc_gemm_pair_kernel<MODE, PBN>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PSMEM_BYTES) != cudaSuccess) {
+        set_error_detail("cudaFuncSetAttribute failed: %s", cudaGetErrorString(cudaGetLastError()));
+        return TP_ERR_CUDA;
+      }
+      attr_done[dev] = true;
+    }
+  }
+  prm.wait.err = c.err_word;
+  prm.wait.timeout_ns = c.timeout_ns;
+  prm.debug_drop = c.debug_drop;
+  int clusters = c.num_sms / 2;
+  if (clusters > prm.num_tiles) clusters = prm.num_tiles;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = PSMEM_BYTES;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_allowed() ? 2 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<MODE, PBN>, a, b0, b1, prm);
+  note_launch();
+  if (e != cudaSuccess) {
+    set_error_detail("paired GEMM launch failed: %s", cudaGetErrorString(e));
+    return TP_ERR_CUDA;
+  }
+  return TP_OK;
+}
+
+// Tile space of the pair kernel for a layer: 256-row m-tiles, `pbn`-column
+// (SwiGLU: pbn/2 output columns) n-tiles.
+tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMap& a,
+                         const CUtensorMap& b0, const CUtensorMap& b1, TcParams prm) {
+  const int out_cols = mode == kModeColumnSwiglu ? pbn / 2 : pbn;
+  prm.m_tiles = ceil_div(prm.T, PBM);
+  prm.n_tiles = ceil_div(prm.n_total, out_cols);
+  prm.num_tiles = prm.m_tiles * prm.n_tiles * prm.batches;
+  if (pbn == 128) {
+    switch (mode) {
+      case kModeColumn: return launch_pair_mode<kModeColumn, 128>(c, a, b0, b1, prm);
+      case kModeColumnSwiglu: return launch_pair_mode<kModeColumnSwiglu, 128>(c, a, b0, b1, prm);
+      case kModeRowPartial: return launch_pair_mode<kModeRowPartial, 128>(c, a, b0, b1, prm);
+      default: return launch_pair_mode<kModeRowSplitK, 128>(c, a, b0, b1, prm);
+    }
+  }
+  switch (mode) {
+    case kModeColumn: return launch_pair_mode<kModeColumn, 256>(c, a, b0, b1, prm);
+    case kModeColumnSwiglu: return launch_pair_mode<kModeColumnSwiglu, 256>(c, a, b0, b1, prm);
+    case kModeRowPartial: return launch_pair_mode<kModeRowPartial, 256>(c, a, b0, b1, prm);
+    default: return launch_pair_mode<kModeRowSplitK, 256>(c, a, b0, b1, prm);
+  }
+}
+
+}  // namespace tpk

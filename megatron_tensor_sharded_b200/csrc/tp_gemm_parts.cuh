@@ -11,6 +11,7 @@
 
 #include "tp_act.cuh"
 #include "tp_device.cuh"
+#include "tp_internal.h"
 
 namespace tpk {
 namespace gemm {
@@ -278,4 +279,10 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& P, const TileCoord
 }
 
 }  // namespace gemm
+
+// Per-layer GEMM on CTA pairs (tp_gemm2_sm100.cu): 256 x pbn tiles (pbn 128
+// or 256); `mode` is a gemm::Mode; prm's tile space is recomputed.
+tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMap& a,
+                         const CUtensorMap& b0, const CUtensorMap& b1, gemm::TcParams prm);
+
 }  // namespace tpk

@@ -295,9 +295,11 @@ tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, co
   prm.act = act;
   prm.bias = b1;
   prm.out = Y;
-  const int bn = pick_bn(prm.m_tiles, k, 1, c.num_sms, swiglu);
-  if (swiglu) return launch_bn<kModeColumnSwiglu>(c, bn, mA, mB0, mB1, prm);
-  return launch_bn<kModeColumn>(c, bn, mA, mB0, mB1, prm);
+  const TileChoice tch = pick_tile(T, k, 1, prm.k_blocks, c.num_sms, swiglu, pair_allowed());
+  const int mode = swiglu ? kModeColumnSwiglu : kModeColumn;
+  if (tch.pair) return launch_tc_pair(c, mode, tch.bn, mA, mB0, mB1, prm);
+  if (swiglu) return launch_bn<kModeColumnSwiglu>(c, tch.bn, mA, mB0, mB1, prm);
+  return launch_bn<kModeColumn>(c, tch.bn, mA, mB0, mB1, prm);
 }
 
 tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float* P, int64_t T,
@@ -317,8 +319,9 @@ tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float
   prm.act = kActIdentity;
   prm.bias = nullptr;
   prm.out = P;
-  const int bn = pick_bn(prm.m_tiles, d, p, c.num_sms, false);
-  return launch_bn<kModeRowPartial>(c, bn, mA, mB, mB, prm);
+  const TileChoice tch = pick_tile(T, d, p, prm.k_blocks, c.num_sms, false, pair_allowed());
+  if (tch.pair) return launch_tc_pair(c, kModeRowPartial, tch.bn, mA, mB, mB, prm);
+  return launch_bn<kModeRowPartial>(c, tch.bn, mA, mB, mB, prm);
 }
 
 tp_status launch_tc_row_splitk(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
@@ -338,8 +341,9 @@ tp_status launch_tc_row_splitk(const LaunchCtx& c, const void* Y, const void* W2
   prm.act = kActIdentity;
   prm.bias = b2;
   prm.out = Z;
-  const int bn = pick_bn(prm.m_tiles, d, 1, c.num_sms, false);
-  return launch_bn<kModeRowSplitK>(c, bn, mA, mB, mB, prm);
+  const TileChoice tch = pick_tile(T, d, 1, prm.k_blocks, c.num_sms, false, pair_allowed());
+  if (tch.pair) return launch_tc_pair(c, kModeRowSplitK, tch.bn, mA, mB, mB, prm);
+  return launch_bn<kModeRowSplitK>(c, tch.bn, mA, mB, mB, prm);
 }
 
 }  // namespace tpk

@@ -55,8 +55,15 @@ bool make_map(CUtensorMap* m, const void* gaddr, int rank, const uint64_t* dims,
 bool make_map_a(CUtensorMap* m, const void* g, int64_t inner, int64_t rows, int64_t batches);
 // [rows][cols] bf16 weight, N-contiguous, boxes of 64 rows x 64 columns (N-major B tiles).
 bool make_map_b(CUtensorMap* m, const void* g, int64_t cols, int64_t rows);
-// Tile width (accumulator columns) for a GEMM with this tile space.
-int pick_bn(int64_t m_tiles, int64_t n_total, int64_t batches, int num_sms, bool swiglu);
+// Tile width (accumulator columns) and whether to use CTA-pair tiles
+// (256 rows on two SMs) for one GEMM layer of T rows, n_total output
+// columns, `batches` shards and k_blocks 64-deep k slots per tile.
+struct TileChoice {
+  int bn;
+  bool pair;
+};
+TileChoice pick_tile(int64_t T, int64_t n_total, int64_t batches, int64_t k_blocks, int num_sms,
+                     bool swiglu, bool allow_pair);
 
 inline int32_t ceil_div(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
 

@@ -19,6 +19,16 @@ inline bool pdl_allowed() {
   return on;
 }
 
+// CTA-pair (cta_group::2) GEMMs for wide tiles; TP_DISABLE_PAIR=1 keeps the
+// one-CTA kernel (for comparisons).
+inline bool pair_allowed() {
+  static const bool on = [] {
+    const char* e = std::getenv("TP_DISABLE_PAIR");
+    return !(e != nullptr && e[0] == '1');
+  }();
+  return on;
+}
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t stream, Args&&... args) {

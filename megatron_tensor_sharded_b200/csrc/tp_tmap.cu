@@ -5,6 +5,7 @@
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <climits>
 #include <cstdint>
 #include <cstring>
@@ -123,29 +124,43 @@ bool make_map_b(CUtensorMap* m, const void* g, int64_t cols, int64_t rows) {
 }
 
 
-// Tile width: minimise (waves of tiles over the SMs) x (per-tile cost), the
-// per-tile cost taken as BN plus a fixed 64-column overhead (pipeline fill,
-// epilogue).  Wide problems keep BN = 256, the most efficient per FLOP.
-int pick_bn(int64_t m_tiles, int64_t n_total, int64_t batches, int num_sms, bool swiglu) {
-  static const int cand_all[4] = {256, 192, 128, 64};
-  static const int cand_swiglu[2] = {256, 128};
-  const int* cand = swiglu ? cand_swiglu : cand_all;
-  const int n = swiglu ? 2 : 4;
-  int best = 256;
-  int64_t best_cost = INT64_MAX;
-  for (int i = 0; i < n; ++i) {
-    const int bn = cand[i];
+// Tile choice for one GEMM layer.  Per tile: k slots x max(MMA cycles,
+// operand bytes / ingest rate) + a fixed cost (pipeline fill, epilogue);
+// waves = tiles over the SMs (single-CTA tiles) or SM pairs (pair tiles);
+// minimise waves x per-tile cost.  Per 64-deep k slot, a single-CTA tile of
+// width BN issues 2*BN MMA cycles and loads 16 KiB of A + 128*BN bytes of B;
+// a pair tile of width PBN loads 16 KiB + 64*PBN bytes per CTA for 2*PBN
+// cycles.  Ingest is taken as 80 bytes per SM cycle and the fixed cost as
+// 2000 cycles (both from the measured kernels).  Pair tiles need at least
+// 256 rows.  Ties prefer pair tiles, then wider tiles.
+TileChoice pick_tile(int64_t T, int64_t n_total, int64_t batches, int64_t k_blocks, int num_sms,
+                     bool swiglu, bool allow_pair) {
+  constexpr double kIngest = 80.0, kFixed = 2000.0;
+  TileChoice best{256, false};
+  double best_cost = 1e300;
+  auto consider = [&](int bn, bool pair) {
     const int64_t out_cols = swiglu ? bn / 2 : bn;
-    const int64_t tiles = m_tiles * ((n_total + out_cols - 1) / out_cols) * batches;
-    const int64_t waves = (tiles + num_sms - 1) / num_sms;
-    const int64_t cost = waves * (bn + 64);
-    if (cost < best_cost) {
+    const int64_t rows = pair ? 256 : 128;
+    const int64_t tiles = ((T + rows - 1) / rows) * ((n_total + out_cols - 1) / out_cols) * batches;
+    const int64_t slots = pair ? num_sms / 2 : num_sms;
+    const double waves = static_cast<double>((tiles + slots - 1) / slots);
+    const double b_bytes = pair ? 64.0 * bn : 128.0 * bn;
+    const double kb = std::max(2.0 * bn, (16384.0 + b_bytes) / kIngest);
+    const double cost = waves * (static_cast<double>(k_blocks) * kb + kFixed);
+    if (cost < best_cost * (1.0 - 1e-9)) {
       best_cost = cost;
-      best = bn;
+      best = TileChoice{bn, pair};
     }
+  };
+  if (allow_pair && T >= 256) {
+    consider(256, true);
+    consider(128, true);
   }
+  consider(256, false);
+  if (!swiglu) consider(192, false);
+  consider(128, false);
+  if (!swiglu) consider(64, false);
   return best;
 }
-
 
 }  // namespace tpk

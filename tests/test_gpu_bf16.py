@@ -143,7 +143,8 @@ def test_full_size_configs_sampled_rows(name):
     assert O.rel_err(host_f32(blk.P.index_select(1, idx)), ref["P"]) <= TOL_BF16
     assert O.rel_err(host_f32(blk.Z.index_select(0, idx)), ref["Z"]) <= TOL_BF16
     assert not torch.isnan(blk.Z).any().item()
-    for flags in (tp.TP_FLAG_NONE, tp.TP_FLAG_SPLITK_FUSED):
+    for flags in (tp.TP_FLAG_NONE, tp.TP_FLAG_SPLITK_FUSED, tp.TP_FLAG_FUSED_LAUNCH,
+                  tp.TP_FLAG_SPLITK_FUSED | tp.TP_FLAG_FUSED_LAUNCH):
         Z2 = torch.full_like(blk.Z, float("nan"))
         ws = blk.block(flags, Z=Z2)
         blk.sync()
@@ -165,15 +166,15 @@ def test_fused_block_matches_separate_kernels(T, d, s, p, act):
     blk = DeviceBlock(inp, T, d, k, p, act)
     Zf = torch.full_like(blk.Z, float("nan"))
     Zu = torch.full_like(blk.Z, float("nan"))
-    blk.block(tp.TP_FLAG_NONE, Z=Zf)
-    blk.block(tp.TP_FLAG_UNFUSED, Z=Zu)
+    blk.block(tp.TP_FLAG_FUSED_LAUNCH, Z=Zf)
+    blk.block(tp.TP_FLAG_NONE, Z=Zu)
     blk.sync()
     assert np.array_equal(bits(host_f32(Zf)), bits(host_f32(Zu)))
     ref = _oracle(inp, p, act)
     assert O.rel_err(host_f32(Zf), ref["Z"]) <= TOL_BF16
     if s % 64 == 0:
         Zs = torch.full_like(blk.Z, float("nan"))
-        blk.block(tp.TP_FLAG_SPLITK_FUSED, Z=Zs)
+        blk.block(tp.TP_FLAG_SPLITK_FUSED | tp.TP_FLAG_FUSED_LAUNCH, Z=Zs)
         blk.sync()
         assert O.rel_err(host_f32(Zs), ref["Z"]) <= TOL_BF16
 
@@ -189,8 +190,33 @@ def test_fused_block_repeated_calls_reuse_counters():
     for _ in range(3):
         Z = torch.full_like(blk.Z, float("nan"))
         tp.tp_mlp_block(blk.X, blk.W1, blk.Wu, blk.b1, blk.W2, blk.b2, Z, ws, n, w.T, w.d, w.k,
-                        w.p, blk.dtype, blk.act)
+                        w.p, blk.dtype, blk.act, tp.TP_FLAG_FUSED_LAUNCH)
         outs.append(Z)
     blk.sync()
     for Z in outs[1:]:
         assert torch.equal(Z, outs[0])
+
+
+@pytest.mark.parametrize("act,with_bias", [("gelu_tanh", True), ("swiglu", False)])
+def test_cta_pair_tiles(act, with_bias):
+    """Shapes whose per-layer GEMMs take 256-wide tiles on CTA pairs
+    (tcgen05 cta_group::2): ragged T=1000 (a partial second row of a 256-row
+    pair tile), four shards; every element against the oracle, and the
+    per-layer results against the fused block bit for bit."""
+    T, d, k, p = 1000, 2048, 8192, 4
+    inp = _random_bf16(T, d, k, act, with_bias, seed=11)
+    ref = _oracle(inp, p, act)
+    blk = DeviceBlock(inp, T, d, k, p, act)
+    blk.column()
+    blk.row()
+    blk.reduce()
+    blk.sync()
+    Y = host_f32(blk.Y)
+    for i in range(p):
+        assert O.rel_err(Y[i], ref["Y"][i]) <= TOL_BF16, i
+    assert O.rel_err(host_f32(blk.P), ref["P"]) <= TOL_BF16
+    assert O.rel_err(host_f32(blk.Z), ref["Z"]) <= TOL_BF16
+    Zf = torch.full_like(blk.Z, float("nan"))
+    blk.block(tp.TP_FLAG_FUSED_LAUNCH, Z=Zf)
+    blk.sync()
+    assert np.array_equal(bits(host_f32(Zf)), bits(host_f32(blk.Z)))

@@ -65,7 +65,7 @@ def test_dropped_load_in_column_gemm_times_out(short_timeout, slot):
 def test_dropped_load_in_fused_block_times_out(short_timeout):
     inp, blk = _block()
     tp.tp_debug_drop_load(2)
-    blk.block()
+    blk.block(tp.TP_FLAG_FUSED_LAUNCH)
     st = tp.tp_sync_status(check=False)
     assert st == 6, tp.tp_status_string(st)
     _check_healthy(inp, blk)
@@ -78,3 +78,26 @@ def test_drop_applies_to_one_launch_only(short_timeout):
     assert tp.tp_sync_status(check=False) == 6
     blk.column()   # no drop armed any more
     assert tp.tp_sync_status(check=False) == 0
+
+
+def test_dropped_load_in_cta_pair_gemm_times_out(short_timeout):
+    """A shape whose column layer runs on CTA pairs (256 x 256 tiles): the
+    even CTA's MMA wait runs out, both CTAs of every pair stop, meet at the
+    cluster barrier and free their TMEM."""
+    rng = np.random.default_rng(1)
+    c = W.f32_to_bf16_bits
+    T, d, k, p = 1000, 2048, 8192, 4
+    inp = W.Inputs(c(rng.standard_normal((T, d), dtype=np.float32)),
+                   c(rng.standard_normal((d, k), dtype=np.float32) * 0.02), None, None,
+                   c(rng.standard_normal((k, d), dtype=np.float32) * 0.02), None, "bf16")
+    blk = DeviceBlock(inp, T, d, k, p, "gelu_tanh")
+    tp.tp_debug_drop_load(5)
+    blk.column()
+    assert tp.tp_sync_status(check=False) == 6
+    blk.column()
+    blk.row()
+    blk.reduce()
+    assert tp.tp_sync_status(check=False) == 0
+    ref = O.mlp_sharded(inp.values("X")[:64], inp.values("W1"), None, inp.values("W2"), None, p,
+                        "gelu_tanh")["Z"]
+    assert O.rel_err(host_f32(blk.Z)[:64], ref) <= 1e-2
