@@ -132,12 +132,14 @@ bool make_map_b(CUtensorMap* m, const void* g, int64_t cols, int64_t rows) {
 // a pair tile of width PBN loads 16 KiB + 64*PBN bytes per CTA for 2*PBN
 // cycles.  Ingest is taken as 80 bytes per SM cycle and the fixed cost as
 // 2000 cycles (both from the measured kernels).  Pair tiles need at least
-// 256 rows.  Ties prefer pair tiles, then wider tiles.
+// 256 rows and are considered only when single-CTA tiles need more than one
+// wave.  Ties keep the earlier (wider, single-CTA) choice.
 TileChoice pick_tile(int64_t T, int64_t n_total, int64_t batches, int64_t k_blocks, int num_sms,
                      bool swiglu, bool allow_pair) {
   constexpr double kIngest = 80.0, kFixed = 2000.0;
   TileChoice best{256, false};
   double best_cost = 1e300;
+  int64_t best_tiles = 0;
   auto consider = [&](int bn, bool pair) {
     const int64_t out_cols = swiglu ? bn / 2 : bn;
     const int64_t rows = pair ? 256 : 128;
@@ -150,16 +152,19 @@ TileChoice pick_tile(int64_t T, int64_t n_total, int64_t batches, int64_t k_bloc
     if (cost < best_cost * (1.0 - 1e-9)) {
       best_cost = cost;
       best = TileChoice{bn, pair};
+      best_tiles = tiles;
     }
   };
-  if (allow_pair && T >= 256) {
-    consider(256, true);
-    consider(128, true);
-  }
   consider(256, false);
   if (!swiglu) consider(192, false);
   consider(128, false);
   if (!swiglu) consider(64, false);
+  // Pair tiles only pay once the layer takes more than one wave of
+  // single-CTA tiles (measured: they slowed the one-wave GPT-2 layers).
+  if (allow_pair && T >= 256 && best_tiles > num_sms) {
+    consider(256, true);
+    consider(128, true);
+  }
   return best;
 }
 
