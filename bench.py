@@ -430,6 +430,7 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
                 "frac": achieved / peak, "traffic": ncu_traffic(f"{w.name}/{a.mode}"),
                 "kernel": kernel_name,
                 "duration": "block step time (graph replay, CUDA events on the launching stream)",
+                "traffic_scope": "dram bytes of all kernels of one step (ncu)",
                 "peak_source": f"{peak_src} bf16 dense (burst)"}
     else:
         achieved = block_bytes(w) / (ms_step * 1e-3) / 1e9
