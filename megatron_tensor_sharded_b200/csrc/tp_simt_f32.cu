@@ -5,7 +5,7 @@
 //
 // One 64x64 output tile per block of 256 threads; each thread owns a 4x4
 // strided sub-tile and sums k in ascending order with fmaf, so the result
-// is deterministic.
+// is deterministic.  Very few rows take the skinny kernel below.
 #include <cuda_runtime.h>
 
 #include <cstdint>
@@ -142,11 +142,94 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(SimtArgs a) {
   }
 }
 
+// Few rows (T <= 32, e.g. the day-41 walkthrough's X[4,512]): a 64x64 tile
+// would be mostly padding and its k loop pays one memory latency per step.
+// Instead a block owns 32 output columns (one per lane) and splits k across
+// its 8 warps, each streaming its k range with many weight loads in flight;
+// the 8 warp sums are then added in warp order, so the result is
+// deterministic.
+constexpr int kSkinnyRows = 8;
+
+template <int KIND>
+__global__ void __launch_bounds__(256) skinny_f32_kernel(SimtArgs a) {
+  constexpr bool kTwo = (KIND == kColSwiglu);
+  __shared__ float part[8][kSkinnyRows][33];
+  __shared__ float partu[kTwo ? 8 : 1][kTwo ? kSkinnyRows : 1][33];
+  const int lane = threadIdx.x % 32, w = threadIdx.x / 32;
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * 32 + lane;
+  const int64_t batch = blockIdx.z;
+  pdl_wait();
+  pdl_launch_dependents();
+  const int64_t kchunk = (a.K + 7) / 8;
+  const int64_t k0 = w * kchunk;
+  const int64_t k1 = k0 + kchunk < a.K ? k0 + kchunk : a.K;
+  for (int64_t r0 = 0; r0 < a.M; r0 += kSkinnyRows) {
+    float acc[kSkinnyRows], accu[kSkinnyRows];
+#pragma unroll
+    for (int r = 0; r < kSkinnyRows; ++r) acc[r] = accu[r] = 0.0f;
+    if (c < a.N) {
+#pragma unroll 8
+      for (int64_t kk = k0; kk < k1; ++kk) {
+        const float b = load_b<KIND>(a.B0, a, batch, kk, c);
+        float u = 0.0f;
+        if constexpr (kTwo) u = load_b<KIND>(a.B1, a, batch, kk, c);
+#pragma unroll
+        for (int r = 0; r < kSkinnyRows; ++r) {
+          const float x = load_a<KIND>(a, batch, r0 + r, kk);
+          acc[r] = fmaf(x, b, acc[r]);
+          if constexpr (kTwo) accu[r] = fmaf(x, u, accu[r]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kSkinnyRows; ++r) {
+      part[w][r][lane] = acc[r];
+      if constexpr (kTwo) partu[w][r][lane] = accu[r];
+    }
+    __syncthreads();
+    {
+      const int r = threadIdx.x / 32;   // 8 rows x 32 columns, one per thread
+      const int64_t row = r0 + r;
+      if (row < a.M && c < a.N) {
+        float v = part[0][r][lane], vu = 0.0f;
+        if constexpr (kTwo) vu = partu[0][r][lane];
+#pragma unroll
+        for (int q = 1; q < 8; ++q) {
+          v += part[q][r][lane];
+          if constexpr (kTwo) vu += partu[q][r][lane];
+        }
+        if constexpr (KIND == kCol || KIND == kColSwiglu) {
+          if (a.bias != nullptr) v = v + a.bias[c];
+          if constexpr (kTwo) {
+            v = silu_f32(v) * vu;
+          } else {
+            v = act_unary(a.act, v);
+          }
+          const int64_t shard = c / a.s, cc = c - shard * a.s;
+          a.out[(shard * a.M + row) * a.s + cc] = v;
+        } else if constexpr (KIND == kRowPartial) {
+          a.out[(batch * a.M + row) * a.N + c] = v;
+        } else {
+          if (a.bias != nullptr) v = __fadd_rn(v, a.bias[c]);
+          a.out[row * a.N + c] = v;
+        }
+      }
+    }
+    __syncthreads();
+  }
+}
+
 template <int KIND>
 cudaError_t run(const LaunchCtx& c, const SimtArgs& a, int64_t batches) {
-  dim3 grid(static_cast<unsigned>((a.N + TN - 1) / TN), static_cast<unsigned>((a.M + TM - 1) / TM),
-            static_cast<unsigned>(batches));
-  const cudaError_t e = launch_pdl(simt_gemm_kernel<KIND>, grid, dim3(256), 0, c.stream, a);
+  cudaError_t e;
+  if (a.M <= 32) {
+    dim3 grid(static_cast<unsigned>((a.N + 31) / 32), 1, static_cast<unsigned>(batches));
+    e = launch_pdl(skinny_f32_kernel<KIND>, grid, dim3(256), 0, c.stream, a);
+  } else {
+    dim3 grid(static_cast<unsigned>((a.N + TN - 1) / TN), static_cast<unsigned>((a.M + TM - 1) / TM),
+              static_cast<unsigned>(batches));
+    e = launch_pdl(simt_gemm_kernel<KIND>, grid, dim3(256), 0, c.stream, a);
+  }
   note_launch();
   return e;
 }

@@ -21,6 +21,15 @@ What it computes, and where the pages state it:
   sum.  On one device this is a fixed-order fp32 fold (day-41 post,
   ``sum(partial_sums) + bias``; "Building GPT from Scratch -- Part 9",
   "Implementation Sketch", RowParallelLinear.forward).
+* Tensor-parallel attention -- QKV projections column-parallel by heads,
+  attention local to each shard's heads, row-parallel output projection,
+  one reduction (day-41 post, "Attention heads: naturally parallel";
+  "Tensor parallel math", "Attention: parallel across heads"; "Tensor
+  Parallelism Explained", section 2.A; "Building GPT from Scratch -- Part 9",
+  "Splitting the Attention Layer").  Grouped key/value heads (the aquanode
+  Llama worked example: 64 query heads, 8 key/value heads, 1 per GPU at
+  TP = 8) are supported; the mask is optional (the pages write the plain
+  softmax(Q K^T / sqrt(d_k)) V).
 * The Megatron MLP pairing -- column-parallel first layer, element-wise
   activation applied per shard, row-parallel second layer, one reduction
   ("Tensor parallel math", "The MLP block: column then row, one all-reduce";
@@ -243,3 +252,105 @@ def rel_err(got: np.ndarray, want: np.ndarray) -> float:
     if den == 0.0:
         return num
     return num / den
+
+
+# --------------------------------------------------------------------------
+# tensor-parallel attention block (column-parallel QKV by heads, local
+# attention per head, row-parallel output projection, one reduction)
+# --------------------------------------------------------------------------
+
+def heads_per_shard(n_heads: int, p: int) -> int:
+    """h/p heads on every shard; the head count must divide evenly ("Tensor
+    Parallelism Explained", section 4, head-divisibility failure mode; day-41
+    post, "Attention heads: naturally parallel")."""
+    if p < 1:
+        raise ValueError("p must be >= 1")
+    if n_heads % p != 0:
+        raise ValueError(f"number of attention heads ({n_heads}) must be divisible by "
+                         f"tensor_parallel_size ({p})")
+    return n_heads // p
+
+
+def sdpa_head(q: np.ndarray, k: np.ndarray, v: np.ndarray, causal: bool) -> np.ndarray:
+    """softmax(q k^T / sqrt(d_k)) v for one head, float64 ("Tensor parallel
+    math", "Attention: parallel across heads").  q [T, dh], k/v [S, dh].
+    With `causal`, query t sees keys 0..t only."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    scores = (q @ k.T) / math.sqrt(q.shape[1])
+    if causal:
+        T, S = scores.shape
+        mask = np.arange(S)[None, :] > np.arange(T)[:, None]
+        scores = np.where(mask, -np.inf, scores)
+    scores = scores - np.max(scores, axis=1, keepdims=True)
+    w = np.exp(scores)
+    w = w / np.sum(w, axis=1, keepdims=True)
+    return w @ v
+
+
+def attention_unsharded(X, Wq, Wk, Wv, Wo, bo, n_heads: int, n_kv_heads: int, head_dim: int,
+                        causal: bool) -> np.ndarray:
+    """Plain multi-head attention with grouped key/value heads, float64:
+    Z = concat_h softmax(Q_h K_g(h)^T / sqrt(dh)) V_g(h) @ Wo + bo, where query
+    head h uses key/value head g(h) = h // (n_heads / n_kv_heads).  Weights
+    [in, out]: Wq [d, n_heads*dh], Wk/Wv [d, n_kv_heads*dh], Wo [n_heads*dh, d]."""
+    X64 = _f64(X)
+    Q = X64 @ _f64(Wq)
+    K = X64 @ _f64(Wk)
+    V = X64 @ _f64(Wv)
+    group = n_heads // n_kv_heads
+    outs = []
+    for h in range(n_heads):
+        g = h // group
+        outs.append(sdpa_head(Q[:, h * head_dim:(h + 1) * head_dim],
+                              K[:, g * head_dim:(g + 1) * head_dim],
+                              V[:, g * head_dim:(g + 1) * head_dim], causal))
+    Z = np.concatenate(outs, axis=1) @ _f64(Wo)
+    if bo is not None:
+        Z = Z + _f64(bo)[None, :]
+    return Z
+
+
+def attention_sharded(X, Wq, Wk, Wv, Wo, bo, p: int, n_heads: int, n_kv_heads: int,
+                      head_dim: int, causal: bool, hidden_round: Optional[str] = None) -> dict:
+    """The attention block on p simulated shards, written shard by shard:
+    shard i takes query heads [i*h/p, (i+1)*h/p) and key/value heads
+    [i*hkv/p, (i+1)*hkv/p) -- column blocks of Wq, Wk, Wv -- runs attention
+    on them locally, and multiplies by its row block of Wo; the partials are
+    folded in shard order (float32), bias last (day-41 post, "Attention
+    heads: naturally parallel"; "Building GPT from Scratch -- Part 9",
+    TensorParallelAttention).
+
+    Returns Q, K, V shards (float64, as the column layer produces them), the
+    attention outputs O_i [T, h/p*dh] (optionally rounded to bf16 storage),
+    float32 partials P [p, T, d] and the float32 result Z."""
+    hq = heads_per_shard(n_heads, p)
+    hkv = heads_per_shard(n_kv_heads, p)
+    if n_heads % n_kv_heads != 0:
+        raise ValueError("n_heads must be a multiple of n_kv_heads")
+    group = n_heads // n_kv_heads
+    X64 = _f64(X)
+    Qs, Ks, Vs, Os, Ps = [], [], [], [], []
+    for i in range(p):
+        Qi = X64 @ np.asarray(_column_slice(Wq, i, hq * head_dim), dtype=np.float64)
+        Ki = X64 @ np.asarray(_column_slice(Wk, i, hkv * head_dim), dtype=np.float64)
+        Vi = X64 @ np.asarray(_column_slice(Wv, i, hkv * head_dim), dtype=np.float64)
+        if hidden_round == "bf16":
+            Qi, Ki, Vi = round_to_bf16(Qi), round_to_bf16(Ki), round_to_bf16(Vi)
+        heads = []
+        for hh in range(hq):
+            g = hh // group
+            heads.append(sdpa_head(Qi[:, hh * head_dim:(hh + 1) * head_dim],
+                                   Ki[:, g * head_dim:(g + 1) * head_dim],
+                                   Vi[:, g * head_dim:(g + 1) * head_dim], causal))
+        Oi = np.concatenate(heads, axis=1)
+        if hidden_round == "bf16":
+            Oi = round_to_bf16(Oi)
+        Wo_i = np.asarray(_row_slice(Wo, i, hq * head_dim), dtype=np.float64)
+        Ps.append((Oi @ Wo_i).astype(np.float32))
+        Qs.append(Qi); Ks.append(Ki); Vs.append(Vi); Os.append(Oi)
+    P = np.stack(Ps)
+    bo32 = None if bo is None else np.asarray(bo, dtype=np.float32)
+    Z = reduce_partials_fixed_order(P, bo32)
+    return {"Q": Qs, "K": Ks, "V": Vs, "O": Os, "P": P, "Z": Z}
