@@ -184,6 +184,52 @@ tp_status tp_mlp_block_noalloc(const void* X, const void* W1, const void* W_up, 
 size_t tp_mlp_block_workspace_size(int64_t T, int64_t d, int64_t k, int p,
                                    tp_dtype dtype, tp_act act, int flags);
 
+/*
+ * Attention of every shard's own heads (the local step of the
+ * tensor-parallel attention block: each shard holds h/p query heads and
+ * h_kv/p key/value heads and attends with no communication; day-41 post,
+ * "Attention heads: naturally parallel"; "Tensor parallel math", "Attention:
+ * parallel across heads").  Per head: O = softmax(Q K^T / sqrt(head_dim)) V,
+ * query head j of a shard using key/value head j / (n_heads / n_kv_heads).
+ *
+ *   Q  [p][T][(n_heads/p) * head_dim]     bf16 (the column-parallel layout)
+ *   K  [p][T][(n_kv_heads/p) * head_dim]  bf16
+ *   V  [p][T][(n_kv_heads/p) * head_dim]  bf16
+ *   O  [p][T][(n_heads/p) * head_dim]     bf16 output, the input of the
+ *                                         row-parallel output projection
+ *   causal  nonzero: query t attends to keys 0..t only
+ * head_dim must be 128 (else TP_ERR_UNSUPPORTED); n_heads and n_kv_heads
+ * must be divisible by p (else TP_ERR_INDIVISIBLE -- "Tensor Parallelism
+ * Explained", section 4) and n_heads by n_kv_heads.
+ */
+tp_status tp_attention_heads(const void* Q, const void* K, const void* V, void* O, int64_t T,
+                             int p, int n_heads, int n_kv_heads, int head_dim, int causal,
+                             void* stream);
+
+/*
+ * The tensor-parallel attention block, Z = sum_i Attn_i(X) Wo_i [+ bo]:
+ * column-parallel Q, K, V projections by heads (tp_column_linear, identity),
+ * tp_attention_heads, row-parallel output projection (tp_row_linear) and the
+ * fixed-order fold (tp_reduce_partials) -- one reduction per block ("Tensor
+ * parallel math", "Attention: parallel across heads"; "Tensor Parallelism
+ * Explained", section 2.A).
+ *
+ *   X [T][d]; Wq [d][n_heads*head_dim]; Wk, Wv [d][n_kv_heads*head_dim];
+ *   Wo [n_heads*head_dim][d]  (all bf16, [in, out]);  bo [d] fp32 nullable;
+ *   Z [T][d] fp32.
+ *   workspace: tp_attn_block_workspace_size(...) bytes, 256-byte aligned
+ *   (Q, K, V, O shards, then the fp32 partials).
+ */
+tp_status tp_attn_block(const void* X, const void* Wq, const void* Wk, const void* Wv,
+                        const void* Wo, const float* bo, float* Z,
+                        void* workspace, size_t workspace_bytes,
+                        int64_t T, int64_t d, int n_heads, int n_kv_heads, int head_dim, int p,
+                        int causal, void* stream);
+
+/* Workspace bytes tp_attn_block needs (0 if the arguments are invalid). */
+size_t tp_attn_block_workspace_size(int64_t T, int64_t d, int n_heads, int n_kv_heads,
+                                    int head_dim, int p);
+
 /* Synchronise `stream`, then report (and clear) the device status word of
  * the current device: TP_ERR_DEVICE_TIMEOUT if a bounded wait ran out since
  * the last call, TP_ERR_CUDA if the stream reported an error, else TP_OK. */

@@ -21,7 +21,7 @@ __all__ = [
     "TPError", "TP_F32", "TP_BF16", "TP_ACT_GELU_TANH", "TP_ACT_SWIGLU", "TP_ACT_IDENTITY",
     "TP_ACT_RELU", "TP_FLAG_NONE", "TP_FLAG_SPLITK_FUSED", "TP_FLAG_FUSED_LAUNCH", "STATUS", "ACT", "DTYPE",
     "tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
-    "tp_mlp_block_noalloc",
+    "tp_mlp_block_noalloc", "tp_attention_heads", "tp_attn_block", "tp_attn_block_workspace_size",
     "tp_mlp_block_workspace_size", "tp_sync_status", "tp_set_wait_timeout_ns",
     "tp_debug_drop_load", "tp_status_string", "tp_last_error_detail",
     "tp_kernel_launch_count", "tp_abi_version", "LIB_PATH",
@@ -60,6 +60,11 @@ def _load() -> ctypes.CDLL:
                                  i32, vp]
     lib.tp_mlp_block_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32,
                                          i32, vp]
+    lib.tp_attention_heads.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, vp]
+    lib.tp_attn_block.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sz, i64, i64, i32, i32, i32, i32,
+                                  i32, vp]
+    lib.tp_attn_block_workspace_size.argtypes = [i64, i64, i32, i32, i32, i32]
+    lib.tp_attn_block_workspace_size.restype = sz
     lib.tp_mlp_block_workspace_size.argtypes = [i64, i64, i64, i32, i32, i32, i32]
     lib.tp_mlp_block_workspace_size.restype = sz
     lib.tp_sync_status.argtypes = [vp]
@@ -75,7 +80,7 @@ def _load() -> ctypes.CDLL:
     lib.tp_kernel_launch_count.restype = u64
     lib.tp_abi_version.argtypes = []
     for f in ("tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
-              "tp_mlp_block_noalloc",
+              "tp_mlp_block_noalloc", "tp_attention_heads", "tp_attn_block",
               "tp_sync_status", "tp_abi_version"):
         getattr(lib, f).restype = i32
     return lib
@@ -143,6 +148,27 @@ def tp_mlp_block_noalloc(X, W1, W_up, b1, W2, b2, Z, T, d, k, p, dtype, act,
     return _check(_lib.tp_mlp_block_noalloc(_ptr(X), _ptr(W1), _ptr(W_up), _ptr(b1), _ptr(W2),
                                             _ptr(b2), _ptr(Z), T, d, k, p, dtype, act, flags,
                                             _stream(stream)), check)
+
+
+def tp_attention_heads(Q, K, V, O, T, p, n_heads, n_kv_heads, head_dim, causal=False, stream=None,
+                       check=True):
+    """Attention of every shard's own heads: O = softmax(Q K^T / sqrt(dh)) V."""
+    return _check(_lib.tp_attention_heads(_ptr(Q), _ptr(K), _ptr(V), _ptr(O), T, p, n_heads,
+                                          n_kv_heads, head_dim, int(bool(causal)),
+                                          _stream(stream)), check)
+
+
+def tp_attn_block(X, Wq, Wk, Wv, Wo, bo, Z, workspace, workspace_bytes, T, d, n_heads, n_kv_heads,
+                  head_dim, p, causal=False, stream=None, check=True):
+    """The tensor-parallel attention block, Z = sum_i Attn_i(X) Wo_i [+ bo]."""
+    return _check(_lib.tp_attn_block(_ptr(X), _ptr(Wq), _ptr(Wk), _ptr(Wv), _ptr(Wo), _ptr(bo),
+                                     _ptr(Z), _ptr(workspace), workspace_bytes, T, d, n_heads,
+                                     n_kv_heads, head_dim, p, int(bool(causal)),
+                                     _stream(stream)), check)
+
+
+def tp_attn_block_workspace_size(T, d, n_heads, n_kv_heads, head_dim, p) -> int:
+    return int(_lib.tp_attn_block_workspace_size(T, d, n_heads, n_kv_heads, head_dim, p))
 
 
 def tp_mlp_block_workspace_size(T, d, k, p, dtype, act, flags=TP_FLAG_NONE) -> int:

@@ -192,6 +192,43 @@ tp_status reduce_impl(const float* partials, const float* b2, float* Z, int64_t 
   return cuda_status(launch_reduce(c, partials, b2, Z, T, d, p), "reduce launch");
 }
 
+tp_status check_heads(int p, int n_heads, int n_kv_heads, int head_dim) {
+  if (p < 1) return fail(TP_ERR_INVALID_ARG, "p = %d, must be >= 1", p);
+  if (n_heads < 1 || n_kv_heads < 1 || head_dim < 1)
+    return fail(TP_ERR_INVALID_ARG, "heads %d / %d, head_dim %d", n_heads, n_kv_heads, head_dim);
+  if (n_heads % p != 0 || n_kv_heads % p != 0)
+    return fail(TP_ERR_INDIVISIBLE,
+                "number of attention heads (%d) and key/value heads (%d) must be divisible by "
+                "tensor_parallel_size (%d)",
+                n_heads, n_kv_heads, p);
+  if (n_heads % n_kv_heads != 0)
+    return fail(TP_ERR_INVALID_ARG, "n_heads (%d) must be a multiple of n_kv_heads (%d)", n_heads,
+                n_kv_heads);
+  if (head_dim != 128) return fail(TP_ERR_UNSUPPORTED, "head_dim %d (128 is provided)", head_dim);
+  return TP_OK;
+}
+
+tp_status attention_impl(const void* Q, const void* K, const void* V, void* O, int64_t T, int p,
+                         int n_heads, int n_kv_heads, int head_dim, int causal, void* stream) {
+  TP_TRY(check_heads(p, n_heads, n_kv_heads, head_dim));
+  if (T < 0 || T > INT32_MAX) return fail(TP_ERR_INVALID_ARG, "T = %lld", (long long)T);
+  if (T == 0) return TP_OK;
+  TP_TRY(check_ptr(Q, "Q", TP_BF16, true));
+  TP_TRY(check_ptr(K, "K", TP_BF16, true));
+  TP_TRY(check_ptr(V, "V", TP_BF16, true));
+  TP_TRY(check_ptr(O, "O", TP_BF16, true));
+  LaunchCtx c{};
+  TP_TRY(make_ctx(stream, true, &c));
+  return launch_tc_attention(c, Q, K, V, O, T, p, n_heads / p, n_kv_heads / p, causal);
+}
+
+size_t attn_workspace_bytes(int64_t T, int64_t d, int n_heads, int n_kv_heads, int head_dim, int p) {
+  const size_t q = align256(static_cast<size_t>(T) * n_heads * head_dim * 2);
+  const size_t kv = align256(static_cast<size_t>(T) * n_kv_heads * head_dim * 2);
+  const size_t part = align256(static_cast<size_t>(p) * T * d * 4);
+  return 2 * q + 2 * kv + part;
+}
+
 }  // namespace
 
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -292,6 +329,59 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
   }
   TP_TRY(row_impl(Y, W2, P, T, k, d, p, dtype, stream));
   return reduce_impl(P, b2, Z, T, d, p, stream);
+}
+
+tp_status tp_attention_heads(const void* Q, const void* K, const void* V, void* O, int64_t T,
+                             int p, int n_heads, int n_kv_heads, int head_dim, int causal,
+                             void* stream) {
+  g_detail[0] = 0;
+  return attention_impl(Q, K, V, O, T, p, n_heads, n_kv_heads, head_dim, causal, stream);
+}
+
+size_t tp_attn_block_workspace_size(int64_t T, int64_t d, int n_heads, int n_kv_heads,
+                                    int head_dim, int p) {
+  if (check_heads(p, n_heads, n_kv_heads, head_dim) != TP_OK || T < 0 || d < 1) return 0;
+  return attn_workspace_bytes(T, d, n_heads, n_kv_heads, head_dim, p);
+}
+
+tp_status tp_attn_block(const void* X, const void* Wq, const void* Wk, const void* Wv,
+                        const void* Wo, const float* bo, float* Z, void* workspace,
+                        size_t workspace_size, int64_t T, int64_t d, int n_heads, int n_kv_heads,
+                        int head_dim, int p, int causal, void* stream) {
+  g_detail[0] = 0;
+  TP_TRY(check_heads(p, n_heads, n_kv_heads, head_dim));
+  const int64_t kq = static_cast<int64_t>(n_heads) * head_dim;
+  const int64_t kkv = static_cast<int64_t>(n_kv_heads) * head_dim;
+  TP_TRY(check_shape(T, d, kq, p, TP_BF16));
+  if (T == 0) return TP_OK;
+  TP_TRY(check_ptr(X, "X", TP_BF16, true));
+  TP_TRY(check_ptr(Wq, "Wq", TP_BF16, true));
+  TP_TRY(check_ptr(Wk, "Wk", TP_BF16, true));
+  TP_TRY(check_ptr(Wv, "Wv", TP_BF16, true));
+  TP_TRY(check_ptr(Wo, "Wo", TP_BF16, true));
+  if (Z == nullptr) return fail(TP_ERR_INVALID_ARG, "Z is NULL");
+  if (!aligned16(Z)) return fail(TP_ERR_ALIGNMENT, "Z must be 16-byte aligned");
+  if (bo != nullptr && !aligned4(bo)) return fail(TP_ERR_ALIGNMENT, "bo must be 4-byte aligned");
+  const size_t need = attn_workspace_bytes(T, d, n_heads, n_kv_heads, head_dim, p);
+  if (workspace == nullptr || workspace_size < need)
+    return fail(TP_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need,
+                workspace == nullptr ? size_t(0) : workspace_size);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(TP_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t qb = align256(static_cast<size_t>(T) * kq * 2);
+  const size_t kvb = align256(static_cast<size_t>(T) * kkv * 2);
+  void* Q = ws;
+  void* K = ws + qb;
+  void* V = ws + qb + kvb;
+  void* O = ws + qb + 2 * kvb;
+  float* P = reinterpret_cast<float*>(ws + 2 * qb + 2 * kvb);
+  TP_TRY(column_impl(X, Wq, nullptr, nullptr, Q, T, d, kq, p, TP_BF16, TP_ACT_IDENTITY, stream));
+  TP_TRY(column_impl(X, Wk, nullptr, nullptr, K, T, d, kkv, p, TP_BF16, TP_ACT_IDENTITY, stream));
+  TP_TRY(column_impl(X, Wv, nullptr, nullptr, V, T, d, kkv, p, TP_BF16, TP_ACT_IDENTITY, stream));
+  TP_TRY(attention_impl(Q, K, V, O, T, p, n_heads, n_kv_heads, head_dim, causal, stream));
+  TP_TRY(row_impl(O, Wo, P, T, kq, d, p, TP_BF16, stream));
+  return reduce_impl(P, bo, Z, T, d, p, stream);
 }
 
 tp_status tp_sync_status(void* stream) {

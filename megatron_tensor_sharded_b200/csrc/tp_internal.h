@@ -76,6 +76,10 @@ tp_status launch_tc_block(const LaunchCtx& c, const void* X, const void* W1, con
                           float* Z, int* counters, int64_t T, int64_t d, int64_t k, int p, int act,
                           bool splitk);
 
+// ---- attention of every shard's heads (tp_attn_sm100.cu), head_dim 128, bf16
+tp_status launch_tc_attention(const LaunchCtx& c, const void* Q, const void* K, const void* V,
+                              void* O, int64_t T, int p, int hq, int hkv, int causal);
+
 // Records a human-readable detail for tp_last_error_detail().
 void set_error_detail(const char* fmt, ...);
 

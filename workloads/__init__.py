@@ -77,6 +77,95 @@ WORKLOADS = {
 }
 
 
+@dataclasses.dataclass(frozen=True)
+class AttnWorkload:
+    """The tensor-parallel attention block: Q, K, V column-parallel by heads,
+    attention per shard, output projection row-parallel, one fold."""
+    name: str
+    T: int            # tokens (one sequence)
+    d: int            # model width
+    n_heads: int      # query heads h
+    n_kv_heads: int   # key/value heads (h for plain multi-head attention)
+    head_dim: int
+    p: int
+    causal: bool
+    description: str
+
+    def flops(self) -> dict:
+        """Algorithmic FLOPs: projections 2*T*d*(h + 2*h_kv)*dh and 2*T*h*dh*d;
+        attention 4*T*T*h*dh (Q K^T and P V), halved when causal."""
+        qkv = 2 * self.T * self.d * (self.n_heads + 2 * self.n_kv_heads) * self.head_dim
+        out = 2 * self.T * self.n_heads * self.head_dim * self.d
+        attn = 4 * self.T * self.T * self.n_heads * self.head_dim
+        if self.causal:
+            attn //= 2
+        return {"qkv": qkv, "attention": attn, "out": out, "total": qkv + attn + out}
+
+
+ATTN_WORKLOADS = {
+    "attn_wide": AttnWorkload("attn_wide", 4096, 4096, 32, 32, 128, 4, True,
+                              "attention block: T=4096 d=4096 32 heads x 128 on p=4 shards "
+                              "(8 heads each), causal, bf16"),
+    "attn_llama": AttnWorkload("attn_llama", 4096, 8192, 64, 8, 128, 8, True,
+                               "grouped-query attention block: T=4096 d=8192 64 query heads, "
+                               "8 key/value heads x 128 on p=8 shards, causal, bf16"),
+}
+
+
+@dataclasses.dataclass
+class AttnInputs:
+    """bf16 bit patterns (uint16) of X and the four projection weights
+    ([in, out] layout), plus the fp32 output bias (or None)."""
+    X: np.ndarray
+    Wq: np.ndarray
+    Wk: np.ndarray
+    Wv: np.ndarray
+    Wo: np.ndarray
+    bo: Optional[np.ndarray]
+
+    def values(self, name: str) -> Optional[np.ndarray]:
+        a = getattr(self, name)
+        if a is None:
+            return None
+        return bf16_bits_to_f32(a) if a.dtype == np.uint16 else a
+
+
+def make_attn_inputs(T: int, d: int, n_heads: int, n_kv_heads: int, head_dim: int,
+                     seed: int = 42, with_bias: bool = False, w_std: float = 0.02) -> AttnInputs:
+    """``default_rng(seed)`` float32 normals in the order X (std 1), Wq, Wk,
+    Wv, Wo (std ``w_std``), bo (std 0.02), rounded to bf16 (bo kept as fp32
+    holding bf16-representable values)."""
+    rng = np.random.default_rng(seed)
+
+    def draw(shape, std):
+        v = rng.standard_normal(shape, dtype=np.float32)
+        if std != 1.0:
+            v *= np.float32(std)
+        return v
+
+    c = f32_to_bf16_bits
+    X = c(draw((T, d), 1.0))
+    Wq = c(draw((d, n_heads * head_dim), w_std))
+    Wk = c(draw((d, n_kv_heads * head_dim), w_std))
+    Wv = c(draw((d, n_kv_heads * head_dim), w_std))
+    Wo = c(draw((n_heads * head_dim, d), w_std))
+    bo = bf16_bits_to_f32(c(draw((d,), 0.02))) if with_bias else None
+    return AttnInputs(X, Wq, Wk, Wv, Wo, bo)
+
+
+def make_qkv(p: int, T: int, hq: int, hkv: int, head_dim: int, seed: int, std: float = 1.0):
+    """Per-shard bf16 (uint16) Q [p][T][hq*dh], K and V [p][T][hkv*dh] with
+    standard-normal entries times ``std``, drawn in the order Q, K, V."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for cols in (hq * head_dim, hkv * head_dim, hkv * head_dim):
+        v = rng.standard_normal((p, T, cols), dtype=np.float32)
+        if std != 1.0:
+            v *= np.float32(std)
+        out.append(f32_to_bf16_bits(v))
+    return tuple(out)
+
+
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float32 values to bf16 (round to nearest, ties to even) and
     return the 16-bit patterns as uint16.  Inputs here are finite."""
