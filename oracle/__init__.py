@@ -8,6 +8,7 @@ from .tp_oracle import (  # noqa: F401
     column_parallel_linear,
     gelu_tanh,
     heads_per_shard,
+    layer_norm,
     mlp_sharded,
     mlp_unsharded,
     reduce_partials_fixed_order,
@@ -18,4 +19,6 @@ from .tp_oracle import (  # noqa: F401
     row_parallel_partials,
     shard_width,
     silu,
+    transformer_block_sharded,
+    transformer_block_unsharded,
 )

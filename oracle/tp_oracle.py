@@ -30,6 +30,11 @@ What it computes, and where the pages state it:
   Llama worked example: 64 query heads, 8 key/value heads, 1 per GPU at
   TP = 8) are supported; the mask is optional (the pages write the plain
   softmax(Q K^T / sqrt(d_k)) V).
+* The transformer block -- LayerNorm, attention block, residual add,
+  LayerNorm, MLP block, residual add: two reductions per layer, the
+  residual added in each fold ("Building GPT from Scratch -- Part 9",
+  "Communication Pattern per Transformer Block"; "Tensor parallel math",
+  "Counting all-reduces").  Pre-norm order as the diagram draws it.
 * The Megatron MLP pairing -- column-parallel first layer, element-wise
   activation applied per shard, row-parallel second layer, one reduction
   ("Tensor parallel math", "The MLP block: column then row, one all-reduce";
@@ -187,12 +192,18 @@ def row_parallel_partials(Y_shards: Sequence[np.ndarray], W2, p: int) -> List[np
     return out
 
 
-def reduce_partials_fixed_order(P: np.ndarray, b2: Optional[np.ndarray] = None) -> np.ndarray:
-    """Z = ((P_0 + P_1) + ...) + P_{p-1}  [+ b2], every addition a single
-    float32 round-to-nearest-even operation, shard index ascending.
+def reduce_partials_fixed_order(P: np.ndarray, b2: Optional[np.ndarray] = None,
+                                residual: Optional[np.ndarray] = None) -> np.ndarray:
+    """Z = ((P_0 + P_1) + ...) + P_{p-1}  [+ b2]  [+ residual], every
+    addition a single float32 round-to-nearest-even operation, shard index
+    ascending, the bias after the partials and the residual stream last (the
+    transformer block's "residual connection (element-wise add)" after each
+    reduced block; "Building GPT from Scratch -- Part 9", "Communication
+    Pattern per Transformer Block").
 
     ``P`` is float32 [p][T][d] (or a sequence of [T][d] float32 arrays);
-    ``b2`` is float32 [d] or None.  Returns float32 [T][d]."""
+    ``b2`` is float32 [d] or None; ``residual`` float32 [T][d] or None.
+    Returns float32 [T][d]."""
     parts = [np.asarray(x) for x in P]
     for x in parts:
         if x.dtype != np.float32:
@@ -205,6 +216,11 @@ def reduce_partials_fixed_order(P: np.ndarray, b2: Optional[np.ndarray] = None) 
         if b.dtype != np.float32:
             raise TypeError("b2 must be float32")
         acc = np.add(acc, b[None, :], dtype=np.float32)
+    if residual is not None:
+        r = np.asarray(residual)
+        if r.dtype != np.float32:
+            raise TypeError("residual must be float32")
+        acc = np.add(acc, r, dtype=np.float32)
     return acc
 
 
@@ -354,3 +370,69 @@ def attention_sharded(X, Wq, Wk, Wv, Wo, bo, p: int, n_heads: int, n_kv_heads: i
     bo32 = None if bo is None else np.asarray(bo, dtype=np.float32)
     Z = reduce_partials_fixed_order(P, bo32)
     return {"Q": Qs, "K": Ks, "V": Vs, "O": Os, "P": P, "Z": Z}
+
+
+# --------------------------------------------------------------------------
+# the tensor-parallel transformer block: LayerNorm -> attention (one
+# reduction) -> residual -> LayerNorm -> MLP (one reduction) -> residual
+# --------------------------------------------------------------------------
+
+def layer_norm(X, gamma, beta, eps: float = 1e-5) -> np.ndarray:
+    """Per row of X [T, d]: (x - mean) / sqrt(var + eps) * gamma + beta, with
+    the biased (divide by d) variance, float64.  The pages only name the
+    step ("LayerNorm (replicated, no communication)", "Building GPT from
+    Scratch -- Part 9", "Communication Pattern per Transformer Block"); this
+    is the standard layer normalisation (Ba, Kiros & Hinton) with a learned
+    gain and bias."""
+    x = _f64(X)
+    mean = x.mean(axis=1, keepdims=True)
+    c = x - mean
+    var = (c * c).mean(axis=1, keepdims=True)
+    y = c / np.sqrt(var + eps)
+    return y * _f64(gamma)[None, :] + _f64(beta)[None, :]
+
+
+def transformer_block_unsharded(X, prm: dict, n_heads: int, n_kv_heads: int, head_dim: int,
+                                act: str, causal: bool, eps: float = 1e-5) -> np.ndarray:
+    """Pre-norm block, float64: H = X + Attn(LN1(X)); out = H + MLP(LN2(H)).
+    ``prm`` holds ln1_g, ln1_b, Wq, Wk, Wv, Wo, bo, ln2_g, ln2_b, W1, W_up, b1,
+    W2, b2 (bo, W_up, b1, b2 may be None)."""
+    X64 = _f64(X)
+    a = layer_norm(X64, prm["ln1_g"], prm["ln1_b"], eps)
+    H = X64 + attention_unsharded(a, prm["Wq"], prm["Wk"], prm["Wv"], prm["Wo"], prm["bo"],
+                                  n_heads, n_kv_heads, head_dim, causal)
+    m = layer_norm(H, prm["ln2_g"], prm["ln2_b"], eps)
+    return H + mlp_unsharded(m, prm["W1"], prm["b1"], prm["W2"], prm["b2"], act,
+                             W_up=prm.get("W_up"))
+
+
+def transformer_block_sharded(X, prm: dict, p: int, n_heads: int, n_kv_heads: int, head_dim: int,
+                              act: str, causal: bool, eps: float = 1e-5,
+                              hidden_round: Optional[str] = None) -> dict:
+    """The block on p simulated shards: the attention and MLP blocks each end
+    in one fixed-order float32 fold, with the residual stream added in that
+    fold (two reductions per layer; "Building GPT from Scratch -- Part 9",
+    "Communication Pattern per Transformer Block"; "Tensor parallel math",
+    "Counting all-reduces").  The residual stream X, H, out is float32.
+    With ``hidden_round == "bf16"`` every tensor a GEMM reads (the LayerNorm
+    outputs, Q, K, V, the attention output, the MLP hidden shards) is
+    rounded to bf16, as the device stores them.
+
+    Returns LN1 output ``A``, ``H`` (float32), LN2 output ``M`` and ``out``
+    (float32)."""
+    X32 = np.asarray(X, dtype=np.float32)
+    A = layer_norm(X32, prm["ln1_g"], prm["ln1_b"], eps)
+    if hidden_round == "bf16":
+        A = round_to_bf16(A)
+    att = attention_sharded(A, prm["Wq"], prm["Wk"], prm["Wv"], prm["Wo"], None, p, n_heads,
+                            n_kv_heads, head_dim, causal, hidden_round=hidden_round)
+    bo = None if prm["bo"] is None else np.asarray(prm["bo"], dtype=np.float32)
+    H = reduce_partials_fixed_order(att["P"], bo, residual=X32)
+    M = layer_norm(H, prm["ln2_g"], prm["ln2_b"], eps)
+    if hidden_round == "bf16":
+        M = round_to_bf16(M)
+    mlp = mlp_sharded(M, prm["W1"], prm["b1"], prm["W2"], None, p, act, W_up=prm.get("W_up"),
+                      hidden_round=hidden_round)
+    b2 = None if prm["b2"] is None else np.asarray(prm["b2"], dtype=np.float32)
+    out = reduce_partials_fixed_order(mlp["P"], b2, residual=H)
+    return {"A": A, "H": H, "M": M, "out": out}
