@@ -395,13 +395,13 @@ def layer_norm(X, gamma, beta, eps: float = 1e-5) -> np.ndarray:
 def transformer_block_unsharded(X, prm: dict, n_heads: int, n_kv_heads: int, head_dim: int,
                                 act: str, causal: bool, eps: float = 1e-5) -> np.ndarray:
     """Pre-norm block, float64: H = X + Attn(LN1(X)); out = H + MLP(LN2(H)).
-    ``prm`` holds ln1_g, ln1_b, Wq, Wk, Wv, Wo, bo, ln2_g, ln2_b, W1, W_up, b1,
+    ``prm`` holds ln1_gamma, ln1_beta, Wq, Wk, Wv, Wo, bo, ln2_gamma, ln2_beta, W1, W_up, b1,
     W2, b2 (bo, W_up, b1, b2 may be None)."""
     X64 = _f64(X)
-    a = layer_norm(X64, prm["ln1_g"], prm["ln1_b"], eps)
+    a = layer_norm(X64, prm["ln1_gamma"], prm["ln1_beta"], eps)
     H = X64 + attention_unsharded(a, prm["Wq"], prm["Wk"], prm["Wv"], prm["Wo"], prm["bo"],
                                   n_heads, n_kv_heads, head_dim, causal)
-    m = layer_norm(H, prm["ln2_g"], prm["ln2_b"], eps)
+    m = layer_norm(H, prm["ln2_gamma"], prm["ln2_beta"], eps)
     return H + mlp_unsharded(m, prm["W1"], prm["b1"], prm["W2"], prm["b2"], act,
                              W_up=prm.get("W_up"))
 
@@ -421,14 +421,14 @@ def transformer_block_sharded(X, prm: dict, p: int, n_heads: int, n_kv_heads: in
     Returns LN1 output ``A``, ``H`` (float32), LN2 output ``M`` and ``out``
     (float32)."""
     X32 = np.asarray(X, dtype=np.float32)
-    A = layer_norm(X32, prm["ln1_g"], prm["ln1_b"], eps)
+    A = layer_norm(X32, prm["ln1_gamma"], prm["ln1_beta"], eps)
     if hidden_round == "bf16":
         A = round_to_bf16(A)
     att = attention_sharded(A, prm["Wq"], prm["Wk"], prm["Wv"], prm["Wo"], None, p, n_heads,
                             n_kv_heads, head_dim, causal, hidden_round=hidden_round)
     bo = None if prm["bo"] is None else np.asarray(prm["bo"], dtype=np.float32)
     H = reduce_partials_fixed_order(att["P"], bo, residual=X32)
-    M = layer_norm(H, prm["ln2_g"], prm["ln2_b"], eps)
+    M = layer_norm(H, prm["ln2_gamma"], prm["ln2_beta"], eps)
     if hidden_round == "bf16":
         M = round_to_bf16(M)
     mlp = mlp_sharded(M, prm["W1"], prm["b1"], prm["W2"], None, p, act, W_up=prm.get("W_up"),
@@ -436,3 +436,121 @@ def transformer_block_sharded(X, prm: dict, p: int, n_heads: int, n_kv_heads: in
     b2 = None if prm["b2"] is None else np.asarray(prm["b2"], dtype=np.float32)
     out = reduce_partials_fixed_order(mlp["P"], b2, residual=H)
     return {"A": A, "H": H, "M": M, "out": out}
+
+
+# --------------------------------------------------------------------------
+# backward pass of the MLP block: the f / g conjugate operators ("Tensor
+# parallel math", "The f and g conjugate operators"; "Counting all-reduces":
+# one all-reduce per block in the backward pass as well)
+# --------------------------------------------------------------------------
+
+def gelu_tanh_grad(h: np.ndarray) -> np.ndarray:
+    """d/dh of the tanh-form GELU, float64:
+    0.5 (1 + tanh u) + 0.5 h (1 - tanh^2 u) sqrt(2/pi) (1 + 3 * 0.044715 h^2),
+    u = sqrt(2/pi) (h + 0.044715 h^3)."""
+    h = np.asarray(h, dtype=np.float64)
+    t = np.tanh(_SQRT_2_OVER_PI * (h + 0.044715 * h * h * h))
+    du = _SQRT_2_OVER_PI * (1.0 + 3.0 * 0.044715 * h * h)
+    return 0.5 * (1.0 + t) + 0.5 * h * (1.0 - t * t) * du
+
+
+def silu_grad(h: np.ndarray) -> np.ndarray:
+    """d/dh of h * sigma(h): sigma(h) (1 + h (1 - sigma(h))), float64."""
+    h = np.asarray(h, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        sg = 1.0 / (1.0 + np.exp(-h))
+    return sg * (1.0 + h * (1.0 - sg))
+
+
+def activation_backward(act: str, dY, h, up=None):
+    """Gradient through the element-wise activation: returns (dH, dUp) where
+    dUp is None except for SwiGLU (Y = SiLU(h) * up)."""
+    dY = np.asarray(dY, dtype=np.float64)
+    h = np.asarray(h, dtype=np.float64)
+    if act == "gelu_tanh":
+        return dY * gelu_tanh_grad(h), None
+    if act == "relu":
+        return dY * (h > 0.0), None
+    if act == "identity":
+        return dY.copy(), None
+    if act == "swiglu":
+        u = np.asarray(up, dtype=np.float64)
+        return dY * u * silu_grad(h), dY * silu(h)
+    raise ValueError(f"unknown activation {act!r}")
+
+
+def mlp_backward_unsharded(X, W1, b1, W2, dZ, act: str, W_up=None) -> dict:
+    """Gradients of Z = act(X W1 + b1) W2 + b2 for the upstream gradient dZ,
+    float64, no sharding: dX, dW1, dW_up (SwiGLU), db1, dW2, db2."""
+    X, W1, W2, dZ = _f64(X), _f64(W1), _f64(W2), _f64(dZ)
+    H = X @ W1
+    if b1 is not None:
+        H = H + _f64(b1)[None, :]
+    U = X @ _f64(W_up) if act == "swiglu" else None
+    Y = apply_activation(act, H, U)
+    dY = dZ @ W2.T
+    dH, dU = activation_backward(act, dY, H, U)
+    out = {"dW2": Y.T @ dZ, "db2": dZ.sum(axis=0), "dW1": X.T @ dH, "db1": dH.sum(axis=0),
+           "dX": dH @ W1.T, "dW_up": None}
+    if dU is not None:
+        out["dW_up"] = X.T @ dU
+        out["dX"] = out["dX"] + dU @ _f64(W_up).T
+    return out
+
+
+def mlp_backward_sharded(X, W1, b1, W2, dZ, p: int, act: str, W_up=None,
+                         hidden_round: Optional[str] = None) -> dict:
+    """The backward pass on p simulated shards, shard by shard.
+
+    g (after the row-parallel layer) is the identity backward: every shard
+    receives the whole dZ.  Shard i forms dY_i = dZ W2_i^T, goes back through
+    its activation locally (dH_i), and computes its own weight gradients
+    dW2_i = Y_i^T dZ, dW1_i = X^T dH_i, db1_i = sum_t dH_i -- no
+    communication.  f (before the column-parallel layer) is the all-reduce
+    backward: the input gradient dX = sum_i dH_i W1_i^T (+ dU_i W_up,i^T) is
+    a sum of full-shape partials, folded in shard order in float32 ("Tensor
+    parallel math", "The f and g conjugate operators").  db2 belongs to the
+    replicated bias: sum_t dZ, once.
+
+    ``hidden_round == "bf16"`` rounds what the device stores in bf16: the
+    pre-activations H_i (and up projections), the activations Y_i and dH_i
+    (and dU_i).  Returns per-shard lists and the assembled gradients:
+    dW1 [d, k], dW_up, db1 [k], dW2 [k, d], db2 [d] (float64), the dX partials
+    (float32 [p, T, d]) and dX (float32 fold)."""
+    rnd = round_to_bf16 if hidden_round == "bf16" else (lambda a: a)
+    if hidden_round not in (None, "bf16"):
+        raise ValueError(hidden_round)
+    k = np.shape(W1)[1]
+    s = shard_width(k, p)
+    X64, dZ64 = _f64(X), _f64(dZ)
+    dW1, dWu, db1, dW2, parts = [], [], [], [], []
+    for i in range(p):
+        W1i = np.asarray(_column_slice(W1, i, s), dtype=np.float64)
+        Hi = X64 @ W1i
+        if b1 is not None:
+            Hi = Hi + np.asarray(_vector_slice(b1, i, s), dtype=np.float64)[None, :]
+        Ui = Wui = None
+        if act == "swiglu":
+            Wui = np.asarray(_column_slice(W_up, i, s), dtype=np.float64)
+            Ui = X64 @ Wui
+        Yi = rnd(apply_activation(act, Hi, Ui))
+        Hi = rnd(Hi)
+        Ui = None if Ui is None else rnd(Ui)
+        W2i = np.asarray(_row_slice(W2, i, s), dtype=np.float64)
+        dYi = dZ64 @ W2i.T
+        dHi, dUi = activation_backward(act, dYi, Hi, Ui)
+        dHi = rnd(dHi)
+        dUi = None if dUi is None else rnd(dUi)
+        dW2.append(Yi.T @ dZ64)
+        dW1.append(X64.T @ dHi)
+        db1.append(dHi.sum(axis=0))
+        part = dHi @ W1i.T
+        if dUi is not None:
+            dWu.append(X64.T @ dUi)
+            part = part + dUi @ Wui.T
+        parts.append(part.astype(np.float32))
+    P = np.stack(parts)
+    return {"dW1": np.concatenate(dW1, axis=1), "db1": np.concatenate(db1),
+            "dW_up": np.concatenate(dWu, axis=1) if dWu else None,
+            "dW2": np.concatenate(dW2, axis=0), "db2": dZ64.sum(axis=0),
+            "dX_partials": P, "dX": reduce_partials_fixed_order(P)}
