@@ -2,6 +2,9 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload gpt2|toy|wide|decode|llama]
                     [--mode partials|splitk] [--impl tp|reference]
+    python bench.py --workload attn_wide|attn_llama     (the attention block)
+    python bench.py --workload block_wide|block_llama   (the transformer block)
+    python bench.py --workload wide --mode backward     (the MLP block's backward pass)
 
 One step = one pass of the whole hot path over one batch of synthetic input:
 tp_mlp_block, i.e. the column-parallel GEMM + activation (all p shards), the
@@ -20,11 +23,23 @@ so there is no data-path collective; the step time is the max over ranks and
 
 `--impl reference` times the CPU oracle (float64 numpy) on the host cores on a
 bounded token-row sample of the same workload, in the same metric.
+
+The attention workloads time tp_attn_block the same way (one graph replay per
+step: column Q, K, V projections, attention of every shard's heads,
+row-parallel output projection, fold), with a per-call breakdown; the CPU
+oracle runs on a causal prefix of the tokens (with a causal mask the first n
+rows of the block depend only on the first n tokens).
+
+The transformer-block workloads time tp_transformer_block (LayerNorm,
+attention block with the residual folded into its reduction and the second
+LayerNorm fused behind it, MLP block, reduction with the residual), with a
+breakdown over the public calls run one after another.
 """
 
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import datetime
 import hashlib
 import json
@@ -43,6 +58,9 @@ import numpy as np  # noqa: E402
 import workloads as WL  # noqa: E402
 
 METRIC = "sharded-MLP TFLOP/s & % BF16 tensor peak; partial-sum reduce HBM GB/s"
+ATTN_METRIC = "tensor-parallel attention block TFLOP/s & % BF16 tensor peak"
+BLOCK_METRIC = "tensor-parallel transformer block TFLOP/s & % BF16 tensor peak"
+BWD_METRIC = "sharded-MLP backward TFLOP/s & % BF16 tensor peak"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_FLUSH_BYTES = 256 << 20
@@ -250,6 +268,184 @@ def run_reference(a, w: WL.Workload, rank: int, world: int):
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+def attn_flops_prefix(w: WL.AttnWorkload, n: int) -> dict:
+    """Algorithmic FLOPs of the block on the first n tokens."""
+    return dataclasses.replace(w, T=n).flops()
+
+
+def attn_oracle_rows(w: WL.AttnWorkload, target_flops: float = 3e10) -> int:
+    n = 16
+    while n < w.T and attn_flops_prefix(w, min(w.T, 2 * n))["total"] <= target_flops:
+        n *= 2
+    return min(n, w.T)
+
+
+def time_attn_oracle(w: WL.AttnWorkload, inp, rows: int, min_seconds: float, max_reps: int):
+    from oracle import tp_oracle as O
+    X = inp.values("X")[:rows]
+    args = (inp.values("Wq"), inp.values("Wk"), inp.values("Wv"), inp.values("Wo"), inp.bo)
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        O.attention_sharded(X, *args, w.p, w.n_heads, w.n_kv_heads, w.head_dim, w.causal)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or reps >= max_reps:
+            return el / reps, reps
+
+
+def attn_config(w: WL.AttnWorkload, world: int) -> dict:
+    return {"workload": w.name, "T": w.T, "d": w.d, "n_heads": w.n_heads,
+            "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "p": w.p, "causal": w.causal,
+            "parallelism": f"replicas{world}" if world > 1 else "single"}
+
+
+def run_reference_attn(a, w: WL.AttnWorkload, rank: int, world: int):
+    if rank != 0:
+        return 0
+    inp = WL.make_attn_inputs(w.T, w.d, w.n_heads, w.n_kv_heads, w.head_dim)
+    rows = attn_oracle_rows(w)
+    flops = attn_flops_prefix(w, rows)["total"]
+    for _ in range(a.warmup):
+        time_attn_oracle(w, inp, rows, 0.0, 1)
+    times = [time_attn_oracle(w, inp, rows, 0.0, 1)[0] for _ in range(a.steps)]
+    ms = 1e3 * sum(times) / len(times)
+    value = flops / (ms * 1e-3) / 1e12
+    cfg = attn_config(w, world)
+    cfg["sample_rows"] = rows
+    line = {
+        "impl": "reference", "metric": ATTN_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"causal prefix: first {rows} of {w.T} tokens per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def block_flops_prefix(w: WL.BlockWorkload, n: int) -> dict:
+    return dataclasses.replace(w, T=n).flops()
+
+
+def block_oracle_rows(w: WL.BlockWorkload, target_flops: float = 3e10) -> int:
+    n = 8
+    while n < w.T and block_flops_prefix(w, min(w.T, 2 * n))["total"] <= target_flops:
+        n *= 2
+    return min(n, w.T)
+
+
+def time_block_oracle(w: WL.BlockWorkload, inp, rows: int, min_seconds: float, max_reps: int):
+    from oracle import tp_oracle as O
+    X = inp.X[:rows]
+    prm = inp.value_dict()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        O.transformer_block_sharded(X, prm, w.p, w.n_heads, w.n_kv_heads, w.head_dim, w.act,
+                                    w.causal)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds or reps >= max_reps:
+            return el / reps, reps
+
+
+def block_config(w: WL.BlockWorkload, world: int) -> dict:
+    return {"workload": w.name, "T": w.T, "d": w.d, "n_heads": w.n_heads,
+            "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "k": w.k, "p": w.p, "act": w.act,
+            "causal": w.causal, "parallelism": f"replicas{world}" if world > 1 else "single"}
+
+
+def run_reference_block(a, w: WL.BlockWorkload, rank: int, world: int):
+    if rank != 0:
+        return 0
+    inp = WL.make_block_inputs(w.T, w.d, w.n_heads, w.n_kv_heads, w.head_dim, w.k, w.act)
+    rows = block_oracle_rows(w)
+    flops = block_flops_prefix(w, rows)["total"]
+    for _ in range(a.warmup):
+        time_block_oracle(w, inp, rows, 0.0, 1)
+    times = [time_block_oracle(w, inp, rows, 0.0, 1)[0] for _ in range(a.steps)]
+    ms = 1e3 * sum(times) / len(times)
+    value = flops / (ms * 1e-3) / 1e12
+    cfg = block_config(w, world)
+    cfg["sample_rows"] = rows
+    line = {
+        "impl": "reference", "metric": BLOCK_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": cfg,
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"causal prefix: first {rows} of {w.T} tokens per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+class Harness:
+    """Warm-up, CUDA-graph capture and the timed loop of the transformer-block
+    arm."""
+
+    def __init__(self, a, torch, tp, device, barrier):
+        self.a, self.torch, self.tp, self.device, self.barrier = a, torch, tp, device, barrier
+        self.stream = torch.cuda.current_stream(device)
+        self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+
+    def capture(self, fn, graph: bool):
+        """Warm up eagerly, then (with `graph`) capture one step; returns
+        (graph or None, library kernels per step or None)."""
+        torch, tp = self.torch, self.tp
+        for _ in range(self.a.warmup):
+            self.flush.zero_()
+            fn(self.stream)
+        tp.tp_sync_status(self.stream)
+        if not graph:
+            return None, None
+        g = torch.cuda.CUDAGraph()
+        n0 = tp.tp_kernel_launch_count()
+        with torch.cuda.graph(g):
+            fn(torch.cuda.current_stream())
+        per_step = tp.tp_kernel_launch_count() - n0
+        for _ in range(self.a.warmup):
+            self.flush.zero_()
+            g.replay()
+        torch.cuda.synchronize(self.device)
+        return g, per_step
+
+    def time_steps(self, fn, graph: bool = True, events=None):
+        """K timed steps, L2 flushed before each (outside the events).  Returns
+        the step times (ms), or with `events` (recorded inside the step) the
+        per-step lists of their successive intervals; plus the library
+        launches in the timed region and its wall time."""
+        torch, tp = self.torch, self.tp
+        g, per_step = self.capture(fn, graph and not self.a.no_graph)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        out = []
+        self.barrier()
+        torch.cuda.synchronize(self.device)
+        n0 = tp.tp_kernel_launch_count()
+        t_wall = time.perf_counter()
+        for _ in range(self.a.steps):
+            self.flush.zero_()
+            e0.record(self.stream)
+            if g is not None:
+                g.replay()
+            else:
+                fn(self.stream)
+            e1.record(self.stream)
+            torch.cuda.synchronize(self.device)
+            if events is None:
+                out.append(e0.elapsed_time(e1))
+            else:
+                out.append([events[i].elapsed_time(events[i + 1]) for i in range(len(events) - 1)])
+        t_wall = time.perf_counter() - t_wall
+        launches = tp.tp_kernel_launch_count() - n0
+        if g is not None:
+            launches = per_step * self.a.steps
+        self.barrier()
+        tp.tp_sync_status(self.stream)
+        return out, launches, t_wall
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -489,14 +685,560 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
     return 0
 
 
+def run_tp_attn(a, w: WL.AttnWorkload, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    import megatron_tensor_sharded_b200 as tp
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    grp = dist if world > 1 else None
+    inp = WL.make_attn_inputs(w.T, w.d, w.n_heads, w.n_kv_heads, w.head_dim)
+
+    def dev(x):
+        if x is None:
+            return None
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(x).to(device)
+
+    X, Wq, Wk, Wv, Wo, bo = (dev(inp.X), dev(inp.Wq), dev(inp.Wk), dev(inp.Wv), dev(inp.Wo),
+                             dev(inp.bo))
+    T, d, h, hkv, dh, p, causal = w.T, w.d, w.n_heads, w.n_kv_heads, w.head_dim, w.p, w.causal
+    Z = torch.empty((T, d), dtype=torch.float32, device=device)
+    nbytes = tp.tp_attn_block_workspace_size(T, d, h, hkv, dh, p)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    # separate buffers for the per-call breakdown
+    Qs = torch.empty((p, T, h // p * dh), dtype=torch.bfloat16, device=device)
+    Ks = torch.empty((p, T, hkv // p * dh), dtype=torch.bfloat16, device=device)
+    Vs = torch.empty_like(Ks)
+    Os = torch.empty_like(Qs)
+    Ps = torch.empty((p, T, d), dtype=torch.float32, device=device)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    ident = tp.TP_ACT_IDENTITY
+
+    def block_step(st):
+        tp.tp_attn_block(X, Wq, Wk, Wv, Wo, bo, Z, ws, nbytes, T, d, h, hkv, dh, p, causal,
+                         stream=st)
+
+    def calls_step(st, ev):
+        ev[0].record(st)
+        tp.tp_column_linear(X, Wq, None, None, Qs, T, d, h * dh, p, tp.TP_BF16, ident, stream=st)
+        tp.tp_column_linear(X, Wk, None, None, Ks, T, d, hkv * dh, p, tp.TP_BF16, ident, stream=st)
+        tp.tp_column_linear(X, Wv, None, None, Vs, T, d, hkv * dh, p, tp.TP_BF16, ident, stream=st)
+        ev[1].record(st)
+        tp.tp_attention_heads(Qs, Ks, Vs, Os, T, p, h, hkv, dh, causal, stream=st)
+        ev[2].record(st)
+        tp.tp_row_linear(Os, Wo, Ps, T, h * dh, d, p, tp.TP_BF16, stream=st)
+        ev[3].record(st)
+        tp.tp_reduce_partials(Ps, bo, Z, T, d, p, stream=st)
+        ev[4].record(st)
+
+    def capture(fn):
+        for _ in range(a.warmup):
+            flush.zero_()
+            fn(stream)
+        tp.tp_sync_status(stream)
+        if a.no_graph:
+            return None, None
+        g = torch.cuda.CUDAGraph()
+        n0 = tp.tp_kernel_launch_count()
+        with torch.cuda.graph(g):
+            fn(torch.cuda.current_stream())
+        per_step = tp.tp_kernel_launch_count() - n0
+        for _ in range(a.warmup):
+            flush.zero_()
+            g.replay()
+        torch.cuda.synchronize(device)
+        return g, per_step
+
+    g_block, k_block = capture(block_step)
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    step_ms = []
+    with ClockSampler(local_rank) as clocks:
+        barrier()
+        torch.cuda.synchronize(device)
+        n0 = tp.tp_kernel_launch_count()
+        t_wall = time.perf_counter()
+        for _ in range(a.steps):
+            flush.zero_()
+            e0.record(stream)
+            if g_block is not None:
+                g_block.replay()
+            else:
+                block_step(stream)
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            step_ms.append(e0.elapsed_time(e1))
+        t_wall = time.perf_counter() - t_wall
+        launches = tp.tp_kernel_launch_count() - n0
+        if g_block is not None:
+            launches = k_block * a.steps
+        barrier()
+    tp.tp_sync_status(stream)
+    ms_step, launches = reduce_max([statistics.mean(step_ms), float(launches)], grp, device)
+
+    fl = w.flops()
+    peaks, peak_src = load_peaks()
+    breakdown = None
+    if not a.no_breakdown:
+        evs = [torch.cuda.Event(enable_timing=True, external=not a.no_graph) for _ in range(5)]
+        g_calls, _ = capture(lambda st: calls_step(st, evs))
+        parts = [[], [], [], []]
+        barrier()
+        for _ in range(a.steps):
+            flush.zero_()
+            if g_calls is not None:
+                g_calls.replay()
+            else:
+                calls_step(stream, evs)
+            torch.cuda.synchronize(device)
+            for i in range(4):
+                parts[i].append(evs[i].elapsed_time(evs[i + 1]))
+        barrier()
+        tp.tp_sync_status(stream)
+        qkv_ms, att_ms, out_ms, red_ms = reduce_max([statistics.mean(x) for x in parts], grp, device)
+        red_bytes = (p + 1) * T * d * 4 + (d * 4 if bo is not None else 0)
+
+        def tf(f, ms):
+            return f / (ms * 1e-3) / 1e12
+        breakdown = {
+            "qkv": {"ms": qkv_ms, "TFLOP/s": tf(fl["qkv"], qkv_ms)},
+            "attention": {"ms": att_ms, "TFLOP/s": tf(fl["attention"], att_ms)},
+            "out": {"ms": out_ms, "TFLOP/s": tf(fl["out"], out_ms)},
+            "reduce": {"ms": red_ms, "GB/s": red_bytes / (red_ms * 1e-3) / 1e9, "bytes": red_bytes},
+            "how": "the six C-ABI calls as one graph, external timing events between them",
+        }
+        for k in ("qkv", "attention", "out"):
+            breakdown[k]["frac_bf16_peak"] = breakdown[k]["TFLOP/s"] / peaks["bf16_tflops"]
+
+    e2e = None
+    if not a.no_e2e:
+        Xh = X.cpu().pin_memory()
+        Zh = torch.empty(Z.shape, dtype=Z.dtype).pin_memory()
+        Xd = torch.empty_like(X)
+
+        def e2e_step():
+            Xd.copy_(Xh, non_blocking=True)
+            tp.tp_attn_block(Xd, Wq, Wk, Wv, Wo, bo, Z, ws, nbytes, T, d, h, hkv, dh, p, causal,
+                             stream=stream)
+            Zh.copy_(Z, non_blocking=True)
+
+        for _ in range(a.warmup):
+            flush.zero_()
+            e2e_step()
+        torch.cuda.synchronize(device)
+        barrier()
+        t_e2e = []
+        for _ in range(a.steps):
+            flush.zero_()
+            e0.record(stream)
+            e2e_step()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            t_e2e.append(e0.elapsed_time(e1))
+        barrier()
+        tp.tp_sync_status(stream)
+        e_ms = reduce_max([statistics.mean(t_e2e)], grp, device)[0]
+        e2e = {"value": whole_job_value(fl["total"], world, e_ms) / 1e12, "unit": UNIT,
+               "ms_per_step": e_ms, "h2d_bytes_per_step": Xh.numel() * Xh.element_size(),
+               "d2h_bytes_per_step": Zh.numel() * Zh.element_size(),
+               "call": "tp_attn_block, X host->device and Z device->host inside the timed step"}
+
+    value = whole_job_value(fl["total"], world, ms_step) / 1e12
+    achieved = fl["total"] / (ms_step * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+            "traffic": ncu_traffic(f"{w.name}/block"),
+            "kernel": "tp_attn_block: QKV column GEMMs -> tc_attn_kernel -> row GEMM -> fold",
+            "duration": "block step time (graph replay, CUDA events on the launching stream)",
+            "peak_source": f"{peak_src} bf16 dense (burst)",
+            "flops_per_step": fl}
+    line = {
+        "metric": ATTN_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(attn_config(w, world),
+                       launch="eager" if g_block is None else "cuda-graph replay of tp_attn_block",
+                       l2="flushed before every step (256 MiB write, outside the timed events)"),
+        "pct_bf16_peak": 100.0 * value / (peaks["bf16_tflops"] * world),
+        "breakdown": breakdown,
+        "roofline": roof,
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "wall_s_timed_region": t_wall,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        rows = attn_oracle_rows(w)
+        sec, reps = time_attn_oracle(w, inp, rows, min_seconds=10.0, max_reps=1000)
+        line["cpu_baseline"] = {"value": attn_flops_prefix(w, rows)["total"] / sec / 1e12,
+                                "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"causal prefix: first {rows} of {w.T} tokens, {reps} reps, "
+                                          "float64"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def run_tp_block(a, w: WL.BlockWorkload, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    import megatron_tensor_sharded_b200 as tp
+
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    grp = dist if world > 1 else None
+    H = Harness(a, torch, tp, device, barrier)
+    inp = WL.make_block_inputs(w.T, w.d, w.n_heads, w.n_kv_heads, w.head_dim, w.k, w.act)
+
+    def dev(x):
+        if x is None:
+            return None
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(x).to(device)
+
+    T, d, h, hkv, dh, k, p = w.T, w.d, w.n_heads, w.n_kv_heads, w.head_dim, w.k, w.p
+    act, causal = tp.ACT[w.act], w.causal
+    X = dev(inp.X)
+    t = {name: dev(v) for name, v in inp.prm.items()}
+    prm = tp.block_params(**t)
+    out = torch.empty((T, d), dtype=torch.float32, device=device)
+    nbytes = tp.tp_transformer_block_workspace_size(T, d, h, hkv, dh, k, p)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+    def block_step(st):
+        tp.tp_transformer_block(X, prm, out, ws, nbytes, T, d, h, hkv, dh, k, p, act, causal,
+                                stream=st)
+
+    with ClockSampler(local_rank) as clocks:
+        step_ms, launches, t_wall = H.time_steps(block_step)
+    ms_step, launches = reduce_max([statistics.mean(step_ms), float(launches)], grp, device)
+    fl = w.flops()
+    peaks, peak_src = load_peaks()
+
+    breakdown = None
+    if not a.no_breakdown:
+        A = torch.empty((T, d), dtype=torch.bfloat16, device=device)
+        Hs = torch.empty((T, d), dtype=torch.float32, device=device)
+        Qs = torch.empty((p, T, h // p * dh), dtype=torch.bfloat16, device=device)
+        Ks = torch.empty((p, T, hkv // p * dh), dtype=torch.bfloat16, device=device)
+        Vs = torch.empty_like(Ks)
+        Os = torch.empty_like(Qs)
+        Ys = torch.empty((p, T, k // p), dtype=torch.bfloat16, device=device)
+        Ps = torch.empty((p, T, d), dtype=torch.float32, device=device)
+        Zs = torch.empty((T, d), dtype=torch.float32, device=device)
+        names = ["ln1", "qkv", "attention", "out_proj", "fold1", "ln2", "mlp_column", "mlp_row",
+                 "fold2"]
+        evs = [torch.cuda.Event(enable_timing=True, external=not a.no_graph)
+               for _ in range(len(names) + 1)]
+        ident, bf = tp.TP_ACT_IDENTITY, tp.TP_BF16
+
+        def calls_step(st):
+            evs[0].record(st)
+            tp.tp_layer_norm(X, t["ln1_gamma"], t["ln1_beta"], A, T, d, stream=st)
+            evs[1].record(st)
+            tp.tp_column_linear(A, t["Wq"], None, None, Qs, T, d, h * dh, p, bf, ident, stream=st)
+            tp.tp_column_linear(A, t["Wk"], None, None, Ks, T, d, hkv * dh, p, bf, ident, stream=st)
+            tp.tp_column_linear(A, t["Wv"], None, None, Vs, T, d, hkv * dh, p, bf, ident, stream=st)
+            evs[2].record(st)
+            tp.tp_attention_heads(Qs, Ks, Vs, Os, T, p, h, hkv, dh, causal, stream=st)
+            evs[3].record(st)
+            tp.tp_row_linear(Os, t["Wo"], Ps, T, h * dh, d, p, bf, stream=st)
+            evs[4].record(st)
+            tp.tp_reduce_partials_residual(Ps, t["bo"], X, Hs, T, d, p, stream=st)
+            evs[5].record(st)
+            tp.tp_layer_norm(Hs, t["ln2_gamma"], t["ln2_beta"], A, T, d, stream=st)
+            evs[6].record(st)
+            tp.tp_column_linear(A, t["W1"], t["W_up"], t["b1"], Ys, T, d, k, p, bf, act, stream=st)
+            evs[7].record(st)
+            tp.tp_row_linear(Ys, t["W2"], Ps, T, k, d, p, bf, stream=st)
+            evs[8].record(st)
+            tp.tp_reduce_partials_residual(Ps, t["b2"], Hs, Zs, T, d, p, stream=st)
+            evs[9].record(st)
+
+        parts, _, _ = H.time_steps(calls_step, events=evs)
+        means = reduce_max([statistics.mean(col) for col in zip(*parts)], grp, device)
+        af = w.attn().flops()
+        mlp_col = 2 * T * d * k * (2 if w.act == "swiglu" else 1)
+        flops_of = {"qkv": af["qkv"], "attention": af["attention"], "out_proj": af["out"],
+                    "mlp_column": mlp_col, "mlp_row": 2 * T * k * d}
+        bytes_of = {"ln1": T * d * 6, "ln2": T * d * 6, "fold1": (p + 2) * T * d * 4,
+                    "fold2": (p + 2) * T * d * 4}
+        breakdown = {"how": "the public calls one after another as one graph, external timing "
+                            "events between them (unfused: the block fuses fold1 with ln2)"}
+        for name, ms in zip(names, means):
+            ent = {"ms": ms}
+            if name in flops_of:
+                ent["TFLOP/s"] = flops_of[name] / (ms * 1e-3) / 1e12
+                ent["frac_bf16_peak"] = ent["TFLOP/s"] / peaks["bf16_tflops"]
+            else:
+                ent["GB/s"] = bytes_of[name] / (ms * 1e-3) / 1e9
+                ent["frac_hbm"] = ent["GB/s"] / peaks["hbm_gbs"]
+            breakdown[name] = ent
+        breakdown["sum_ms"] = sum(means)
+
+    e2e = None
+    if not a.no_e2e:
+        Xh = X.cpu().pin_memory()
+        Oh = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        Xd = torch.empty_like(X)
+
+        def e2e_step(st):
+            Xd.copy_(Xh, non_blocking=True)
+            tp.tp_transformer_block(Xd, prm, out, ws, nbytes, T, d, h, hkv, dh, k, p, act, causal,
+                                    stream=st)
+            Oh.copy_(out, non_blocking=True)
+
+        t_e2e, _, _ = H.time_steps(e2e_step, graph=False)
+        e_ms = reduce_max([statistics.mean(t_e2e)], grp, device)[0]
+        e2e = {"value": whole_job_value(fl["total"], world, e_ms) / 1e12, "unit": UNIT,
+               "ms_per_step": e_ms, "h2d_bytes_per_step": Xh.numel() * Xh.element_size(),
+               "d2h_bytes_per_step": Oh.numel() * Oh.element_size(),
+               "call": "tp_transformer_block, X host->device and out device->host inside the "
+                       "timed step"}
+
+    value = whole_job_value(fl["total"], world, ms_step) / 1e12
+    achieved = fl["total"] / (ms_step * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+            "traffic": ncu_traffic(f"{w.name}/block"),
+            "kernel": "tp_transformer_block: LN -> QKV GEMMs -> tc_attn_kernel -> Wo GEMM -> "
+                      "fold+residual+LN -> MLP GEMMs -> fold+residual",
+            "duration": "block step time (graph replay, CUDA events on the launching stream)",
+            "peak_source": f"{peak_src} bf16 dense (burst)", "flops_per_step": fl}
+    line = {
+        "metric": BLOCK_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": dict(block_config(w, world),
+                       launch="eager" if a.no_graph else "cuda-graph replay of tp_transformer_block",
+                       l2="flushed before every step (256 MiB write, outside the timed events)"),
+        "pct_bf16_peak": 100.0 * value / (peaks["bf16_tflops"] * world),
+        "breakdown": breakdown,
+        "roofline": roof,
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "wall_s_timed_region": t_wall,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        rows = block_oracle_rows(w)
+        sec, reps = time_block_oracle(w, inp, rows, min_seconds=10.0, max_reps=1000)
+        line["cpu_baseline"] = {"value": block_flops_prefix(w, rows)["total"] / sec / 1e12,
+                                "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"causal prefix: first {rows} of {w.T} tokens, {reps} "
+                                          "reps, float64"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def backward_flops(w: WL.Workload, T=None) -> int:
+    """GEMM FLOPs of the backward pass: dY = dZ W2^T, dW2 = Y^T dZ, dW1 = X^T dH,
+    dX = dH W1^T (SwiGLU: dW_up and dU W_up^T as well), 2*T*d*k each."""
+    T = w.T if T is None else T
+    return 2 * T * w.d * w.k * (6 if w.act == "swiglu" else 4)
+
+
+def backward_inputs(w: WL.Workload, seed: int = 42):
+    """The forward inputs of the workload plus an upstream gradient dZ
+    (bf16, standard normal), drawn after them."""
+    inp = WL.make_inputs(w, seed)
+    rng = np.random.default_rng(seed + 1)
+    dZ = WL.f32_to_bf16_bits(rng.standard_normal((w.T, w.d), dtype=np.float32))
+    return inp, dZ
+
+
+def run_reference_backward(a, w: WL.Workload, rank: int, world: int):
+    if rank != 0:
+        return 0
+    from oracle import tp_oracle as O
+    inp, dZ = backward_inputs(w)
+    rows = int(max(1, min(w.T, 3e10 // (backward_flops(w) / w.T))))
+    X = inp.values("X")[:rows]
+    dz = WL.bf16_bits_to_f32(dZ)[:rows]
+    args = (inp.values("W1"), inp.values("b1"), inp.values("W2"), dz, w.p, w.act)
+
+    def once():
+        t0 = time.perf_counter()
+        O.mlp_backward_sharded(X, *args, W_up=inp.values("W_up"))
+        return time.perf_counter() - t0
+
+    for _ in range(a.warmup):
+        once()
+    ms = 1e3 * statistics.mean(once() for _ in range(a.steps))
+    value = backward_flops(w, rows) / (ms * 1e-3) / 1e12
+    line = {
+        "impl": "reference", "metric": BWD_METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": a.steps, "warmup": a.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "mode": "backward", "T": w.T, "d": w.d, "k": w.k, "p": w.p,
+                   "act": w.act, "sample_rows": rows,
+                   "parallelism": f"replicas{world}" if world > 1 else "single"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"first {rows} of {w.T} token rows per step, full weights"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_tp_backward(a, w: WL.Workload, rank: int, world: int, local_rank: int):
+    import torch
+    import torch.distributed as dist
+    import megatron_tensor_sharded_b200 as tp
+
+    if w.dtype != "bf16":
+        raise SystemExit("the backward pass is provided for the bf16 workloads")
+    torch.cuda.set_device(local_rank)
+    device = torch.device("cuda", local_rank)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=device)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    grp = dist if world > 1 else None
+    H = Harness(a, torch, tp, device, barrier)
+    inp, dZh = backward_inputs(w)
+
+    def dev(x):
+        if x is None:
+            return None
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
+        return torch.from_numpy(x).to(device)
+
+    T, d, k, p = w.T, w.d, w.k, w.p
+    act, bf = tp.ACT[w.act], tp.TP_BF16
+    X, W1, Wu, b1, W2 = dev(inp.X), dev(inp.W1), dev(inp.W_up), dev(inp.b1), dev(inp.W2)
+    dZ = dev(dZh)
+    sh = (p, T, k // p)
+    Hp = torch.empty(sh, dtype=torch.bfloat16, device=device)
+    Hu = torch.empty(sh, dtype=torch.bfloat16, device=device) if w.act == "swiglu" else None
+    Y = torch.empty(sh, dtype=torch.bfloat16, device=device)
+    ident = tp.TP_ACT_IDENTITY
+    tp.tp_column_linear(X, W1, None, b1, Hp, T, d, k, p, bf, ident)
+    if Hu is not None:
+        tp.tp_column_linear(X, Wu, None, None, Hu, T, d, k, p, bf, ident)
+    tp.tp_column_linear(X, W1, Wu, b1, Y, T, d, k, p, bf, act)
+    f32 = dict(dtype=torch.float32, device=device)
+    dX, dW1, db1 = torch.empty((T, d), **f32), torch.empty((d, k), **f32), torch.empty(k, **f32)
+    dWu = torch.empty((d, k), **f32) if Hu is not None else None
+    dW2, db2 = torch.empty((k, d), **f32), torch.empty(d, **f32)
+    nbytes = tp.tp_mlp_block_backward_workspace_size(T, d, k, p, act)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+
+    def step(st, dz=dZ):
+        tp.tp_mlp_block_backward(X, W1, Wu, W2, Hp, Hu, Y, dz, dX, dW1, dWu, db1, dW2, db2, ws,
+                                 nbytes, T, d, k, p, act, stream=st)
+
+    with ClockSampler(local_rank) as clocks:
+        step_ms, launches, t_wall = H.time_steps(step)
+    ms_step, launches = reduce_max([statistics.mean(step_ms), float(launches)], grp, device)
+    fl = backward_flops(w)
+    peaks, peak_src = load_peaks()
+
+    e2e = None
+    if not a.no_e2e:
+        dZpin = dZ.cpu().pin_memory()
+        dXh = torch.empty((T, d), dtype=torch.float32).pin_memory()
+        dZd = torch.empty_like(dZ)
+
+        def e2e_step(st):
+            dZd.copy_(dZpin, non_blocking=True)
+            step(st, dZd)
+            dXh.copy_(dX, non_blocking=True)
+
+        t_e2e, _, _ = H.time_steps(e2e_step, graph=False)
+        e_ms = reduce_max([statistics.mean(t_e2e)], grp, device)[0]
+        e2e = {"value": whole_job_value(fl, world, e_ms) / 1e12, "unit": UNIT, "ms_per_step": e_ms,
+               "h2d_bytes_per_step": dZpin.numel() * dZpin.element_size(),
+               "d2h_bytes_per_step": dXh.numel() * dXh.element_size(),
+               "call": "tp_mlp_block_backward, dZ host->device and dX device->host inside the "
+                       "timed step (weight gradients stay on the device)"}
+
+    value = whole_job_value(fl, world, ms_step) / 1e12
+    achieved = fl / (ms_step * 1e-3) / 1e12
+    roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
+            "traffic": ncu_traffic(f"{w.name}/backward"),
+            "kernel": "tp_mlp_block_backward: dH GEMM (act' epilogue) -> dW2, dW1 GEMMs -> "
+                      "bias-gradient column sums -> dX partial GEMM -> fold",
+            "duration": "backward step time (graph replay, CUDA events on the launching stream)",
+            "peak_source": f"{peak_src} bf16 dense (burst)"}
+    line = {
+        "metric": BWD_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
+        "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "mode": "backward", "T": T, "d": d, "k": k, "p": p,
+                   "act": w.act, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "launch": "eager" if a.no_graph else "cuda-graph replay of tp_mlp_block_backward",
+                   "l2": "flushed before every step (256 MiB write, outside the timed events)"},
+        "pct_bf16_peak": 100.0 * value / (peaks["bf16_tflops"] * world),
+        "roofline": roof,
+        "gpu_launches": int(launches),
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+        "wall_s_timed_region": t_wall,
+    }
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        from oracle import tp_oracle as O
+        rows = int(max(1, min(T, 3e10 // (fl / T))))
+        Xs = inp.values("X")[:rows]
+        dzs = WL.bf16_bits_to_f32(dZh)[:rows]
+        reps, t0 = 0, time.perf_counter()
+        while time.perf_counter() - t0 < 10.0 and reps < 1000:
+            O.mlp_backward_sharded(Xs, inp.values("W1"), inp.values("b1"), inp.values("W2"), dzs,
+                                   p, w.act, W_up=inp.values("W_up"))
+            reps += 1
+        sec = (time.perf_counter() - t0) / reps
+        line["cpu_baseline"] = {"value": backward_flops(w, rows) / sec / 1e12, "unit": UNIT,
+                                "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"first {rows} of {T} token rows, {reps} reps, float64"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tp", "reference"], default="tp")
-    ap.add_argument("--workload", choices=sorted(WL.WORKLOADS), default="gpt2")
-    ap.add_argument("--mode", choices=["partials", "splitk", "fused"], default="partials")
+    ap.add_argument("--workload", choices=sorted(WL.WORKLOADS) + sorted(WL.ATTN_WORKLOADS)
+                    + sorted(WL.BLOCK_WORKLOADS), default="gpt2")
+    ap.add_argument("--mode", choices=["partials", "splitk", "fused", "backward"],
+                    default="partials")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of graph replay")
     ap.add_argument("--no-breakdown", action="store_true", help="skip the per-kernel loop")
@@ -509,7 +1251,21 @@ def main(argv=None):
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if world != a.gpus:
         ap.error(f"--gpus {a.gpus} but WORLD_SIZE={world}")
+    if a.workload in WL.BLOCK_WORKLOADS:
+        w = WL.BLOCK_WORKLOADS[a.workload]
+        if a.impl == "reference":
+            return run_reference_block(a, w, rank, world)
+        return run_tp_block(a, w, rank, world, local_rank)
+    if a.workload in WL.ATTN_WORKLOADS:
+        w = WL.ATTN_WORKLOADS[a.workload]
+        if a.impl == "reference":
+            return run_reference_attn(a, w, rank, world)
+        return run_tp_attn(a, w, rank, world, local_rank)
     w = WL.WORKLOADS[a.workload]
+    if a.mode == "backward":
+        if a.impl == "reference":
+            return run_reference_backward(a, w, rank, world)
+        return run_tp_backward(a, w, rank, world, local_rank)
     if a.impl == "reference":
         return run_reference(a, w, rank, world)
     return run_tp(a, w, rank, world, local_rank)

@@ -230,6 +230,111 @@ tp_status tp_attn_block(const void* X, const void* Wq, const void* Wk, const voi
 size_t tp_attn_block_workspace_size(int64_t T, int64_t d, int n_heads, int n_kv_heads,
                                     int head_dim, int p);
 
+/*
+ * LayerNorm of every row ("Building GPT from Scratch -- Part 9",
+ * "Communication Pattern per Transformer Block": LayerNorm, replicated, no
+ * communication): Y = (x - mean) / sqrt(var + eps) * gamma + beta with the
+ * biased variance, computed in fp32, Y rounded to bf16 (the input of the
+ * next block's column-parallel GEMMs).
+ *
+ *   X [T][d] fp32, gamma [d], beta [d] fp32, Y [T][d] bf16 (all 16-byte
+ *   aligned); d % 4 == 0 and d <= 16384 (else TP_ERR_UNSUPPORTED); eps > 0.
+ */
+tp_status tp_layer_norm(const float* X, const float* gamma, const float* beta, void* Y, int64_t T,
+                        int64_t d, float eps, void* stream);
+
+/*
+ * The reduction that ends a transformer sub-block, with the residual
+ * connection folded in: Z = ((P_0 + ... + P_{p-1}) + bias) + residual, each
+ * addition one fp32 round-to-nearest-even operation in that order
+ * (bit-reproducible).  ("Building GPT from Scratch -- Part 9",
+ * "Communication Pattern per Transformer Block": all-reduce after the
+ * output projection / W2, then the element-wise residual add.)
+ *
+ *   partials [p][T][d] fp32, bias [d] fp32 or NULL, residual [T][d] fp32 or
+ *   NULL (may equal Z; no other overlap), Z [T][d] fp32; 16-byte aligned;
+ *   d % 4 == 0 and d <= 16384.
+ */
+tp_status tp_reduce_partials_residual(const float* partials, const float* bias,
+                                      const float* residual, float* Z, int64_t T, int64_t d, int p,
+                                      void* stream);
+
+/* Weights of one transformer block (bf16 matrices [in, out], fp32 vectors;
+ * bo, W_up, b1, b2 may be NULL; W_up is required for TP_ACT_SWIGLU, b1 is bf16
+ * like the column-parallel layer's bias). */
+typedef struct tp_block_params {
+  const float* ln1_gamma;
+  const float* ln1_beta;
+  const void* Wq;   /* [d][n_heads * head_dim]    */
+  const void* Wk;   /* [d][n_kv_heads * head_dim] */
+  const void* Wv;   /* [d][n_kv_heads * head_dim] */
+  const void* Wo;   /* [n_heads * head_dim][d]    */
+  const float* bo;  /* [d]                        */
+  const float* ln2_gamma;
+  const float* ln2_beta;
+  const void* W1;   /* [d][k] (W_gate for SwiGLU) */
+  const void* W_up; /* [d][k]                     */
+  const void* b1;   /* [k] bf16                   */
+  const void* W2;   /* [k][d]                     */
+  const float* b2;  /* [d]                        */
+} tp_block_params;
+
+/*
+ * One pre-norm tensor-parallel transformer block on p simulated shards
+ * ("Building GPT from Scratch -- Part 9", "Communication Pattern per
+ * Transformer Block"; "Tensor parallel math", "Counting all-reduces": two
+ * reductions per layer):
+ *
+ *   H   = X + tp_attn_block(LayerNorm(X; ln1))        (reduction #1 + residual)
+ *   out = H + tp_mlp_block(LayerNorm(H; ln2))          (reduction #2 + residual)
+ *
+ * X, out [T][d] fp32 (out may equal X); every GEMM reads bf16 and
+ * accumulates fp32; head_dim 128; d % 8 == 0 and d <= 16384.  workspace:
+ * tp_transformer_block_workspace_size(...) bytes, 256-byte aligned.
+ */
+tp_status tp_transformer_block(const float* X, const tp_block_params* params, float* out,
+                               void* workspace, size_t workspace_bytes, int64_t T, int64_t d,
+                               int n_heads, int n_kv_heads, int head_dim, int64_t k, int p,
+                               int act, int causal, float eps, void* stream);
+
+/* Workspace bytes tp_transformer_block needs (0 if the arguments are invalid). */
+size_t tp_transformer_block_workspace_size(int64_t T, int64_t d, int n_heads, int n_kv_heads,
+                                           int head_dim, int64_t k, int p);
+
+/*
+ * Backward pass of the MLP block through the f / g conjugate operators
+ * ("Tensor parallel math", "The f and g conjugate operators": f is the
+ * identity forward and an all-reduce backward, g the reverse; "Counting
+ * all-reduces": one all-reduce per block in the backward pass).  g's
+ * identity backward hands every shard the whole dZ; shard i then computes
+ * locally
+ *     dY_i = dZ W2_i^T,  dH_i = dY_i * act'(H_i)   (SwiGLU: dG_i, dU_i),
+ *     dW2_i = Y_i^T dZ,  dW1_i = X^T dH_i,  db1_i = sum_t dH_i,
+ * and f's all-reduce becomes the fixed-order fold of the p full-shape
+ * partials dX = sum_i dH_i W1_i^T (+ dU_i Wup_i^T).  db2 = sum_t dZ.
+ *
+ *   X [T][d], W1 / W_up [d][k], W2 [k][d]   bf16, as in the forward call
+ *   H     [p][T][k/p] bf16 pre-activation X W1_i + b1_i (SwiGLU: the gate),
+ *         e.g. from tp_column_linear with TP_ACT_IDENTITY
+ *   H_up  [p][T][k/p] bf16 up projection X Wup_i (SwiGLU only, else NULL)
+ *   Y     [p][T][k/p] bf16 activation output (tp_column_linear's Y)
+ *   dZ    [T][d] bf16 upstream gradient
+ * Outputs (fp32, each may be NULL to skip it): dX [T][d]; dW1, dW_up
+ * [d][k] (column blocks per shard); db1 [k]; dW2 [k][d] (row blocks);
+ * db2 [d].  workspace: tp_mlp_block_backward_workspace_size(...) bytes,
+ * 256-byte aligned.  k/p must be a multiple of 64 (else
+ * TP_ERR_UNSUPPORTED).  Bias gradients are summed over tokens in a fixed
+ * order (reproducible).
+ */
+tp_status tp_mlp_block_backward(const void* X, const void* W1, const void* W_up, const void* W2,
+                                const void* H, const void* H_up, const void* Y, const void* dZ,
+                                float* dX, float* dW1, float* dW_up, float* db1, float* dW2,
+                                float* db2, void* workspace, size_t workspace_bytes, int64_t T,
+                                int64_t d, int64_t k, int p, int act, void* stream);
+
+/* Workspace bytes tp_mlp_block_backward needs (0 if the arguments are invalid). */
+size_t tp_mlp_block_backward_workspace_size(int64_t T, int64_t d, int64_t k, int p, int act);
+
 /* Synchronise `stream`, then report (and clear) the device status word of
  * the current device: TP_ERR_DEVICE_TIMEOUT if a bounded wait ran out since
  * the last call, TP_ERR_CUDA if the stream reported an error, else TP_OK. */

@@ -21,7 +21,12 @@ __all__ = [
     "TPError", "TP_F32", "TP_BF16", "TP_ACT_GELU_TANH", "TP_ACT_SWIGLU", "TP_ACT_IDENTITY",
     "TP_ACT_RELU", "TP_FLAG_NONE", "TP_FLAG_SPLITK_FUSED", "TP_FLAG_FUSED_LAUNCH", "STATUS", "ACT", "DTYPE",
     "tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
-    "tp_mlp_block_noalloc", "tp_attention_heads", "tp_attn_block", "tp_attn_block_workspace_size",
+    "tp_mlp_block_noalloc", "tp_attention_heads", "tp_attn_block",
+              "tp_layer_norm", "tp_reduce_partials_residual", "tp_transformer_block",
+              "tp_mlp_block_backward", "tp_attn_block_workspace_size",
+    "tp_layer_norm", "tp_reduce_partials_residual", "tp_transformer_block",
+    "tp_transformer_block_workspace_size", "BlockParams", "tp_mlp_block_backward",
+    "tp_mlp_block_backward_workspace_size",
     "tp_mlp_block_workspace_size", "tp_sync_status", "tp_set_wait_timeout_ns",
     "tp_debug_drop_load", "tp_status_string", "tp_last_error_detail",
     "tp_kernel_launch_count", "tp_abi_version", "LIB_PATH",
@@ -47,6 +52,13 @@ class TPError(RuntimeError):
         super().__init__(f"{self.name}: {detail}")
 
 
+class BlockParams(ctypes.Structure):
+    """tp_block_params: device pointers of one transformer block's weights."""
+    _fields_ = [(name, ctypes.c_void_p) for name in (
+        "ln1_gamma", "ln1_beta", "Wq", "Wk", "Wv", "Wo", "bo", "ln2_gamma", "ln2_beta", "W1",
+        "W_up", "b1", "W2", "b2")]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is not built; run "
@@ -65,6 +77,15 @@ def _load() -> ctypes.CDLL:
                                   i32, vp]
     lib.tp_attn_block_workspace_size.argtypes = [i64, i64, i32, i32, i32, i32]
     lib.tp_attn_block_workspace_size.restype = sz
+    lib.tp_layer_norm.argtypes = [vp, vp, vp, vp, i64, i64, ctypes.c_float, vp]
+    lib.tp_reduce_partials_residual.argtypes = [vp, vp, vp, vp, i64, i64, i32, vp]
+    lib.tp_transformer_block.argtypes = [vp, ctypes.POINTER(BlockParams), vp, vp, sz, i64, i64,
+                                         i32, i32, i32, i64, i32, i32, i32, ctypes.c_float, vp]
+    lib.tp_transformer_block_workspace_size.argtypes = [i64, i64, i32, i32, i32, i64, i32]
+    lib.tp_transformer_block_workspace_size.restype = sz
+    lib.tp_mlp_block_backward.argtypes = [vp] * 15 + [sz, i64, i64, i64, i32, i32, vp]
+    lib.tp_mlp_block_backward_workspace_size.argtypes = [i64, i64, i64, i32, i32]
+    lib.tp_mlp_block_backward_workspace_size.restype = sz
     lib.tp_mlp_block_workspace_size.argtypes = [i64, i64, i64, i32, i32, i32, i32]
     lib.tp_mlp_block_workspace_size.restype = sz
     lib.tp_sync_status.argtypes = [vp]
@@ -169,6 +190,54 @@ def tp_attn_block(X, Wq, Wk, Wv, Wo, bo, Z, workspace, workspace_bytes, T, d, n_
 
 def tp_attn_block_workspace_size(T, d, n_heads, n_kv_heads, head_dim, p) -> int:
     return int(_lib.tp_attn_block_workspace_size(T, d, n_heads, n_kv_heads, head_dim, p))
+
+
+def tp_layer_norm(X, gamma, beta, Y, T, d, eps=1e-5, stream=None, check=True):
+    """Y = LayerNorm(X) * gamma + beta per row, fp32 statistics, bf16 Y."""
+    return _check(_lib.tp_layer_norm(_ptr(X), _ptr(gamma), _ptr(beta), _ptr(Y), T, d, eps,
+                                     _stream(stream)), check)
+
+
+def tp_reduce_partials_residual(partials, bias, residual, Z, T, d, p, stream=None, check=True):
+    """Z = ((P_0 + ... + P_{p-1}) + bias) + residual, fixed order, fp32."""
+    return _check(_lib.tp_reduce_partials_residual(_ptr(partials), _ptr(bias), _ptr(residual),
+                                                   _ptr(Z), T, d, p, _stream(stream)), check)
+
+
+def block_params(**tensors) -> BlockParams:
+    """BlockParams from device tensors (or None) named like its fields."""
+    prm = BlockParams()
+    for name, _ in BlockParams._fields_:
+        setattr(prm, name, _ptr(tensors.get(name)))
+    return prm
+
+
+def tp_transformer_block(X, params: BlockParams, out, workspace, workspace_bytes, T, d, n_heads,
+                         n_kv_heads, head_dim, k, p, act, causal=True, eps=1e-5, stream=None,
+                         check=True):
+    """H = X + attn(LN1(X)); out = H + mlp(LN2(H)), both reductions fixed-order."""
+    return _check(_lib.tp_transformer_block(_ptr(X), ctypes.byref(params), _ptr(out),
+                                            _ptr(workspace), workspace_bytes, T, d, n_heads,
+                                            n_kv_heads, head_dim, k, p, act, int(bool(causal)),
+                                            eps, _stream(stream)), check)
+
+
+def tp_transformer_block_workspace_size(T, d, n_heads, n_kv_heads, head_dim, k, p) -> int:
+    return int(_lib.tp_transformer_block_workspace_size(T, d, n_heads, n_kv_heads, head_dim, k, p))
+
+
+def tp_mlp_block_backward(X, W1, W_up, W2, H, H_up, Y, dZ, dX, dW1, dW_up, db1, dW2, db2,
+                          workspace, workspace_bytes, T, d, k, p, act, stream=None, check=True):
+    """Gradients of the MLP block: dX (fold of p partials), dW1, dW_up, db1,
+    dW2, db2 (any output may be None)."""
+    return _check(_lib.tp_mlp_block_backward(
+        _ptr(X), _ptr(W1), _ptr(W_up), _ptr(W2), _ptr(H), _ptr(H_up), _ptr(Y), _ptr(dZ), _ptr(dX),
+        _ptr(dW1), _ptr(dW_up), _ptr(db1), _ptr(dW2), _ptr(db2), _ptr(workspace), workspace_bytes,
+        T, d, k, p, act, _stream(stream)), check)
+
+
+def tp_mlp_block_backward_workspace_size(T, d, k, p, act) -> int:
+    return int(_lib.tp_mlp_block_backward_workspace_size(T, d, k, p, act))
 
 
 def tp_mlp_block_workspace_size(T, d, k, p, dtype, act, flags=TP_FLAG_NONE) -> int:

@@ -222,12 +222,120 @@ tp_status attention_impl(const void* Q, const void* K, const void* V, void* O, i
   return launch_tc_attention(c, Q, K, V, O, T, p, n_heads / p, n_kv_heads / p, causal);
 }
 
+tp_status check_rows(int64_t T, int64_t d) {
+  if (T < 0 || d < 1) return fail(TP_ERR_INVALID_ARG, "sizes T=%lld d=%lld", (long long)T, (long long)d);
+  if (T > INT32_MAX) return fail(TP_ERR_UNSUPPORTED, "T = %lld", (long long)T);
+  if (d % 4 != 0 || d > 16384)
+    return fail(TP_ERR_UNSUPPORTED, "row kernels need d %% 4 == 0 and d <= 16384 (d = %lld)",
+                (long long)d);
+  return TP_OK;
+}
+
+tp_status check_vec16(const void* ptr, const char* name, bool nullable) {
+  if (ptr == nullptr) return nullable ? TP_OK : fail(TP_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(ptr)) return fail(TP_ERR_ALIGNMENT, "%s must be 16-byte aligned", name);
+  return TP_OK;
+}
+
+tp_status layer_norm_impl(const float* X, const float* gamma, const float* beta, void* Y, int64_t T,
+                          int64_t d, float eps, void* stream) {
+  TP_TRY(check_rows(T, d));
+  if (!(eps > 0.0f)) return fail(TP_ERR_INVALID_ARG, "eps must be > 0");
+  if (T == 0) return TP_OK;
+  TP_TRY(check_vec16(X, "X", false));
+  TP_TRY(check_vec16(gamma, "gamma", false));
+  TP_TRY(check_vec16(beta, "beta", false));
+  TP_TRY(check_vec16(Y, "Y", false));
+  LaunchCtx c{};
+  TP_TRY(make_ctx(stream, false, &c));
+  return cuda_status(launch_row_fold_ln(c, nullptr, 0, nullptr, X, nullptr, gamma, beta, Y, T, d, eps),
+                     "layer norm launch");
+}
+
+tp_status fold_residual_impl(const float* P, const float* b, const float* R, float* Z, int64_t T,
+                             int64_t d, int p, const float* gamma, const float* beta, void* Y,
+                             float eps, void* stream) {
+  if (p < 1) return fail(TP_ERR_INVALID_ARG, "p = %d, must be >= 1", p);
+  TP_TRY(check_rows(T, d));
+  if (T == 0) return TP_OK;
+  TP_TRY(check_vec16(P, "partials", false));
+  TP_TRY(check_vec16(b, "bias", true));
+  TP_TRY(check_vec16(R, "residual", true));
+  TP_TRY(check_vec16(Z, "Z", false));
+  const uintptr_t p0 = reinterpret_cast<uintptr_t>(P);
+  const uintptr_t p1 = p0 + static_cast<uintptr_t>(p) * T * d * 4;
+  const uintptr_t z0 = reinterpret_cast<uintptr_t>(Z);
+  const uintptr_t z1 = z0 + static_cast<uintptr_t>(T) * d * 4;
+  if (z0 < p1 && p0 < z1) return fail(TP_ERR_INVALID_ARG, "Z overlaps the partials");
+  if (R != nullptr && R != Z) {
+    const uintptr_t r0 = reinterpret_cast<uintptr_t>(R);
+    const uintptr_t r1 = r0 + static_cast<uintptr_t>(T) * d * 4;
+    if (z0 < r1 && r0 < z1) return fail(TP_ERR_INVALID_ARG, "Z partly overlaps the residual");
+  }
+  LaunchCtx c{};
+  TP_TRY(make_ctx(stream, false, &c));
+  return cuda_status(launch_row_fold_ln(c, P, p, b, R, Z, gamma, beta, Y, T, d, eps),
+                     "fold launch");
+}
+
 size_t attn_workspace_bytes(int64_t T, int64_t d, int n_heads, int n_kv_heads, int head_dim, int p) {
   const size_t q = align256(static_cast<size_t>(T) * n_heads * head_dim * 2);
   const size_t kv = align256(static_cast<size_t>(T) * n_kv_heads * head_dim * 2);
   const size_t part = align256(static_cast<size_t>(p) * T * d * 4);
   return 2 * q + 2 * kv + part;
 }
+
+struct BwdLayout {
+  size_t dh, du, part, scratch, total;
+};
+
+BwdLayout bwd_layout(int64_t T, int64_t d, int64_t k, int p, bool swiglu) {
+  BwdLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align256(bytes);
+    return at;
+  };
+  const size_t t = static_cast<size_t>(T);
+  const size_t chunks = (t + 127) / 128;
+  const size_t s = static_cast<size_t>(k / p);
+  L.dh = take(t * k * 2);
+  L.du = swiglu ? take(t * k * 2) : 0;
+  L.part = take(static_cast<size_t>(p) * t * d * 4);
+  const size_t sc = chunks * (static_cast<size_t>(p) * s > static_cast<size_t>(d)
+                                  ? static_cast<size_t>(p) * s : static_cast<size_t>(d));
+  L.scratch = take(sc * 4);
+  L.total = off;
+  return L;
+}
+
+struct BlockLayout {
+  size_t a, h, q, k, v, o, y, p, total;
+};
+
+BlockLayout block_layout(int64_t T, int64_t d, int n_heads, int n_kv_heads, int head_dim,
+                         int64_t k, int p) {
+  BlockLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align256(bytes);
+    return at;
+  };
+  const size_t t = static_cast<size_t>(T);
+  L.a = take(t * d * 2);
+  L.h = take(t * d * 4);
+  L.q = take(t * n_heads * head_dim * 2);
+  L.k = take(t * n_kv_heads * head_dim * 2);
+  L.v = take(t * n_kv_heads * head_dim * 2);
+  L.o = take(t * n_heads * head_dim * 2);
+  L.y = take(t * k * 2);
+  L.p = take(static_cast<size_t>(p) * t * d * 4);
+  L.total = off;
+  return L;
+}
+
 
 }  // namespace
 
@@ -382,6 +490,143 @@ tp_status tp_attn_block(const void* X, const void* Wq, const void* Wk, const voi
   TP_TRY(attention_impl(Q, K, V, O, T, p, n_heads, n_kv_heads, head_dim, causal, stream));
   TP_TRY(row_impl(O, Wo, P, T, kq, d, p, TP_BF16, stream));
   return reduce_impl(P, bo, Z, T, d, p, stream);
+}
+
+tp_status tp_layer_norm(const float* X, const float* gamma, const float* beta, void* Y, int64_t T,
+                        int64_t d, float eps, void* stream) {
+  g_detail[0] = 0;
+  return layer_norm_impl(X, gamma, beta, Y, T, d, eps, stream);
+}
+
+tp_status tp_reduce_partials_residual(const float* partials, const float* bias,
+                                      const float* residual, float* Z, int64_t T, int64_t d, int p,
+                                      void* stream) {
+  g_detail[0] = 0;
+  return fold_residual_impl(partials, bias, residual, Z, T, d, p, nullptr, nullptr, nullptr, 1e-5f,
+                            stream);
+}
+
+
+size_t tp_transformer_block_workspace_size(int64_t T, int64_t d, int n_heads, int n_kv_heads,
+                                           int head_dim, int64_t k, int p) {
+  if (check_heads(p, n_heads, n_kv_heads, head_dim) != TP_OK || T < 0 || d < 1 || k < 1) return 0;
+  return block_layout(T, d, n_heads, n_kv_heads, head_dim, k, p).total;
+}
+
+tp_status tp_transformer_block(const float* X, const tp_block_params* prm, float* out,
+                               void* workspace, size_t workspace_bytes, int64_t T, int64_t d,
+                               int n_heads, int n_kv_heads, int head_dim, int64_t k, int p, int act,
+                               int causal, float eps, void* stream) {
+  g_detail[0] = 0;
+  if (prm == nullptr) return fail(TP_ERR_INVALID_ARG, "params is NULL");
+  TP_TRY(check_heads(p, n_heads, n_kv_heads, head_dim));
+  TP_TRY(check_rows(T, d));
+  TP_TRY(check_shape(T, d, k, p, TP_BF16));
+  TP_TRY(check_act(act, prm->W_up));
+  if (!(eps > 0.0f)) return fail(TP_ERR_INVALID_ARG, "eps must be > 0");
+  if (T == 0) return TP_OK;
+  TP_TRY(check_vec16(X, "X", false));
+  TP_TRY(check_vec16(out, "out", false));
+  TP_TRY(check_vec16(prm->ln1_gamma, "ln1_gamma", false));
+  TP_TRY(check_vec16(prm->ln1_beta, "ln1_beta", false));
+  TP_TRY(check_vec16(prm->ln2_gamma, "ln2_gamma", false));
+  TP_TRY(check_vec16(prm->ln2_beta, "ln2_beta", false));
+  TP_TRY(check_vec16(prm->bo, "bo", true));
+  TP_TRY(check_vec16(prm->b2, "b2", true));
+  const BlockLayout L = block_layout(T, d, n_heads, n_kv_heads, head_dim, k, p);
+  if (workspace == nullptr || workspace_bytes < L.total)
+    return fail(TP_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", L.total,
+                workspace == nullptr ? size_t(0) : workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(TP_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* A = ws + L.a;                       // LN1(X), later LN2(H): bf16 [T][d]
+  float* H = reinterpret_cast<float*>(ws + L.h);
+  void* Q = ws + L.q;
+  void* K = ws + L.k;
+  void* V = ws + L.v;
+  void* O = ws + L.o;
+  void* Yh = ws + L.y;
+  float* P = reinterpret_cast<float*>(ws + L.p);
+  const int64_t kq = static_cast<int64_t>(n_heads) * head_dim;
+  const int64_t kkv = static_cast<int64_t>(n_kv_heads) * head_dim;
+  const int ident = TP_ACT_IDENTITY;
+  // LayerNorm -> attention (column Q, K, V by heads; local attention; row Wo)
+  TP_TRY(layer_norm_impl(X, prm->ln1_gamma, prm->ln1_beta, A, T, d, eps, stream));
+  TP_TRY(column_impl(A, prm->Wq, nullptr, nullptr, Q, T, d, kq, p, TP_BF16, ident, stream));
+  TP_TRY(column_impl(A, prm->Wk, nullptr, nullptr, K, T, d, kkv, p, TP_BF16, ident, stream));
+  TP_TRY(column_impl(A, prm->Wv, nullptr, nullptr, V, T, d, kkv, p, TP_BF16, ident, stream));
+  TP_TRY(attention_impl(Q, K, V, O, T, p, n_heads, n_kv_heads, head_dim, causal, stream));
+  TP_TRY(row_impl(O, prm->Wo, P, T, kq, d, p, TP_BF16, stream));
+  // reduction #1 with the residual: H = X + fold + bo; then LayerNorm of H
+  TP_TRY(fold_residual_impl(P, prm->bo, X, H, T, d, p, prm->ln2_gamma, prm->ln2_beta, A, eps,
+                            stream));
+  // MLP: column W1 (+ activation), row W2
+  TP_TRY(column_impl(A, prm->W1, prm->W_up, prm->b1, Yh, T, d, k, p, TP_BF16, act, stream));
+  TP_TRY(row_impl(Yh, prm->W2, P, T, k, d, p, TP_BF16, stream));
+  // reduction #2 with the residual: out = H + fold + b2
+  return fold_residual_impl(P, prm->b2, H, out, T, d, p, nullptr, nullptr, nullptr, eps, stream);
+}
+
+size_t tp_mlp_block_backward_workspace_size(int64_t T, int64_t d, int64_t k, int p, int act) {
+  if (p < 1 || T < 0 || d < 1 || k < 1 || k % p != 0) return 0;
+  return bwd_layout(T, d, k, p, act == TP_ACT_SWIGLU).total;
+}
+
+tp_status tp_mlp_block_backward(const void* X, const void* W1, const void* W_up, const void* W2,
+                                const void* H, const void* H_up, const void* Y, const void* dZ,
+                                float* dX, float* dW1, float* dW_up, float* db1, float* dW2,
+                                float* db2, void* workspace, size_t workspace_bytes, int64_t T,
+                                int64_t d, int64_t k, int p, int act, void* stream) {
+  g_detail[0] = 0;
+  TP_TRY(check_shape(T, d, k, p, TP_BF16));
+  const bool swiglu = act == TP_ACT_SWIGLU;
+  TP_TRY(check_act(act, W_up));
+  if ((k / p) % 64 != 0)
+    return fail(TP_ERR_UNSUPPORTED, "backward needs k/p %% 64 == 0 (k/p = %lld)",
+                (long long)(k / p));
+  if (T > 65535LL * 128) return fail(TP_ERR_UNSUPPORTED, "T = %lld", (long long)T);
+  if (T == 0) return TP_OK;
+  for (const void* ptr : {X, W1, W2, H, Y, dZ})
+    if (ptr == nullptr || !aligned16(ptr))
+      return fail(ptr == nullptr ? TP_ERR_INVALID_ARG : TP_ERR_ALIGNMENT,
+                  "X, W1, W2, H, Y, dZ must be non-NULL and 16-byte aligned");
+  if (swiglu && (H_up == nullptr || !aligned16(H_up) || !aligned16(W_up)))
+    return fail(TP_ERR_INVALID_ARG, "SwiGLU needs W_up and H_up (16-byte aligned)");
+  for (const float* ptr : {dX, dW1, dW_up, db1, dW2, db2})
+    if (ptr != nullptr && !aligned16(ptr))
+      return fail(TP_ERR_ALIGNMENT, "gradient outputs must be 16-byte aligned");
+  const BwdLayout L = bwd_layout(T, d, k, p, swiglu);
+  if (workspace == nullptr || workspace_bytes < L.total)
+    return fail(TP_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", L.total,
+                workspace == nullptr ? size_t(0) : workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(TP_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  void* dH = ws + L.dh;
+  void* dU = swiglu ? ws + L.du : nullptr;
+  float* part = reinterpret_cast<float*>(ws + L.part);
+  float* scratch = reinterpret_cast<float*>(ws + L.scratch);
+  const int64_t s = k / p;
+  LaunchCtx c{};
+  TP_TRY(make_ctx(stream, true, &c));
+  // g backward (identity): every shard uses the whole dZ
+  TP_TRY(launch_bwd_act_grad(c, dZ, W2, H, H_up, dH, dU, T, d, k, p, act));
+  c.debug_drop = -1;   // an armed fault injection applies to the first launch only
+  if (dW2 != nullptr) TP_TRY(launch_bwd_dw2(c, Y, dZ, dW2, T, d, k, p));
+  if (dW1 != nullptr) TP_TRY(launch_bwd_dw1(c, X, dH, dU, dW1, swiglu ? dW_up : nullptr, T, d, k, p));
+  if (swiglu && dW1 == nullptr && dW_up != nullptr)
+    return fail(TP_ERR_INVALID_ARG, "dW_up without dW1 is not provided");
+  if (db1 != nullptr)
+    TP_TRY(cuda_status(launch_colsum(c, dH, db1, scratch, p, T, s, s), "bias gradient launch"));
+  if (db2 != nullptr)
+    TP_TRY(cuda_status(launch_colsum(c, dZ, db2, scratch, 1, T, d, d), "bias gradient launch"));
+  if (dX != nullptr) {
+    // f backward (all-reduce): p input-gradient partials, folded in shard order
+    TP_TRY(launch_bwd_dx_partials(c, dH, dU, W1, W_up, part, T, d, k, p));
+    TP_TRY(cuda_status(launch_reduce(c, part, nullptr, dX, T, d, p), "fold launch"));
+  }
+  return TP_OK;
 }
 
 tp_status tp_sync_status(void* stream) {

@@ -43,6 +43,25 @@ __device__ __forceinline__ float act_unary_mufu(int act, float h) {
   return h;
 }
 
+// Derivatives for the backward pass (results are stored as bf16).
+// d/dh GELU_tanh = 0.5 (1 + tanh u) + 0.5 h (1 - tanh^2 u) u', u = c (h + 0.044715 h^3).
+__device__ __forceinline__ float gelu_tanh_grad_mufu(float h) {
+  const float kSqrt2OverPi = 0.7978845608028654f;
+  const float h2 = h * h;
+  const float t = tanh_mufu(kSqrt2OverPi * (h + 0.044715f * h2 * h));
+  const float du = kSqrt2OverPi * (1.0f + 3.0f * 0.044715f * h2);
+  return 0.5f * (1.0f + t) + 0.5f * h * (1.0f - t * t) * du;
+}
+
+// sigmoid(h) = (1 + tanh(h / 2)) / 2; d/dh SiLU = sigmoid (1 + h (1 - sigmoid)).
+__device__ __forceinline__ float sigmoid_mufu(float h) { return 0.5f + 0.5f * tanh_mufu(0.5f * h); }
+
+__device__ __forceinline__ float act_grad_unary_mufu(int act, float h) {
+  if (act == kActGeluTanh) return gelu_tanh_grad_mufu(h);
+  if (act == kActRelu) return h > 0.0f ? 1.0f : 0.0f;
+  return 1.0f;
+}
+
 // Single-input activations (GELU / identity / ReLU).
 __device__ __forceinline__ float act_unary(int act, float h) {
   if (act == kActGeluTanh) return gelu_tanh_f32(h);

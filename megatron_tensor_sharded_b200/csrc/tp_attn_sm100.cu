@@ -7,24 +7,30 @@
 // math", "Attention: parallel across heads": softmax(Q K^T / sqrt(d_k)) V per
 // head).  This kernel computes it for all shards and heads at once.
 //
-// Work unit: (shard, query head, block of 128 queries); key/value blocks of
-// 128.  Roles (256 threads):
-//   warp 0 lane 0  TMA: the unit's Q tile [128 x 128] once, then K_j, V_j per
-//                  key block through a 2-slot ring (128-byte swizzle);
-//   warp 1 lane 0  MMA: S_j = Q K_j^T into one of two TMEM score buffers
-//                  (128 x 128 fp32), O += P_j V_j into a TMEM accumulator;
-//                  S_{j+1} is issued before O += P_j V_j so the tensor core
-//                  works while the softmax of block j runs;
+// Work unit: (shard, query head, pair of 128-query tiles); the two tiles share
+// every K/V block load.  Key/value blocks of 128.  Roles (384 threads):
+//   warp 0 lane 0  TMA: the unit's two Q tiles once, then K_j and V_j per key
+//                  block through a 2-slot ring (128-byte swizzle);
+//   warp 1 lane 0  MMA: S_t = Q_t K_j^T into tile t's TMEM score buffer
+//                  (128 x 128 fp32); O_t += P_t V_j with P_t read from TMEM,
+//                  where the softmax left it (bf16, over the first 64 columns
+//                  of the score buffer).  Issue order per block:
+//                  PV_0 -> S_0(next) -> PV_1 -> S_1(next), so the tensor core
+//                  runs one tile's products while the other tile's softmax
+//                  runs;
 //   warp 2         TMEM allocation;
-//   warps 4..7     online softmax: thread = query row (its TMEM lane), so
-//                  the row maximum and sum never leave the thread; scores
-//                  in the log2 domain with ex2.approx; when the row maximum
-//                  grows, the thread rescales its O row in TMEM before the
-//                  next O += P V; P is written as bf16 into shared memory in
-//                  the MMA's K-major 128-byte-swizzled layout; at the end O
-//                  is divided by the row sum, converted to bf16 and stored.
-// Keys beyond T and (causal) keys after the query are masked.  Every
-// barrier wait is bounded.
+//   warps 4..7     online softmax of tile 0, warps 8..11 of tile 1: thread =
+//                  query row (its TMEM lane); scores in the log2 domain with
+//                  ex2.approx.  The running maximum is only moved when it grows
+//                  by more than 2^8 (the stale maximum is exact once the sum
+//                  and O share it), so O is rarely rescaled; when it is, the
+//                  thread scales its O row in TMEM -- safe without a wait,
+//                  because the score block it just read was committed after
+//                  the previous O += P V.  At the end O is divided by the row
+//                  sum, converted to bf16 and stored.
+// Keys beyond T and (causal) keys after the query are masked, on the blocks
+// that hold any.  Causal units are taken longest first.  Every barrier wait
+// is bounded.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -42,20 +48,22 @@ namespace tpk {
 namespace {
 
 constexpr int DH = 128;                 // head dimension
-constexpr int BQ = 128;                 // queries per unit (TMEM lanes)
+constexpr int BQ = 128;                 // queries per tile (TMEM lanes)
 constexpr int BKV = 128;                // keys per block
+constexpr int NQT = 2;                  // query tiles per unit
 constexpr int NST = 2;                  // K/V ring slots
 constexpr int TILE_BYTES = 128 * 128 * 2;   // one 128 x 128 bf16 tile (two 64-column boxes)
 constexpr int HALF_BYTES = TILE_BYTES / 2;  // one box: 128 rows x 64 columns
-constexpr int SMEM_BYTES = 1024 + 2 * TILE_BYTES /* Q, P */ + NST * 2 * TILE_BYTES /* K, V */ + 256;
-constexpr int NUM_THREADS = 256;
+constexpr int SMEM_BYTES = 1024 + NQT * TILE_BYTES + NST * 2 * TILE_BYTES + 256;
+constexpr int NUM_THREADS = 384;
 constexpr uint32_t IDESC_S = idesc_bf16_f32(BQ, BKV, /*a_mn=*/0, /*b_mn=*/0);  // Q K^T
 constexpr uint32_t IDESC_O = idesc_bf16_f32(BQ, DH, /*a_mn=*/0, /*b_mn=*/1);   // P V
-constexpr uint32_t S_COL0 = 0, O_COL = 2 * BKV, TMEM_COLS = 512;
+constexpr uint32_t O_COL0 = NQT * BKV, TMEM_COLS = 512;   // S_t at t*128, O_t at 256 + t*128
+constexpr float RESCALE_LOG2 = 8.0f;    // move the running maximum only past this growth
 constexpr unsigned kErrWaitAttn = 1u << 6;
 
 struct AttnParams {
-  int32_t T, p, hq, hkv, group, q_blocks, num_units, causal;
+  int32_t T, p, hq, hkv, group, q_blocks, q_pairs, num_units, causal;
   float scale_log2;          // log2(e) / sqrt(DH)
   __nv_bfloat16* O;          // [p][T][hq*DH]
   WaitCtl wait;
@@ -63,18 +71,29 @@ struct AttnParams {
 };
 
 struct Unit {
-  int32_t shard, head, qb, kvh, nkb;
+  int32_t shard, head, kvh, qb0, nkb0, nkb1, nmax;
+  // key blocks of query tile t (0 when the tile lies beyond T)
+  __device__ __forceinline__ int32_t nkb(int t) const { return t == 0 ? nkb0 : nkb1; }
 };
 
 __device__ __forceinline__ Unit decode_unit(const AttnParams& P, int32_t u) {
   Unit x;
-  x.qb = u % P.q_blocks;          // query blocks fastest: neighbours share K, V
-  const int32_t r = u / P.q_blocks;
-  x.head = r % P.hq;
-  x.shard = r / P.hq;
+  const int32_t heads = P.p * P.hq;
+  const int32_t level = u / heads;
+  const int32_t hh = u % heads;
+  // causal: the longest query pairs first
+  const int32_t qp = P.causal ? P.q_pairs - 1 - level : level;
+  x.shard = hh / P.hq;
+  x.head = hh % P.hq;
   x.kvh = x.head / P.group;
+  x.qb0 = qp * NQT;
   const int32_t all = (P.T + BKV - 1) / BKV;
-  x.nkb = P.causal ? (x.qb + 1 < all ? x.qb + 1 : all) : all;
+  auto blocks = [&](int32_t qb) {
+    return qb >= P.q_blocks ? 0 : (P.causal ? (qb + 1 < all ? qb + 1 : all) : all);
+  };
+  x.nkb0 = blocks(x.qb0);
+  x.nkb1 = blocks(x.qb0 + 1);
+  x.nmax = x.nkb0 > x.nkb1 ? x.nkb0 : x.nkb1;   // causal: tile 1 never has fewer
   return x;
 }
 
@@ -91,29 +110,83 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return u;
 }
 
+// One softmax step of a thread's row over a 128-key block already in TMEM
+// columns [tS, tS+128): returns the block's probabilities' sum and leaves
+// the probabilities (bf16 pairs) in columns [tS, tS+64).  MASK: apply the
+// key < T and causal (key <= q) masks.
+template <bool MASK>
+__device__ __forceinline__ float softmax_block(uint32_t tS, float scale, float m_use, int32_t key0,
+                                               int32_t T, int32_t causal, int32_t q, float& mx_out,
+                                               bool max_only) {
+  if (max_only) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < BKV / 32; ++c) {
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tS + c * 32, v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) {
+        float xv = __uint_as_float(v[e]);
+        if (MASK) {
+          const int32_t key = key0 + c * 32 + e;
+          if (key >= T || (causal && key > q)) xv = -INFINITY;
+        }
+        mx = fmaxf(mx, xv);
+      }
+    }
+    mx_out = mx;
+    return 0.0f;
+  }
+  float sum = 0.0f;
+  const float neg = -m_use;
+  // chunk c: scores of columns [32c, 32c+32) -> probabilities in columns
+  // [16c, 16c+16), all of which were read by this or an earlier chunk
+#pragma unroll
+  for (int c = 0; c < BKV / 32; ++c) {
+    uint32_t v[32], pk[16];
+    tmem_ld_32x32b_x32(tS + c * 32, v);
+    tmem_ld_wait();
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      float a0 = ex2(fmaf(__uint_as_float(v[e]), scale, neg));
+      float a1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale, neg));
+      if (MASK) {
+        const int32_t k = key0 + c * 32 + e;
+        if (k >= T || (causal && k > q)) a0 = 0.0f;
+        if (k + 1 >= T || (causal && k + 1 > q)) a1 = 0.0f;
+      }
+      sum += a0 + a1;
+      pk[e / 2] = pack2(a0, a1);
+    }
+    tmem_st_32x32b_x16(tS + c * 16, pk);
+  }
+  tmem_st_wait();
+  return sum;
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_attn_kernel(const __grid_constant__ CUtensorMap mapQ, const __grid_constant__ CUtensorMap mapK,
                    const __grid_constant__ CUtensorMap mapV, const AttnParams P) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  const uint32_t sQ = base, sP = base + TILE_BYTES;
-  auto sK = [&](uint32_t st) { return base + 2 * TILE_BYTES + st * 2 * TILE_BYTES; };
-  auto sV = [&](uint32_t st) { return base + 2 * TILE_BYTES + st * 2 * TILE_BYTES + TILE_BYTES; };
-  uint8_t* const ctrl = smem_raw + (base - raw) + 2 * TILE_BYTES + NST * 2 * TILE_BYTES;
-  uint8_t* const sP_ptr = smem_raw + (base - raw) + TILE_BYTES;
+  auto sQ = [&](uint32_t t) { return base + t * TILE_BYTES; };
+  auto sK = [&](uint32_t st) { return base + NQT * TILE_BYTES + st * 2 * TILE_BYTES; };
+  auto sV = [&](uint32_t st) { return base + NQT * TILE_BYTES + st * 2 * TILE_BYTES + TILE_BYTES; };
+  uint8_t* const ctrl = smem_raw + (base - raw) + NQT * TILE_BYTES + NST * 2 * TILE_BYTES;
   uint64_t* const bars = reinterpret_cast<uint64_t*>(ctrl);
   // barrier slots
   const uint32_t q_full = smem_u32(&bars[0]), q_empty = smem_u32(&bars[1]);
   auto kv_full = [&](uint32_t s) { return smem_u32(&bars[2 + s]); };
   auto kv_empty = [&](uint32_t s) { return smem_u32(&bars[2 + NST + s]); };
-  auto s_full = [&](uint32_t b) { return smem_u32(&bars[2 + 2 * NST + b]); };
-  auto s_empty = [&](uint32_t b) { return smem_u32(&bars[4 + 2 * NST + b]); };
-  const uint32_t p_full = smem_u32(&bars[6 + 2 * NST]);
-  const uint32_t o_done = smem_u32(&bars[7 + 2 * NST]);
-  const uint32_t o_empty = smem_u32(&bars[8 + 2 * NST]);
-  const uint32_t drain = smem_u32(&bars[9 + 2 * NST]);
-  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * (10 + 2 * NST));
+  auto s_full = [&](uint32_t t) { return smem_u32(&bars[2 + 2 * NST + t]); };
+  auto p_full = [&](uint32_t t) { return smem_u32(&bars[2 + 2 * NST + NQT + t]); };
+  auto o_full = [&](uint32_t t) { return smem_u32(&bars[2 + 2 * NST + 2 * NQT + t]); };
+  auto o_empty = [&](uint32_t t) { return smem_u32(&bars[2 + 2 * NST + 3 * NQT + t]); };
+  const uint32_t drain = smem_u32(&bars[2 + 2 * NST + 4 * NQT]);
+  constexpr int NBARS = 3 + 2 * NST + 4 * NQT;
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * NBARS);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -124,13 +197,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(kv_full(s), 1);
       mbar_init(kv_empty(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(s_full(b), 1);
-      mbar_init(s_empty(b), 128);
+    for (int t = 0; t < NQT; ++t) {
+      mbar_init(s_full(t), 1);
+      mbar_init(p_full(t), 128);
+      mbar_init(o_full(t), 1);
+      mbar_init(o_empty(t), 128);
     }
-    mbar_init(p_full, 128);
-    mbar_init(o_done, 1);
-    mbar_init(o_empty, 128);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -162,11 +234,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int32_t u = blockIdx.x; ok && u < P.num_units; u += gridDim.x, ++lu) {
         const Unit x = decode_unit(P, u);
         if (!wait_bounded(q_empty, (lu & 1) ^ 1u, abort_flag, P.wait, kErrWaitAttn)) break;
-        mbar_arrive_expect_tx(q_full, TILE_BYTES);
-        for (int c = 0; c < 2; ++c)
-          tma_load_3d(sQ + c * HALF_BYTES, &mapQ, q_full, x.head * DH + c * 64, x.qb * BQ, x.shard);
+        const int ntiles = x.nkb1 > 0 ? 2 : 1;
+        mbar_arrive_expect_tx(q_full, ntiles * TILE_BYTES);
+        for (int t = 0; t < ntiles; ++t)
+          for (int c = 0; c < 2; ++c)
+            tma_load_3d(sQ(t) + c * HALF_BYTES, &mapQ, q_full, x.head * DH + c * 64,
+                        (x.qb0 + t) * BQ, x.shard);
         last_q = lu;
-        for (int32_t j = 0; j < x.nkb; ++j) {
+        for (int32_t j = 0; j < x.nmax; ++j) {
           if (!wait_bounded(kv_empty(st), ph ^ 1u, abort_flag, P.wait, kErrWaitEmpty)) {
             ok = false;
             break;
@@ -200,67 +275,77 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ---------------------------------------------------------- MMA issuer
-      // K/V blocks are consumed in the producer's order: block n of the whole
+      // K/V blocks arrive in the producer's order: block n of the whole
       // sequence sits in ring slot n % NST, phase (n / NST) & 1.
-      uint32_t kv_n = 0;         // K/V blocks taken by S MMAs so far
-      uint32_t gs = 0;           // S buffers used so far
-      uint32_t gb = 0;           // P V products issued so far
+      uint32_t kv_n = 0;             // K/V blocks of finished units
+      uint32_t pv[NQT] = {0, 0};     // O += P V products per tile (p_full phases)
+      uint32_t ou[NQT] = {0, 0};     // units per tile with an output (o_empty phases)
       int32_t lu = 0;
       bool ok = true;
-      auto issue_s = [&](uint32_t kst) {
-        const uint32_t b = gs & 1;
-        const uint32_t d = tmem_base + S_COL0 + b * BKV;
+      auto wait_kv = [&](uint32_t n) {
+        return wait_bounded(kv_full(n % NST), (n / NST) & 1, abort_flag, P.wait, kErrWaitFull);
+      };
+      auto issue_s = [&](uint32_t t, uint32_t n) {
+        const uint32_t kst = n % NST;
 #pragma unroll
         for (int kk = 0; kk < DH / 16; ++kk) {
           const uint32_t off = (kk >> 2) * HALF_BYTES + (kk & 3) * 32;
-          tc_mma_f16(d, smem_desc_sw128(sQ + off, 16, 1024), smem_desc_sw128(sK(kst) + off, 16, 1024),
-                     IDESC_S, kk > 0 ? 1u : 0u);
+          tc_mma_f16(tmem_base + t * BKV, smem_desc_sw128(sQ(t) + off, 16, 1024),
+                     smem_desc_sw128(sK(kst) + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
         }
-        tc_commit(s_full(b));
-        ++gs;
-      };
-      // wait for K/V block n and a free S buffer, then issue S = Q K_n^T
-      auto next_s = [&](uint32_t n) -> bool {
-        if (!wait_bounded(kv_full(n % NST), (n / NST) & 1, abort_flag, P.wait, kErrWaitFull) ||
-            !wait_bounded(s_empty(gs & 1), ((gs >> 1) & 1) ^ 1u, abort_flag, P.wait, kErrWaitAttn))
-          return false;
-        tc_fence_after();
-        issue_s(n % NST);
-        return true;
+        tc_commit(s_full(t));
       };
       for (int32_t u = blockIdx.x; ok && u < P.num_units; u += gridDim.x, ++lu) {
         const Unit x = decode_unit(P, u);
         if (!wait_bounded(q_full, lu & 1, abort_flag, P.wait, kErrWaitAttn)) break;
         const uint32_t n0 = kv_n;
-        if (!next_s(n0)) break;
-        for (int32_t j = 0; j < x.nkb; ++j) {
-          if (j + 1 < x.nkb && !next_s(n0 + j + 1)) {
-            ok = false;
-            break;
-          }
-          if (j == 0 && lu > 0 &&
-              !wait_bounded(o_empty, (lu - 1) & 1, abort_flag, P.wait, kErrWaitAttn)) {
-            ok = false;
-            break;
-          }
-          if (!wait_bounded(p_full, gb & 1, abort_flag, P.wait, kErrWaitAttn)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
+        if (!wait_kv(n0)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int t = 0; t < NQT; ++t)
+          if (x.nkb(t) > 0) issue_s(t, n0);
+        for (int32_t j = 0; ok && j < x.nmax; ++j) {
           const uint32_t vst = (n0 + j) % NST;
 #pragma unroll
-          for (int kk = 0; kk < BKV / 16; ++kk) {
-            const uint64_t adesc = smem_desc_sw128(sP + (kk >> 2) * HALF_BYTES + (kk & 3) * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(sV(vst) + kk * 16 * 128, HALF_BYTES, 1024);
-            tc_mma_f16(tmem_base + O_COL, adesc, bdesc, IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+          for (int t = 0; t < NQT; ++t) {
+            if (j >= x.nkb(t)) continue;
+            if (j == 0 && ou[t] > 0 &&
+                !wait_bounded(o_empty(t), (ou[t] - 1) & 1, abort_flag, P.wait, kErrWaitAttn)) {
+              ok = false;
+              break;
+            }
+            if (!wait_bounded(p_full(t), pv[t] & 1, abort_flag, P.wait, kErrWaitAttn)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < BKV / 16; ++kk) {
+              const uint64_t bdesc = smem_desc_sw128(sV(vst) + kk * 16 * 128, HALF_BYTES, 1024);
+              tc_mma_f16_ts(tmem_base + O_COL0 + t * DH, tmem_base + t * BKV + kk * 8, bdesc,
+                            IDESC_O, (j > 0 || kk > 0) ? 1u : 0u);
+            }
+            ++pv[t];
+            // the last tile that uses block j releases its ring slot
+            const bool last_user = (t == NQT - 1) || (j >= x.nkb1);
+            if (last_user) tc_commit(kv_empty(vst));
+            if (j + 1 < x.nkb(t)) {
+              if (!wait_kv(n0 + j + 1)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              issue_s(t, n0 + j + 1);
+            } else {
+              tc_commit(o_full(t));
+            }
           }
-          tc_commit(o_done);
-          tc_commit(kv_empty(vst));
-          ++gb;
         }
         if (!ok) break;
-        kv_n = n0 + x.nkb;
+#pragma unroll
+        for (int t = 0; t < NQT; ++t)
+          if (x.nkb(t) > 0) ++ou[t];
+        kv_n = n0 + x.nmax;
         tc_commit(q_empty);
       }
       tc_commit(drain);
@@ -269,75 +354,43 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     __syncwarp();
   } else if (warp >= 4) {
     // ------------------------------------------------------- softmax / output
-    const int quad = warp & 3;
+    const int t = (warp - 4) / 4;          // query tile of this warpgroup
+    const int quad = warp & 3;             // TMEM lane quarter this warp may access
     const uint32_t lane_off = static_cast<uint32_t>(quad * 32) << 16;
-    uint32_t gs = 0, gb = 0;
-    int32_t lu = 0;
-    for (int32_t u = blockIdx.x; u < P.num_units; u += gridDim.x, ++lu) {
+    const uint32_t tS = tmem_base + lane_off + t * BKV;
+    const uint32_t tO = tmem_base + lane_off + O_COL0 + t * DH;
+    const float scale = P.scale_log2;
+    uint32_t sc = 0, uc = 0;
+    for (int32_t u = blockIdx.x; u < P.num_units; u += gridDim.x) {
       const Unit x = decode_unit(P, u);
-      const int32_t q = x.qb * BQ + quad * 32 + lane;
+      const int32_t nkb = x.nkb(t);
+      if (nkb == 0) continue;
+      const int32_t q0 = (x.qb0 + t) * BQ;
+      const int32_t q = q0 + quad * 32 + lane;
       float m = -INFINITY, l = 0.0f;
       bool ok = true;
-      for (int32_t j = 0; j < x.nkb; ++j) {
-        const uint32_t b = gs & 1;
-        ok = wait_bounded(s_full(b), (gs >> 1) & 1, abort_flag, P.wait, kErrWaitAttn);
+      for (int32_t j = 0; j < nkb; ++j) {
+        ok = wait_bounded(s_full(t), sc & 1, abort_flag, P.wait, kErrWaitAttn);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const uint32_t tS = tmem_base + lane_off + S_COL0 + b * BKV;
         const int32_t key0 = j * BKV;
-        // pass 1: row maximum (log2 domain)
-        float mx = -INFINITY;
-#pragma unroll
-        for (int c = 0; c < BKV / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tS + c * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int32_t key = key0 + c * 32 + e;
-            const bool valid = key < P.T && (!P.causal || key <= q);
-            const float xv = valid ? __uint_as_float(v[e]) * P.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, xv);
-          }
-        }
-        const float m_new = fmaxf(m, mx);
-        // pass 2: probabilities (bf16, packed) and their sum
-        uint32_t pk[BKV / 2];
-        float sum = 0.0f;
-#pragma unroll
-        for (int c = 0; c < BKV / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld_32x32b_x32(tS + c * 32, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            float pr[2];
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              const int32_t key = key0 + c * 32 + e + t;
-              const bool valid = key < P.T && (!P.causal || key <= q);
-              pr[t] = valid ? ex2(__uint_as_float(v[e + t]) * P.scale_log2 - m_new) : 0.0f;
-              sum += pr[t];
-            }
-            pk[(c * 32 + e) / 2] = pack2(pr[0], pr[1]);
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(s_empty(b));
-        ++gs;
-        const float alpha = ex2(m - m_new);   // 0 for the first block (m = -inf)
-        l = l * alpha + sum;
-        m = m_new;
-        // P's buffer and O are busy until the previous O += P V has finished
-        if (gb > 0) {
-          ok = wait_bounded(o_done, (gb - 1) & 1, abort_flag, P.wait, kErrWaitAttn);
-          ok = __all_sync(0xffffffffu, ok);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        if (j > 0 && __any_sync(0xffffffffu, alpha < 1.0f)) {
-          const uint32_t tO = tmem_base + lane_off + O_COL;
+        const bool masked = (key0 + BKV > P.T) || (P.causal && key0 + BKV - 1 > q0);
+        float mx;
+        if (masked)
+          softmax_block<true>(tS, scale, 0.0f, key0, P.T, P.causal, q, mx, true);
+        else
+          softmax_block<false>(tS, scale, 0.0f, key0, P.T, P.causal, q, mx, true);
+        const float m_cand = mx * scale;
+        const bool grow = m_cand > m + RESCALE_LOG2;
+        const float m_use = grow ? m_cand : m;
+        const float alpha = grow ? ex2(m - m_cand) : 1.0f;   // 0 on the first block
+        const float sum = masked
+                              ? softmax_block<true>(tS, scale, m_use, key0, P.T, P.causal, q, mx, false)
+                              : softmax_block<false>(tS, scale, m_use, key0, P.T, P.causal, q, mx, false);
+        if (j > 0 && __any_sync(0xffffffffu, grow)) {
+          // O += P V of the previous block has completed (it was issued
+          // before this score block, whose commit we waited for)
 #pragma unroll
           for (int c = 0; c < DH / 32; ++c) {
             uint32_t v[32];
@@ -349,30 +402,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tmem_st_wait();
         }
-        // P row -> shared memory, K-major with 128-byte swizzle
-        const int r = quad * 32 + lane;
-#pragma unroll
-        for (int c = 0; c < 2; ++c) {
-#pragma unroll
-          for (int un = 0; un < 8; ++un) {
-            const uint32_t off = c * HALF_BYTES + r * 128 + ((un ^ (r & 7)) * 16);
-            const int w0 = c * 32 + un * 4;
-            *reinterpret_cast<uint4*>(sP_ptr + off) = make_uint4(pk[w0], pk[w0 + 1], pk[w0 + 2], pk[w0 + 3]);
-          }
-        }
-        fence_proxy_async_smem();
+        l = l * alpha + sum;
+        m = m_use;
         tc_fence_before();
-        mbar_arrive(p_full);
-        ++gb;
+        mbar_arrive(p_full(t));
+        ++sc;
       }
       if (!ok) break;
-      // the unit's last O += P V
-      bool ok2 = wait_bounded(o_done, (gb - 1) & 1, abort_flag, P.wait, kErrWaitAttn);
+      // the tile's last O += P V
+      bool ok2 = wait_bounded(o_full(t), uc & 1, abort_flag, P.wait, kErrWaitAttn);
       ok2 = __all_sync(0xffffffffu, ok2);
       if (!ok2) break;
       tc_fence_after();
       const float inv_l = 1.0f / l;
-      const uint32_t tO = tmem_base + lane_off + O_COL;
       __nv_bfloat16* dst = P.O + ((static_cast<int64_t>(x.shard) * P.T + q) * P.hq + x.head) * DH;
 #pragma unroll
       for (int c = 0; c < DH / 32; ++c) {
@@ -392,7 +434,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
       }
       tc_fence_before();
-      mbar_arrive(o_empty);
+      mbar_arrive(o_empty(t));
+      ++uc;
     }
   }
 
@@ -433,7 +476,8 @@ tp_status launch_tc_attention(const LaunchCtx& c, const void* Q, const void* K, 
   prm.hkv = hkv;
   prm.group = hq / hkv;
   prm.q_blocks = ceil_div(T, BQ);
-  prm.num_units = p * hq * prm.q_blocks;
+  prm.q_pairs = ceil_div(prm.q_blocks, NQT);
+  prm.num_units = p * hq * prm.q_pairs;
   prm.causal = causal ? 1 : 0;
   prm.scale_log2 = static_cast<float>(1.4426950408889634 / std::sqrt(static_cast<double>(DH)));
   prm.O = static_cast<__nv_bfloat16*>(O);

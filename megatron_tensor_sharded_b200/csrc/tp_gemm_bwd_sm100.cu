@@ -1,0 +1,538 @@
+// Backward pass of the sharded MLP block on sm_100a tensor cores.
+//
+// The f / g conjugate operators ("Tensor parallel math", "The f and g
+// conjugate operators"): g after the row-parallel layer is the identity in
+// the backward pass, so every shard takes the whole upstream gradient dZ;
+// everything up to the column-parallel layer's input is local to the shard;
+// f before the column-parallel layer is the all-reduce, here the sum of p
+// full-shape input-gradient partials folded in shard order.
+//
+// Four batched GEMMs (batch = shard), one persistent warp-specialised kernel
+// template with the operand layouts as parameters:
+//
+//   G1  dH_i = (dZ W2_i^T) * act'(H_i)   A = dZ [T x d] K-major,
+//                                        B = W2_i (rows of W2) K-major;
+//                                        epilogue reads H_i (and the up
+//                                        projection for SwiGLU) and writes
+//                                        dH_i (and dU_i), bf16 [p][T][s]
+//   G2  dX_i = dH_i W1_i^T (+ dU_i Wup_i^T)   A = dH_i K-major, B = W1_i
+//                                        (column block of W1) K-major; the
+//                                        SwiGLU pair is one K loop over both
+//                                        halves; fp32 partials [p][T][d]
+//   G3  dW1_i = X^T dH_i                 A = X^T (M-major), B = dH_i
+//                                        N-major; written into the column
+//                                        block i of dW1 [d][k] (SwiGLU: a
+//                                        second half of batches for dW_up)
+//   G4  dW2_i = Y_i^T dZ                 A = Y_i^T (M-major), B = dZ
+//                                        N-major; written into row block i
+//                                        of dW2 [k][d]
+//
+// Every operand is a 3-D tensor map (inner, outer, batch) with the shard as
+// the batch, except W1's column blocks, read from the whole [d][k] map at a
+// K offset of s per shard (s is a multiple of 64, so no K block crosses into
+// the next shard).  TMA zero-fills beyond each extent, so ragged M, N and K
+// need no special code.  Roles as in the forward GEMM:
+// warp 0 TMA, warp 1 MMA (two TMEM accumulators), warp 2 TMEM allocation,
+// warps 4..11 epilogue; every wait bounded.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "tp_gemm_parts.cuh"
+#include "tp_internal.h"
+#include "tp_launch.cuh"
+
+namespace tpk {
+namespace {
+
+using namespace gemm;
+
+constexpr int A_CHUNK_BYTES = BK * 64 * 2;   // M-major A: one 64-wide M atom column, 8 KiB
+
+enum BwdEpi : int { kEpiF32 = 0, kEpiActGrad = 1, kEpiSwigluGrad = 2 };
+
+struct GParams {
+  int32_t M, N, K;              // per batch
+  int32_t p, halves;            // batch b -> shard b % p, half b / p
+  int32_t m_tiles, n_tiles, num_tiles, k_blocks, kb_half;  // kb_half > 0: K-concat of two sources
+  int32_t a_batched, b_batched; // operand batch coordinate = shard (else 0)
+  int32_t b_koff;               // K-major B: K coordinate offset per shard (W1's column blocks)
+  int32_t act;
+  // epilogue
+  void* out[2];                 // per half
+  int64_t out_shard_stride;     // elements
+  int64_t ldc;                  // elements
+  const void* aux0;             // H (pre-activation / gate) bf16, same layout as out
+  const void* aux1;             // up projection (SwiGLU)
+  WaitCtl wait;
+  int64_t debug_drop;
+};
+
+struct GTile {
+  int32_t b, shard, half, m, n;
+};
+
+__device__ __forceinline__ GTile decode(const GParams& P, int32_t t) {
+  const int32_t per = P.m_tiles * P.n_tiles;
+  GTile g;
+  g.b = t / per;
+  const int32_t r = t - g.b * per;
+  g.n = r / P.m_tiles;
+  g.m = r - g.n * P.m_tiles;
+  g.shard = g.b % P.p;
+  g.half = g.b / P.p;
+  return g;
+}
+
+template <int AMN, int BMN, int BN>
+__device__ __forceinline__ void issue(const GParams& P, const CUtensorMap* mA0,
+                                      const CUtensorMap* mA1, const CUtensorMap* mB0,
+                                      const CUtensorMap* mB1, const GTile& g, int32_t kb,
+                                      uint32_t sa, uint32_t sb, uint32_t bar) {
+  // K-concat (kb_half > 0): the second half of the K loop reads the second
+  // sources; halves > 1: the second half of the batches reads B1.
+  bool second = false;
+  if (P.kb_half > 0 && kb >= P.kb_half) {
+    second = true;
+    kb -= P.kb_half;
+  }
+  const CUtensorMap* mA = second ? mA1 : mA0;
+  const CUtensorMap* mB = (second || g.half > 0) ? mB1 : mB0;
+  const int32_t za = P.a_batched ? g.shard : 0;
+  const int32_t zb = P.b_batched ? g.shard : 0;
+  const int32_t m0 = g.m * BM, n0 = g.n * BN, k0 = kb * BK;
+  if constexpr (AMN == 0) {
+    tma_load_3d(sa, mA, bar, k0, m0, za);
+  } else {
+#pragma unroll
+    for (int c = 0; c < BM / 64; ++c) tma_load_3d(sa + c * A_CHUNK_BYTES, mA, bar, m0 + c * 64, k0, za);
+  }
+  if constexpr (BMN == 0) {
+    tma_load_3d(sb, mB, bar, k0 + g.shard * P.b_koff, n0, zb);
+  } else {
+#pragma unroll
+    for (int c = 0; c < BN / 64; ++c) tma_load_3d(sb + c * B_CHUNK_BYTES, mB, bar, n0 + c * 64, k0, zb);
+  }
+}
+
+__device__ __forceinline__ void store_bf16x8_at(__nv_bfloat16* dst, const float (&y)[8]) {
+  const uint4 pk = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
+                              pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
+  *reinterpret_cast<uint4*>(dst) = pk;
+}
+
+template <int EPI, int BN>
+__device__ __forceinline__ void epilogue(const GParams& P, const GTile& g, uint32_t tacc, int row,
+                                         int half) {
+  const bool row_ok = row < P.M;
+  const int64_t rbase = static_cast<int64_t>(g.shard) * P.out_shard_stride +
+                        static_cast<int64_t>(row) * P.ldc;
+#pragma unroll 1
+  for (int q = 0; q < BN / 64; ++q) {
+    const int c0 = half * (BN / 2) + q * 32;
+    const int32_t j0 = g.n * BN + c0;
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(tacc + c0, v);
+    tmem_ld_wait();
+    if (!row_ok) continue;
+    if constexpr (EPI == kEpiF32) {
+      float* dst = static_cast<float*>(P.out[g.half]) + rbase;
+#pragma unroll
+      for (int e4 = 0; e4 < 8; ++e4) {
+        const int32_t j = j0 + e4 * 4;
+        if (j >= P.N) break;
+        *reinterpret_cast<float4*>(dst + j) =
+            make_float4(__uint_as_float(v[e4 * 4 + 0]), __uint_as_float(v[e4 * 4 + 1]),
+                        __uint_as_float(v[e4 * 4 + 2]), __uint_as_float(v[e4 * 4 + 3]));
+      }
+    } else {
+      const __nv_bfloat16* H = static_cast<const __nv_bfloat16*>(P.aux0) + rbase;
+      __nv_bfloat16* dH = static_cast<__nv_bfloat16*>(P.out[0]) + rbase;
+#pragma unroll
+      for (int e8 = 0; e8 < 4; ++e8) {
+        const int32_t j = j0 + e8 * 8;
+        if (j >= P.N) break;
+        float h[8], dy[8], o[8];
+        unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(H + j)), h);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) dy[e] = __uint_as_float(v[e8 * 8 + e]);
+        if constexpr (EPI == kEpiActGrad) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) o[e] = dy[e] * act_grad_unary_mufu(P.act, h[e]);
+          store_bf16x8_at(dH + j, o);
+        } else {
+          const __nv_bfloat16* U = static_cast<const __nv_bfloat16*>(P.aux1) + rbase;
+          __nv_bfloat16* dU = static_cast<__nv_bfloat16*>(P.out[1]) + rbase;
+          float u[8], ou[8];
+          unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(U + j)), u);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float sg = sigmoid_mufu(h[e]);
+            o[e] = dy[e] * u[e] * (sg * (1.0f + h[e] * (1.0f - sg)));   // d gate
+            ou[e] = dy[e] * (h[e] * sg);                                // d up
+          }
+          store_bf16x8_at(dH + j, o);
+          store_bf16x8_at(dU + j, ou);
+        }
+      }
+    }
+  }
+}
+
+template <int AMN, int BMN, int EPI, int BN>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    tc_gemm_bwd_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
+                       const __grid_constant__ CUtensorMap mapB0, const __grid_constant__ CUtensorMap mapB1,
+                       const GParams P) {
+  using C = Cfg<BN>;
+  constexpr int STAGES = C::STAGES;
+  constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, AMN, BMN);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const ctrl = smem_raw + (base - raw) + STAGES * C::STAGE_BYTES;
+  uint64_t* const bars = reinterpret_cast<uint64_t*>(ctrl);
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * (2 * STAGES + 5));
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto full_bar = [&](uint32_t s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](uint32_t s) { return smem_u32(&bars[STAGES + s]); };
+  auto accf_bar = [&](uint32_t b) { return smem_u32(&bars[2 * STAGES + b]); };
+  auto acce_bar = [&](uint32_t b) { return smem_u32(&bars[2 * STAGES + 2 + b]); };
+  const uint32_t drain_bar = smem_u32(&bars[2 * STAGES + 4]);
+  auto slot_a = [&](uint32_t s) { return base + s * C::STAGE_BYTES; };
+  auto slot_b = [&](uint32_t s) { return base + s * C::STAGE_BYTES + A_BYTES; };
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), NUM_EPI_WARPS * 32);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&mapA0);
+    tma_prefetch_map(&mapB0);
+  }
+  if (warp == 2) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  pdl_wait();
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int32_t t = blockIdx.x; ok && t < P.num_tiles; t += gridDim.x) {
+        const GTile g = decode(P, t);
+        for (int32_t kb = 0; kb < P.k_blocks; ++kb) {
+          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, P.wait, kErrWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          if (issued != P.debug_drop) {
+            mbar_arrive_expect_tx(full_bar(stage), C::STAGE_BYTES);
+            issue<AMN, BMN, BN>(P, &mapA0, &mapA1, &mapB0, &mapB1, g, kb, slot_a(stage),
+                                slot_b(stage), full_bar(stage));
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      const int64_t first = issued > STAGES ? issued - STAGES : 0;
+      for (int64_t q = first; q < issued; ++q) {
+        if (q == P.debug_drop) continue;
+        wait_teardown(full_bar(static_cast<uint32_t>(q % STAGES)),
+                      static_cast<uint32_t>((q / STAGES) & 1), P.wait);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      int32_t lt = 0;
+      for (int32_t t = blockIdx.x; ok && t < P.num_tiles; t += gridDim.x, ++lt) {
+        const uint32_t b = lt & 1, ap = (lt >> 1) & 1;
+        if (!wait_bounded(acce_bar(b), ap ^ 1u, abort_flag, P.wait, kErrWaitAccEmpty)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + b * BN;
+        for (int32_t kb = 0; kb < P.k_blocks; ++kb) {
+          if (!wait_bounded(full_bar(stage), phase, abort_flag, P.wait, kErrWaitFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = slot_a(stage), sb = slot_b(stage);
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk) {
+            // K-major: a 16-element k step is 32 B inside the 128-byte swizzle
+            // row; M/N-major: 64-wide atoms a chunk apart, a k step is 16
+            // rows of 128 B.
+            const uint64_t adesc = AMN == 0 ? smem_desc_sw128(sa + kk * UK * 2, 16, 1024)
+                                            : smem_desc_sw128(sa + kk * UK * 128, A_CHUNK_BYTES, 1024);
+            const uint64_t bdesc = BMN == 0 ? smem_desc_sw128(sb + kk * UK * 2, 16, 1024)
+                                            : smem_desc_sw128(sb + kk * UK * 128, B_CHUNK_BYTES, 1024);
+            tc_mma_f16(d_tmem, adesc, bdesc, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit(empty_bar(stage));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(accf_bar(b));
+      }
+      tc_commit(drain_bar);
+      wait_teardown(drain_bar, 0, P.wait);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    const int quad = warp & 3;
+    const int half = (warp - 4) >> 2;
+    int32_t lt = 0;
+    for (int32_t t = blockIdx.x; t < P.num_tiles; t += gridDim.x, ++lt) {
+      const uint32_t b = lt & 1, ap = (lt >> 1) & 1;
+      const GTile g = decode(P, t);
+      bool ok = wait_bounded(accf_bar(b), ap, abort_flag, P.wait, kErrWaitAccFull);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * BN;
+      epilogue<EPI, BN>(P, g, tacc, g.m * BM + quad * 32 + lane, half);
+      tc_fence_before();
+      mbar_arrive(acce_bar(b));
+    }
+  }
+
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+template <int AMN, int BMN, int EPI, int BN>
+tp_status launch_g(const LaunchCtx& c, const CUtensorMap* maps, GParams prm) {
+  using Cf = Cfg<BN>;
+  static bool attr_done[64] = {};
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    const int dev = c.device & 63;
+    if (!attr_done[dev]) {
+      if (cudaFuncSetAttribute(tc_gemm_bwd_kernel<AMN, BMN, EPI, BN>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cf::SMEM_BYTES) != cudaSuccess) {
+        set_error_detail("cudaFuncSetAttribute failed: %s", cudaGetErrorString(cudaGetLastError()));
+        return TP_ERR_CUDA;
+      }
+      attr_done[dev] = true;
+    }
+  }
+  prm.n_tiles = ceil_div(prm.N, BN);
+  prm.num_tiles = prm.m_tiles * prm.n_tiles * prm.p * prm.halves;
+  prm.wait.err = c.err_word;
+  prm.wait.timeout_ns = c.timeout_ns;
+  prm.debug_drop = c.debug_drop;
+  if (prm.num_tiles == 0) return TP_OK;
+  const int grid = prm.num_tiles < c.num_sms ? prm.num_tiles : c.num_sms;
+  const cudaError_t e = launch_pdl(tc_gemm_bwd_kernel<AMN, BMN, EPI, BN>, dim3(grid),
+                                   dim3(NUM_THREADS), Cf::SMEM_BYTES, c.stream, maps[0], maps[1],
+                                   maps[2], maps[3], prm);
+  note_launch();
+  if (e != cudaSuccess) {
+    set_error_detail("backward GEMM launch failed: %s", cudaGetErrorString(e));
+    return TP_ERR_CUDA;
+  }
+  return TP_OK;
+}
+
+// Tile width for an (M x N) x batches problem with K / 64 slots: the
+// forward cost model, restricted to single-CTA tiles of 64, 128 or 256.
+int pick_bn(int64_t M, int64_t N, int64_t batches, int64_t k_blocks, int num_sms) {
+  const TileChoice t = pick_tile(M, N, batches, k_blocks, num_sms, false, false);
+  return t.bn == 192 ? 128 : t.bn;
+}
+
+template <int AMN, int BMN, int EPI>
+tp_status launch_any(const LaunchCtx& c, const CUtensorMap* maps, GParams prm, int batches) {
+  const int bn = pick_bn(prm.M, prm.N, batches, prm.k_blocks, c.num_sms);
+  if (bn == 256) return launch_g<AMN, BMN, EPI, 256>(c, maps, prm);
+  if (bn == 128) return launch_g<AMN, BMN, EPI, 128>(c, maps, prm);
+  return launch_g<AMN, BMN, EPI, 64>(c, maps, prm);
+}
+
+// 3-D bf16 map: dims (inner, outer, batch), row stride and batch stride in
+// elements; box (inner 64, outer box_outer).
+bool map3(CUtensorMap* m, const void* g, int64_t inner, int64_t outer, int64_t batch,
+          int64_t row_stride, int64_t batch_stride, uint32_t box_outer) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(inner), static_cast<uint64_t>(outer),
+                            static_cast<uint64_t>(batch)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(row_stride) * 2,
+                               static_cast<uint64_t>(batch > 1 ? batch_stride : row_stride * outer) * 2};
+  const uint32_t box[3] = {64, box_outer, 1};
+  return make_map(m, g, 3, dims, strides, box);
+}
+
+GParams base_params(int64_t M, int64_t N, int64_t K, int p, int halves) {
+  GParams prm{};
+  prm.M = static_cast<int32_t>(M);
+  prm.N = static_cast<int32_t>(N);
+  prm.K = static_cast<int32_t>(K);
+  prm.p = p;
+  prm.halves = halves;
+  prm.m_tiles = ceil_div(M, BM);
+  prm.k_blocks = ceil_div(K, BK);
+  return prm;
+}
+
+}  // namespace
+
+// G1: dH_i = (dZ W2_i^T) * act'(H_i)   [SwiGLU: dG_i, dU_i]
+tp_status launch_bwd_act_grad(const LaunchCtx& c, const void* dZ, const void* W2, const void* H,
+                              const void* Hup, void* dH, void* dU, int64_t T, int64_t d, int64_t k,
+                              int p, int act) {
+  const int64_t s = k / p;
+  GParams prm = base_params(T, s, d, p, 1);
+  prm.a_batched = 0;
+  prm.b_batched = 1;
+  prm.act = act;
+  prm.out[0] = dH;
+  prm.out[1] = dU;
+  prm.out_shard_stride = T * s;
+  prm.ldc = s;
+  prm.aux0 = H;
+  prm.aux1 = Hup;
+  const int bn = pick_bn(T, s, p, prm.k_blocks, c.num_sms);
+  CUtensorMap maps[4];
+  // A = dZ [T][d] K-major; B = W2 rows of shard i: [p][s][d] K-major (N rows)
+  if (!map3(&maps[0], dZ, d, T, 1, d, 0, BM) || !map3(&maps[2], W2, d, s, p, d, s * d, bn))
+    return TP_ERR_CUDA;
+  maps[1] = maps[0];
+  maps[3] = maps[2];
+  if (act == kActSwiglu) {
+    if (bn == 256) return launch_g<0, 0, kEpiSwigluGrad, 256>(c, maps, prm);
+    if (bn == 128) return launch_g<0, 0, kEpiSwigluGrad, 128>(c, maps, prm);
+    return launch_g<0, 0, kEpiSwigluGrad, 64>(c, maps, prm);
+  }
+  if (bn == 256) return launch_g<0, 0, kEpiActGrad, 256>(c, maps, prm);
+  if (bn == 128) return launch_g<0, 0, kEpiActGrad, 128>(c, maps, prm);
+  return launch_g<0, 0, kEpiActGrad, 64>(c, maps, prm);
+}
+
+// G2: dX partials P_i = dH_i W1_i^T (+ dU_i Wup_i^T), fp32 [p][T][d]
+tp_status launch_bwd_dx_partials(const LaunchCtx& c, const void* dH, const void* dU,
+                                 const void* W1, const void* Wup, float* P, int64_t T, int64_t d,
+                                 int64_t k, int p) {
+  const int64_t s = k / p;
+  const bool two = dU != nullptr;
+  GParams prm = base_params(T, d, two ? 2 * s : s, p, 1);
+  if (two) {
+    prm.kb_half = ceil_div(s, BK);
+    prm.k_blocks = 2 * prm.kb_half;
+  }
+  prm.a_batched = 1;
+  prm.b_batched = 0;
+  prm.b_koff = static_cast<int32_t>(s);
+  prm.out[0] = P;
+  prm.out[1] = P;
+  prm.out_shard_stride = T * d;
+  prm.ldc = d;
+  const int bn = pick_bn(T, d, p, prm.k_blocks, c.num_sms);
+  CUtensorMap maps[4];
+  // A = dH [p][T][s] K-major; B = W1 [d][k] K-major (inner k, outer d = N
+  // rows), shard i's block at K offset i s
+  if (!map3(&maps[0], dH, s, T, p, s, T * s, BM) || !map3(&maps[2], W1, k, d, 1, k, 0, bn))
+    return TP_ERR_CUDA;
+  if (two) {
+    if (!map3(&maps[1], dU, s, T, p, s, T * s, BM) || !map3(&maps[3], Wup, k, d, 1, k, 0, bn))
+      return TP_ERR_CUDA;
+  } else {
+    maps[1] = maps[0];
+    maps[3] = maps[2];
+  }
+  if (bn == 256) return launch_g<0, 0, kEpiF32, 256>(c, maps, prm);
+  if (bn == 128) return launch_g<0, 0, kEpiF32, 128>(c, maps, prm);
+  return launch_g<0, 0, kEpiF32, 64>(c, maps, prm);
+}
+
+// G3: dW1[:, i s:(i+1) s] = X^T dH_i  (SwiGLU: dW_up from dU as a second
+// half of the batches), fp32 [d][k]
+tp_status launch_bwd_dw1(const LaunchCtx& c, const void* X, const void* dH, const void* dU,
+                         float* dW1, float* dWup, int64_t T, int64_t d, int64_t k, int p) {
+  const int64_t s = k / p;
+  const bool two = dU != nullptr && dWup != nullptr;
+  GParams prm = base_params(d, s, T, p, two ? 2 : 1);
+  prm.a_batched = 0;
+  prm.b_batched = 1;
+  prm.out[0] = dW1;
+  prm.out[1] = two ? dWup : dW1;
+  prm.out_shard_stride = s;
+  prm.ldc = k;
+  const int bn = pick_bn(d, s, p * prm.halves, prm.k_blocks, c.num_sms);
+  CUtensorMap maps[4];
+  // A = X^T: M-major view of X [T][d] (inner d = M, outer T = K);
+  // B = dH [p][T][s] N-major (inner s = N, outer T = K)
+  if (!map3(&maps[0], X, d, T, 1, d, 0, BK) || !map3(&maps[2], dH, s, T, p, s, T * s, BK))
+    return TP_ERR_CUDA;
+  maps[1] = maps[0];
+  if (two) {
+    if (!map3(&maps[3], dU, s, T, p, s, T * s, BK)) return TP_ERR_CUDA;
+  } else {
+    maps[3] = maps[2];
+  }
+  if (bn == 256) return launch_g<1, 1, kEpiF32, 256>(c, maps, prm);
+  if (bn == 128) return launch_g<1, 1, kEpiF32, 128>(c, maps, prm);
+  return launch_g<1, 1, kEpiF32, 64>(c, maps, prm);
+}
+
+// G4: dW2[i s:(i+1) s, :] = Y_i^T dZ, fp32 [k][d]
+tp_status launch_bwd_dw2(const LaunchCtx& c, const void* Y, const void* dZ, float* dW2, int64_t T,
+                         int64_t d, int64_t k, int p) {
+  const int64_t s = k / p;
+  GParams prm = base_params(s, d, T, p, 1);
+  prm.a_batched = 1;
+  prm.b_batched = 0;
+  prm.out[0] = dW2;
+  prm.out[1] = dW2;
+  prm.out_shard_stride = s * d;
+  prm.ldc = d;
+  const int bn = pick_bn(s, d, p, prm.k_blocks, c.num_sms);
+  CUtensorMap maps[4];
+  // A = Y_i^T: M-major view of Y [p][T][s]; B = dZ [T][d] N-major
+  if (!map3(&maps[0], Y, s, T, p, s, T * s, BK) || !map3(&maps[2], dZ, d, T, 1, d, 0, BK))
+    return TP_ERR_CUDA;
+  maps[1] = maps[0];
+  maps[3] = maps[2];
+  if (bn == 256) return launch_g<1, 1, kEpiF32, 256>(c, maps, prm);
+  if (bn == 128) return launch_g<1, 1, kEpiF32, 128>(c, maps, prm);
+  return launch_g<1, 1, kEpiF32, 64>(c, maps, prm);
+}
+
+}  // namespace tpk

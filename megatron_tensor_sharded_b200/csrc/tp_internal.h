@@ -76,6 +76,26 @@ tp_status launch_tc_block(const LaunchCtx& c, const void* X, const void* W1, con
                           float* Z, int* counters, int64_t T, int64_t d, int64_t k, int p, int act,
                           bool splitk);
 
+// ---- row-wise fold (+ bias, + residual) and LayerNorm (tp_rowops.cu)
+cudaError_t launch_row_fold_ln(const LaunchCtx& c, const float* P, int p, const float* bias,
+                               const float* R, float* H, const float* gamma, const float* beta,
+                               void* Y, int64_t T, int64_t d, float eps);
+
+cudaError_t launch_colsum(const LaunchCtx& c, const void* A, float* out, float* scratch,
+                          int64_t batches, int64_t R, int64_t n, int64_t out_batch_stride);
+
+// ---- backward pass of the MLP block (tp_gemm_bwd_sm100.cu)
+tp_status launch_bwd_act_grad(const LaunchCtx& c, const void* dZ, const void* W2, const void* H,
+                              const void* Hup, void* dH, void* dU, int64_t T, int64_t d, int64_t k,
+                              int p, int act);
+tp_status launch_bwd_dx_partials(const LaunchCtx& c, const void* dH, const void* dU,
+                                 const void* W1, const void* Wup, float* P, int64_t T, int64_t d,
+                                 int64_t k, int p);
+tp_status launch_bwd_dw1(const LaunchCtx& c, const void* X, const void* dH, const void* dU,
+                         float* dW1, float* dWup, int64_t T, int64_t d, int64_t k, int p);
+tp_status launch_bwd_dw2(const LaunchCtx& c, const void* Y, const void* dZ, float* dW2, int64_t T,
+                         int64_t d, int64_t k, int p);
+
 // ---- attention of every shard's heads (tp_attn_sm100.cu), head_dim 128, bf16
 tp_status launch_tc_attention(const LaunchCtx& c, const void* Q, const void* K, const void* V,
                               void* O, int64_t T, int p, int hq, int hkv, int causal);

@@ -10,9 +10,14 @@ maxima, sums and the O accumulator in fp32; it rounds the probabilities
 P = exp(s - m) to bf16 before P V and rounds O to bf16 once at the end.  A
 relative error of at most 2^-9 on every probability moves O by at most
 2^-9 * max|v| (a convex combination of the value rows), and the final
-rounding adds at most 2^-9 * |O|; fp32 accumulation and the exp2
-approximation stay orders of magnitude below.  So
-    |O_gpu - O_ref| <= 2^-9 * (max|v| + |O_ref|) (+ 1e-6 slack)."""
+rounding adds at most 2^-9 * |O|.  The scores themselves carry fp32
+rounding: the tensor core's fp32 sum of 128 exact bf16 products is off by at
+most 128 * 2^-24 * sum|q_i k_i| (about 2.5e-3 for the std-2 inputs of the
+peaked test, far less for the others); scaled by log2(e)/sqrt(128) = 0.1275
+and turned into a relative error of the probability by ln 2, that is below
+2^-12 on every probability, so at most 2^-12 * max|v| on O (the fma forming
+the exponent argument and the exp2 approximation add about 2^-20).  So
+    |O_gpu - O_ref| <= 2^-9 * (max|v| + |O_ref|) + 2^-12 * max|v|."""
 
 import math
 
@@ -27,7 +32,8 @@ from oracle import tp_oracle as O
 
 pytestmark = pytest.mark.gpu
 
-EPS = 2.0 ** -9
+EPS = 2.0 ** -9          # bf16 rounding of P and of O
+EPS_SCORE = 2.0 ** -12   # fp32 rounding of the scores and exponent argument
 
 
 def _bf16_vals(a):
@@ -44,7 +50,7 @@ def _run_heads(Qb, Kb, Vb, p, T, h, hkv, causal):
 
 def _check_head(got, q, k, v, causal):
     want = O.sdpa_head(q, k, v, causal)
-    bound = EPS * (np.abs(v).max() + np.abs(want)) + 1e-6
+    bound = EPS * (np.abs(v).max() + np.abs(want)) + EPS_SCORE * np.abs(v).max()
     err = np.abs(got - want)
     assert np.all(err <= bound), (float(err.max()), float((err / bound).max()))
     return want
@@ -78,7 +84,7 @@ def test_attention_heads_match_oracle(p, T, h, hkv, causal):
 
 
 def test_attention_heads_peaked_scores():
-    """Large scores (std 4 inputs): the running maximum changes from block to
+    """Large scores (std 2 inputs): the running maximum changes from block to
     block and the O rescaling in tensor memory is exercised."""
     p, T, h, hkv = 1, 700, 2, 2
     Qb, Kb, Vb = W.make_qkv(p, T, h, hkv, 128, seed=5, std=2.0)
@@ -110,7 +116,7 @@ def test_attention_heads_full_size_sampled(name):
                 q = _bf16_vals(Qb[i][t:t + 1, cs])
                 n = t + 1 if w.causal else T
                 want = O.sdpa_head(q, K[:n], V[:n], False)[0]
-                bound = EPS * (np.abs(V[:n]).max() + np.abs(want)) + 1e-6
+                bound = EPS * (np.abs(V[:n]).max() + np.abs(want)) + EPS_SCORE * np.abs(V[:n]).max()
                 assert np.all(np.abs(got[i][t, cs] - want) <= bound), (i, j, t)
 
 

@@ -45,9 +45,9 @@ def check_layer_norm_closed_forms():
 def _params(rng, d, h, hkv, dh, k, act, bias=True, scale=0.1):
     def r(*shape):
         return rng.standard_normal(shape) * scale
-    return {"ln1_g": 1.0 + r(d), "ln1_b": r(d), "Wq": r(d, h * dh), "Wk": r(d, hkv * dh),
+    return {"ln1_gamma": 1.0 + r(d), "ln1_beta": r(d), "Wq": r(d, h * dh), "Wk": r(d, hkv * dh),
             "Wv": r(d, hkv * dh), "Wo": r(h * dh, d), "bo": r(d) if bias else None,
-            "ln2_g": 1.0 + r(d), "ln2_b": r(d), "W1": r(d, k),
+            "ln2_gamma": 1.0 + r(d), "ln2_beta": r(d), "W1": r(d, k),
             "W_up": r(d, k) if act == "swiglu" else None, "b1": r(k) if bias else None,
             "W2": r(k, d), "b2": r(d) if bias else None}
 

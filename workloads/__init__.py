@@ -166,6 +166,101 @@ def make_qkv(p: int, T: int, hq: int, hkv: int, head_dim: int, seed: int, std: f
     return tuple(out)
 
 
+@dataclasses.dataclass(frozen=True)
+class BlockWorkload:
+    """One pre-norm transformer block: LayerNorm, the attention block, the
+    residual add, LayerNorm, the MLP block, the residual add."""
+    name: str
+    T: int
+    d: int
+    n_heads: int
+    n_kv_heads: int
+    head_dim: int
+    k: int            # FFN width
+    p: int
+    act: str
+    causal: bool
+    description: str
+
+    def attn(self) -> AttnWorkload:
+        return AttnWorkload(self.name + "/attn", self.T, self.d, self.n_heads, self.n_kv_heads,
+                            self.head_dim, self.p, self.causal, "")
+
+    def mlp_flops(self) -> int:
+        return 2 * self.T * self.d * self.k * (3 if self.act == "swiglu" else 2)
+
+    def flops(self) -> dict:
+        a = self.attn().flops()
+        m = self.mlp_flops()
+        return {"attention_block": a["total"], "mlp_block": m, "total": a["total"] + m}
+
+
+BLOCK_WORKLOADS = {
+    "block_wide": BlockWorkload("block_wide", 4096, 4096, 32, 32, 128, 16384, 4, "gelu_tanh", True,
+                                "transformer block: T=4096 d=4096, 32 heads x 128, d_ff=16384, "
+                                "GELU(tanh), p=4, causal, bf16 GEMMs, fp32 residual stream"),
+    "block_llama": BlockWorkload("block_llama", 4096, 8192, 64, 8, 128, 28672, 8, "swiglu", True,
+                                 "Llama-70B-shaped block: T=4096 d=8192, 64 query / 8 key-value "
+                                 "heads x 128, SwiGLU d_ff=28672, p=8, causal"),
+}
+
+
+@dataclasses.dataclass
+class BlockInputs:
+    """X (fp32 residual stream), LayerNorm gains/biases (fp32), projection
+    weights and b1 as bf16 bit patterns (uint16), bo and b2 fp32."""
+    X: np.ndarray
+    prm: dict
+
+    def values(self, name: str) -> Optional[np.ndarray]:
+        a = self.X if name == "X" else self.prm[name]
+        if a is None:
+            return None
+        return bf16_bits_to_f32(a) if a.dtype == np.uint16 else a
+
+    def value_dict(self) -> dict:
+        return {k: self.values(k) for k in self.prm}
+
+
+def make_block_inputs(T: int, d: int, n_heads: int, n_kv_heads: int, head_dim: int, k: int,
+                      act: str, seed: int = 42, w_std: float = 0.02,
+                      with_bias: bool = True) -> BlockInputs:
+    """``default_rng(seed)`` float32 normals in the order X (std 1), ln1 gain
+    (1 + 0.1 N), ln1 bias (0.1 N), Wq, Wk, Wv, Wo (std ``w_std``), bo
+    (0.02 N), ln2 gain, ln2 bias, W1, W_up (SwiGLU only), b1, W2, b2; matrices
+    and b1 rounded to bf16, bo and b2 kept fp32 holding bf16 values."""
+    rng = np.random.default_rng(seed)
+
+    def draw(shape, std, mean=0.0):
+        v = rng.standard_normal(shape, dtype=np.float32)
+        if std != 1.0:
+            v *= np.float32(std)
+        if mean != 0.0:
+            v += np.float32(mean)
+        return v
+
+    c = f32_to_bf16_bits
+
+    def vec_bf16_f32(n):
+        return bf16_bits_to_f32(c(draw((n,), 0.02)))
+
+    X = draw((T, d), 1.0)
+    prm = {"ln1_gamma": draw((d,), 0.1, 1.0), "ln1_beta": draw((d,), 0.1)}
+    prm["Wq"] = c(draw((d, n_heads * head_dim), w_std))
+    prm["Wk"] = c(draw((d, n_kv_heads * head_dim), w_std))
+    prm["Wv"] = c(draw((d, n_kv_heads * head_dim), w_std))
+    prm["Wo"] = c(draw((n_heads * head_dim, d), w_std))
+    prm["bo"] = vec_bf16_f32(d) if with_bias else None
+    prm["ln2_gamma"] = draw((d,), 0.1, 1.0)
+    prm["ln2_beta"] = draw((d,), 0.1)
+    prm["W1"] = c(draw((d, k), w_std))
+    prm["W_up"] = c(draw((d, k), w_std)) if act == "swiglu" else None
+    prm["b1"] = c(draw((k,), 0.02)) if with_bias else None
+    prm["W2"] = c(draw((k, d), w_std))
+    prm["b2"] = vec_bf16_f32(d) if with_bias else None
+    return BlockInputs(X, prm)
+
+
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
     """Round float32 values to bf16 (round to nearest, ties to even) and
     return the 16-bit patterns as uint16.  Inputs here are finite."""
