@@ -20,13 +20,19 @@
 //                  runs;
 //   warp 2         TMEM allocation;
 //   warps 4..7     online softmax of tile 0, warps 8..11 of tile 1: thread =
-//                  query row (its TMEM lane); scores in the log2 domain with
-//                  ex2.approx.  The running maximum is only moved when it grows
-//                  by more than 2^8 (the stale maximum is exact once the sum
-//                  and O share it), so O is rarely rescaled; when it is, the
-//                  thread scales its O row in TMEM -- safe without a wait,
-//                  because the score block it just read was committed after
-//                  the previous O += P V.  At the end O is divided by the row
+//                  query row (its TMEM lane), one round trip to TMEM per
+//                  block (all 128 scores loaded at once); scores in the log2
+//                  domain; the row max in registers (3-input max, four
+//                  independent chains); exponent arguments, sums in packed
+//                  fp32 pairs; exp2 by MUFU (ex2.approx) for 3/4 of the
+//                  elements and by a polynomial on the FMA pipe for 1/4, so
+//                  the MUFU unit (16 per clock per SM) is not the only one.
+//                  The running maximum is only moved when it grows by more
+//                  than 2^8 (the stale maximum is exact once the sum and O
+//                  share it), so O is rarely rescaled; when it is, the thread
+//                  scales its O row in TMEM -- safe without a wait, because
+//                  the score block it just read was committed after the
+//                  previous O += P V.  At the end O is divided by the row
 //                  sum, converted to bf16 and stored.
 // Keys beyond T and (causal) keys after the query are masked, on the blocks
 // that hold any.  Causal units are taken longest first.  Every barrier wait
@@ -59,7 +65,9 @@ constexpr int NUM_THREADS = 384;
 constexpr uint32_t IDESC_S = idesc_bf16_f32(BQ, BKV, /*a_mn=*/0, /*b_mn=*/0);  // Q K^T
 constexpr uint32_t IDESC_O = idesc_bf16_f32(BQ, DH, /*a_mn=*/0, /*b_mn=*/1);   // P V
 constexpr uint32_t O_COL0 = NQT * BKV, TMEM_COLS = 512;   // S_t at t*128, O_t at 256 + t*128
-constexpr float RESCALE_LOG2 = 8.0f;    // move the running maximum only past this growth
+constexpr float RESCALE_LOG2 = 8.0f;
+constexpr int POLY_PAIRS = 2;           // of every 8 probability pairs, this many use the
+                                        // polynomial exp2 on the FMA pipe, the rest MUFU    // move the running maximum only past this growth
 constexpr unsigned kErrWaitAttn = 1u << 6;
 
 struct AttnParams {
@@ -110,59 +118,124 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
   return u;
 }
 
-// One softmax step of a thread's row over a 128-key block already in TMEM
-// columns [tS, tS+128): returns the block's probabilities' sum and leaves
-// the probabilities (bf16 pairs) in columns [tS, tS+64).  MASK: apply the
-// key < T and causal (key <= q) masks.
+// Packed fp32 pairs (sm_100 FFMA2 / FADD2): two lanes of arithmetic per
+// instruction on the softmax's hot loop.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x on the FMA pipe, for part of the probabilities so that the MUFU unit
+// (16 exp2 per clock per SM) is not the only one computing them: range
+// reduction to the nearest integer n (x = n + f, |f| <= 1/2, by the
+// 1.5 * 2^23 rounding constant), a degree-4 polynomial for 2^f whose
+// coefficients were fitted to minimise the relative error on [-1/2, 1/2]
+// (iteratively reweighted least squares; max relative error 2.6e-6), and n
+// added to the exponent field.  x is clamped to >= -126 (the probabilities
+// are bf16, so 2^-126 and 0 are the same to them).  Two lanes per call.
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
+  x2 = f2_pack(fmaxf(x0, -126.0f), fmaxf(x1, -126.0f));
+  const uint64_t magic = f2_pack(12582912.0f, 12582912.0f);
+  const uint64_t t = f2_add(x2, magic);
+  const uint64_t n = f2_add(t, f2_pack(-12582912.0f, -12582912.0f));
+  const uint64_t f = f2_fma(n, f2_pack(-1.0f, -1.0f), x2);
+  uint64_t p = f2_fma(f2_pack(0.009570101276040077f, 0.009570101276040077f), f,
+                      f2_pack(0.05591785907745361f, 0.05591785907745361f));
+  p = f2_fma(p, f, f2_pack(0.240247443318367f, 0.240247443318367f));
+  p = f2_fma(p, f, f2_pack(0.6931217908859253f, 0.6931217908859253f));
+  p = f2_fma(p, f, f2_pack(0.9999992847442627f, 0.9999992847442627f));
+  float p0, p1, t0, t1;
+  f2_unpack(p, p0, p1);
+  f2_unpack(t, t0, t1);
+  return f2_pack(__int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23)),
+                 __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23)));
+}
+
+// One softmax step of a thread's row over a 128-key block in TMEM columns
+// [tS, tS+128), with a single round trip to tensor memory: all 128 scores
+// are loaded at once (one wait), the maximum is taken in registers, the
+// running maximum updated (moved only past RESCALE_LOG2 growth), and the
+// probabilities written back as bf16 pairs into columns [tS, tS+64).
+// Returns the block's probability sum; m and alpha are updated in place.
 template <bool MASK>
-__device__ __forceinline__ float softmax_block(uint32_t tS, float scale, float m_use, int32_t key0,
-                                               int32_t T, int32_t causal, int32_t q, float& mx_out,
-                                               bool max_only) {
-  if (max_only) {
-    float mx = -INFINITY;
+__device__ __forceinline__ float softmax_one_pass(uint32_t tS, float scale, float& m, float& alpha,
+                                                  bool& grow, int32_t key0, int32_t T,
+                                                  int32_t causal, int32_t q) {
+  uint32_t v[128];
 #pragma unroll
-    for (int c = 0; c < BKV / 32; ++c) {
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tS + c * 32, v);
-      tmem_ld_wait();
+  for (int c = 0; c < 4; ++c)
+    tmem_ld_32x32b_x32(tS + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&v[c * 32]));
+  tmem_ld_wait();
+  if (MASK) {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) {
-        float xv = __uint_as_float(v[e]);
-        if (MASK) {
-          const int32_t key = key0 + c * 32 + e;
-          if (key >= T || (causal && key > q)) xv = -INFINITY;
-        }
-        mx = fmaxf(mx, xv);
-      }
+    for (int e = 0; e < 128; ++e) {
+      const int32_t key = key0 + e;
+      if (key >= T || (causal && key > q)) v[e] = __float_as_uint(-INFINITY);
     }
-    mx_out = mx;
-    return 0.0f;
   }
-  float sum = 0.0f;
-  const float neg = -m_use;
-  // chunk c: scores of columns [32c, 32c+32) -> probabilities in columns
-  // [16c, 16c+16), all of which were read by this or an earlier chunk
+  float acc[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-  for (int c = 0; c < BKV / 32; ++c) {
-    uint32_t v[32], pk[16];
-    tmem_ld_32x32b_x32(tS + c * 32, v);
-    tmem_ld_wait();
+  for (int e = 0; e < 128; e += 8) {
+    const int a = (e / 8) & 3;
+    acc[a] = max3(acc[a], __uint_as_float(v[e]), __uint_as_float(v[e + 1]));
+    acc[a] = max3(acc[a], __uint_as_float(v[e + 2]), __uint_as_float(v[e + 3]));
+    acc[a] = max3(acc[a], __uint_as_float(v[e + 4]), __uint_as_float(v[e + 5]));
+    acc[a] = max3(acc[a], __uint_as_float(v[e + 6]), __uint_as_float(v[e + 7]));
+  }
+  const float m_cand = max3(acc[0], acc[1], fmaxf(acc[2], acc[3])) * scale;
+  grow = m_cand > m + RESCALE_LOG2;
+  alpha = grow ? ex2(m - m_cand) : 1.0f;
+  if (grow) m = m_cand;
+  const uint64_t sc2 = f2_pack(scale, scale);
+  const uint64_t nm2 = f2_pack(-m, -m);
+  uint64_t sum2[2] = {f2_pack(0.0f, 0.0f), f2_pack(0.0f, 0.0f)};
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint32_t pk[16];
 #pragma unroll
     for (int e = 0; e < 32; e += 2) {
-      float a0 = ex2(fmaf(__uint_as_float(v[e]), scale, neg));
-      float a1 = ex2(fmaf(__uint_as_float(v[e + 1]), scale, neg));
-      if (MASK) {
-        const int32_t k = key0 + c * 32 + e;
-        if (k >= T || (causal && k > q)) a0 = 0.0f;
-        if (k + 1 >= T || (causal && k + 1 > q)) a1 = 0.0f;
+      const int i = c * 32 + e;
+      const uint64_t xa = f2_fma(f2_pack(__uint_as_float(v[i]), __uint_as_float(v[i + 1])), sc2, nm2);
+      float a0, a1;
+      if ((e / 2) % 8 < POLY_PAIRS) {
+        f2_unpack(exp2_poly2(xa), a0, a1);
+      } else {
+        float x0, x1;
+        f2_unpack(xa, x0, x1);
+        a0 = ex2(x0);
+        a1 = ex2(x1);
       }
-      sum += a0 + a1;
+      sum2[(e / 2) & 1] = f2_add(sum2[(e / 2) & 1], f2_pack(a0, a1));
       pk[e / 2] = pack2(a0, a1);
     }
     tmem_st_32x32b_x16(tS + c * 16, pk);
   }
   tmem_st_wait();
-  return sum;
+  float s0, s1, s2, s3;
+  f2_unpack(sum2[0], s0, s1);
+  f2_unpack(sum2[1], s2, s3);
+  return (s0 + s1) + (s2 + s3);
 }
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -376,18 +449,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const int32_t key0 = j * BKV;
         const bool masked = (key0 + BKV > P.T) || (P.causal && key0 + BKV - 1 > q0);
-        float mx;
-        if (masked)
-          softmax_block<true>(tS, scale, 0.0f, key0, P.T, P.causal, q, mx, true);
-        else
-          softmax_block<false>(tS, scale, 0.0f, key0, P.T, P.causal, q, mx, true);
-        const float m_cand = mx * scale;
-        const bool grow = m_cand > m + RESCALE_LOG2;
-        const float m_use = grow ? m_cand : m;
-        const float alpha = grow ? ex2(m - m_cand) : 1.0f;   // 0 on the first block
+        float alpha;
+        bool grow;
         const float sum = masked
-                              ? softmax_block<true>(tS, scale, m_use, key0, P.T, P.causal, q, mx, false)
-                              : softmax_block<false>(tS, scale, m_use, key0, P.T, P.causal, q, mx, false);
+            ? softmax_one_pass<true>(tS, scale, m, alpha, grow, key0, P.T, P.causal, q)
+            : softmax_one_pass<false>(tS, scale, m, alpha, grow, key0, P.T, P.causal, q);
         if (j > 0 && __any_sync(0xffffffffu, grow)) {
           // O += P V of the previous block has completed (it was issued
           // before this score block, whose commit we waited for)
@@ -403,7 +469,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_st_wait();
         }
         l = l * alpha + sum;
-        m = m_use;
         tc_fence_before();
         mbar_arrive(p_full(t));
         ++sc;

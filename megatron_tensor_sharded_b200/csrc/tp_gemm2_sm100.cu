@@ -35,13 +35,14 @@ using namespace gemm;
 constexpr int PBM = 2 * BM;  // rows of a pair tile
 
 // Pair tile of PBN accumulator columns: each CTA holds PBN/2 columns of B.
-template <int PBN>
+template <int PBN, int EPI_BYTES_ = 0>
 struct PCfg {
+  static constexpr int EPI_BYTES = EPI_BYTES_;   // bulk-store staging (fp32 row layers)
   static constexpr int B_CHUNKS = PBN / 2 / B_BOX_COLS;
   static constexpr int STAGE_BYTES = A_BYTES + B_CHUNKS * B_CHUNK_BYTES;
-  static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - CTRL_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - CTRL_BYTES - EPI_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTRL_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + CTRL_BYTES;
   static constexpr int TMEM_COLS = 2 * PBN <= 256 ? 256 : 512;
   static constexpr uint32_t IDESC = idesc_bf16_f32(PBM, PBN, /*a_mn=*/0, /*b_mn=*/1);
   static_assert(PBN == 128 || PBN == 256, "pair tile width");
@@ -90,18 +91,26 @@ __device__ __forceinline__ void issue_slot_pair(const TcParams& P, const CUtenso
   }
 }
 
+template <int MODE>
+constexpr bool kPairBulkOut = (MODE == kModeRowPartial || MODE == kModeRowSplitK);
+
+template <int MODE, int PBN>
+using PKCfg = PCfg<PBN, kPairBulkOut<MODE> ? EPI_STAGE_BYTES : 0>;
+
 template <int MODE, int PBN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA,
                         const __grid_constant__ CUtensorMap mapB0,
-                        const __grid_constant__ CUtensorMap mapB1, const TcParams P) {
-  using C = PCfg<PBN>;
+                        const __grid_constant__ CUtensorMap mapB1,
+                        const __grid_constant__ CUtensorMap mapC, const TcParams P) {
+  using C = PKCfg<MODE, PBN>;
   constexpr int PSTAGES = C::STAGES;
   constexpr int PSTAGE_BYTES = C::STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* const ctrl = smem_raw + (base - raw) + PSTAGES * PSTAGE_BYTES;
+  const uint32_t epi_stage = base + PSTAGES * PSTAGE_BYTES;   // C::EPI_BYTES of staging
+  uint8_t* const ctrl = smem_raw + (base - raw) + PSTAGES * PSTAGE_BYTES + C::EPI_BYTES;
   uint64_t* const bars = reinterpret_cast<uint64_t*>(ctrl);
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * (2 * PSTAGES + 5));
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -241,12 +250,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * PBN;
-      const int row = tc.m * PBM + static_cast<int>(rank) * BM + quad * 32 + lane;
-      epilogue_tile<MODE, PBN>(P, tc, tacc, row, half, eb);
+      const int row0 = tc.m * PBM + static_cast<int>(rank) * BM + quad * 32;
+      if constexpr (kPairBulkOut<MODE>) {
+        epilogue_tile_bulk<MODE, PBN>(P, tc, tacc, row0, half,
+                                      epi_stage + (warp - 4) * EPI_WARP_STAGE_BYTES, &mapC, lane);
+      } else {
+        epilogue_tile<MODE, PBN>(P, tc, tacc, row0 + lane, half, eb);
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(b), 0));
     }
+    // the staging tiles must be read out before shared memory is released
+    if (kPairBulkOut<MODE> && lane == 0) bulk_wait_all0();
   }
 
   tc_fence_before();
@@ -261,8 +277,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 template <int MODE, int PBN>
 tp_status launch_pair_mode(const LaunchCtx& c, const CUtensorMap& a, const CUtensorMap& b0,
-                           const CUtensorMap& b1, TcParams prm) {
-  constexpr int PSMEM_BYTES = PCfg<PBN>::SMEM_BYTES;
+                           const CUtensorMap& b1, const CUtensorMap& cm, TcParams prm) {
+  constexpr int PSMEM_BYTES = PKCfg<MODE, PBN>::SMEM_BYTES;
   static bool attr_done[64] = {};
   static std::mutex mu;
   {
@@ -297,7 +313,7 @@ tp_status launch_pair_mode(const LaunchCtx& c, const CUtensorMap& a, const CUten
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_allowed() ? 2 : 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<MODE, PBN>, a, b0, b1, prm);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<MODE, PBN>, a, b0, b1, cm, prm);
   note_launch();
   if (e != cudaSuccess) {
     set_error_detail("paired GEMM launch failed: %s", cudaGetErrorString(e));
@@ -309,24 +325,25 @@ tp_status launch_pair_mode(const LaunchCtx& c, const CUtensorMap& a, const CUten
 // Tile space of the pair kernel for a layer: 256-row m-tiles, `pbn`-column
 // (SwiGLU: pbn/2 output columns) n-tiles.
 tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMap& a,
-                         const CUtensorMap& b0, const CUtensorMap& b1, TcParams prm) {
+                         const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& cm,
+                         TcParams prm) {
   const int out_cols = mode == kModeColumnSwiglu ? pbn / 2 : pbn;
   prm.m_tiles = ceil_div(prm.T, PBM);
   prm.n_tiles = ceil_div(prm.n_total, out_cols);
   prm.num_tiles = prm.m_tiles * prm.n_tiles * prm.batches;
   if (pbn == 128) {
     switch (mode) {
-      case kModeColumn: return launch_pair_mode<kModeColumn, 128>(c, a, b0, b1, prm);
-      case kModeColumnSwiglu: return launch_pair_mode<kModeColumnSwiglu, 128>(c, a, b0, b1, prm);
-      case kModeRowPartial: return launch_pair_mode<kModeRowPartial, 128>(c, a, b0, b1, prm);
-      default: return launch_pair_mode<kModeRowSplitK, 128>(c, a, b0, b1, prm);
+      case kModeColumn: return launch_pair_mode<kModeColumn, 128>(c, a, b0, b1, cm, prm);
+      case kModeColumnSwiglu: return launch_pair_mode<kModeColumnSwiglu, 128>(c, a, b0, b1, cm, prm);
+      case kModeRowPartial: return launch_pair_mode<kModeRowPartial, 128>(c, a, b0, b1, cm, prm);
+      default: return launch_pair_mode<kModeRowSplitK, 128>(c, a, b0, b1, cm, prm);
     }
   }
   switch (mode) {
-    case kModeColumn: return launch_pair_mode<kModeColumn, 256>(c, a, b0, b1, prm);
-    case kModeColumnSwiglu: return launch_pair_mode<kModeColumnSwiglu, 256>(c, a, b0, b1, prm);
-    case kModeRowPartial: return launch_pair_mode<kModeRowPartial, 256>(c, a, b0, b1, prm);
-    default: return launch_pair_mode<kModeRowSplitK, 256>(c, a, b0, b1, prm);
+    case kModeColumn: return launch_pair_mode<kModeColumn, 256>(c, a, b0, b1, cm, prm);
+    case kModeColumnSwiglu: return launch_pair_mode<kModeColumnSwiglu, 256>(c, a, b0, b1, cm, prm);
+    case kModeRowPartial: return launch_pair_mode<kModeRowPartial, 256>(c, a, b0, b1, cm, prm);
+    default: return launch_pair_mode<kModeRowSplitK, 256>(c, a, b0, b1, cm, prm);
   }
 }
 

@@ -27,16 +27,22 @@ constexpr int NUM_THREADS = 128 + 32 * NUM_EPI_WARPS;
 constexpr int CTRL_BYTES = 256;
 constexpr int SMEM_LIMIT = 232448;          // max dynamic shared memory per block
 
-template <int BN_>
+// Staging for the bulk-store epilogue of the fp32 row layers: one 32 x 32
+// fp32 tile (4 KiB, a 128-byte swizzle pattern of 32 rows) per epilogue warp.
+constexpr int EPI_WARP_STAGE_BYTES = 32 * 32 * 4;
+constexpr int EPI_STAGE_BYTES = NUM_EPI_WARPS * EPI_WARP_STAGE_BYTES;
+
+template <int BN_, int EPI_BYTES_ = 0>
 struct Cfg {
   static constexpr int BN = BN_;
+  static constexpr int EPI_BYTES = EPI_BYTES_;   // after the stages, before the control block
   static constexpr int B_CHUNKS = BN / B_BOX_COLS;
   static constexpr int B_BYTES = B_CHUNKS * B_CHUNK_BYTES;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - CTRL_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - CTRL_BYTES - EPI_BYTES) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr int TMEM_COLS = 2 * BN <= 128 ? 128 : (2 * BN <= 256 ? 256 : 512);
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + CTRL_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + CTRL_BYTES;
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, /*a_mn=*/0, /*b_mn=*/1);
   static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "tile width");
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
@@ -278,11 +284,63 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& P, const TileCoord
   }
 }
 
+// Bulk-store epilogue of the fp32 row layers (partials [p][T][d], or split-K
+// Z [T][d] + b2): for each 32-column chunk the warp moves its 32 rows from
+// TMEM to registers, writes them into its 4 KiB staging tile in the 128-byte
+// swizzled layout (16-byte chunk c of row r at c ^ (r % 8): no bank
+// conflicts), and one lane issues a TMA tensor store of the 32 x 32 box.
+// Whole cache lines leave the SM instead of 16-byte pieces of 32 rows per
+// instruction.  The box is clipped at T and d by the tensor map.  `row0` is
+// the warp's first output row; the caller waits for the last stores
+// (bulk_wait_all0) before the CTA's shared memory is released.
+template <int MODE, int BN>
+__device__ __forceinline__ void epilogue_tile_bulk(const TcParams& P, const TileCoord& tc,
+                                                   uint32_t tacc, int32_t row0, int half,
+                                                   uint32_t stage, const CUtensorMap* mapC,
+                                                   int lane) {
+  const float* __restrict__ bias = static_cast<const float*>(P.bias);
+#pragma unroll 1
+  for (int q = 0; q < BN / 64; ++q) {
+    const int c0 = half * (BN / 2) + q * 32;
+    const int32_t j0 = tc.n * BN + c0;
+    float bv[32];
+    if (MODE == kModeRowSplitK && bias != nullptr) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) bv[e] = (j0 + e < P.n_total) ? __ldg(bias + j0 + e) : 0.0f;
+    }
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(tacc + c0, v);
+    tmem_ld_wait();
+    if (j0 >= P.n_total) continue;   // warp-uniform
+    if (MODE == kModeRowSplitK && bias != nullptr) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__fadd_rn(__uint_as_float(v[e]), bv[e]));
+    }
+    // the staging tile is free once the previous store has read it
+    if (lane == 0) bulk_wait_read0();
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t addr = stage + lane * 128 + ((c ^ (lane & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[4 * c]),
+                   "r"(v[4 * c + 1]), "r"(v[4 * c + 2]), "r"(v[4 * c + 3])
+                   : "memory");
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(mapC, stage, j0, row0, MODE == kModeRowPartial ? tc.batch : 0);
+      bulk_commit();
+    }
+  }
+}
+
 }  // namespace gemm
 
 // Per-layer GEMM on CTA pairs (tp_gemm2_sm100.cu): 256 x pbn tiles (pbn 128
 // or 256); `mode` is a gemm::Mode; prm's tile space is recomputed.
 tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMap& a,
-                         const CUtensorMap& b0, const CUtensorMap& b1, gemm::TcParams prm);
+                         const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& cm,
+                         gemm::TcParams prm);
 
 }  // namespace tpk

@@ -50,16 +50,25 @@ namespace {
 
 using namespace gemm;
 
+// fp32 row layers store through shared memory with bulk tensor stores
+template <int MODE>
+constexpr bool kBulkOut = (MODE == kModeRowPartial || MODE == kModeRowSplitK);
+
+template <int MODE, int BN>
+using KCfg = Cfg<BN, kBulkOut<MODE> ? EPI_STAGE_BYTES : 0>;
+
 template <int MODE, int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB0,
-                   const __grid_constant__ CUtensorMap mapB1, const TcParams P) {
-  using C = Cfg<BN>;
+                   const __grid_constant__ CUtensorMap mapB1, const __grid_constant__ CUtensorMap mapC,
+                   const TcParams P) {
+  using C = KCfg<MODE, BN>;
   constexpr int STAGES = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;  // swizzle atoms need 1024-byte alignment
-  uint8_t* const ctrl = smem_raw + (base - raw) + STAGES * C::STAGE_BYTES;
+  const uint32_t epi_stage = base + STAGES * C::STAGE_BYTES;   // C::EPI_BYTES of staging
+  uint8_t* const ctrl = smem_raw + (base - raw) + STAGES * C::STAGE_BYTES + C::EPI_BYTES;
   uint64_t* const bars = reinterpret_cast<uint64_t*>(ctrl);
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * (2 * STAGES + 5));
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -93,6 +102,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_map(&mapA);
     tma_prefetch_map(&mapB0);
     if (MODE == kModeColumnSwiglu) tma_prefetch_map(&mapB1);
+    if (kBulkOut<MODE>) tma_prefetch_map(&mapC);
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -203,10 +213,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * BN;
-      epilogue_tile<MODE, BN>(P, tc, tacc, tc.m * BM + quad * 32 + lane, half, eb);
+      if constexpr (kBulkOut<MODE>) {
+        epilogue_tile_bulk<MODE, BN>(P, tc, tacc, tc.m * BM + quad * 32, half,
+                                     epi_stage + (warp - 4) * EPI_WARP_STAGE_BYTES, &mapC, lane);
+      } else {
+        epilogue_tile<MODE, BN>(P, tc, tacc, tc.m * BM + quad * 32 + lane, half, eb);
+      }
       tc_fence_before();
       mbar_arrive(acce_bar(b));
     }
+    // the staging tiles must be read out before shared memory is released
+    if (kBulkOut<MODE> && lane == 0) bulk_wait_all0();
   }
 
   __syncthreads();
@@ -220,8 +237,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 template <int MODE, int BN>
 tp_status launch_mode(const LaunchCtx& c, const CUtensorMap& a, const CUtensorMap& b0,
-                      const CUtensorMap& b1, TcParams prm) {
-  using Cf = Cfg<BN>;
+                      const CUtensorMap& b1, const CUtensorMap& cm, TcParams prm) {
+  using Cf = KCfg<MODE, BN>;
   static bool attr_done[64] = {};
   static std::mutex mu;
   {
@@ -242,7 +259,7 @@ tp_status launch_mode(const LaunchCtx& c, const CUtensorMap& a, const CUtensorMa
   prm.debug_drop = c.debug_drop;
   const int grid = prm.num_tiles < c.num_sms ? prm.num_tiles : c.num_sms;
   const cudaError_t e = launch_pdl(tc_gemm_kernel<MODE, BN>, dim3(grid), dim3(NUM_THREADS),
-                                   Cf::SMEM_BYTES, c.stream, a, b0, b1, prm);
+                                   Cf::SMEM_BYTES, c.stream, a, b0, b1, cm, prm);
   note_launch();
   if (e != cudaSuccess) {
     set_error_detail("tensor-core GEMM launch failed: %s", cudaGetErrorString(e));
@@ -253,18 +270,18 @@ tp_status launch_mode(const LaunchCtx& c, const CUtensorMap& a, const CUtensorMa
 
 template <int MODE>
 tp_status launch_bn(const LaunchCtx& c, int bn, const CUtensorMap& a, const CUtensorMap& b0,
-                    const CUtensorMap& b1, TcParams prm) {
+                    const CUtensorMap& b1, const CUtensorMap& cm, TcParams prm) {
   const int out_cols = MODE == kModeColumnSwiglu ? bn / 2 : bn;
   prm.n_tiles = ceil_div(prm.n_total, out_cols);
   prm.num_tiles = prm.m_tiles * prm.n_tiles * prm.batches;
   switch (bn) {
-    case 256: return launch_mode<MODE, 256>(c, a, b0, b1, prm);
-    case 128: return launch_mode<MODE, 128>(c, a, b0, b1, prm);
+    case 256: return launch_mode<MODE, 256>(c, a, b0, b1, cm, prm);
+    case 128: return launch_mode<MODE, 128>(c, a, b0, b1, cm, prm);
     default: break;
   }
   if constexpr (MODE != kModeColumnSwiglu) {
-    if (bn == 192) return launch_mode<MODE, 192>(c, a, b0, b1, prm);
-    if (bn == 64) return launch_mode<MODE, 64>(c, a, b0, b1, prm);
+    if (bn == 192) return launch_mode<MODE, 192>(c, a, b0, b1, cm, prm);
+    if (bn == 64) return launch_mode<MODE, 64>(c, a, b0, b1, cm, prm);
   }
   set_error_detail("no tile width %d", bn);
   return TP_ERR_UNSUPPORTED;
@@ -297,16 +314,18 @@ tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, co
   prm.out = Y;
   const TileChoice tch = pick_tile(T, k, 1, prm.k_blocks, c.num_sms, swiglu, pair_allowed());
   const int mode = swiglu ? kModeColumnSwiglu : kModeColumn;
-  if (tch.pair) return launch_tc_pair(c, mode, tch.bn, mA, mB0, mB1, prm);
-  if (swiglu) return launch_bn<kModeColumnSwiglu>(c, tch.bn, mA, mB0, mB1, prm);
-  return launch_bn<kModeColumn>(c, tch.bn, mA, mB0, mB1, prm);
+  if (tch.pair) return launch_tc_pair(c, mode, tch.bn, mA, mB0, mB1, mA, prm);
+  if (swiglu) return launch_bn<kModeColumnSwiglu>(c, tch.bn, mA, mB0, mB1, mA, prm);
+  return launch_bn<kModeColumn>(c, tch.bn, mA, mB0, mB1, mA, prm);
 }
 
 tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float* P, int64_t T,
                         int64_t k, int64_t d, int p) {
   const int64_t s = k / p;
-  CUtensorMap mA, mB;
-  if (!make_map_a(&mA, Y, s, T, p) || !make_map_b(&mB, W2, d, k)) return TP_ERR_CUDA;
+  CUtensorMap mA, mB, mC;
+  if (!make_map_a(&mA, Y, s, T, p) || !make_map_b(&mB, W2, d, k) ||
+      !make_map_f32_out(&mC, P, d, T, p))
+    return TP_ERR_CUDA;
   TcParams prm{};
   prm.T = static_cast<int32_t>(T);
   prm.n_total = static_cast<int32_t>(d);
@@ -320,15 +339,17 @@ tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float
   prm.bias = nullptr;
   prm.out = P;
   const TileChoice tch = pick_tile(T, d, p, prm.k_blocks, c.num_sms, false, pair_allowed());
-  if (tch.pair) return launch_tc_pair(c, kModeRowPartial, tch.bn, mA, mB, mB, prm);
-  return launch_bn<kModeRowPartial>(c, tch.bn, mA, mB, mB, prm);
+  if (tch.pair) return launch_tc_pair(c, kModeRowPartial, tch.bn, mA, mB, mB, mC, prm);
+  return launch_bn<kModeRowPartial>(c, tch.bn, mA, mB, mB, mC, prm);
 }
 
 tp_status launch_tc_row_splitk(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
                                float* Z, int64_t T, int64_t k, int64_t d, int p) {
   const int64_t s = k / p;
-  CUtensorMap mA, mB;
-  if (!make_map_a(&mA, Y, s, T, p) || !make_map_b(&mB, W2, d, k)) return TP_ERR_CUDA;
+  CUtensorMap mA, mB, mC;
+  if (!make_map_a(&mA, Y, s, T, p) || !make_map_b(&mB, W2, d, k) ||
+      !make_map_f32_out(&mC, Z, d, T, 1))
+    return TP_ERR_CUDA;
   TcParams prm{};
   prm.T = static_cast<int32_t>(T);
   prm.n_total = static_cast<int32_t>(d);
@@ -342,8 +363,8 @@ tp_status launch_tc_row_splitk(const LaunchCtx& c, const void* Y, const void* W2
   prm.bias = b2;
   prm.out = Z;
   const TileChoice tch = pick_tile(T, d, 1, prm.k_blocks, c.num_sms, false, pair_allowed());
-  if (tch.pair) return launch_tc_pair(c, kModeRowSplitK, tch.bn, mA, mB, mB, prm);
-  return launch_bn<kModeRowSplitK>(c, tch.bn, mA, mB, mB, prm);
+  if (tch.pair) return launch_tc_pair(c, kModeRowSplitK, tch.bn, mA, mB, mB, mC, prm);
+  return launch_bn<kModeRowSplitK>(c, tch.bn, mA, mB, mB, mC, prm);
 }
 
 }  // namespace tpk

@@ -38,6 +38,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 // call, and an encode is pure host work.
 struct MapKey {
   const void* g;
+  int dtype;
   uint64_t dims[3], strides[2];
   uint32_t box[3];
   int rank;
@@ -56,11 +57,12 @@ std::mutex g_map_mu;
 }  // namespace
 
 // bf16 tensor map, 128-byte swizzle, zero fill outside the tensor.
-bool make_map(CUtensorMap* m, const void* gaddr, int rank, const uint64_t* dims,
-              const uint64_t* strides_bytes, const uint32_t* box) {
+bool make_map_typed(CUtensorMap* m, const void* gaddr, int rank, const uint64_t* dims,
+                    const uint64_t* strides_bytes, const uint32_t* box, bool f32) {
   MapKey key;
   memset(&key, 0, sizeof(key));
   key.g = gaddr;
+  key.dtype = f32 ? 1 : 0;
   key.rank = rank;
   for (int i = 0; i < rank; ++i) {
     key.dims[i] = dims[i];
@@ -88,7 +90,7 @@ bool make_map(CUtensorMap* m, const void* gaddr, int rank, const uint64_t* dims,
   }
   for (int i = 0; i < rank - 1; ++i) st[i] = strides_bytes[i];
   const CUresult r =
-      fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
+      fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
          const_cast<void*>(gaddr), d, st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -103,6 +105,22 @@ bool make_map(CUtensorMap* m, const void* gaddr, int rank, const uint64_t* dims,
   e.map = *m;
   e.used = true;
   return true;
+}
+
+bool make_map(CUtensorMap* m, const void* gaddr, int rank, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box) {
+  return make_map_typed(m, gaddr, rank, dims, strides_bytes, box, false);
+}
+
+// fp32 output [batches][rows][cols] for bulk tensor stores of 32 x 32 boxes
+// (one 128-byte swizzle row of fp32 per box row).
+bool make_map_f32_out(CUtensorMap* m, void* g, int64_t cols, int64_t rows, int64_t batches) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
+                            static_cast<uint64_t>(batches)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(cols) * 4,
+                               static_cast<uint64_t>(cols) * rows * 4};
+  const uint32_t box[3] = {32, 32, 1};
+  return make_map_typed(m, g, 3, dims, strides, box, true);
 }
 
 // [rows][inner] bf16 matrices stacked `batches` times, boxes of 128 x 64.
