@@ -95,7 +95,7 @@ template <int MODE>
 constexpr bool kPairBulkOut = (MODE == kModeRowPartial || MODE == kModeRowSplitK);
 
 template <int MODE, int PBN>
-using PKCfg = PCfg<PBN, kPairBulkOut<MODE> ? EPI_STAGE_BYTES : 0>;
+using PKCfg = PCfg<PBN, EPI_STAGE_BYTES>;
 
 template <int MODE, int PBN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -251,18 +251,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * PBN;
       const int row0 = tc.m * PBM + static_cast<int>(rank) * BM + quad * 32;
+      const uint32_t stage_w = epi_stage + (warp - 4) * EPI_WARP_STAGE_BYTES;
       if constexpr (kPairBulkOut<MODE>) {
-        epilogue_tile_bulk<MODE, PBN>(P, tc, tacc, row0, half,
-                                      epi_stage + (warp - 4) * EPI_WARP_STAGE_BYTES, &mapC, lane);
+        epilogue_tile_bulk<MODE, PBN>(P, tc, tacc, row0, half, stage_w, &mapC, lane);
       } else {
-        epilogue_tile<MODE, PBN>(P, tc, tacc, row0 + lane, half, eb);
+        if (P.bulk_out)
+          epilogue_tile_bulk_col<MODE, PBN>(P, tc, tacc, row0, half, eb, stage_w, &mapC, lane);
+        else
+          epilogue_tile<MODE, PBN>(P, tc, tacc, row0 + lane, half, eb);
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(b), 0));
     }
     // the staging tiles must be read out before shared memory is released
-    if (kPairBulkOut<MODE> && lane == 0) bulk_wait_all0();
+    if (lane == 0) bulk_wait_all0();
   }
 
   tc_fence_before();

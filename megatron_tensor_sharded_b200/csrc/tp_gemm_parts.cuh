@@ -62,6 +62,7 @@ struct TcParams {
   int32_t act;
   const void* bias;      // b1 (bf16, column) or b2 (fp32, split-K row); may be null
   void* out;             // Y bf16 [p][T][s] | P fp32 [p][T][d] | Z fp32 [T][d]
+  int32_t bulk_out;      // column layers: 1 = bulk tensor stores through shared memory
   WaitCtl wait;
   int64_t debug_drop;    // slot (in issue order) whose load is skipped; -1 none
 };
@@ -330,6 +331,81 @@ __device__ __forceinline__ void epilogue_tile_bulk(const TcParams& P, const Tile
     __syncwarp();
     if (lane == 0) {
       tma_store_3d(mapC, stage, j0, row0, MODE == kModeRowPartial ? tc.batch : 0);
+      bulk_commit();
+    }
+  }
+}
+
+// Bulk-store epilogue of the column layers (bf16 Y [p][T][s], s % 32 == 0 so
+// a 32-column chunk never straddles two shards): bias + activation as in
+// epilogue_tile, then each warp writes its 32 rows x 32 columns (64 bytes a
+// row) into its staging tile in the 64-byte swizzled layout (16-byte chunk c
+// of row r at c ^ ((r / 2) % 4): conflict-free) and one lane issues a TMA
+// tensor store, clipped at T by the tensor map.
+template <int MODE, int BN>
+__device__ __forceinline__ void epilogue_tile_bulk_col(const TcParams& P, const TileCoord& tc,
+                                                       uint32_t tacc, int32_t row0, int half,
+                                                       const EpiBias<MODE, BN>& eb,
+                                                       uint32_t stage, const CUtensorMap* mapY,
+                                                       int lane) {
+  using S = EpiShape<MODE, BN>;
+  const bool has_bias = P.bias != nullptr;
+#pragma unroll
+  for (int q = 0; q < S::kChunks; ++q) {
+    int32_t j0;
+    float y[32];
+    if constexpr (MODE == kModeColumn) {
+      const int c0 = half * (BN / 2) + q * 32;
+      uint32_t v[32];
+      tmem_ld_32x32b_x32(tacc + c0, v);
+      tmem_ld_wait();
+      j0 = tc.n * BN + c0;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        float bv[8];
+        unpack_bf16x8(eb.v[q * 4 + g], bv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float h = __uint_as_float(v[g * 8 + e]);
+          if (has_bias) h += bv[e];
+          y[g * 8 + e] = act_unary_mufu(P.act, h);
+        }
+      }
+    } else {
+      const int c0 = half * (BN / 4) + q * 32;   // gate column inside the accumulator
+      uint32_t g32[32], u32[32];
+      tmem_ld_32x32b_x32(tacc + c0, g32);
+      tmem_ld_32x32b_x32(tacc + BN / 2 + c0, u32);
+      tmem_ld_wait();
+      j0 = tc.n * (BN / 2) + c0;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        float bv[8];
+        unpack_bf16x8(eb.v[q * 4 + g], bv);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float gate = __uint_as_float(g32[g * 8 + e]);
+          if (has_bias) gate += bv[e];
+          y[g * 8 + e] = silu_mufu(gate) * __uint_as_float(u32[g * 8 + e]);
+        }
+      }
+    }
+    if (j0 >= P.n_total) continue;   // warp-uniform
+    if (lane == 0) bulk_wait_read0();
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t addr = stage + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
+                   "r"(pack_bf16x2(y[8 * c], y[8 * c + 1])), "r"(pack_bf16x2(y[8 * c + 2], y[8 * c + 3])),
+                   "r"(pack_bf16x2(y[8 * c + 4], y[8 * c + 5])), "r"(pack_bf16x2(y[8 * c + 6], y[8 * c + 7]))
+                   : "memory");
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      const int32_t shard = j0 / P.s;
+      tma_store_3d(mapY, stage, j0 - shard * P.s, row0, shard);
       bulk_commit();
     }
   }

@@ -50,12 +50,13 @@ namespace {
 
 using namespace gemm;
 
-// fp32 row layers store through shared memory with bulk tensor stores
+// Epilogues store through shared memory with bulk tensor stores (the column
+// layers when every shard is a whole number of 32-column chunks).
 template <int MODE>
 constexpr bool kBulkOut = (MODE == kModeRowPartial || MODE == kModeRowSplitK);
 
 template <int MODE, int BN>
-using KCfg = Cfg<BN, kBulkOut<MODE> ? EPI_STAGE_BYTES : 0>;
+using KCfg = Cfg<BN, EPI_STAGE_BYTES>;
 
 template <int MODE, int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -102,7 +103,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tma_prefetch_map(&mapA);
     tma_prefetch_map(&mapB0);
     if (MODE == kModeColumnSwiglu) tma_prefetch_map(&mapB1);
-    if (kBulkOut<MODE>) tma_prefetch_map(&mapC);
+    if (kBulkOut<MODE> || P.bulk_out) tma_prefetch_map(&mapC);
   }
   if (warp == 2) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
@@ -213,17 +214,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * BN;
+      const uint32_t stage_w = epi_stage + (warp - 4) * EPI_WARP_STAGE_BYTES;
       if constexpr (kBulkOut<MODE>) {
-        epilogue_tile_bulk<MODE, BN>(P, tc, tacc, tc.m * BM + quad * 32, half,
-                                     epi_stage + (warp - 4) * EPI_WARP_STAGE_BYTES, &mapC, lane);
+        epilogue_tile_bulk<MODE, BN>(P, tc, tacc, tc.m * BM + quad * 32, half, stage_w, &mapC,
+                                     lane);
       } else {
-        epilogue_tile<MODE, BN>(P, tc, tacc, tc.m * BM + quad * 32 + lane, half, eb);
+        if (P.bulk_out)
+          epilogue_tile_bulk_col<MODE, BN>(P, tc, tacc, tc.m * BM + quad * 32, half, eb, stage_w,
+                                           &mapC, lane);
+        else
+          epilogue_tile<MODE, BN>(P, tc, tacc, tc.m * BM + quad * 32 + lane, half, eb);
       }
       tc_fence_before();
       mbar_arrive(acce_bar(b));
     }
     // the staging tiles must be read out before shared memory is released
-    if (kBulkOut<MODE> && lane == 0) bulk_wait_all0();
+    if (lane == 0) bulk_wait_all0();
   }
 
   __syncthreads();
@@ -292,8 +298,11 @@ tp_status launch_bn(const LaunchCtx& c, int bn, const CUtensorMap& a, const CUte
 tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, const void* Wup,
                            const void* b1, void* Y, int64_t T, int64_t d, int64_t k, int p,
                            int act) {
-  CUtensorMap mA, mB0, mB1;
+  CUtensorMap mA, mB0, mB1, mY;
   if (!make_map_a(&mA, X, d, T, 1) || !make_map_b(&mB0, W1, k, d)) return TP_ERR_CUDA;
+  const bool bulk = (k / p) % 32 == 0;
+  if (bulk && !make_map_bf16_out(&mY, Y, k / p, T, p)) return TP_ERR_CUDA;
+  if (!bulk) mY = mA;
   const bool swiglu = (act == kActSwiglu);
   if (swiglu) {
     if (!make_map_b(&mB1, Wup, k, d)) return TP_ERR_CUDA;
@@ -312,11 +321,12 @@ tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, co
   prm.act = act;
   prm.bias = b1;
   prm.out = Y;
+  prm.bulk_out = bulk ? 1 : 0;
   const TileChoice tch = pick_tile(T, k, 1, prm.k_blocks, c.num_sms, swiglu, pair_allowed());
   const int mode = swiglu ? kModeColumnSwiglu : kModeColumn;
-  if (tch.pair) return launch_tc_pair(c, mode, tch.bn, mA, mB0, mB1, mA, prm);
-  if (swiglu) return launch_bn<kModeColumnSwiglu>(c, tch.bn, mA, mB0, mB1, mA, prm);
-  return launch_bn<kModeColumn>(c, tch.bn, mA, mB0, mB1, mA, prm);
+  if (tch.pair) return launch_tc_pair(c, mode, tch.bn, mA, mB0, mB1, mY, prm);
+  if (swiglu) return launch_bn<kModeColumnSwiglu>(c, tch.bn, mA, mB0, mB1, mY, prm);
+  return launch_bn<kModeColumn>(c, tch.bn, mA, mB0, mB1, mY, prm);
 }
 
 tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float* P, int64_t T,

@@ -58,11 +58,12 @@ std::mutex g_map_mu;
 
 // bf16 tensor map, 128-byte swizzle, zero fill outside the tensor.
 bool make_map_typed(CUtensorMap* m, const void* gaddr, int rank, const uint64_t* dims,
-                    const uint64_t* strides_bytes, const uint32_t* box, bool f32) {
+                    const uint64_t* strides_bytes, const uint32_t* box, bool f32,
+                    bool swizzle64 = false) {
   MapKey key;
   memset(&key, 0, sizeof(key));
   key.g = gaddr;
-  key.dtype = f32 ? 1 : 0;
+  key.dtype = (f32 ? 1 : 0) | (swizzle64 ? 2 : 0);
   key.rank = rank;
   for (int i = 0; i < rank; ++i) {
     key.dims[i] = dims[i];
@@ -92,7 +93,8 @@ bool make_map_typed(CUtensorMap* m, const void* gaddr, int rank, const uint64_t*
   const CUresult r =
       fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, static_cast<cuuint32_t>(rank),
          const_cast<void*>(gaddr), d, st, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         swizzle64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_error_detail("cuTensorMapEncodeTiled failed (%d)", static_cast<int>(r));
@@ -121,6 +123,17 @@ bool make_map_f32_out(CUtensorMap* m, void* g, int64_t cols, int64_t rows, int64
                                static_cast<uint64_t>(cols) * rows * 4};
   const uint32_t box[3] = {32, 32, 1};
   return make_map_typed(m, g, 3, dims, strides, box, true);
+}
+
+// bf16 output [batches][rows][cols] for bulk tensor stores of 32 x 32 boxes
+// (64-byte rows, 64-byte swizzle).
+bool make_map_bf16_out(CUtensorMap* m, void* g, int64_t cols, int64_t rows, int64_t batches) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
+                            static_cast<uint64_t>(batches)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(cols) * 2,
+                               static_cast<uint64_t>(cols) * rows * 2};
+  const uint32_t box[3] = {32, 32, 1};
+  return make_map_typed(m, g, 3, dims, strides, box, false, true);
 }
 
 // [rows][inner] bf16 matrices stacked `batches` times, boxes of 128 x 64.
