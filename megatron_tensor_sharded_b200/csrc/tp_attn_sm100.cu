@@ -105,6 +105,15 @@ __device__ __forceinline__ Unit decode_unit(const AttnParams& P, int32_t u) {
   return x;
 }
 
+// The CTA's r-th unit: rounds of gridDim.x units, alternately walked
+// forwards and backwards across the CTAs ("snake" order), so that with the
+// longest causal units first every CTA gets a similar total (the plain
+// round-robin left one CTA with 1.3x the average on the 4-shard shape).
+__device__ __forceinline__ int32_t unit_of(int32_t r) {
+  const int32_t g = static_cast<int32_t>(gridDim.x), b = static_cast<int32_t>(blockIdx.x);
+  return r * g + ((r & 1) ? g - 1 - b : b);
+}
+
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -304,7 +313,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int64_t issued = 0, last_q = -1;
       int32_t lu = 0;
       bool ok = true;
-      for (int32_t u = blockIdx.x; ok && u < P.num_units; u += gridDim.x, ++lu) {
+      for (int32_t u = unit_of(0); ok && u < P.num_units; u = unit_of(++lu)) {
         const Unit x = decode_unit(P, u);
         if (!wait_bounded(q_empty, (lu & 1) ^ 1u, abort_flag, P.wait, kErrWaitAttn)) break;
         const int ntiles = x.nkb1 > 0 ? 2 : 1;
@@ -368,7 +377,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         tc_commit(s_full(t));
       };
-      for (int32_t u = blockIdx.x; ok && u < P.num_units; u += gridDim.x, ++lu) {
+      for (int32_t u = unit_of(0); ok && u < P.num_units; u = unit_of(++lu)) {
         const Unit x = decode_unit(P, u);
         if (!wait_bounded(q_full, lu & 1, abort_flag, P.wait, kErrWaitAttn)) break;
         const uint32_t n0 = kv_n;
@@ -434,7 +443,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tO = tmem_base + lane_off + O_COL0 + t * DH;
     const float scale = P.scale_log2;
     uint32_t sc = 0, uc = 0;
-    for (int32_t u = blockIdx.x; u < P.num_units; u += gridDim.x) {
+    int32_t ru = 0;
+    for (int32_t u = unit_of(0); u < P.num_units; u = unit_of(++ru)) {
       const Unit x = decode_unit(P, u);
       const int32_t nkb = x.nkb(t);
       if (nkb == 0) continue;

@@ -15,6 +15,7 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cstdint>
 #include <cstring>
 
@@ -50,12 +51,13 @@ template <int NV>
 __global__ void __launch_bounds__(kThreads) row_fold_ln_kernel(
     const float* __restrict__ part, int p, int64_t part_stride, const float* __restrict__ bias,
     const float* R, float* H, const float* __restrict__ gamma, const float* __restrict__ beta,
-    __nv_bfloat16* __restrict__ Y, int64_t d, float eps) {
+    __nv_bfloat16* __restrict__ Y, int64_t T, int64_t d, float eps) {
   __shared__ float red[kThreads / 32];
   pdl_wait();
   pdl_launch_dependents();
-  const int64_t row = blockIdx.x;
   const int64_t d4 = d / 4;
+  // persistent: a fixed grid of resident CTAs walks the rows
+  for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
   const int64_t base = row * d;
   float4 h[NV];
 #pragma unroll
@@ -78,7 +80,7 @@ __global__ void __launch_bounds__(kThreads) row_fold_ln_kernel(
       h[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
-  if (Y == nullptr) return;
+  if (Y == nullptr) continue;
   float s = 0.0f;
 #pragma unroll
   for (int k = 0; k < NV; ++k) s += (h[k].x + h[k].y) + (h[k].z + h[k].w);
@@ -109,6 +111,7 @@ __global__ void __launch_bounds__(kThreads) row_fold_ln_kernel(
       memcpy(&u.y, &hi, 4);
       reinterpret_cast<uint2*>(Y + base)[c] = u;
     }
+  }
   }
 }
 
@@ -190,20 +193,34 @@ cudaError_t launch_row_fold_ln(const LaunchCtx& c, const float* P, int p, const 
   if (T == 0) return cudaSuccess;
   const int64_t d4 = d / 4;
   const int nv = static_cast<int>((d4 + kThreads - 1) / kThreads);
-  const dim3 g(static_cast<unsigned>(T)), b(kThreads);
   __nv_bfloat16* y = static_cast<__nv_bfloat16*>(Y);
   const int64_t ps = T * d;
+  // a persistent grid: as many CTAs as fit on the SMs at once (by the
+  // kernel's register use), each walking rows blockIdx.x, + gridDim.x, ...
+  auto go = [&](auto kern) {
+    static std::atomic<int> cached{0};   // per kernel instantiation
+    int per_sm = cached.load(std::memory_order_relaxed);
+    if (per_sm == 0) {
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess ||
+          per_sm < 1)
+        per_sm = 1;
+      cached.store(per_sm, std::memory_order_relaxed);
+    }
+    const int64_t resident = static_cast<int64_t>(c.num_sms) * per_sm;
+    const dim3 g(static_cast<unsigned>(T < resident ? T : resident)), b(kThreads);
+    return launch_pdl(kern, g, b, 0, c.stream, P, p, ps, bias, R, H, gamma, beta, y, T, d, eps);
+  };
   cudaError_t e;
   if (nv <= 1)
-    e = launch_pdl(row_fold_ln_kernel<1>, g, b, 0, c.stream, P, p, ps, bias, R, H, gamma, beta, y, d, eps);
+    e = go(row_fold_ln_kernel<1>);
   else if (nv <= 2)
-    e = launch_pdl(row_fold_ln_kernel<2>, g, b, 0, c.stream, P, p, ps, bias, R, H, gamma, beta, y, d, eps);
+    e = go(row_fold_ln_kernel<2>);
   else if (nv <= 4)
-    e = launch_pdl(row_fold_ln_kernel<4>, g, b, 0, c.stream, P, p, ps, bias, R, H, gamma, beta, y, d, eps);
+    e = go(row_fold_ln_kernel<4>);
   else if (nv <= 8)
-    e = launch_pdl(row_fold_ln_kernel<8>, g, b, 0, c.stream, P, p, ps, bias, R, H, gamma, beta, y, d, eps);
+    e = go(row_fold_ln_kernel<8>);
   else
-    e = launch_pdl(row_fold_ln_kernel<kMaxV>, g, b, 0, c.stream, P, p, ps, bias, R, H, gamma, beta, y, d, eps);
+    e = go(row_fold_ln_kernel<kMaxV>);
   note_launch();
   return e;
 }
