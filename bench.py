@@ -639,6 +639,34 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
     roof["intensity_flop_per_byte"] = intensity
     roof["ridge_flop_per_byte"] = ridge
 
+    # The dominant kernel (largest share of the separately timed layers):
+    # algorithmic FLOPs (or bytes) per launch over its CUDA-event duration.
+    if kernels is not None:
+        cand = {
+            "column": (column_flops(w), column_bytes(w), kernels["column"],
+                       "tc_gemm_kernel/tc_gemm_pair_kernel, column layer (all shards)"),
+            "row": (row_flops(w), row_bytes(w), kernels["row"],
+                    "tc_gemm_kernel/tc_gemm_pair_kernel, row layer to partials (all shards)"),
+            "reduce": (0, reduce_bytes(w), kernels["reduce"], "reduce_vec_kernel, fixed-order fold"),
+        }
+        name = max(cand, key=lambda n: cand[n][2])
+        fl_k, by_k, ms_k, desc = cand[name]
+        if w.dtype == "bf16" and fl_k > 0 and fl_k / by_k >= ridge:
+            ach = fl_k / (ms_k * 1e-3) / 1e12
+            kroof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                     "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                     "flops_per_launch": fl_k, "peak_source": f"{peak_src} bf16 dense (burst)"}
+        else:
+            ach = by_k / (ms_k * 1e-3) / 1e9
+            kroof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": ach / peaks["hbm_gbs"], "bytes_per_launch": by_k,
+                     "peak_source": f"{peak_src} hbm copy"}
+        kroof.update({"traffic": ncu_traffic(f"{w.name}/{name}"), "kernel": f"{name}: {desc}",
+                      "duration": "average launch duration, CUDA events on the launching stream "
+                                  "around the layer's call inside a replayed graph",
+                      "launch_ms": ms_k, "step": roof})
+        roof = kroof
+
     breakdown = None
     if kernels is not None:
         def tfl(f, ms):
@@ -864,6 +892,18 @@ def run_tp_attn(a, w: WL.AttnWorkload, rank: int, world: int, local_rank: int):
             "duration": "block step time (graph replay, CUDA events on the launching stream)",
             "peak_source": f"{peak_src} bf16 dense (burst)",
             "flops_per_step": fl}
+    if breakdown is not None:
+        # the attention kernel, the row's own hot kernel: FLOPs per launch over
+        # its event-timed duration
+        att_ms = breakdown["attention"]["ms"]
+        ach = fl["attention"] / (att_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
+                "flops_per_launch": fl["attention"], "traffic": ncu_traffic(f"{w.name}/attention"),
+                "kernel": "tc_attn_kernel (all shards and heads, one launch)",
+                "duration": "average launch duration, CUDA events on the launching stream around "
+                            "tp_attention_heads inside a replayed graph",
+                "launch_ms": att_ms, "peak_source": f"{peak_src} bf16 dense (burst)", "step": roof}
     line = {
         "metric": ATTN_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -1028,6 +1068,20 @@ def run_tp_block(a, w: WL.BlockWorkload, rank: int, world: int, local_rank: int)
                       "fold+residual+LN -> MLP GEMMs -> fold+residual",
             "duration": "block step time (graph replay, CUDA events on the launching stream)",
             "peak_source": f"{peak_src} bf16 dense (burst)", "flops_per_step": fl}
+    if breakdown is not None:
+        # the dominant single kernel launch (the Q, K, V GEMMs are three launches)
+        per_launch = {n: breakdown[n]["ms"] / (3 if n == "qkv" else 1)
+                      for n in ("qkv", "attention", "out_proj", "mlp_column", "mlp_row")}
+        name = max(per_launch, key=per_launch.get)
+        fl_k = flops_of[name] / (3 if name == "qkv" else 1)
+        ach = fl_k / (per_launch[name] * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"], "flops_per_launch": fl_k,
+                "traffic": ncu_traffic(f"{w.name}/{name}"), "kernel": name,
+                "duration": "average launch duration, CUDA events on the launching stream around "
+                            "the call inside a replayed graph",
+                "launch_ms": per_launch[name], "peak_source": f"{peak_src} bf16 dense (burst)",
+                "step": roof}
     line = {
         "metric": BLOCK_METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
