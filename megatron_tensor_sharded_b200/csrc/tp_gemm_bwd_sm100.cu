@@ -62,6 +62,7 @@ struct GParams {
   int32_t a_batched, b_batched; // operand batch coordinate = shard (else 0)
   int32_t b_koff;               // K-major B: K coordinate offset per shard (W1's column blocks)
   int32_t act;
+  int32_t bulk_out;             // fp32 epilogue through shared memory + TMA tensor stores
   // epilogue
   void* out[2];                 // per half
   int64_t out_shard_stride;     // elements
@@ -125,6 +126,40 @@ __device__ __forceinline__ void store_bf16x8_at(__nv_bfloat16* dst, const float 
   *reinterpret_cast<uint4*>(dst) = pk;
 }
 
+// fp32 outputs through shared memory: per 32-column chunk the warp's 32 rows
+// go into its 4 KiB staging tile (128-byte swizzle) and one lane issues a TMA
+// tensor store of the box at (column, row, shard) of the half's output map,
+// which clips it at the shard's extents.
+template <int BN>
+__device__ __forceinline__ void epilogue_f32_bulk(const GParams& P, const GTile& g, uint32_t tacc,
+                                                  int32_t row0, int half, uint32_t stage,
+                                                  const CUtensorMap* mapC, int lane) {
+#pragma unroll 1
+  for (int q = 0; q < BN / 64; ++q) {
+    const int c0 = half * (BN / 2) + q * 32;
+    const int32_t j0 = g.n * BN + c0;
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(tacc + c0, v);
+    tmem_ld_wait();
+    if (j0 >= P.N) continue;   // warp-uniform
+    if (lane == 0) bulk_wait_read0();
+    __syncwarp();
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t addr = stage + lane * 128 + ((c ^ (lane & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[4 * c]),
+                   "r"(v[4 * c + 1]), "r"(v[4 * c + 2]), "r"(v[4 * c + 3])
+                   : "memory");
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(mapC, stage, j0, row0, g.shard);
+      bulk_commit();
+    }
+  }
+}
+
 template <int EPI, int BN>
 __device__ __forceinline__ void epilogue(const GParams& P, const GTile& g, uint32_t tacc, int row,
                                          int half) {
@@ -183,18 +218,23 @@ __device__ __forceinline__ void epilogue(const GParams& P, const GTile& g, uint3
   }
 }
 
+template <int EPI, int BN>
+using BCfg = Cfg<BN, EPI == kEpiF32 ? EPI_STAGE_BYTES : 0>;
+
 template <int AMN, int BMN, int EPI, int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_bwd_kernel(const __grid_constant__ CUtensorMap mapA0, const __grid_constant__ CUtensorMap mapA1,
                        const __grid_constant__ CUtensorMap mapB0, const __grid_constant__ CUtensorMap mapB1,
+                       const __grid_constant__ CUtensorMap mapC0, const __grid_constant__ CUtensorMap mapC1,
                        const GParams P) {
-  using C = Cfg<BN>;
+  using C = BCfg<EPI, BN>;
   constexpr int STAGES = C::STAGES;
   constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, AMN, BMN);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
-  uint8_t* const ctrl = smem_raw + (base - raw) + STAGES * C::STAGE_BYTES;
+  const uint32_t epi_stage = base + STAGES * C::STAGE_BYTES;   // C::EPI_BYTES of staging
+  uint8_t* const ctrl = smem_raw + (base - raw) + STAGES * C::STAGE_BYTES + C::EPI_BYTES;
   uint64_t* const bars = reinterpret_cast<uint64_t*>(ctrl);
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * (2 * STAGES + 5));
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -324,10 +364,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * BN;
-      epilogue<EPI, BN>(P, g, tacc, g.m * BM + quad * 32 + lane, half);
+      if (EPI == kEpiF32 && P.bulk_out)
+        epilogue_f32_bulk<BN>(P, g, tacc, g.m * BM + quad * 32, half,
+                              epi_stage + (warp - 4) * EPI_WARP_STAGE_BYTES,
+                              g.half > 0 ? &mapC1 : &mapC0, lane);
+      else
+        epilogue<EPI, BN>(P, g, tacc, g.m * BM + quad * 32 + lane, half);
       tc_fence_before();
       mbar_arrive(acce_bar(b));
     }
+    if (lane == 0) bulk_wait_all0();   // staging read out before shared memory is released
   }
 
   __syncthreads();
@@ -339,7 +385,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 template <int AMN, int BMN, int EPI, int BN>
 tp_status launch_g(const LaunchCtx& c, const CUtensorMap* maps, GParams prm) {
-  using Cf = Cfg<BN>;
+  using Cf = BCfg<EPI, BN>;
   static bool attr_done[64] = {};
   static std::mutex mu;
   {
@@ -364,7 +410,7 @@ tp_status launch_g(const LaunchCtx& c, const CUtensorMap* maps, GParams prm) {
   const int grid = prm.num_tiles < c.num_sms ? prm.num_tiles : c.num_sms;
   const cudaError_t e = launch_pdl(tc_gemm_bwd_kernel<AMN, BMN, EPI, BN>, dim3(grid),
                                    dim3(NUM_THREADS), Cf::SMEM_BYTES, c.stream, maps[0], maps[1],
-                                   maps[2], maps[3], prm);
+                                   maps[2], maps[3], maps[4], maps[5], prm);
   note_launch();
   if (e != cudaSuccess) {
     set_error_detail("backward GEMM launch failed: %s", cudaGetErrorString(e));
@@ -430,12 +476,13 @@ tp_status launch_bwd_act_grad(const LaunchCtx& c, const void* dZ, const void* W2
   prm.aux0 = H;
   prm.aux1 = Hup;
   const int bn = pick_bn(T, s, p, prm.k_blocks, c.num_sms);
-  CUtensorMap maps[4];
+  CUtensorMap maps[6];
   // A = dZ [T][d] K-major; B = W2 rows of shard i: [p][s][d] K-major (N rows)
   if (!map3(&maps[0], dZ, d, T, 1, d, 0, BM) || !map3(&maps[2], W2, d, s, p, d, s * d, bn))
     return TP_ERR_CUDA;
   maps[1] = maps[0];
   maps[3] = maps[2];
+  maps[4] = maps[5] = maps[0];   // bf16 outputs: per-thread stores
   if (act == kActSwiglu) {
     if (bn == 256) return launch_g<0, 0, kEpiSwigluGrad, 256>(c, maps, prm);
     if (bn == 128) return launch_g<0, 0, kEpiSwigluGrad, 128>(c, maps, prm);
@@ -465,7 +512,7 @@ tp_status launch_bwd_dx_partials(const LaunchCtx& c, const void* dH, const void*
   prm.out_shard_stride = T * d;
   prm.ldc = d;
   const int bn = pick_bn(T, d, p, prm.k_blocks, c.num_sms);
-  CUtensorMap maps[4];
+  CUtensorMap maps[6];
   // A = dH [p][T][s] K-major; B = W1 [d][k] K-major (inner k, outer d = N
   // rows), shard i's block at K offset i s
   if (!map3(&maps[0], dH, s, T, p, s, T * s, BM) || !map3(&maps[2], W1, k, d, 1, k, 0, bn))
@@ -477,6 +524,9 @@ tp_status launch_bwd_dx_partials(const LaunchCtx& c, const void* dH, const void*
     maps[1] = maps[0];
     maps[3] = maps[2];
   }
+  if (!make_map_f32_out(&maps[4], P, d, T, p)) return TP_ERR_CUDA;
+  maps[5] = maps[4];
+  prm.bulk_out = 1;
   if (bn == 256) return launch_g<0, 0, kEpiF32, 256>(c, maps, prm);
   if (bn == 128) return launch_g<0, 0, kEpiF32, 128>(c, maps, prm);
   return launch_g<0, 0, kEpiF32, 64>(c, maps, prm);
@@ -496,7 +546,7 @@ tp_status launch_bwd_dw1(const LaunchCtx& c, const void* X, const void* dH, cons
   prm.out_shard_stride = s;
   prm.ldc = k;
   const int bn = pick_bn(d, s, p * prm.halves, prm.k_blocks, c.num_sms);
-  CUtensorMap maps[4];
+  CUtensorMap maps[6];
   // A = X^T: M-major view of X [T][d] (inner d = M, outer T = K);
   // B = dH [p][T][s] N-major (inner s = N, outer T = K)
   if (!map3(&maps[0], X, d, T, 1, d, 0, BK) || !map3(&maps[2], dH, s, T, p, s, T * s, BK))
@@ -507,6 +557,13 @@ tp_status launch_bwd_dw1(const LaunchCtx& c, const void* X, const void* dH, cons
   } else {
     maps[3] = maps[2];
   }
+  // dW1's column block i: (s columns, d rows, shard i at a column offset of
+  // i s); the bulk path needs the driver to accept the interleaved batch
+  // stride, else the per-thread epilogue writes it
+  prm.bulk_out = make_map_f32_strided(&maps[4], dW1, s, d, p, k, s) ? 1 : 0;
+  if (prm.bulk_out && two) prm.bulk_out = make_map_f32_strided(&maps[5], dWup, s, d, p, k, s) ? 1 : 0;
+  if (!prm.bulk_out) maps[4] = maps[0];
+  if (!two || !prm.bulk_out) maps[5] = maps[4];
   if (bn == 256) return launch_g<1, 1, kEpiF32, 256>(c, maps, prm);
   if (bn == 128) return launch_g<1, 1, kEpiF32, 128>(c, maps, prm);
   return launch_g<1, 1, kEpiF32, 64>(c, maps, prm);
@@ -524,12 +581,16 @@ tp_status launch_bwd_dw2(const LaunchCtx& c, const void* Y, const void* dZ, floa
   prm.out_shard_stride = s * d;
   prm.ldc = d;
   const int bn = pick_bn(s, d, p, prm.k_blocks, c.num_sms);
-  CUtensorMap maps[4];
+  CUtensorMap maps[6];
   // A = Y_i^T: M-major view of Y [p][T][s]; B = dZ [T][d] N-major
   if (!map3(&maps[0], Y, s, T, p, s, T * s, BK) || !map3(&maps[2], dZ, d, T, 1, d, 0, BK))
     return TP_ERR_CUDA;
   maps[1] = maps[0];
   maps[3] = maps[2];
+  // dW2's row block i as shard i of a [p][s][d] tensor
+  if (!make_map_f32_out(&maps[4], dW2, d, s, p)) return TP_ERR_CUDA;
+  maps[5] = maps[4];
+  prm.bulk_out = 1;
   if (bn == 256) return launch_g<1, 1, kEpiF32, 256>(c, maps, prm);
   if (bn == 128) return launch_g<1, 1, kEpiF32, 128>(c, maps, prm);
   return launch_g<1, 1, kEpiF32, 64>(c, maps, prm);

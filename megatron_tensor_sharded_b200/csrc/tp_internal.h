@@ -55,6 +55,8 @@ bool make_map(CUtensorMap* m, const void* gaddr, int rank, const uint64_t* dims,
 bool make_map_a(CUtensorMap* m, const void* g, int64_t inner, int64_t rows, int64_t batches);
 bool make_map_f32_out(CUtensorMap* m, void* g, int64_t cols, int64_t rows, int64_t batches);
 bool make_map_bf16_out(CUtensorMap* m, void* g, int64_t cols, int64_t rows, int64_t batches);
+bool make_map_f32_strided(CUtensorMap* m, void* g, int64_t cols, int64_t rows, int64_t batches,
+                          int64_t row_stride, int64_t batch_stride);
 // [rows][cols] bf16 weight, N-contiguous, boxes of 64 rows x 64 columns (N-major B tiles).
 bool make_map_b(CUtensorMap* m, const void* g, int64_t cols, int64_t rows);
 // Tile width (accumulator columns) and whether to use CTA-pair tiles

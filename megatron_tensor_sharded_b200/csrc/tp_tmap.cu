@@ -125,6 +125,19 @@ bool make_map_f32_out(CUtensorMap* m, void* g, int64_t cols, int64_t rows, int64
   return make_map_typed(m, g, 3, dims, strides, box, true);
 }
 
+// fp32 output with explicit row and batch strides (elements), boxes 32 x 32
+// (a shard's column block inside a wider matrix: batch stride = the block's
+// width); false if the driver does not accept the layout.
+bool make_map_f32_strided(CUtensorMap* m, void* g, int64_t cols, int64_t rows, int64_t batches,
+                          int64_t row_stride, int64_t batch_stride) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows),
+                            static_cast<uint64_t>(batches)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(row_stride) * 4,
+                               static_cast<uint64_t>(batch_stride) * 4};
+  const uint32_t box[3] = {32, 32, 1};
+  return make_map_typed(m, g, 3, dims, strides, box, true);
+}
+
 // bf16 output [batches][rows][cols] for bulk tensor stores of 32 x 32 boxes
 // (64-byte rows, 64-byte swizzle).
 bool make_map_bf16_out(CUtensorMap* m, void* g, int64_t cols, int64_t rows, int64_t batches) {
