@@ -487,6 +487,8 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
     flags = tp.TP_FLAG_SPLITK_FUSED if a.mode == "splitk" else tp.TP_FLAG_NONE
     if a.mode == "fused":
         flags = tp.TP_FLAG_FUSED_LAUNCH
+    if a.mode == "fold":
+        flags = tp.TP_FLAG_ROW_FOLD
     nbytes = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, w.p, dtype, act, flags)
     ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
 
@@ -613,6 +615,8 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
     peaks, peak_src = load_peaks()
     value = whole_job_value(w.gemm_flops(), world, ms_step) / 1e12
     kernel_name = {"partials": "tp_mlp_block: column GEMM -> row GEMM -> fixed-order fold (PDL-chained)",
+                   "fold": "tp_mlp_block row-fold: column GEMM -> row GEMM folding the p partials "
+                           "in its epilogue (bit-identical to partials + fold)",
                    "splitk": "tp_mlp_block split-K: column GEMM -> row GEMM accumulating all shards",
                    "fused": "tc_block_kernel (both GEMM layers, one launch) -> fold"}[a.mode]
     # Roofline side: tensor peak unless the step's arithmetic intensity
@@ -1291,7 +1295,7 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["tp", "reference"], default="tp")
     ap.add_argument("--workload", choices=sorted(WL.WORKLOADS) + sorted(WL.ATTN_WORKLOADS)
                     + sorted(WL.BLOCK_WORKLOADS), default="gpt2")
-    ap.add_argument("--mode", choices=["partials", "splitk", "fused", "backward"],
+    ap.add_argument("--mode", choices=["partials", "fold", "splitk", "fused", "backward"],
                     default="partials")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of graph replay")

@@ -83,6 +83,16 @@ typedef enum {
  * launch per layer.  Same bits either way; the default per-layer launches
  * were faster on every measured shape (they use CTA-pair tiles). */
 #define TP_FLAG_FUSED_LAUNCH 2
+/* bf16: the row-parallel layer computes the p partials of each output tile
+ * one after another in tensor memory and folds them in its epilogue in shard
+ * order (then + b2), so the partials never reach HBM and no separate
+ * reduction runs.  Bit-identical to the default (partials + fixed-order
+ * fold).  Needs s % 64 == 0; combines with no other flag; the workspace
+ * holds only the hidden shards (no p * T * d * 4 bytes of partials).  Slower
+ * than the default on every measured shape: its 128-column single-CTA tiles
+ * (the accumulator ring and the running sum share TMEM) read twice the
+ * operand bytes per FLOP of the default row layer's CTA-pair tiles. */
+#define TP_FLAG_ROW_FOLD 4
 
 /*
  * Column-parallel linear + activation, all p shards in one launch.

@@ -19,7 +19,7 @@ import os
 
 __all__ = [
     "TPError", "TP_F32", "TP_BF16", "TP_ACT_GELU_TANH", "TP_ACT_SWIGLU", "TP_ACT_IDENTITY",
-    "TP_ACT_RELU", "TP_FLAG_NONE", "TP_FLAG_SPLITK_FUSED", "TP_FLAG_FUSED_LAUNCH", "STATUS", "ACT", "DTYPE",
+    "TP_ACT_RELU", "TP_FLAG_NONE", "TP_FLAG_SPLITK_FUSED", "TP_FLAG_FUSED_LAUNCH", "TP_FLAG_ROW_FOLD", "STATUS", "ACT", "DTYPE",
     "tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
     "tp_mlp_block_noalloc", "tp_attention_heads", "tp_attn_block",
               "tp_layer_norm", "tp_reduce_partials_residual", "tp_transformer_block",
@@ -36,7 +36,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtpmlp.so
 
 TP_F32, TP_BF16 = 0, 1
 TP_ACT_GELU_TANH, TP_ACT_SWIGLU, TP_ACT_IDENTITY, TP_ACT_RELU = 0, 1, 2, 3
-TP_FLAG_NONE, TP_FLAG_SPLITK_FUSED, TP_FLAG_FUSED_LAUNCH = 0, 1, 2
+TP_FLAG_NONE, TP_FLAG_SPLITK_FUSED, TP_FLAG_FUSED_LAUNCH, TP_FLAG_ROW_FOLD = 0, 1, 2, 4
 DTYPE = {"f32": TP_F32, "bf16": TP_BF16}
 ACT = {"gelu_tanh": TP_ACT_GELU_TANH, "swiglu": TP_ACT_SWIGLU, "identity": TP_ACT_IDENTITY,
        "relu": TP_ACT_RELU}

@@ -130,7 +130,7 @@ size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 size_t workspace_bytes(int64_t T, int64_t d, int64_t k, int p, int dtype, int flags) {
   const size_t esize = dtype == TP_BF16 ? 2 : 4;
   size_t bytes = align256(static_cast<size_t>(T) * static_cast<size_t>(k) * esize);
-  if (!(flags & TP_FLAG_SPLITK_FUSED))
+  if (!(flags & (TP_FLAG_SPLITK_FUSED | TP_FLAG_ROW_FOLD)))
     bytes += align256(static_cast<size_t>(p) * static_cast<size_t>(T) * static_cast<size_t>(d) * 4);
   return bytes + block_counter_bytes(T, d);
 }
@@ -387,9 +387,14 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
   g_detail[0] = 0;
   TP_TRY(check_shape(T, d, k, p, dtype));
   TP_TRY(check_act(act, W_up));
-  if (flags & ~(TP_FLAG_SPLITK_FUSED | TP_FLAG_FUSED_LAUNCH))
+  if (flags & ~(TP_FLAG_SPLITK_FUSED | TP_FLAG_FUSED_LAUNCH | TP_FLAG_ROW_FOLD))
     return fail(TP_ERR_INVALID_ARG, "flags 0x%x", flags);
   const bool splitk = (flags & TP_FLAG_SPLITK_FUSED) != 0;
+  const bool row_fold = (flags & TP_FLAG_ROW_FOLD) != 0;
+  if (row_fold && (flags & (TP_FLAG_SPLITK_FUSED | TP_FLAG_FUSED_LAUNCH)))
+    return fail(TP_ERR_INVALID_ARG, "TP_FLAG_ROW_FOLD combines with no other flag");
+  if (row_fold && (dtype != TP_BF16 || (k / p) % 64 != 0))
+    return fail(TP_ERR_UNSUPPORTED, "the epilogue fold needs bf16 and k/p %% 64 == 0");
   if (splitk && dtype == TP_BF16 && (k / p) % 64 != 0)
     return fail(TP_ERR_UNSUPPORTED, "split-K over shards needs k/p %% 64 == 0 for bf16");
   if (T == 0) return TP_OK;
@@ -412,7 +417,7 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
   void* Y = ws;
   const size_t esize = dtype == TP_BF16 ? 2 : 4;
   const size_t y_bytes = align256(static_cast<size_t>(T) * k * esize);
-  float* P = splitk ? nullptr : reinterpret_cast<float*>(ws + y_bytes);
+  float* P = (splitk || row_fold) ? nullptr : reinterpret_cast<float*>(ws + y_bytes);
   if (dtype == TP_BF16 && (flags & TP_FLAG_FUSED_LAUNCH)) {
     // Both GEMM layers in one persistent launch (its tile counters start at
     // 0), then the fixed-order fold of the partials.
@@ -427,6 +432,11 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
     return reduce_impl(P, b2, Z, T, d, p, stream);
   }
   TP_TRY(column_impl(X, W1, W_up, b1, Y, T, d, k, p, dtype, act, stream));
+  if (row_fold) {
+    LaunchCtx c{};
+    TP_TRY(make_ctx(stream, true, &c));
+    return launch_tc_row_fold(c, Y, W2, b2, Z, T, k, d, p);
+  }
   if (splitk) {
     LaunchCtx c{};
     TP_TRY(make_ctx(stream, dtype == TP_BF16, &c));

@@ -80,6 +80,10 @@ tp_status launch_tc_block(const LaunchCtx& c, const void* X, const void* W1, con
                           float* Z, int* counters, int64_t T, int64_t d, int64_t k, int p, int act,
                           bool splitk);
 
+// ---- row layer with the fixed-order fold in its epilogue (tp_gemm_fold_sm100.cu)
+tp_status launch_tc_row_fold(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
+                             float* Z, int64_t T, int64_t k, int64_t d, int p);
+
 // ---- row-wise fold (+ bias, + residual) and LayerNorm (tp_rowops.cu)
 cudaError_t launch_row_fold_ln(const LaunchCtx& c, const float* P, int p, const float* bias,
                                const float* R, float* H, const float* gamma, const float* beta,

@@ -127,7 +127,9 @@ def test_block_validation():
     assert blk(ws=0x40000 + 16) == 3
     assert blk(k=255) == 2
     assert blk(flags=8) == 1
-    assert blk(flags=4) == 1
+    assert blk(flags=16) == 1
+    assert blk(flags=tp.TP_FLAG_ROW_FOLD | tp.TP_FLAG_SPLITK_FUSED) == 1
+    assert blk(k=4 * 72, flags=tp.TP_FLAG_ROW_FOLD) == 4      # s = 72, not a multiple of 64
     assert blk(k=4 * 72, flags=tp.TP_FLAG_SPLITK_FUSED) == 4   # s = 72, not a multiple of 64
     assert blk(Z=None) == 1
 

@@ -220,3 +220,55 @@ def test_cta_pair_tiles(act, with_bias):
     blk.block(tp.TP_FLAG_FUSED_LAUNCH, Z=Zf)
     blk.sync()
     assert np.array_equal(bits(host_f32(Zf)), bits(host_f32(blk.Z)))
+
+
+@pytest.mark.parametrize("T,d,s,p,act,bias", [(1, 64, 64, 1, "gelu_tanh", True),
+                                              (130, 200, 64, 4, "relu", True),
+                                              (300, 192, 128, 3, "swiglu", False),
+                                              (1024, 768, 1536, 2, "gelu_tanh", True),
+                                              (16, 512, 448, 8, "swiglu", False),
+                                              (700, 1000, 256, 4, "gelu_tanh", True),
+                                              (2000, 2048, 512, 2, "swiglu", True)])
+def test_row_fold_is_bit_identical_to_partials_and_fold(T, d, s, p, act, bias):
+    """TP_FLAG_ROW_FOLD folds the p partials in the row layer's epilogue: the
+    same fp32 accumulators and the same additions in the same order as the
+    partials layer followed by the fixed-order reduction, so Z has the same
+    bits."""
+    k = s * p
+    inp = _random_bf16(T, d, k, act, with_bias=bias, seed=T + s + p)
+    blk = DeviceBlock(inp, T, d, k, p, act)
+    Zr = torch.full_like(blk.Z, float("nan"))
+    Zd = torch.full_like(blk.Z, float("nan"))
+    blk.block(tp.TP_FLAG_ROW_FOLD, Z=Zr)
+    blk.block(tp.TP_FLAG_NONE, Z=Zd)
+    blk.sync()
+    assert np.array_equal(bits(host_f32(Zr)), bits(host_f32(Zd)))
+    if T <= 1024:
+        assert O.rel_err(host_f32(Zr), _oracle(inp, p, act)["Z"]) <= TOL_BF16
+
+
+@pytest.mark.parametrize("name", ["gpt2", "wide", "llama"])
+def test_row_fold_full_size(name):
+    w = W.WORKLOADS[name]
+    blk = DeviceBlock(W.make_inputs(w), w.T, w.d, w.k, w.p, w.act)
+    Zr = torch.full_like(blk.Z, float("nan"))
+    blk.block(tp.TP_FLAG_ROW_FOLD, Z=Zr)
+    blk.block(tp.TP_FLAG_NONE)
+    blk.sync()
+    assert np.array_equal(bits(host_f32(Zr)), bits(host_f32(blk.Z)))
+
+
+def test_row_fold_argument_errors():
+    w = W.WORKLOADS["gpt2"]
+    blk = DeviceBlock(W.make_inputs(w), w.T, w.d, w.k, w.p, w.act)
+    for bad in (tp.TP_FLAG_ROW_FOLD | tp.TP_FLAG_SPLITK_FUSED,
+                tp.TP_FLAG_ROW_FOLD | tp.TP_FLAG_FUSED_LAUNCH):
+        assert tp.tp_mlp_block(blk.X, blk.W1, None, blk.b1, blk.W2, blk.b2, blk.Z, None, 0, w.T,
+                               w.d, w.k, w.p, blk.dtype, blk.act, bad, check=False) == 1
+    # k/p not a multiple of 64
+    inp = _random_bf16(64, 128, 2 * 72, "relu", with_bias=False, seed=1)
+    b2 = DeviceBlock(inp, 64, 128, 144, 2, "relu")
+    n = tp.tp_mlp_block_workspace_size(64, 128, 144, 2, b2.dtype, b2.act, tp.TP_FLAG_ROW_FOLD)
+    ws = torch.empty(max(n, 256), dtype=torch.uint8, device="cuda")
+    assert tp.tp_mlp_block(b2.X, b2.W1, None, None, b2.W2, None, b2.Z, ws, n, 64, 128, 144, 2,
+                           b2.dtype, b2.act, tp.TP_FLAG_ROW_FOLD, check=False) == 4

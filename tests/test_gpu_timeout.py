@@ -101,3 +101,4 @@ def test_dropped_load_in_cta_pair_gemm_times_out(short_timeout):
     ref = O.mlp_sharded(inp.values("X")[:64], inp.values("W1"), None, inp.values("W2"), None, p,
                         "gelu_tanh")["Z"]
     assert O.rel_err(host_f32(blk.Z)[:64], ref) <= 1e-2
+
