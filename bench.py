@@ -47,6 +47,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -148,7 +149,10 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu_index = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_gpu{gpu_index}.csv")
+        # raw samples: $TP_BENCH_CLOCK_DIR if set (kept for inspection), else a
+        # temporary directory
+        out_dir = os.environ.get("TP_BENCH_CLOCK_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"tp_bench_clocks_gpu{gpu_index}_{os.getpid()}.csv")
 
     def __enter__(self):
         try:
