@@ -16,7 +16,9 @@
 //   empty[s]  in each CTA: the MMA's commit multicast to both;
 //   accf[b]   in each CTA: the MMA's commit multicast to both;
 //   acce[b]   on the even CTA: one arrival per epilogue warp of both CTAs.
-// No load uses cluster multicast: every CTA reads its own tiles.
+// No load uses cluster multicast: every CTA reads its own tiles.  Epilogues
+// store through shared memory with TMA tensor stores, as in the single-CTA
+// kernel.
 #include <cuda.h>
 #include <cuda_runtime.h>
 

@@ -26,7 +26,10 @@
 //   warp 2         TMEM allocation / release;
 //   warps 4..11    epilogue: warp w reads TMEM lanes 32*(w%4).. (the lane
 //                  quadrant it may access) and one half of the columns;
-//                  bias + activation (or none), convert, store.
+//                  bias + activation (or none), convert, then stages 32 x 32
+//                  tiles in shared memory and bulk-stores them with TMA
+//                  tensor stores (per-thread stores for column layers whose
+//                  shard width is not a multiple of 32).
 // Tile width BN (64..256) is picked per problem so that the tiles of a small
 // problem still cover the SMs.  Every barrier wait is bounded.  Launches use
 // programmatic dependent launch: the prologue overlaps the previous kernel,
