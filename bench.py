@@ -387,8 +387,8 @@ def run_reference_block(a, w: WL.BlockWorkload, rank: int, world: int):
 
 
 class Harness:
-    """Warm-up, CUDA-graph capture and the timed loop of the transformer-block
-    arm."""
+    """Warm-up, CUDA-graph capture and the timed loop of the attention,
+    transformer-block and backward arms."""
 
     def __init__(self, a, torch, tp, device, barrier):
         self.a, self.torch, self.tp, self.device, self.barrier = a, torch, tp, device, barrier
@@ -758,92 +758,39 @@ def run_tp_attn(a, w: WL.AttnWorkload, rank: int, world: int, local_rank: int):
     Vs = torch.empty_like(Ks)
     Os = torch.empty_like(Qs)
     Ps = torch.empty((p, T, d), dtype=torch.float32, device=device)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
-    stream = torch.cuda.current_stream(device)
     ident = tp.TP_ACT_IDENTITY
+    H = Harness(a, torch, tp, device, barrier)
 
     def block_step(st):
         tp.tp_attn_block(X, Wq, Wk, Wv, Wo, bo, Z, ws, nbytes, T, d, h, hkv, dh, p, causal,
                          stream=st)
 
-    def calls_step(st, ev):
-        ev[0].record(st)
+    evs = [torch.cuda.Event(enable_timing=True, external=not a.no_graph) for _ in range(5)]
+
+    def calls_step(st):
+        evs[0].record(st)
         tp.tp_column_linear(X, Wq, None, None, Qs, T, d, h * dh, p, tp.TP_BF16, ident, stream=st)
         tp.tp_column_linear(X, Wk, None, None, Ks, T, d, hkv * dh, p, tp.TP_BF16, ident, stream=st)
         tp.tp_column_linear(X, Wv, None, None, Vs, T, d, hkv * dh, p, tp.TP_BF16, ident, stream=st)
-        ev[1].record(st)
+        evs[1].record(st)
         tp.tp_attention_heads(Qs, Ks, Vs, Os, T, p, h, hkv, dh, causal, stream=st)
-        ev[2].record(st)
+        evs[2].record(st)
         tp.tp_row_linear(Os, Wo, Ps, T, h * dh, d, p, tp.TP_BF16, stream=st)
-        ev[3].record(st)
+        evs[3].record(st)
         tp.tp_reduce_partials(Ps, bo, Z, T, d, p, stream=st)
-        ev[4].record(st)
+        evs[4].record(st)
 
-    def capture(fn):
-        for _ in range(a.warmup):
-            flush.zero_()
-            fn(stream)
-        tp.tp_sync_status(stream)
-        if a.no_graph:
-            return None, None
-        g = torch.cuda.CUDAGraph()
-        n0 = tp.tp_kernel_launch_count()
-        with torch.cuda.graph(g):
-            fn(torch.cuda.current_stream())
-        per_step = tp.tp_kernel_launch_count() - n0
-        for _ in range(a.warmup):
-            flush.zero_()
-            g.replay()
-        torch.cuda.synchronize(device)
-        return g, per_step
-
-    g_block, k_block = capture(block_step)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    step_ms = []
     with ClockSampler(local_rank) as clocks:
-        barrier()
-        torch.cuda.synchronize(device)
-        n0 = tp.tp_kernel_launch_count()
-        t_wall = time.perf_counter()
-        for _ in range(a.steps):
-            flush.zero_()
-            e0.record(stream)
-            if g_block is not None:
-                g_block.replay()
-            else:
-                block_step(stream)
-            e1.record(stream)
-            torch.cuda.synchronize(device)
-            step_ms.append(e0.elapsed_time(e1))
-        t_wall = time.perf_counter() - t_wall
-        launches = tp.tp_kernel_launch_count() - n0
-        if g_block is not None:
-            launches = k_block * a.steps
-        barrier()
-    tp.tp_sync_status(stream)
+        step_ms, launches, t_wall = H.time_steps(block_step)
     ms_step, launches = reduce_max([statistics.mean(step_ms), float(launches)], grp, device)
 
     fl = w.flops()
     peaks, peak_src = load_peaks()
     breakdown = None
     if not a.no_breakdown:
-        evs = [torch.cuda.Event(enable_timing=True, external=not a.no_graph) for _ in range(5)]
-        g_calls, _ = capture(lambda st: calls_step(st, evs))
-        parts = [[], [], [], []]
-        barrier()
-        for _ in range(a.steps):
-            flush.zero_()
-            if g_calls is not None:
-                g_calls.replay()
-            else:
-                calls_step(stream, evs)
-            torch.cuda.synchronize(device)
-            for i in range(4):
-                parts[i].append(evs[i].elapsed_time(evs[i + 1]))
-        barrier()
-        tp.tp_sync_status(stream)
-        qkv_ms, att_ms, out_ms, red_ms = reduce_max([statistics.mean(x) for x in parts], grp, device)
+        parts, _, _ = H.time_steps(calls_step, events=evs)
+        qkv_ms, att_ms, out_ms, red_ms = reduce_max([statistics.mean(col) for col in zip(*parts)],
+                                                    grp, device)
         red_bytes = (p + 1) * T * d * 4 + (d * 4 if bo is not None else 0)
 
         def tf(f, ms):
@@ -864,27 +811,13 @@ def run_tp_attn(a, w: WL.AttnWorkload, rank: int, world: int, local_rank: int):
         Zh = torch.empty(Z.shape, dtype=Z.dtype).pin_memory()
         Xd = torch.empty_like(X)
 
-        def e2e_step():
+        def e2e_step(st):
             Xd.copy_(Xh, non_blocking=True)
             tp.tp_attn_block(Xd, Wq, Wk, Wv, Wo, bo, Z, ws, nbytes, T, d, h, hkv, dh, p, causal,
-                             stream=stream)
+                             stream=st)
             Zh.copy_(Z, non_blocking=True)
 
-        for _ in range(a.warmup):
-            flush.zero_()
-            e2e_step()
-        torch.cuda.synchronize(device)
-        barrier()
-        t_e2e = []
-        for _ in range(a.steps):
-            flush.zero_()
-            e0.record(stream)
-            e2e_step()
-            e1.record(stream)
-            torch.cuda.synchronize(device)
-            t_e2e.append(e0.elapsed_time(e1))
-        barrier()
-        tp.tp_sync_status(stream)
+        t_e2e, _, _ = H.time_steps(e2e_step, graph=False)
         e_ms = reduce_max([statistics.mean(t_e2e)], grp, device)[0]
         e2e = {"value": whole_job_value(fl["total"], world, e_ms) / 1e12, "unit": UNIT,
                "ms_per_step": e_ms, "h2d_bytes_per_step": Xh.numel() * Xh.element_size(),
@@ -917,7 +850,7 @@ def run_tp_attn(a, w: WL.AttnWorkload, rank: int, world: int, local_rank: int):
         "warmup": a.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": dict(attn_config(w, world),
-                       launch="eager" if g_block is None else "cuda-graph replay of tp_attn_block",
+                       launch="eager" if a.no_graph else "cuda-graph replay of tp_attn_block",
                        l2="flushed before every step (256 MiB write, outside the timed events)"),
         "pct_bf16_peak": 100.0 * value / (peaks["bf16_tflops"] * world),
         "breakdown": breakdown,
