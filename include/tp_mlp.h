@@ -345,6 +345,26 @@ tp_status tp_mlp_block_backward(const void* X, const void* W1, const void* W_up,
 /* Workspace bytes tp_mlp_block_backward needs (0 if the arguments are invalid). */
 size_t tp_mlp_block_backward_workspace_size(int64_t T, int64_t d, int64_t k, int p, int act);
 
+/*
+ * The same backward pass from the forward inputs alone (activation
+ * recomputation): the column-parallel layer is run again to rebuild the
+ * pre-activations H (and the up projection) and the activations Y in the
+ * workspace, then tp_mlp_block_backward runs on them.  Same results as
+ * calling tp_column_linear (identity, then act) and tp_mlp_block_backward.
+ *   b1 [k] bf16 or NULL (the forward's bias); other arguments as in
+ *   tp_mlp_block_backward.  workspace:
+ *   tp_mlp_block_backward_recompute_workspace_size(...) bytes, 256-aligned.
+ */
+tp_status tp_mlp_block_backward_recompute(const void* X, const void* W1, const void* W_up,
+                                          const void* b1, const void* W2, const void* dZ,
+                                          float* dX, float* dW1, float* dW_up, float* db1,
+                                          float* dW2, float* db2, void* workspace,
+                                          size_t workspace_bytes, int64_t T, int64_t d, int64_t k,
+                                          int p, int act, void* stream);
+
+size_t tp_mlp_block_backward_recompute_workspace_size(int64_t T, int64_t d, int64_t k, int p,
+                                                      int act);
+
 /* Synchronise `stream`, then report (and clear) the device status word of
  * the current device: TP_ERR_DEVICE_TIMEOUT if a bounded wait ran out since
  * the last call, TP_ERR_CUDA if the stream reported an error, else TP_OK. */

@@ -23,10 +23,11 @@ __all__ = [
     "tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
     "tp_mlp_block_noalloc", "tp_attention_heads", "tp_attn_block",
               "tp_layer_norm", "tp_reduce_partials_residual", "tp_transformer_block",
-              "tp_mlp_block_backward", "tp_attn_block_workspace_size",
+              "tp_mlp_block_backward", "tp_mlp_block_backward_recompute", "tp_attn_block_workspace_size",
     "tp_layer_norm", "tp_reduce_partials_residual", "tp_transformer_block",
     "tp_transformer_block_workspace_size", "BlockParams", "tp_mlp_block_backward",
-    "tp_mlp_block_backward_workspace_size",
+    "tp_mlp_block_backward_workspace_size", "tp_mlp_block_backward_recompute",
+    "tp_mlp_block_backward_recompute_workspace_size",
     "tp_mlp_block_workspace_size", "tp_sync_status", "tp_set_wait_timeout_ns",
     "tp_debug_drop_load", "tp_status_string", "tp_last_error_detail",
     "tp_kernel_launch_count", "tp_abi_version", "LIB_PATH",
@@ -84,6 +85,9 @@ def _load() -> ctypes.CDLL:
     lib.tp_transformer_block_workspace_size.argtypes = [i64, i64, i32, i32, i32, i64, i32]
     lib.tp_transformer_block_workspace_size.restype = sz
     lib.tp_mlp_block_backward.argtypes = [vp] * 15 + [sz, i64, i64, i64, i32, i32, vp]
+    lib.tp_mlp_block_backward_recompute.argtypes = [vp] * 13 + [sz, i64, i64, i64, i32, i32, vp]
+    lib.tp_mlp_block_backward_recompute_workspace_size.argtypes = [i64, i64, i64, i32, i32]
+    lib.tp_mlp_block_backward_recompute_workspace_size.restype = sz
     lib.tp_mlp_block_backward_workspace_size.argtypes = [i64, i64, i64, i32, i32]
     lib.tp_mlp_block_backward_workspace_size.restype = sz
     lib.tp_mlp_block_workspace_size.argtypes = [i64, i64, i64, i32, i32, i32, i32]
@@ -234,6 +238,20 @@ def tp_mlp_block_backward(X, W1, W_up, W2, H, H_up, Y, dZ, dX, dW1, dW_up, db1, 
         _ptr(X), _ptr(W1), _ptr(W_up), _ptr(W2), _ptr(H), _ptr(H_up), _ptr(Y), _ptr(dZ), _ptr(dX),
         _ptr(dW1), _ptr(dW_up), _ptr(db1), _ptr(dW2), _ptr(db2), _ptr(workspace), workspace_bytes,
         T, d, k, p, act, _stream(stream)), check)
+
+
+def tp_mlp_block_backward_recompute(X, W1, W_up, b1, W2, dZ, dX, dW1, dW_up, db1, dW2, db2,
+                                    workspace, workspace_bytes, T, d, k, p, act, stream=None,
+                                    check=True):
+    """The backward pass from the forward inputs (H, H_up, Y recomputed)."""
+    return _check(_lib.tp_mlp_block_backward_recompute(
+        _ptr(X), _ptr(W1), _ptr(W_up), _ptr(b1), _ptr(W2), _ptr(dZ), _ptr(dX), _ptr(dW1),
+        _ptr(dW_up), _ptr(db1), _ptr(dW2), _ptr(db2), _ptr(workspace), workspace_bytes, T, d, k, p,
+        act, _stream(stream)), check)
+
+
+def tp_mlp_block_backward_recompute_workspace_size(T, d, k, p, act) -> int:
+    return int(_lib.tp_mlp_block_backward_recompute_workspace_size(T, d, k, p, act))
 
 
 def tp_mlp_block_backward_workspace_size(T, d, k, p, act) -> int:

@@ -639,6 +639,49 @@ tp_status tp_mlp_block_backward(const void* X, const void* W1, const void* W_up,
   return TP_OK;
 }
 
+size_t tp_mlp_block_backward_recompute_workspace_size(int64_t T, int64_t d, int64_t k, int p,
+                                                      int act) {
+  const size_t base = tp_mlp_block_backward_workspace_size(T, d, k, p, act);
+  if (base == 0) return 0;
+  const size_t h = align256(static_cast<size_t>(T) * static_cast<size_t>(k) * 2);
+  return base + h * (act == TP_ACT_SWIGLU ? 3 : 2);
+}
+
+tp_status tp_mlp_block_backward_recompute(const void* X, const void* W1, const void* W_up,
+                                          const void* b1, const void* W2, const void* dZ,
+                                          float* dX, float* dW1, float* dW_up, float* db1,
+                                          float* dW2, float* db2, void* workspace,
+                                          size_t workspace_bytes, int64_t T, int64_t d, int64_t k,
+                                          int p, int act, void* stream) {
+  g_detail[0] = 0;
+  TP_TRY(check_shape(T, d, k, p, TP_BF16));
+  TP_TRY(check_act(act, W_up));
+  const size_t need = tp_mlp_block_backward_recompute_workspace_size(T, d, k, p, act);
+  if (need == 0) return fail(TP_ERR_INVALID_ARG, "sizes");
+  if (T == 0) return TP_OK;
+  if (workspace == nullptr || workspace_bytes < need)
+    return fail(TP_ERR_WORKSPACE, "workspace needs %zu bytes, got %zu", need,
+                workspace == nullptr ? size_t(0) : workspace_bytes);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    return fail(TP_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  // Activation recomputation: the forward column layer again, keeping the
+  // pre-activations (identity epilogue) and the activations, then the
+  // backward pass proper in the rest of the workspace.
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t h = align256(static_cast<size_t>(T) * static_cast<size_t>(k) * 2);
+  const bool swiglu = act == TP_ACT_SWIGLU;
+  void* H = ws;
+  void* Y = ws + h;
+  void* Hu = swiglu ? ws + 2 * h : nullptr;
+  uint8_t* rest = ws + h * (swiglu ? 3 : 2);
+  TP_TRY(column_impl(X, W1, nullptr, b1, H, T, d, k, p, TP_BF16, TP_ACT_IDENTITY, stream));
+  if (swiglu)
+    TP_TRY(column_impl(X, W_up, nullptr, nullptr, Hu, T, d, k, p, TP_BF16, TP_ACT_IDENTITY, stream));
+  TP_TRY(column_impl(X, W1, W_up, b1, Y, T, d, k, p, TP_BF16, act, stream));
+  return tp_mlp_block_backward(X, W1, W_up, W2, H, Hu, Y, dZ, dX, dW1, dW_up, db1, dW2, db2, rest,
+                               workspace_bytes - (rest - ws), T, d, k, p, act, stream);
+}
+
 tp_status tp_sync_status(void* stream) {
   g_detail[0] = 0;
   int dev = 0, sms = 0, cc = 0;

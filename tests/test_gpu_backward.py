@@ -186,3 +186,28 @@ def test_backward_dropped_load_times_out():
                                  _vals(inp["W2"]), _vals(inp["dZ"]), p, "gelu_tanh",
                                  hidden_round="bf16")
     assert O.rel_err(host_f32(blk.dX), ref["dX"]) <= TOL
+
+
+@pytest.mark.parametrize("T,d,k,p,act", [(300, 256, 512, 2, "gelu_tanh"), (129, 512, 1024, 4, "swiglu")])
+def test_backward_recompute_matches_explicit(T, d, k, p, act):
+    """tp_mlp_block_backward_recompute rebuilds H (and the up projection) and
+    Y with the same column-layer kernels, so its gradients have the same bits
+    as the explicit call on tp_column_linear's outputs."""
+    inp = _inputs(T, d, k, act, seed=T + k)
+    blk = DeviceBackward(inp, T, d, k, p, act)
+    blk.run()
+    want = blk.grads()
+    t = blk.t
+    out = {name: torch.full_like(v, float("nan")) for name, v in
+           (("dX", blk.dX), ("dW1", blk.dW1), ("db1", blk.db1), ("dW2", blk.dW2), ("db2", blk.db2))}
+    if blk.dWu is not None:
+        out["dW_up"] = torch.full_like(blk.dWu, float("nan"))
+    n = tp.tp_mlp_block_backward_recompute_workspace_size(T, d, k, p, blk.act)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    tp.tp_mlp_block_backward_recompute(t["X"], t["W1"], t["W_up"], t["b1"], t["W2"], t["dZ"],
+                                       out["dX"], out["dW1"], out.get("dW_up"), out["db1"],
+                                       out["dW2"], out["db2"], ws, n, T, d, k, p, blk.act)
+    tp.tp_sync_status()
+    for name, v in out.items():
+        got = host_f32(v)
+        assert np.array_equal(got.view(np.uint32), want[name].view(np.uint32)), name
