@@ -198,9 +198,24 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def source_digest(files) -> str:
+    """Digest of the kernels' device sources with comments and whitespace
+    removed, so that a traffic figure stays tied to the code it was measured
+    on, not to its comments."""
+    import re
+    h = hashlib.sha256()
+    for src in files:
+        with open(os.path.join(ROOT, "megatron_tensor_sharded_b200", "csrc", src)) as f:
+            text = f.read()
+        text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", " ", text)
+        h.update(" ".join(text.split()).encode())
+    return h.hexdigest()[:16]
+
+
 def ncu_traffic(kernel_key: str):
     """dram bytes per launch from the committed ncu summary table, if it was
-    taken on the current kernel sources (else None)."""
+    taken on the current kernel code (else None)."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
@@ -210,14 +225,11 @@ def ncu_traffic(kernel_key: str):
     ent = table.get(kernel_key)
     if not ent:
         return None
-    h = hashlib.sha256()
     try:
-        for src in ent["sources"]:
-            with open(os.path.join(ROOT, "megatron_tensor_sharded_b200", "csrc", src), "rb") as f:
-                h.update(f.read())
+        digest = source_digest(ent["sources"])
     except (OSError, KeyError):
         return None
-    if h.hexdigest()[:16] != ent.get("source_sha"):
+    if digest != ent.get("source_sha"):
         return None
     return ent.get("dram_bytes_per_launch")
 
