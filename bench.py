@@ -570,6 +570,23 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
     ms_step, launches = reduce_max([statistics.mean(step_ms), float(launches)],
                                    dist if world > 1 else None, device)
 
+    # ---- the same graph replayed without the L2 flush (operands L2-resident
+    # when they fit): a labelled second figure, not the metric
+    l2_resident = None
+    if g_block is not None:
+        warm = []
+        torch.cuda.synchronize(device)
+        for _ in range(a.steps):
+            e0.record(stream)
+            g_block.replay()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            warm.append(e0.elapsed_time(e1))
+        tp.tp_sync_status(stream)
+        w_ms = reduce_max([statistics.mean(warm)], dist if world > 1 else None, device)[0]
+        l2_resident = {"ms_per_step": w_ms, "value": whole_job_value(w.gemm_flops(), world, w_ms) / 1e12,
+                       "unit": UNIT, "how": "graph replay without the L2 flush between steps"}
+
     # ---- per-kernel breakdown of the same block as three separate calls
     kernels = None
     if a.mode == "partials" and not a.no_breakdown:
@@ -718,6 +735,7 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
         "gpu_launches": int(launches),
         "clocks": clocks.summary(),
         "e2e": e2e,
+        "l2_resident": l2_resident,
         "wall_s_timed_region": t_wall,
     }
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
@@ -726,6 +744,16 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
         line["cpu_baseline"] = {"value": w.gemm_flops() * rows / w.T / sec / 1e12, "unit": UNIT,
                                 "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"first {rows} of {w.T} token rows, {reps} reps, float64"}
+        try:   # the same oracle on one host thread
+            from threadpoolctl import threadpool_limits
+            with threadpool_limits(limits=1):
+                rows1 = max(1, rows // 8)
+                sec1, reps1 = time_oracle(w, inp, rows1, min_seconds=3.0, max_reps=100)
+            line["cpu_baseline"]["single_thread"] = {
+                "value": w.gemm_flops() * rows1 / w.T / sec1 / 1e12, "unit": UNIT, "cores": 1,
+                "sample": f"first {rows1} of {w.T} token rows, {reps1} reps, float64"}
+        except Exception as exc:  # threadpoolctl missing or BLAS not controllable
+            line["cpu_baseline"]["single_thread"] = {"unavailable": str(exc)[:120]}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
