@@ -105,7 +105,9 @@ typedef enum {
  *   W1    [d][k]        dtype   (W_gate for SwiGLU)
  *   W_up  [d][k]        dtype   SwiGLU only (must be non-NULL), else ignored
  *   b1    [k]           dtype   nullable (no bias); with SwiGLU, b1 is added
- *                               to the gate pre-activation
+ *                               to the gate pre-activation; bf16: 16-byte
+ *                               aligned (read as 8-element vectors), else
+ *                               TP_ERR_ALIGNMENT
  *   Y     [p][T][s]     dtype   output: shard i is a dense [T][s] matrix
  *   returns TP_ERR_INDIVISIBLE when k % p != 0.
  */

@@ -144,7 +144,7 @@ tp_status column_impl(const void* X, const void* W1, const void* W_up, const voi
   TP_TRY(check_ptr(W1, "W1", dtype, true));
   if (act == TP_ACT_SWIGLU) TP_TRY(check_ptr(W_up, "W_up", dtype, true));
   TP_TRY(check_ptr(Y, "Y", dtype, true));
-  if (b1 != nullptr) TP_TRY(check_ptr(b1, "b1", dtype, false));
+  if (b1 != nullptr) TP_TRY(check_ptr(b1, "b1", dtype, dtype == TP_BF16));
   LaunchCtx c{};
   TP_TRY(make_ctx(stream, dtype == TP_BF16, &c));
   if (dtype == TP_BF16) return launch_tc_column(c, X, W1, W_up, b1, Y, T, d, k, p, act);
@@ -402,7 +402,7 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
   TP_TRY(check_ptr(W1, "W1", dtype, true));
   if (act == TP_ACT_SWIGLU) TP_TRY(check_ptr(W_up, "W_up", dtype, true));
   TP_TRY(check_ptr(W2, "W2", dtype, true));
-  if (b1 != nullptr) TP_TRY(check_ptr(b1, "b1", dtype, false));
+  if (b1 != nullptr) TP_TRY(check_ptr(b1, "b1", dtype, dtype == TP_BF16));
   if (Z == nullptr) return fail(TP_ERR_INVALID_ARG, "Z is NULL");
   if (!aligned16(Z)) return fail(TP_ERR_ALIGNMENT, "Z must be 16-byte aligned");
   if (b2 != nullptr && !aligned4(b2)) return fail(TP_ERR_ALIGNMENT, "b2 must be 4-byte aligned");

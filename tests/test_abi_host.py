@@ -145,3 +145,11 @@ def test_valid_call_without_gpu_fails_loudly():
     with pytest.raises(tp.TPError):
         tp.tp_column_linear(FAKE, FAKE, None, None, FAKE2, 4, 64, 256, 4, tp.TP_BF16,
                             tp.TP_ACT_GELU_TANH, stream=0)
+
+
+def test_bf16_bias_alignment_is_checked():
+    """The bf16 column epilogue reads b1 as 16-byte vectors: a misaligned
+    bias is refused before any launch."""
+    st = tp.tp_column_linear(FAKE, FAKE, None, FAKE + 2, FAKE2, 4, 64, 256, 4, tp.TP_BF16,
+                             tp.TP_ACT_GELU_TANH, stream=0, check=False)
+    assert st == 3
