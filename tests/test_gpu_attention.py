@@ -65,6 +65,8 @@ HEAD_CASES = [
     (2, 129, 4, 4, True),      # one row past a block
     (4, 517, 8, 4, True),      # several blocks per unit, more units than rounds
     (2, 640, 8, 2, False),     # group of 4 query heads per K/V head
+    (8, 383, 16, 8, True),     # one K/V head per shard, 8 shards
+    (1, 1200, 3, 1, True),     # odd head count, 3 query heads on one K/V head
 ]
 
 

@@ -93,6 +93,7 @@ CASES = [
     (1000, 1024, 4096, 4, "gelu_tanh"),
     (1, 256, 512, 2, "swiglu"),
     (200, 384, 768, 3, "identity"),
+    (513, 1024, 4096, 8, "swiglu"),
 ]
 
 

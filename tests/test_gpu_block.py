@@ -115,6 +115,8 @@ BLOCK_CASES = [
     (129, 512, 4, 4, 1024, 4, "swiglu", True),
     (200, 256, 2, 2, 768, 2, "gelu_tanh", False),
     (1, 128, 2, 1, 256, 1, "swiglu", True),
+    (333, 1024, 8, 8, 2048, 8, "swiglu", True),     # one K/V head per shard, ragged T
+    (257, 768, 6, 2, 3072, 2, "gelu_tanh", True),   # GPT-2 width, 3 query heads per K/V head
 ]
 
 
