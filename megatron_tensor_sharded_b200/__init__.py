@@ -10,6 +10,23 @@ kernels.  Arguments that are device buffers accept a ``torch.Tensor`` (its
 Importing this package fails loudly when the shared library has not been
 built (``python megatron_tensor_sharded_b200/build.py``): there is no CPU or
 PyTorch fallback.
+
+Example -- the MLP block on p = 4 simulated shards, bf16 in, fp32 out::
+
+    import torch, megatron_tensor_sharded_b200 as tp
+    T, d, k, p = 4096, 4096, 16384, 4
+    X = torch.randn(T, d, device="cuda").bfloat16()
+    W1 = (0.02 * torch.randn(d, k, device="cuda")).bfloat16()    # [in, out]
+    W2 = (0.02 * torch.randn(k, d, device="cuda")).bfloat16()
+    Z = torch.empty(T, d, device="cuda")
+    n = tp.tp_mlp_block_workspace_size(T, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    tp.tp_mlp_block(X, W1, None, None, W2, None, Z, ws, n, T, d, k, p,
+                    tp.TP_BF16, tp.TP_ACT_GELU_TANH)
+    tp.tp_sync_status()          # raises TPError if a device wait timed out
+
+The same pattern serves tp_attn_block, tp_transformer_block (weights in a
+BlockParams built by ``block_params(**tensors)``) and tp_mlp_block_backward.
 """
 
 from __future__ import annotations
