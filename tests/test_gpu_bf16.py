@@ -272,3 +272,33 @@ def test_row_fold_argument_errors():
     ws = torch.empty(max(n, 256), dtype=torch.uint8, device="cuda")
     assert tp.tp_mlp_block(b2.X, b2.W1, None, None, b2.W2, None, b2.Z, ws, n, 64, 128, 144, 2,
                            b2.dtype, b2.act, tp.TP_FLAG_ROW_FOLD, check=False) == 4
+
+
+@pytest.mark.parametrize("T,d,s,p,act,bias", [(1, 64, 64, 1, "gelu_tanh", True),
+                                              (130, 200, 40, 4, "relu", True),
+                                              (257, 128, 72, 2, "gelu_tanh", True),
+                                              (300, 192, 128, 3, "swiglu", False),
+                                              (1024, 768, 1536, 2, "gelu_tanh", True),
+                                              (16, 512, 448, 8, "swiglu", False),
+                                              (1000, 2048, 512, 4, "gelu_tanh", True),
+                                              (777, 1000, 256, 5, "relu", False)])
+def test_block_is_bit_identical_to_separate_calls(T, d, s, p, act, bias):
+    """tp_mlp_block's default path (PDL-chained layers, CTA-pair tiles where
+    the cost model picks them) gives the same bits as tp_column_linear +
+    tp_row_linear + tp_reduce_partials, call after call on one workspace."""
+    k = s * p
+    inp = _random_bf16(T, d, k, act, with_bias=bias, seed=T + d + p)
+    blk = DeviceBlock(inp, T, d, k, p, act)
+    blk.column()
+    blk.row()
+    blk.reduce()
+    blk.sync()
+    want = bits(host_f32(blk.Z))
+    n = tp.tp_mlp_block_workspace_size(T, d, k, p, blk.dtype, blk.act)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        Zb = torch.full_like(blk.Z, float("nan"))
+        tp.tp_mlp_block(blk.X, blk.W1, blk.Wu, blk.b1, blk.W2, blk.b2, Zb, ws, n, T, d, k, p,
+                        blk.dtype, blk.act, tp.TP_FLAG_NONE)
+        blk.sync()
+        assert np.array_equal(bits(host_f32(Zb)), want)
