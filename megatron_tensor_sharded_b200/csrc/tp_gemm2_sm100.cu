@@ -241,6 +241,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // -------------------------------------------------------------- epilogue
     const int quad = warp & 3;
     const int half = (warp - 4) >> 2;
+    uint32_t nchunk = 0;   // bf16 chunks this warp has staged (alternating halves)
     int32_t lt = 0;
     for (int32_t t = cluster; t < P.num_tiles; t += nclusters, ++lt) {
       const uint32_t b = lt & 1, ap = (lt >> 1) & 1;
@@ -258,7 +259,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         epilogue_tile_bulk<MODE, PBN>(P, tc, tacc, row0, half, stage_w, &mapC, lane);
       } else {
         if (P.bulk_out)
-          epilogue_tile_bulk_col<MODE, PBN>(P, tc, tacc, row0, half, eb, stage_w, &mapC, lane);
+          epilogue_tile_bulk_col<MODE, PBN>(P, tc, tacc, row0, half, eb, stage_w, &mapC, lane,
+                                            nchunk);
         else
           epilogue_tile<MODE, PBN>(P, tc, tacc, row0 + lane, half, eb);
       }

@@ -128,15 +128,100 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return u;
 }
 
-// 8 consecutive output columns j..j+7 of one row, bf16, into shard storage.
-__device__ __forceinline__ void store_bf16x8(const TcParams& P, int row, int32_t j,
-                                             const float (&y)[8]) {
+// 8 consecutive output columns j..j+7 of one row (4 bf16 pairs) into shard
+// storage.
+__device__ __forceinline__ void store_bf16x8(const TcParams& P, int row, int32_t j, uint4 pk) {
   const int32_t shard = j / P.s;
   const int32_t jj = j - shard * P.s;
-  const uint4 pk = make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
-                              pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7]));
   __nv_bfloat16* __restrict__ Y = static_cast<__nv_bfloat16*>(P.out);
   *reinterpret_cast<uint4*>(Y + (static_cast<int64_t>(shard) * P.T + row) * P.s + jj) = pk;
+}
+
+// ----------------------------------------------- column-layer activations
+// Two adjacent hidden columns of one row at a time, as a packed fp32 pair:
+// sm_100 issues one FFMA2 / FMUL2 / FADD2 for both, so the epilogue's
+// arithmetic takes half the issue slots of the scalar form.  Results are
+// rounded once to a bf16 pair (the stored Y).
+//   GELU, tanh form:  h/2 + (h/2) tanh(u),  u = h (c1 + c3 h^2),
+//                     c1 = sqrt(2/pi), c3 = 0.044715 c1;
+//   SwiGLU:           a + a tanh(g/2),  a = (g/2) up  (= SiLU(g) up, since
+//                     sigmoid(g) = (1 + tanh(g/2)) / 2).
+// tanh is the MUFU approximation (relative error about 2^-11, below the
+// bf16 rounding of the result).
+
+// Two bf16 bias values (one 32-bit word, lower column first) as a pair.
+__device__ __forceinline__ uint64_t bf16_word_to_pair(uint32_t w) {
+  return f2_pack(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+
+__device__ __forceinline__ uint64_t tanh_pair(uint64_t x) {
+  float a, b;
+  f2_unpack(x, a, b);
+  return f2_pack(tanh_mufu(a), tanh_mufu(b));
+}
+
+__device__ __forceinline__ uint32_t pair_to_bf16x2(uint64_t y) {
+  float a, b;
+  f2_unpack(y, a, b);
+  return pack_bf16x2(a, b);
+}
+
+__device__ __forceinline__ uint32_t gelu_pair_bf16(uint64_t h) {
+  const uint64_t c1 = f2_pack(0.7978845608028654f, 0.7978845608028654f);
+  const uint64_t c3 = f2_pack(0.035677408136300125f, 0.035677408136300125f);
+  const uint64_t half = f2_pack(0.5f, 0.5f);
+  const uint64_t u = f2_mul(h, f2_fma(f2_mul(h, h), c3, c1));
+  const uint64_t hh = f2_mul(h, half);
+  return pair_to_bf16x2(f2_fma(hh, tanh_pair(u), hh));
+}
+
+__device__ __forceinline__ uint32_t swiglu_pair_bf16(uint64_t gate, uint64_t up) {
+  const uint64_t hg = f2_mul(gate, f2_pack(0.5f, 0.5f));
+  const uint64_t a = f2_mul(hg, up);
+  return pair_to_bf16x2(f2_fma(a, tanh_pair(hg), a));
+}
+
+// Identity / ReLU (the exact-integer test activations): scalar.
+__device__ __forceinline__ uint32_t plain_pair_bf16(int act, uint64_t h) {
+  float a, b;
+  f2_unpack(h, a, b);
+  return pack_bf16x2(act_unary_mufu(act, a), act_unary_mufu(act, b));
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4& u, int k) {
+  return k == 0 ? u.x : (k == 1 ? u.y : (k == 2 ? u.z : u.w));
+}
+
+// One row's 32-column chunk of the column layer: the accumulator words `a`
+// (gate for SwiGLU, with `up` the matching up-projection words), the bias
+// (4 vectors of 8 bf16, or none) and the activation, into 16 bf16 pairs.
+template <bool kSwiglu>
+__device__ __forceinline__ void act_chunk_bf16(int act, bool has_bias, const uint32_t (&a)[32],
+                                               const uint32_t (&up)[32], const uint4* bias,
+                                               uint32_t (&out)[16]) {
+  if (kSwiglu) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      uint64_t g = f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
+      if (has_bias) g = f2_add(g, bf16_word_to_pair(word_of(bias[i / 4], i % 4)));
+      out[i] = swiglu_pair_bf16(g, f2_pack(__uint_as_float(up[2 * i]),
+                                           __uint_as_float(up[2 * i + 1])));
+    }
+  } else if (act == kActGeluTanh) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      uint64_t h = f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
+      if (has_bias) h = f2_add(h, bf16_word_to_pair(word_of(bias[i / 4], i % 4)));
+      out[i] = gelu_pair_bf16(h);
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      uint64_t h = f2_pack(__uint_as_float(a[2 * i]), __uint_as_float(a[2 * i + 1]));
+      if (has_bias) h = f2_add(h, bf16_word_to_pair(word_of(bias[i / 4], i % 4)));
+      out[i] = plain_pair_bf16(act, h);
+    }
+  }
 }
 
 // 32-column chunks one epilogue warp handles per tile (it owns half of the
@@ -194,58 +279,28 @@ __device__ __forceinline__ void epilogue_tile(const TcParams& P, const TileCoord
                                               const EpiBias<MODE, BN>& eb) {
   using S = EpiShape<MODE, BN>;
   const bool row_ok = row < P.T;
-  if constexpr (MODE == kModeColumn) {
+  if constexpr (S::kColumn) {
+    constexpr bool kSwiglu = (MODE == kModeColumnSwiglu);
     const bool has_bias = P.bias != nullptr;
     // unrolled: the prefetched bias registers are indexed by chunk
 #pragma unroll
     for (int q = 0; q < S::kChunks; ++q) {
-      const int c0 = half * (BN / 2) + q * 32;
-      uint32_t v[32];
+      // gate (or hidden) column inside the accumulator; SwiGLU's up columns
+      // sit BN/2 further
+      const int c0 = half * (S::kOutCols / 2) + q * 32;
+      uint32_t v[32], u[32];
       tmem_ld_32x32b_x32(tacc + c0, v);
+      if (kSwiglu) tmem_ld_32x32b_x32(tacc + BN / 2 + c0, u);
       tmem_ld_wait();
       if (!row_ok) continue;
-      const int32_t j0 = tc.n * BN + c0;
+      const int32_t j0 = tc.n * S::kOutCols + c0;
+      uint32_t y[16];
+      act_chunk_bf16<kSwiglu>(P.act, has_bias, v, u, &eb.v[q * 4], y);
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         const int32_t j = j0 + g * 8;
         if (j >= P.n_total) break;
-        float bv[8];
-        unpack_bf16x8(eb.v[q * 4 + g], bv);
-        float h[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          h[e] = __uint_as_float(v[g * 8 + e]);
-          if (has_bias) h[e] += bv[e];
-          h[e] = act_unary_mufu(P.act, h[e]);
-        }
-        store_bf16x8(P, row, j, h);
-      }
-    }
-  } else if constexpr (MODE == kModeColumnSwiglu) {
-    const bool has_bias = P.bias != nullptr;
-#pragma unroll
-    for (int q = 0; q < S::kChunks; ++q) {
-      const int c0 = half * (BN / 4) + q * 32;   // gate column inside the accumulator
-      uint32_t g32[32], u32[32];
-      tmem_ld_32x32b_x32(tacc + c0, g32);
-      tmem_ld_32x32b_x32(tacc + BN / 2 + c0, u32);
-      tmem_ld_wait();
-      if (!row_ok) continue;
-      const int32_t j0 = tc.n * (BN / 2) + c0;
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int32_t j = j0 + g * 8;
-        if (j >= P.n_total) break;
-        float bv[8];
-        unpack_bf16x8(eb.v[q * 4 + g], bv);
-        float y[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float gate = __uint_as_float(g32[g * 8 + e]);
-          if (has_bias) gate += bv[e];
-          y[e] = silu_mufu(gate) * __uint_as_float(u32[g * 8 + e]);
-        }
-        store_bf16x8(P, row, j, y);
+        store_bf16x8(P, row, j, make_uint4(y[4 * g], y[4 * g + 1], y[4 * g + 2], y[4 * g + 3]));
       }
     }
   } else {
@@ -337,77 +392,54 @@ __device__ __forceinline__ void epilogue_tile_bulk(const TcParams& P, const Tile
 }
 
 // Bulk-store epilogue of the column layers (bf16 Y [p][T][s], s % 32 == 0 so
-// a 32-column chunk never straddles two shards): bias + activation as in
-// epilogue_tile, then each warp writes its 32 rows x 32 columns (64 bytes a
-// row) into its staging tile in the 64-byte swizzled layout (16-byte chunk c
-// of row r at c ^ ((r / 2) % 4): conflict-free) and one lane issues a TMA
-// tensor store, clipped at T by the tensor map.
+// a 32-column chunk never straddles two shards): bias + activation on packed
+// pairs, then each warp writes its 32 rows x 32 columns (64 bytes a row) into
+// one half of its staging tile in the 64-byte swizzled layout (16-byte chunk
+// c of row r at c ^ ((r / 2) % 4): conflict-free) and one lane issues a TMA
+// tensor store, clipped at T by the tensor map.  The two halves alternate
+// (`nchunk` counts the warp's chunks across tiles), so a chunk waits only
+// for the store before last to have read its half, not for the previous one.
 template <int MODE, int BN>
 __device__ __forceinline__ void epilogue_tile_bulk_col(const TcParams& P, const TileCoord& tc,
                                                        uint32_t tacc, int32_t row0, int half,
                                                        const EpiBias<MODE, BN>& eb,
                                                        uint32_t stage, const CUtensorMap* mapY,
-                                                       int lane) {
+                                                       int lane, uint32_t& nchunk) {
   using S = EpiShape<MODE, BN>;
+  constexpr bool kSwiglu = (MODE == kModeColumnSwiglu);
+  constexpr uint32_t kChunkBytes = 32 * 64;
+  static_assert(2 * kChunkBytes <= EPI_WARP_STAGE_BYTES, "two bf16 chunks per staging tile");
   const bool has_bias = P.bias != nullptr;
 #pragma unroll
   for (int q = 0; q < S::kChunks; ++q) {
-    int32_t j0;
-    float y[32];
-    if constexpr (MODE == kModeColumn) {
-      const int c0 = half * (BN / 2) + q * 32;
-      uint32_t v[32];
-      tmem_ld_32x32b_x32(tacc + c0, v);
-      tmem_ld_wait();
-      j0 = tc.n * BN + c0;
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        float bv[8];
-        unpack_bf16x8(eb.v[q * 4 + g], bv);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float h = __uint_as_float(v[g * 8 + e]);
-          if (has_bias) h += bv[e];
-          y[g * 8 + e] = act_unary_mufu(P.act, h);
-        }
-      }
-    } else {
-      const int c0 = half * (BN / 4) + q * 32;   // gate column inside the accumulator
-      uint32_t g32[32], u32[32];
-      tmem_ld_32x32b_x32(tacc + c0, g32);
-      tmem_ld_32x32b_x32(tacc + BN / 2 + c0, u32);
-      tmem_ld_wait();
-      j0 = tc.n * (BN / 2) + c0;
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        float bv[8];
-        unpack_bf16x8(eb.v[q * 4 + g], bv);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          float gate = __uint_as_float(g32[g * 8 + e]);
-          if (has_bias) gate += bv[e];
-          y[g * 8 + e] = silu_mufu(gate) * __uint_as_float(u32[g * 8 + e]);
-        }
-      }
-    }
-    if (j0 >= P.n_total) continue;   // warp-uniform
-    if (lane == 0) bulk_wait_read0();
+    const int c0 = half * (S::kOutCols / 2) + q * 32;
+    const int32_t j0 = tc.n * S::kOutCols + c0;
+    if (j0 >= P.n_total) break;   // warp-uniform; later chunks are further right
+    uint32_t v[32], u[32];
+    tmem_ld_32x32b_x32(tacc + c0, v);
+    if (kSwiglu) tmem_ld_32x32b_x32(tacc + BN / 2 + c0, u);
+    tmem_ld_wait();
+    uint32_t y[16];
+    act_chunk_bf16<kSwiglu>(P.act, has_bias, v, u, &eb.v[q * 4], y);
+    const uint32_t buf = stage + (nchunk & 1u) * kChunkBytes;
+    // the half is free once the store issued two chunks ago has read it
+    if (lane == 0) bulk_wait_read1();
     __syncwarp();
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      const uint32_t addr = stage + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4);
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr),
-                   "r"(pack_bf16x2(y[8 * c], y[8 * c + 1])), "r"(pack_bf16x2(y[8 * c + 2], y[8 * c + 3])),
-                   "r"(pack_bf16x2(y[8 * c + 4], y[8 * c + 5])), "r"(pack_bf16x2(y[8 * c + 6], y[8 * c + 7]))
+      const uint32_t addr = buf + lane * 64 + ((c ^ ((lane >> 1) & 3)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(y[4 * c]),
+                   "r"(y[4 * c + 1]), "r"(y[4 * c + 2]), "r"(y[4 * c + 3])
                    : "memory");
     }
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
       const int32_t shard = j0 / P.s;
-      tma_store_3d(mapY, stage, j0 - shard * P.s, row0, shard);
+      tma_store_3d(mapY, buf, j0 - shard * P.s, row0, shard);
       bulk_commit();
     }
+    ++nchunk;
   }
 }
 

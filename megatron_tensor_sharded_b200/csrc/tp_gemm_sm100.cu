@@ -206,6 +206,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // -------------------------------------------------------------- epilogue
     const int quad = warp & 3;          // TMEM lane quadrant this warp may access
     const int half = (warp - 4) >> 2;   // which half of the accumulator columns
+    uint32_t nchunk = 0;   // bf16 chunks this warp has staged (alternating halves)
     int32_t lt = 0;
     for (int32_t t = blockIdx.x; t < P.num_tiles; t += gridDim.x, ++lt) {
       const uint32_t b = lt & 1, ap = (lt >> 1) & 1;
@@ -224,7 +225,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else {
         if (P.bulk_out)
           epilogue_tile_bulk_col<MODE, BN>(P, tc, tacc, tc.m * BM + quad * 32, half, eb, stage_w,
-                                           &mapC, lane);
+                                           &mapC, lane, nchunk);
         else
           epilogue_tile<MODE, BN>(P, tc, tacc, tc.m * BM + quad * 32 + lane, half, eb);
       }
