@@ -36,18 +36,20 @@ import os
 
 __all__ = [
     "TPError", "TP_F32", "TP_BF16", "TP_ACT_GELU_TANH", "TP_ACT_SWIGLU", "TP_ACT_IDENTITY",
-    "TP_ACT_RELU", "TP_FLAG_NONE", "TP_FLAG_SPLITK_FUSED", "TP_FLAG_FUSED_LAUNCH", "TP_FLAG_ROW_FOLD", "STATUS", "ACT", "DTYPE",
+    "TP_ACT_RELU", "TP_FLAG_NONE", "TP_FLAG_SPLITK_FUSED", "TP_FLAG_FUSED_LAUNCH",
+    "TP_FLAG_ROW_FOLD", "STATUS", "ACT", "DTYPE", "LIB_PATH", "BlockParams", "block_params",
+    # the MLP block and its steps
     "tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
-    "tp_mlp_block_noalloc", "tp_attention_heads", "tp_attn_block",
-              "tp_layer_norm", "tp_reduce_partials_residual", "tp_transformer_block",
-              "tp_mlp_block_backward", "tp_mlp_block_backward_recompute", "tp_attn_block_workspace_size",
+    "tp_mlp_block_workspace_size", "tp_mlp_block_noalloc",
+    # attention, transformer block, backward
+    "tp_attention_heads", "tp_attn_block", "tp_attn_block_workspace_size",
     "tp_layer_norm", "tp_reduce_partials_residual", "tp_transformer_block",
-    "tp_transformer_block_workspace_size", "BlockParams", "tp_mlp_block_backward",
+    "tp_transformer_block_workspace_size", "tp_mlp_block_backward",
     "tp_mlp_block_backward_workspace_size", "tp_mlp_block_backward_recompute",
     "tp_mlp_block_backward_recompute_workspace_size",
-    "tp_mlp_block_workspace_size", "tp_sync_status", "tp_set_wait_timeout_ns",
-    "tp_debug_drop_load", "tp_status_string", "tp_last_error_detail",
-    "tp_kernel_launch_count", "tp_abi_version", "LIB_PATH",
+    # status, timeouts, introspection
+    "tp_sync_status", "tp_set_wait_timeout_ns", "tp_debug_drop_load", "tp_status_string",
+    "tp_last_error_detail", "tp_kernel_launch_count", "tp_abi_version",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libtpmlp.so")
@@ -122,8 +124,9 @@ def _load() -> ctypes.CDLL:
     lib.tp_kernel_launch_count.restype = u64
     lib.tp_abi_version.argtypes = []
     for f in ("tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
-              "tp_mlp_block_noalloc", "tp_attention_heads", "tp_attn_block",
-              "tp_sync_status", "tp_abi_version"):
+              "tp_mlp_block_noalloc", "tp_attention_heads", "tp_attn_block", "tp_layer_norm",
+              "tp_reduce_partials_residual", "tp_transformer_block", "tp_mlp_block_backward",
+              "tp_mlp_block_backward_recompute", "tp_sync_status", "tp_abi_version"):
         getattr(lib, f).restype = i32
     return lib
 
