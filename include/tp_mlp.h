@@ -197,6 +197,51 @@ size_t tp_mlp_block_workspace_size(int64_t T, int64_t d, int64_t k, int p,
                                    tp_dtype dtype, tp_act act, int flags);
 
 /*
+ * tp_mlp_block with the activations in HOST memory: X is read from, and Z
+ * written to, host buffers; the weights and biases are device buffers (they
+ * stay resident between calls).  The block is row-wise (row t of Z depends
+ * only on row t of X: "Tensor parallel math", "The MLP block: column then
+ * row, one all-reduce"), so the call cuts the T token rows into up to four
+ * chunks (multiples of 128 rows, at least 256 each) and pipelines them: the
+ * copy of chunk c+1 into the device, the block on chunk c and the copy of
+ * chunk c-1 back to the host overlap on the GPU's two copy engines and its
+ * SMs.  Z has exactly the bits of copying X in, calling tp_mlp_block on all
+ * rows and copying Z out.
+ *
+ *   X_host     [T][d] host memory (bf16 or fp32 per dtype).  Pinned
+ *              (page-locked) memory lets the copies overlap the compute;
+ *              pageable memory works but copies synchronously.
+ *   Z_host     [T][d] fp32 host memory.
+ *   workspace  device memory of at least tp_mlp_block_host_workspace_size()
+ *              bytes, 256-byte aligned: device copies of X and Z, then the
+ *              block's workspace for one chunk.
+ *   others     as for tp_mlp_block.
+ *
+ * Stream semantics: everything is ordered on `stream`.  The call forks two
+ * library-owned helper streams (one per copy direction, created on the first
+ * call on each device and kept for the process) from `stream` with an event
+ * and joins them back before it returns, so Z_host is complete once `stream`
+ * has reached the point of the call (cudaStreamSynchronize).  The call can be
+ * captured into a CUDA graph from `stream` when both host buffers are pinned
+ * and the device has had one uncaptured call first.  Calls on one device
+ * enqueue under a lock (the helper events are shared).
+ *
+ * Errors: argument errors return before anything is enqueued; a CUDA error
+ * after the fork returns TP_ERR_CUDA with the helper streams still joined
+ * into `stream`.
+ */
+tp_status tp_mlp_block_host(const void* X_host, const void* W1, const void* W_up,
+                            const void* b1, const void* W2, const float* b2, float* Z_host,
+                            void* workspace, size_t workspace_bytes,
+                            int64_t T, int64_t d, int64_t k, int p,
+                            tp_dtype dtype, tp_act act, int flags, void* stream);
+
+/* Workspace bytes tp_mlp_block_host needs (0 if the arguments are invalid
+ * or T == 0). */
+size_t tp_mlp_block_host_workspace_size(int64_t T, int64_t d, int64_t k, int p,
+                                        tp_dtype dtype, tp_act act, int flags);
+
+/*
  * Attention of every shard's own heads (the local step of the
  * tensor-parallel attention block: each shard holds h/p query heads and
  * h_kv/p key/value heads and attends with no communication; day-41 post,

@@ -40,7 +40,8 @@ __all__ = [
     "TP_FLAG_ROW_FOLD", "STATUS", "ACT", "DTYPE", "LIB_PATH", "BlockParams", "block_params",
     # the MLP block and its steps
     "tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
-    "tp_mlp_block_workspace_size", "tp_mlp_block_noalloc",
+    "tp_mlp_block_workspace_size", "tp_mlp_block_noalloc", "tp_mlp_block_host",
+    "tp_mlp_block_host_workspace_size",
     # attention, transformer block, backward
     "tp_attention_heads", "tp_attn_block", "tp_attn_block_workspace_size",
     "tp_layer_norm", "tp_reduce_partials_residual", "tp_transformer_block",
@@ -92,6 +93,10 @@ def _load() -> ctypes.CDLL:
                                  i32, vp]
     lib.tp_mlp_block_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i32, i32, i32,
                                          i32, vp]
+    lib.tp_mlp_block_host.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sz, i64, i64, i64, i32, i32,
+                                      i32, i32, vp]
+    lib.tp_mlp_block_host_workspace_size.argtypes = [i64, i64, i64, i32, i32, i32, i32]
+    lib.tp_mlp_block_host_workspace_size.restype = sz
     lib.tp_attention_heads.argtypes = [vp, vp, vp, vp, i64, i32, i32, i32, i32, i32, vp]
     lib.tp_attn_block.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, sz, i64, i64, i32, i32, i32, i32,
                                   i32, vp]
@@ -124,7 +129,7 @@ def _load() -> ctypes.CDLL:
     lib.tp_kernel_launch_count.restype = u64
     lib.tp_abi_version.argtypes = []
     for f in ("tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
-              "tp_mlp_block_noalloc", "tp_attention_heads", "tp_attn_block", "tp_layer_norm",
+              "tp_mlp_block_noalloc", "tp_mlp_block_host", "tp_attention_heads", "tp_attn_block", "tp_layer_norm",
               "tp_reduce_partials_residual", "tp_transformer_block", "tp_mlp_block_backward",
               "tp_mlp_block_backward_recompute", "tp_sync_status", "tp_abi_version"):
         getattr(lib, f).restype = i32
@@ -183,6 +188,21 @@ def tp_mlp_block(X, W1, W_up, b1, W2, b2, Z, workspace, workspace_bytes, T, d, k
     return _check(_lib.tp_mlp_block(_ptr(X), _ptr(W1), _ptr(W_up), _ptr(b1), _ptr(W2), _ptr(b2),
                                     _ptr(Z), _ptr(workspace), workspace_bytes, T, d, k, p, dtype,
                                     act, flags, _stream(stream)), check)
+
+
+def tp_mlp_block_host(X_host, W1, W_up, b1, W2, b2, Z_host, workspace, workspace_bytes, T, d, k,
+                      p, dtype, act, flags=TP_FLAG_NONE, stream=None, check=True):
+    """The whole block with X and Z in host memory (pinned for overlap): the
+    token rows are pipelined in chunks through copy-in, the block and
+    copy-out on the GPU's copy engines; Z_host is complete once `stream`
+    reaches the call."""
+    return _check(_lib.tp_mlp_block_host(_ptr(X_host), _ptr(W1), _ptr(W_up), _ptr(b1), _ptr(W2),
+                                         _ptr(b2), _ptr(Z_host), _ptr(workspace), workspace_bytes,
+                                         T, d, k, p, dtype, act, flags, _stream(stream)), check)
+
+
+def tp_mlp_block_host_workspace_size(T, d, k, p, dtype, act, flags=TP_FLAG_NONE) -> int:
+    return int(_lib.tp_mlp_block_host_workspace_size(T, d, k, p, dtype, act, flags))
 
 
 def tp_mlp_block_noalloc(X, W1, W_up, b1, W2, b2, Z, T, d, k, p, dtype, act,

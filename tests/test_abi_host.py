@@ -153,3 +153,52 @@ def test_bf16_bias_alignment_is_checked():
     st = tp.tp_column_linear(FAKE, FAKE, None, FAKE + 2, FAKE2, 4, 64, 256, 4, tp.TP_BF16,
                              tp.TP_ACT_GELU_TANH, stream=0, check=False)
     assert st == 3
+
+
+def test_host_entry_workspace_and_validation():
+    """tp_mlp_block_host: device copies of X and Z plus one chunk's block
+    workspace (chunks of >= 256 rows, multiples of 128, at most four); every
+    argument error returns before anything is enqueued, and a valid call
+    without a GPU fails loudly."""
+    def r256(n):
+        return -(-n // 256) * 256
+
+    T, d, k, p = 1024, 768, 3072, 2
+    want = r256(T * d * 2) + r256(T * d * 4) + tp.tp_mlp_block_workspace_size(
+        256, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH)
+    assert tp.tp_mlp_block_host_workspace_size(T, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH) == want
+    # 300 rows -> two chunks of 256 (the second one ragged)
+    assert tp.tp_mlp_block_host_workspace_size(300, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH) == \
+        r256(300 * d * 2) + r256(300 * d * 4) + tp.tp_mlp_block_workspace_size(
+            256, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH)
+    # 4096 rows -> four chunks of 1024
+    assert tp.tp_mlp_block_host_workspace_size(4096, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH) == \
+        r256(4096 * d * 2) + r256(4096 * d * 4) + tp.tp_mlp_block_workspace_size(
+            1024, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH)
+    assert tp.tp_mlp_block_host_workspace_size(T, d, 3071, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH) == 0
+
+    def call(**kw):
+        a = dict(X=FAKE, W1=FAKE, W_up=None, b1=None, W2=FAKE, b2=None, Z=FAKE2, ws=0x40000,
+                 wsb=1 << 30, T=4, d=64, k=256, p=4, dtype=tp.TP_BF16, act=tp.TP_ACT_GELU_TANH,
+                 flags=0)
+        a.update(kw)
+        return tp.tp_mlp_block_host(a["X"], a["W1"], a["W_up"], a["b1"], a["W2"], a["b2"],
+                                    a["Z"], a["ws"], a["wsb"], a["T"], a["d"], a["k"], a["p"],
+                                    a["dtype"], a["act"], a["flags"], stream=0, check=False)
+    n0 = tp.tp_kernel_launch_count()
+    assert call(T=0, X=None, Z=None, ws=None, wsb=0) == 0     # empty: a no-op
+    assert call(k=255) == 2
+    assert call(flags=8) == 1
+    assert call(X=None) == 1
+    assert call(Z=None) == 1
+    assert call(W1=None) == 1
+    assert call(W1=FAKE + 2) == 3
+    assert call(act=tp.TP_ACT_SWIGLU) == 1                   # SwiGLU needs W_up
+    assert call(b1=FAKE + 2) == 3
+    assert call(wsb=16) == 7
+    assert call(ws=0x40000 + 16) == 3
+    assert call(T=-1) == 1
+    assert tp.tp_kernel_launch_count() == n0
+    import torch
+    if not torch.cuda.is_available():
+        assert call() == 5
