@@ -139,6 +139,8 @@ BLOCK_CASES = [
     (300, 256, 4, 4, 4, False, False),
     (1, 128, 2, 2, 1, True, True),
     (520, 512, 8, 2, 2, True, False),
+    (130, 256, 16, 16, 1, True, True),   # 16 heads on one shard: 2048-row W_O shard
+    (200, 384, 32, 8, 2, False, True),   # 4 query heads per K/V head, 16 per shard
 ]
 
 
