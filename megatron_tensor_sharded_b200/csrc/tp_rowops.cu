@@ -59,25 +59,43 @@ __global__ void __launch_bounds__(kThreads) row_fold_ln_kernel(
   // persistent: a fixed grid of resident CTAs walks the rows
   for (int64_t row = blockIdx.x; row < T; row += gridDim.x) {
   const int64_t base = row * d;
+  // The fold, shard by shard over the whole row: each shard's NV vectors are
+  // loaded together (NV loads in flight per thread, not one), and every
+  // element still takes its additions in shard order, then bias, then R.
   float4 h[NV];
+  const float4* src = reinterpret_cast<const float4*>((p > 0 ? part : R) + base);
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
     const int64_t c = threadIdx.x + static_cast<int64_t>(k) * kThreads;
-    if (c < d4) {
-      float4 acc;
-      if (p > 0) {
-        acc = __ldcs(reinterpret_cast<const float4*>(part + base) + c);
-        for (int s = 1; s < p; ++s)
-          acc = add4(acc, __ldcs(reinterpret_cast<const float4*>(part + s * part_stride + base) + c));
-        if (bias != nullptr) acc = add4(acc, __ldg(reinterpret_cast<const float4*>(bias) + c));
-        if (R != nullptr) acc = add4(acc, reinterpret_cast<const float4*>(R + base)[c]);
-      } else {
-        acc = reinterpret_cast<const float4*>(R + base)[c];
+    h[k] = c < d4 ? (p > 0 ? __ldcs(src + c) : src[c]) : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  if (p > 0) {
+    for (int s = 1; s < p; ++s) {
+      const float4* ps = reinterpret_cast<const float4*>(part + s * part_stride + base);
+      float4 v[NV];
+#pragma unroll
+      for (int k = 0; k < NV; ++k) {
+        const int64_t c = threadIdx.x + static_cast<int64_t>(k) * kThreads;
+        if (c < d4) v[k] = __ldcs(ps + c);
       }
-      h[k] = acc;
-      if (H != nullptr) reinterpret_cast<float4*>(H + base)[c] = acc;
-    } else {
-      h[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int k = 0; k < NV; ++k)
+        if (threadIdx.x + static_cast<int64_t>(k) * kThreads < d4) h[k] = add4(h[k], v[k]);
+    }
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      const int64_t c = threadIdx.x + static_cast<int64_t>(k) * kThreads;
+      if (c < d4) {
+        if (bias != nullptr) h[k] = add4(h[k], __ldg(reinterpret_cast<const float4*>(bias) + c));
+        if (R != nullptr) h[k] = add4(h[k], reinterpret_cast<const float4*>(R + base)[c]);
+      }
+    }
+  }
+  if (H != nullptr) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+      const int64_t c = threadIdx.x + static_cast<int64_t>(k) * kThreads;
+      if (c < d4) reinterpret_cast<float4*>(H + base)[c] = h[k];
     }
   }
   if (Y == nullptr) continue;
