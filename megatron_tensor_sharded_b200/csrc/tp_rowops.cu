@@ -18,6 +18,7 @@
 #include <atomic>
 #include <cstdint>
 #include <cstring>
+#include <type_traits>
 
 #include "tp_device.cuh"
 #include "tp_internal.h"
@@ -47,7 +48,9 @@ __device__ __forceinline__ float block_sum(float v, float* red) {
   return s;
 }
 
-template <int NV>
+// FOLD = false is the plain LayerNorm of R (p == 0): no partial loads, so
+// the instance needs fewer registers and more CTAs stay resident.
+template <int NV, bool FOLD>
 __global__ void __launch_bounds__(kThreads) row_fold_ln_kernel(
     const float* __restrict__ part, int p, int64_t part_stride, const float* __restrict__ bias,
     const float* R, float* H, const float* __restrict__ gamma, const float* __restrict__ beta,
@@ -63,13 +66,13 @@ __global__ void __launch_bounds__(kThreads) row_fold_ln_kernel(
   // loaded together (NV loads in flight per thread, not one), and every
   // element still takes its additions in shard order, then bias, then R.
   float4 h[NV];
-  const float4* src = reinterpret_cast<const float4*>((p > 0 ? part : R) + base);
+  const float4* src = reinterpret_cast<const float4*>((FOLD ? part : R) + base);
 #pragma unroll
   for (int k = 0; k < NV; ++k) {
     const int64_t c = threadIdx.x + static_cast<int64_t>(k) * kThreads;
-    h[k] = c < d4 ? (p > 0 ? __ldcs(src + c) : src[c]) : make_float4(0.f, 0.f, 0.f, 0.f);
+    h[k] = c < d4 ? (FOLD ? __ldcs(src + c) : src[c]) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  if (p > 0) {
+  if constexpr (FOLD) {
     for (int s = 1; s < p; ++s) {
       const float4* ps = reinterpret_cast<const float4*>(part + s * part_stride + base);
       float4 v[NV];
@@ -215,30 +218,31 @@ cudaError_t launch_row_fold_ln(const LaunchCtx& c, const float* P, int p, const 
   const int64_t ps = T * d;
   // a persistent grid: as many CTAs as fit on the SMs at once (by the
   // kernel's register use), each walking rows blockIdx.x, + gridDim.x, ...
-  auto go = [&](auto kern) {
-    static std::atomic<int> cached{0};   // per kernel instantiation
-    int per_sm = cached.load(std::memory_order_relaxed);
+  // Residency is looked up once per instantiation: every instantiation has
+  // the same function type, so each gets its own slot (index `slot`).
+  static std::atomic<int> per_sm_cache[10];
+  auto go = [&](auto kern, int slot) {
+    int per_sm = per_sm_cache[slot].load(std::memory_order_relaxed);
     if (per_sm == 0) {
       if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, 0) != cudaSuccess ||
           per_sm < 1)
         per_sm = 1;
-      cached.store(per_sm, std::memory_order_relaxed);
+      per_sm_cache[slot].store(per_sm, std::memory_order_relaxed);
     }
     const int64_t resident = static_cast<int64_t>(c.num_sms) * per_sm;
     const dim3 g(static_cast<unsigned>(T < resident ? T : resident)), b(kThreads);
     return launch_pdl(kern, g, b, 0, c.stream, P, p, ps, bias, R, H, gamma, beta, y, T, d, eps);
   };
-  cudaError_t e;
-  if (nv <= 1)
-    e = go(row_fold_ln_kernel<1>);
-  else if (nv <= 2)
-    e = go(row_fold_ln_kernel<2>);
-  else if (nv <= 4)
-    e = go(row_fold_ln_kernel<4>);
-  else if (nv <= 8)
-    e = go(row_fold_ln_kernel<8>);
-  else
-    e = go(row_fold_ln_kernel<kMaxV>);
+  auto pick = [&](auto fold) {
+    constexpr bool F = decltype(fold)::value;
+    constexpr int f = F ? 5 : 0;
+    if (nv <= 1) return go(row_fold_ln_kernel<1, F>, f + 0);
+    if (nv <= 2) return go(row_fold_ln_kernel<2, F>, f + 1);
+    if (nv <= 4) return go(row_fold_ln_kernel<4, F>, f + 2);
+    if (nv <= 8) return go(row_fold_ln_kernel<8, F>, f + 3);
+    return go(row_fold_ln_kernel<kMaxV, F>, f + 4);
+  };
+  const cudaError_t e = p > 0 ? pick(std::true_type{}) : pick(std::false_type{});
   note_launch();
   return e;
 }
