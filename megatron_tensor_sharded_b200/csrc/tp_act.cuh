@@ -20,8 +20,10 @@ __device__ __forceinline__ float gelu_tanh_f32(float h) {
 __device__ __forceinline__ float silu_f32(float h) { return h / (1.0f + expf(-h)); }
 
 // Hardware tanh (PTX tanh.approx.f32, one MUFU operation, relative error
-// about 2^-11): used where the result is stored as bf16 (8 significant bits),
-// so its error stays well below the storage rounding.
+// about 2^-11): used where the result is stored as bf16 (8 significant bits).
+// Its absolute error (about 2^-11 near |tanh| = 1) is below the storage
+// rounding of the activation except where 1 + tanh cancels (GELU of
+// h below about -2, a value near zero with a tiny absolute error).
 __device__ __forceinline__ float tanh_mufu(float x) {
   float y;
   asm("tanh.approx.f32 %0, %1;" : "=f"(y) : "f"(x));

@@ -146,8 +146,11 @@ __device__ __forceinline__ void store_bf16x8(const TcParams& P, int row, int32_t
 //                     c1 = sqrt(2/pi), c3 = 0.044715 c1;
 //   SwiGLU:           a + a tanh(g/2),  a = (g/2) up  (= SiLU(g) up, since
 //                     sigmoid(g) = (1 + tanh(g/2)) / 2).
-// tanh is the MUFU approximation (relative error about 2^-11, below the
-// bf16 rounding of the result).
+// tanh is the MUFU approximation (relative error about 2^-11 of tanh): the
+// GELU value then carries an absolute error of at most about 2^-11 |h| / 2,
+// below its bf16 rounding wherever |GELU(h)| is not small; in the negative
+// tail (h below about -2, where 1 + tanh(u) cancels) the relative error is
+// larger but the value, and its absolute error, are tiny.
 
 // Two bf16 bias values (one 32-bit word, lower column first) as a pair.
 __device__ __forceinline__ uint64_t bf16_word_to_pair(uint32_t w) {
