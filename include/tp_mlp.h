@@ -201,7 +201,7 @@ size_t tp_mlp_block_workspace_size(int64_t T, int64_t d, int64_t k, int p,
  * written to, host buffers; the weights and biases are device buffers (they
  * stay resident between calls).  The block is row-wise (row t of Z depends
  * only on row t of X: "Tensor parallel math", "The MLP block: column then
- * row, one all-reduce"), so the call cuts the T token rows into up to four
+ * row, one all-reduce"), so the call cuts the T token rows into up to eight
  * chunks (multiples of 128 rows, at least 256 each) and pipelines them: the
  * copy of chunk c+1 into the device, the block on chunk c and the copy of
  * chunk c-1 back to the host overlap on the GPU's two copy engines and its

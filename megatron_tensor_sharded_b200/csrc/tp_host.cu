@@ -28,8 +28,8 @@
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxChunks = 4;
-constexpr int64_t kMinChunkRows = 256;
+constexpr int kMaxChunks = 8;
+constexpr int64_t kMinChunkRows = 256;   // smaller chunks cost more in launches than they hide
 constexpr int64_t kRowAlign = 128;   // keeps every chunk's rows 256-byte aligned
 
 struct Pipe {
@@ -44,8 +44,8 @@ std::mutex g_pipe_mu[kMaxDevices];
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Rows per chunk: up to kMaxChunks chunks of at least kMinChunkRows rows,
-// each a multiple of kRowAlign rows except the last.
+// Rows per chunk: up to kMaxChunks chunks, each a multiple of kRowAlign rows
+// and at least kMinChunkRows long, except the last, which takes what is left.
 int64_t chunk_rows(int64_t T) {
   if (T <= kMinChunkRows) return T;
   int64_t n = (T + kMinChunkRows - 1) / kMinChunkRows;
