@@ -245,13 +245,29 @@ def check_sharded_matches_unsharded():
             assert O.rel_err(Z, want) < 1e-12, (act, p)
 
 
+def check_rel_err():
+    """The parity measure on hand-worked cases: max|got - want| / max|want|,
+    with the largest difference and the largest reference element at
+    different places, a negative reference maximum, a negative difference,
+    a reference whose mean is far below its maximum, an all-zero reference
+    (absolute difference) and empty arrays."""
+    g = _golden("rel_err_by_hand.json")
+    for c in g["cases"]:
+        got = np.array(c["got"], dtype=np.float64)
+        want = np.array(c["want"], dtype=np.float64)
+        expected = c["expected_num"] / c["expected_den"]
+        r = O.rel_err(got, want)
+        assert isinstance(r, float), c["name"]
+        assert r == expected, (c["name"], r, expected)
+
+
 # --------------------------------------------------------------------------
 # tests
 # --------------------------------------------------------------------------
 
 PINS = [check_page_column_concat, check_shard_shapes, check_tiny_block_by_hand, check_fold_order,
         check_brute_force_tiny, check_closed_form_identity, check_activation_values,
-        check_p1_is_the_textbook_block, check_sharded_matches_unsharded]
+        check_p1_is_the_textbook_block, check_sharded_matches_unsharded, check_rel_err]
 
 
 @pytest.mark.parametrize("pin", PINS, ids=lambda f: f.__name__)
@@ -384,6 +400,47 @@ def _mut_relu_leaky(h):
     return np.where(h > 0, h, 0.01 * h)
 
 
+def _mut_rel_err_mean_denominator(got, want):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    if not want.size:
+        return 0.0
+    den = float(np.mean(np.abs(want)))
+    num = float(np.max(np.abs(got - want)))
+    return num if den == 0.0 else num / den
+
+
+def _mut_rel_err_per_element(got, want):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    if not want.size:
+        return 0.0
+    diff = np.abs(got - want)
+    a = np.abs(want)
+    ratio = np.where(a > 0, diff / np.where(a > 0, a, 1.0), diff)
+    return float(np.max(ratio))
+
+
+def _mut_rel_err_signed_max(got, want):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    if not want.size:
+        return 0.0
+    den = float(np.max(want))
+    num = float(np.max(np.abs(got - want)))
+    return num if den == 0.0 else num / den
+
+
+def _mut_rel_err_no_abs(got, want):
+    got = np.asarray(got, dtype=np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    if not want.size:
+        return 0.0
+    den = float(np.max(np.abs(want)))
+    num = float(np.max(got - want))
+    return num if den == 0.0 else num / den
+
+
 MUTATIONS = {
     "row_slice_uses_columns": ("_row_slice", _mut_row_slice_uses_columns),
     "row_slice_wrong_shard": ("_row_slice", _mut_row_slice_off_by_one),
@@ -398,6 +455,10 @@ MUTATIONS = {
     "reduce_reversed_order": ("reduce_partials_fixed_order", _mut_reduce_reversed),
     "reduce_in_float64": ("reduce_partials_fixed_order", _mut_reduce_in_float64),
     "swiglu_gate_up_swapped": ("apply_activation", _mut_swiglu_swapped),
+    "rel_err_mean_denominator": ("rel_err", _mut_rel_err_mean_denominator),
+    "rel_err_per_element_ratio": ("rel_err", _mut_rel_err_per_element),
+    "rel_err_signed_max": ("rel_err", _mut_rel_err_signed_max),
+    "rel_err_abs_missing": ("rel_err", _mut_rel_err_no_abs),
 }
 
 
