@@ -466,6 +466,285 @@ class Harness:
 
 # ----------------------------------------------------------------------------- GPU arm
 
+def clocks_capped(clk: dict) -> bool:
+    """True when the SM clocks of a timed loop were held below their maximum
+    (the power cap active, or a median clock under 97% of the maximum)."""
+    if not clk or clk.get("sm_mhz") is None:
+        return False
+    if "sw_power_cap" in clk.get("reasons", []):
+        return True
+    return bool(clk.get("sm_max_mhz")) and clk["sm_mhz"] < 0.97 * clk["sm_max_mhz"]
+
+
+def tensor_peak(peaks: dict, peak_src: str, clk: dict):
+    """The bf16 denominator for a loop: the burst figure when the loop ran at
+    full clocks, the sustained (power-capped) figure when it did not."""
+    if clocks_capped(clk):
+        return peaks["bf16_tflops_sustained"], f"{peak_src} bf16 dense (sustained, power-capped loop)"
+    return peaks["bf16_tflops"], f"{peak_src} bf16 dense (burst)"
+
+
+def traffic_entry(key: str) -> dict:
+    """roofline.traffic and where it comes from: the committed ncu table,
+    keyed by workload/kernel and by a digest of the kernels' device code."""
+    v = ncu_traffic(key)
+    if v is None:
+        return {"traffic": None,
+                "traffic_source": f"none: no ncu figure for {key} on the current kernel code"}
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    with open(path) as f:
+        ent = json.load(f)[key]
+    return {"traffic": v,
+            "traffic_source": f"profiles/ncu_traffic.json[{key}] (cold-cache ncu capture, "
+                              f"device-code digest {ent['source_sha']})"}
+
+
+class MlpBench:
+    """Device buffers of one MLP workload and the timed loops over them: the
+    block step (one CUDA-graph replay of tp_mlp_block) and the same block as
+    the three separate C-ABI calls with events between them."""
+
+    def __init__(self, a, torch, tp, w: WL.Workload, inp: WL.Inputs, device, mode: str, barrier,
+                 dist, world: int):
+        self.a, self.torch, self.tp, self.w, self.device = a, torch, tp, w, device
+        self.barrier, self.dist, self.world = barrier, dist, world
+        self.inp = inp
+
+        def dev(x):
+            if x is None:
+                return None
+            if x.dtype == np.uint16:
+                return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
+            return torch.from_numpy(x).to(device)
+
+        self.X, self.W1, self.Wu, self.b1 = dev(inp.X), dev(inp.W1), dev(inp.W_up), dev(inp.b1)
+        self.W2, self.b2 = dev(inp.W2), dev(inp.b2)
+        self.dtype = tp.DTYPE[w.dtype]
+        self.act = tp.ACT[w.act]
+        hdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+        self.Y = torch.empty((w.p, w.T, w.s), dtype=hdt, device=device)
+        self.P = torch.empty((w.p, w.T, w.d), dtype=torch.float32, device=device)
+        self.Z = torch.empty((w.T, w.d), dtype=torch.float32, device=device)
+        self.flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
+        self.stream = torch.cuda.current_stream(device)
+        self.mode = mode
+        self.flags = {"partials": tp.TP_FLAG_NONE, "splitk": tp.TP_FLAG_SPLITK_FUSED,
+                      "fused": tp.TP_FLAG_FUSED_LAUNCH, "fold": tp.TP_FLAG_ROW_FOLD}[mode]
+        self.nbytes = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, w.p, self.dtype, self.act,
+                                                     self.flags)
+        self.ws = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        self.evs = None
+
+    def block_step(self, st):
+        w, tp = self.w, self.tp
+        tp.tp_mlp_block(self.X, self.W1, self.Wu, self.b1, self.W2, self.b2, self.Z, self.ws,
+                        self.nbytes, w.T, w.d, w.k, w.p, self.dtype, self.act, self.flags,
+                        stream=st)
+
+    def calls_step(self, st):
+        w, tp, ev = self.w, self.tp, self.evs
+        ev[0].record(st)
+        tp.tp_column_linear(self.X, self.W1, self.Wu, self.b1, self.Y, w.T, w.d, w.k, w.p,
+                            self.dtype, self.act, stream=st)
+        ev[1].record(st)
+        tp.tp_row_linear(self.Y, self.W2, self.P, w.T, w.k, w.d, w.p, self.dtype, stream=st)
+        ev[2].record(st)
+        tp.tp_reduce_partials(self.P, self.b2, self.Z, w.T, w.d, w.p, stream=st)
+        ev[3].record(st)
+
+    def capture(self, fn):
+        """Warm up eagerly, then capture one step as a CUDA graph; returns
+        (graph, kernels of this library per step)."""
+        torch, tp = self.torch, self.tp
+        for _ in range(self.a.warmup):
+            self.flush.zero_()
+            fn(self.stream)
+        tp.tp_sync_status(self.stream)
+        if self.a.no_graph:
+            return None, None
+        g = torch.cuda.CUDAGraph()
+        n0 = tp.tp_kernel_launch_count()
+        with torch.cuda.graph(g):
+            fn(torch.cuda.current_stream())
+        per_step = tp.tp_kernel_launch_count() - n0
+        for _ in range(self.a.warmup):
+            self.flush.zero_()
+            g.replay()
+        torch.cuda.synchronize(self.device)
+        return g, per_step
+
+    def rmax(self, vals):
+        return reduce_max(vals, self.dist if self.world > 1 else None, self.device)
+
+    def time_block(self, gpu_index: int, flush: bool = True):
+        """K steps of the block, one graph replay each, L2 flushed before each
+        step outside the events.  Returns (ms per step max over ranks, library
+        launches in the timed region, clock summary, wall seconds)."""
+        torch, tp = self.torch, self.tp
+        if not hasattr(self, "g_block"):
+            self.g_block, self.k_block = self.capture(self.block_step)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        step_ms = []
+        with ClockSampler(gpu_index) as clocks:
+            self.barrier()
+            torch.cuda.synchronize(self.device)
+            n0 = tp.tp_kernel_launch_count()
+            t_wall = time.perf_counter()
+            for _ in range(self.a.steps):
+                if flush:
+                    self.flush.zero_()
+                e0.record(self.stream)
+                if self.g_block is not None:
+                    self.g_block.replay()
+                else:
+                    self.block_step(self.stream)
+                e1.record(self.stream)
+                torch.cuda.synchronize(self.device)
+                step_ms.append(e0.elapsed_time(e1))
+            t_wall = time.perf_counter() - t_wall
+            launches = tp.tp_kernel_launch_count() - n0
+            if self.g_block is not None:
+                launches = self.k_block * self.a.steps
+            self.barrier()
+        tp.tp_sync_status(self.stream)
+        ms, launches = self.rmax([statistics.mean(step_ms), float(launches)])
+        return ms, int(launches), clocks.summary(), t_wall
+
+    def time_calls(self, gpu_index: int):
+        """The block as the three C-ABI calls (one graph), events between them:
+        per-layer times (max over ranks) and the loop's clock summary."""
+        torch, tp = self.torch, self.tp
+        self.evs = [torch.cuda.Event(enable_timing=True, external=not self.a.no_graph)
+                    for _ in range(4)]
+        g_calls, _ = self.capture(self.calls_step)
+        col, row, red, tot = [], [], [], []
+        with ClockSampler(gpu_index) as clocks:
+            self.barrier()
+            for _ in range(self.a.steps):
+                self.flush.zero_()
+                if g_calls is not None:
+                    g_calls.replay()
+                else:
+                    self.calls_step(self.stream)
+                torch.cuda.synchronize(self.device)
+                ev = self.evs
+                col.append(ev[0].elapsed_time(ev[1]))
+                row.append(ev[1].elapsed_time(ev[2]))
+                red.append(ev[2].elapsed_time(ev[3]))
+                tot.append(ev[0].elapsed_time(ev[3]))
+            self.barrier()
+        tp.tp_sync_status(self.stream)
+        vals = self.rmax([statistics.mean(x) for x in (col, row, red, tot)])
+        return dict(zip(["column", "row", "reduce", "sum"], vals)), clocks.summary()
+
+
+def layer_figures(w: WL.Workload, kernels: dict, clk: dict, peaks: dict, peak_src: str) -> dict:
+    """Per-layer throughput of the three-call loop against the peak that fits
+    that loop's clocks, with the clock record and time x median SM MHz."""
+    peak, src = tensor_peak(peaks, peak_src, clk)
+
+    def tfl(f, ms):
+        return f / (ms * 1e-3) / 1e12
+
+    mhz = clk.get("sm_mhz")
+    out = {}
+    bf16 = w.dtype == "bf16"
+    for name, fl in (("column", column_flops(w)), ("row", row_flops(w))):
+        ms = kernels[name]
+        out[name] = {"ms": ms, "TFLOP/s": tfl(fl, ms),
+                     "frac_bf16_peak": tfl(fl, ms) / peak if bf16 else None,
+                     "frac_bf16_burst": tfl(fl, ms) / peaks["bf16_tflops"] if bf16 else None,
+                     "ms_x_mhz": None if mhz is None else ms * mhz}
+    rb = reduce_bytes(w)
+    gbs = rb / (kernels["reduce"] * 1e-3) / 1e9
+    out["reduce"] = {"ms": kernels["reduce"], "GB/s": gbs, "frac_hbm": gbs / peaks["hbm_gbs"],
+                     "bytes": rb, "ms_x_mhz": None if mhz is None else kernels["reduce"] * mhz}
+    out["step_ms"] = kernels["sum"]
+    out["peak"] = {"bf16_tflops": peak, "source": src, "hbm_gbs": peaks["hbm_gbs"]}
+    out["clocks"] = clk
+    out["how"] = ("the three C-ABI calls as one graph, external timing events between them, "
+                  "L2 flushed before each step; clocks sampled over this loop alone")
+    return out
+
+
+def step_roofline(w: WL.Workload, ms: float, clk: dict, peaks: dict, peak_src: str) -> dict:
+    """Whole-step roofline: tensor side unless the step's arithmetic intensity
+    (FLOPs per minimum HBM byte) is below the measured ridge point."""
+    intensity = w.gemm_flops() / block_bytes(w)
+    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if w.dtype == "bf16" and intensity >= ridge:
+        peak, src = tensor_peak(peaks, peak_src, clk)
+        ach = w.gemm_flops() / (ms * 1e-3) / 1e12
+        r = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+             "frac": ach / peak, "peak_source": src}
+    else:
+        ach = block_bytes(w) / (ms * 1e-3) / 1e9
+        r = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+             "frac": ach / peaks["hbm_gbs"], "bytes_per_step": block_bytes(w),
+             "peak_source": f"{peak_src} hbm copy"}
+    r["intensity_flop_per_byte"] = intensity
+    r["ridge_flop_per_byte"] = ridge
+    return r
+
+
+def measure_e2e(a, torch, tp, B: "MlpBench", w: WL.Workload, world: int, barrier) -> dict:
+    """The block through tp_mlp_block_host: X copied in from pinned host
+    memory and Z copied back inside every timed step (plus the same copies
+    run one after the other around tp_mlp_block, for comparison)."""
+    device = B.device
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    stream = B.stream
+    Xh = B.X.cpu().pin_memory()
+    Zh = torch.empty(B.Z.shape, dtype=B.Z.dtype).pin_memory()
+    n_host = tp.tp_mlp_block_host_workspace_size(w.T, w.d, w.k, w.p, B.dtype, B.act, B.flags)
+    ws_host = torch.empty(max(n_host, 256), dtype=torch.uint8, device=device)
+    Xd = torch.empty_like(B.X)
+
+    def e2e_step():
+        tp.tp_mlp_block_host(Xh, B.W1, B.Wu, B.b1, B.W2, B.b2, Zh, ws_host, n_host, w.T, w.d,
+                             w.k, w.p, B.dtype, B.act, B.flags, stream=stream)
+
+    def serial_step():
+        Xd.copy_(Xh, non_blocking=True)
+        tp.tp_mlp_block(Xd, B.W1, B.Wu, B.b1, B.W2, B.b2, B.Z, B.ws, B.nbytes, w.T, w.d, w.k,
+                        w.p, B.dtype, B.act, B.flags, stream=stream)
+        Zh.copy_(B.Z, non_blocking=True)
+
+    def time_e2e(fn):
+        for _ in range(a.warmup):
+            B.flush.zero_()
+            fn()
+        torch.cuda.synchronize(device)
+        barrier()
+        t = []
+        for _ in range(a.steps):
+            B.flush.zero_()
+            e0.record(stream)
+            fn()
+            e1.record(stream)
+            torch.cuda.synchronize(device)
+            t.append(e0.elapsed_time(e1))
+        barrier()
+        tp.tp_sync_status(stream)
+        return B.rmax([statistics.mean(t)])[0]
+
+    e_ms = time_e2e(e2e_step)
+    s_ms = time_e2e(serial_step)
+    e2e = {"value": whole_job_value(w.gemm_flops(), world, e_ms) / 1e12, "unit": UNIT,
+           "ms_per_step": e_ms, "h2d_bytes_per_step": Xh.numel() * Xh.element_size(),
+           "d2h_bytes_per_step": Zh.numel() * Zh.element_size(),
+           "call": "tp_mlp_block_host: X read from and Z written to pinned host memory, the "
+                   "token rows pipelined in chunks through copy-in, the block and copy-out",
+           "serial_copies": {"value": whole_job_value(w.gemm_flops(), world, s_ms) / 1e12,
+                             "ms_per_step": s_ms,
+                             "how": "copy X in, tp_mlp_block on all rows, copy Z out, one "
+                                    "after the other"}}
+
+    return e2e
+
+
 def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -481,260 +760,75 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
         if world > 1:
             dist.barrier()
 
+    peaks, peak_src = load_peaks()
     inp = WL.make_inputs(w)
-
-    def dev(x):
-        if x is None:
-            return None
-        if x.dtype == np.uint16:
-            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(device)
-        return torch.from_numpy(x).to(device)
-
-    X, W1, Wu, b1, W2 = dev(inp.X), dev(inp.W1), dev(inp.W_up), dev(inp.b1), dev(inp.W2)
-    b2 = dev(inp.b2)
-    dtype = tp.DTYPE[w.dtype]
-    act = tp.ACT[w.act]
-    hdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
-    Y = torch.empty((w.p, w.T, w.s), dtype=hdt, device=device)
-    P = torch.empty((w.p, w.T, w.d), dtype=torch.float32, device=device)
-    Z = torch.empty((w.T, w.d), dtype=torch.float32, device=device)
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=device)
-    stream = torch.cuda.current_stream(device)
-    flags = tp.TP_FLAG_SPLITK_FUSED if a.mode == "splitk" else tp.TP_FLAG_NONE
-    if a.mode == "fused":
-        flags = tp.TP_FLAG_FUSED_LAUNCH
-    if a.mode == "fold":
-        flags = tp.TP_FLAG_ROW_FOLD
-    nbytes = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, w.p, dtype, act, flags)
-    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
-
-    def block_step(st):
-        tp.tp_mlp_block(X, W1, Wu, b1, W2, b2, Z, ws, nbytes, w.T, w.d, w.k, w.p, dtype, act,
-                        flags, stream=st)
-
-    def calls_step(st, ev):
-        ev[0].record(st)
-        tp.tp_column_linear(X, W1, Wu, b1, Y, w.T, w.d, w.k, w.p, dtype, act, stream=st)
-        ev[1].record(st)
-        tp.tp_row_linear(Y, W2, P, w.T, w.k, w.d, w.p, dtype, stream=st)
-        ev[2].record(st)
-        tp.tp_reduce_partials(P, b2, Z, w.T, w.d, w.p, stream=st)
-        ev[3].record(st)
-
-    def capture(fn):
-        """Warm up eagerly, then capture one step as a CUDA graph; returns
-        (graph, kernels of this library per step)."""
-        for _ in range(a.warmup):
-            flush.zero_()
-            fn(stream)
-        tp.tp_sync_status(stream)
-        if a.no_graph:
-            return None, None
-        g = torch.cuda.CUDAGraph()
-        n0 = tp.tp_kernel_launch_count()
-        with torch.cuda.graph(g):
-            fn(torch.cuda.current_stream())
-        per_step = tp.tp_kernel_launch_count() - n0
-        for _ in range(a.warmup):
-            flush.zero_()
-            g.replay()
-        torch.cuda.synchronize(device)
-        return g, per_step
+    B = MlpBench(a, torch, tp, w, inp, device, a.mode, barrier, dist, world)
 
     # ---- the timed region: K steps of the block, one graph replay each
-    g_block, k_block = capture(block_step)
-    e0 = torch.cuda.Event(enable_timing=True)
-    e1 = torch.cuda.Event(enable_timing=True)
-    step_ms = []
-    with ClockSampler(local_rank) as clocks:
-        barrier()
-        torch.cuda.synchronize(device)
-        n0 = tp.tp_kernel_launch_count()
-        t_wall = time.perf_counter()
-        for _ in range(a.steps):
-            flush.zero_()
-            e0.record(stream)
-            if g_block is not None:
-                g_block.replay()
-            else:
-                block_step(stream)
-            e1.record(stream)
-            torch.cuda.synchronize(device)
-            step_ms.append(e0.elapsed_time(e1))
-        t_wall = time.perf_counter() - t_wall
-        launches = tp.tp_kernel_launch_count() - n0
-        if g_block is not None:
-            launches = k_block * a.steps
-        barrier()
-    tp.tp_sync_status(stream)
-    ms_step, launches = reduce_max([statistics.mean(step_ms), float(launches)],
-                                   dist if world > 1 else None, device)
+    ms_step, launches, clocks, t_wall = B.time_block(local_rank)
 
     # ---- the same graph replayed without the L2 flush (operands L2-resident
     # when they fit): a labelled second figure, not the metric
     l2_resident = None
-    if g_block is not None:
-        warm = []
-        torch.cuda.synchronize(device)
-        for _ in range(a.steps):
-            e0.record(stream)
-            g_block.replay()
-            e1.record(stream)
-            torch.cuda.synchronize(device)
-            warm.append(e0.elapsed_time(e1))
-        tp.tp_sync_status(stream)
-        w_ms = reduce_max([statistics.mean(warm)], dist if world > 1 else None, device)[0]
+    if B.g_block is not None:
+        w_ms, _, _, _ = B.time_block(local_rank, flush=False)
         l2_resident = {"ms_per_step": w_ms, "value": whole_job_value(w.gemm_flops(), world, w_ms) / 1e12,
                        "unit": UNIT, "how": "graph replay without the L2 flush between steps"}
 
     # ---- per-kernel breakdown of the same block as three separate calls
-    kernels = None
+    breakdown = None
     if a.mode == "partials" and not a.no_breakdown:
-        evs = [torch.cuda.Event(enable_timing=True, external=not a.no_graph) for _ in range(4)]
-        g_calls, _ = capture(lambda st: calls_step(st, evs))
-        col_ms, row_ms, red_ms, sum_ms = [], [], [], []
-        barrier()
-        for _ in range(a.steps):
-            flush.zero_()
-            if g_calls is not None:
-                g_calls.replay()
-            else:
-                calls_step(stream, evs)
-            torch.cuda.synchronize(device)
-            col_ms.append(evs[0].elapsed_time(evs[1]))
-            row_ms.append(evs[1].elapsed_time(evs[2]))
-            red_ms.append(evs[2].elapsed_time(evs[3]))
-            sum_ms.append(evs[0].elapsed_time(evs[3]))
-        barrier()
-        tp.tp_sync_status(stream)
-        kernels = dict(zip(["column", "row", "reduce", "sum"],
-                           reduce_max([statistics.mean(x) for x in (col_ms, row_ms, red_ms, sum_ms)],
-                                      dist if world > 1 else None, device)))
+        kernels, kclk = B.time_calls(local_rank)
+        breakdown = layer_figures(w, kernels, kclk, peaks, peak_src)
 
     # ---- end to end through the public block call with host buffers: X read
     # from, and Z written to, pinned host memory inside the timed step
-    e2e = None
-    if not a.no_e2e:
-        Xh = X.cpu().pin_memory()
-        Zh = torch.empty(Z.shape, dtype=Z.dtype).pin_memory()
-        n_host = tp.tp_mlp_block_host_workspace_size(w.T, w.d, w.k, w.p, dtype, act, flags)
-        ws_host = torch.empty(max(n_host, 256), dtype=torch.uint8, device=device)
-        Xd = torch.empty_like(X)
+    e2e = None if a.no_e2e else measure_e2e(a, torch, tp, B, w, world, barrier)
 
-        def e2e_step():
-            tp.tp_mlp_block_host(Xh, W1, Wu, b1, W2, b2, Zh, ws_host, n_host, w.T, w.d, w.k, w.p,
-                                 dtype, act, flags, stream=stream)
-
-        def serial_step():
-            Xd.copy_(Xh, non_blocking=True)
-            tp.tp_mlp_block(Xd, W1, Wu, b1, W2, b2, Z, ws, nbytes, w.T, w.d, w.k, w.p, dtype, act,
-                            flags, stream=stream)
-            Zh.copy_(Z, non_blocking=True)
-
-        def time_e2e(fn):
-            for _ in range(a.warmup):
-                flush.zero_()
-                fn()
-            torch.cuda.synchronize(device)
-            barrier()
-            t = []
-            for _ in range(a.steps):
-                flush.zero_()
-                e0.record(stream)
-                fn()
-                e1.record(stream)
-                torch.cuda.synchronize(device)
-                t.append(e0.elapsed_time(e1))
-            barrier()
-            tp.tp_sync_status(stream)
-            return reduce_max([statistics.mean(t)], dist if world > 1 else None, device)[0]
-
-        e_ms = time_e2e(e2e_step)
-        s_ms = time_e2e(serial_step)
-        e2e = {"value": whole_job_value(w.gemm_flops(), world, e_ms) / 1e12, "unit": UNIT,
-               "ms_per_step": e_ms, "h2d_bytes_per_step": Xh.numel() * Xh.element_size(),
-               "d2h_bytes_per_step": Zh.numel() * Zh.element_size(),
-               "call": "tp_mlp_block_host: X read from and Z written to pinned host memory, the "
-                       "token rows pipelined in chunks through copy-in, the block and copy-out",
-               "serial_copies": {"value": whole_job_value(w.gemm_flops(), world, s_ms) / 1e12,
-                                 "ms_per_step": s_ms,
-                                 "how": "copy X in, tp_mlp_block on all rows, copy Z out, one "
-                                        "after the other"}}
-
-    peaks, peak_src = load_peaks()
     value = whole_job_value(w.gemm_flops(), world, ms_step) / 1e12
     kernel_name = {"partials": "tp_mlp_block: column GEMM -> row GEMM -> fixed-order fold (PDL-chained)",
                    "fold": "tp_mlp_block row-fold: column GEMM -> row GEMM folding the p partials "
                            "in its epilogue (bit-identical to partials + fold)",
                    "splitk": "tp_mlp_block split-K: column GEMM -> row GEMM accumulating all shards",
                    "fused": "tc_block_kernel (both GEMM layers, one launch) -> fold"}[a.mode]
-    # Roofline side: tensor peak unless the step's arithmetic intensity
-    # (FLOPs per minimum HBM byte) is below the measured ridge point.
-    intensity = w.gemm_flops() / block_bytes(w)
-    ridge = peaks["bf16_tflops"] * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if w.dtype == "bf16" and intensity >= ridge:
-        achieved = w.gemm_flops() / (ms_step * 1e-3) / 1e12
-        peak = peaks["bf16_tflops"]
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": ncu_traffic(f"{w.name}/{a.mode}"),
-                "kernel": kernel_name,
-                "duration": "block step time (graph replay, CUDA events on the launching stream)",
-                "traffic_scope": "dram bytes of all kernels of one step (ncu)",
-                "peak_source": f"{peak_src} bf16 dense (burst)"}
-    else:
-        achieved = block_bytes(w) / (ms_step * 1e-3) / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak, "traffic": ncu_traffic(f"{w.name}/{a.mode}"),
-                "kernel": kernel_name, "bytes_per_step": block_bytes(w),
-                "duration": "block step time (graph replay, CUDA events on the launching stream)",
-                "peak_source": f"{peak_src} hbm copy"}
-    roof["intensity_flop_per_byte"] = intensity
-    roof["ridge_flop_per_byte"] = ridge
+    roof = step_roofline(w, ms_step, clocks, peaks, peak_src)
+    roof.update(traffic_entry(f"{w.name}/{a.mode}"))
+    roof.update({"kernel": kernel_name,
+                 "duration": "block step time (graph replay, CUDA events on the launching stream)",
+                 "traffic_scope": "dram bytes of all kernels of one step (ncu)"})
 
     # The dominant kernel (largest share of the separately timed layers):
-    # algorithmic FLOPs (or bytes) per launch over its CUDA-event duration.
-    if kernels is not None:
+    # algorithmic FLOPs (or bytes) per launch over its CUDA-event duration,
+    # against the peak that fits the clocks of the loop it was timed in.
+    if breakdown is not None:
+        ridge = roof["ridge_flop_per_byte"]
         cand = {
-            "column": (column_flops(w), column_bytes(w), kernels["column"],
+            "column": (column_flops(w), column_bytes(w), breakdown["column"]["ms"],
                        "tc_gemm_kernel/tc_gemm_pair_kernel, column layer (all shards)"),
-            "row": (row_flops(w), row_bytes(w), kernels["row"],
+            "row": (row_flops(w), row_bytes(w), breakdown["row"]["ms"],
                     "tc_gemm_kernel/tc_gemm_pair_kernel, row layer to partials (all shards)"),
-            "reduce": (0, reduce_bytes(w), kernels["reduce"], "reduce_vec_kernel, fixed-order fold"),
+            "reduce": (0, reduce_bytes(w), breakdown["reduce"]["ms"],
+                       "reduce_vec_kernel, fixed-order fold"),
         }
         name = max(cand, key=lambda n: cand[n][2])
         fl_k, by_k, ms_k, desc = cand[name]
         if w.dtype == "bf16" and fl_k > 0 and fl_k / by_k >= ridge:
+            peak, src = breakdown["peak"]["bf16_tflops"], breakdown["peak"]["source"]
             ach = fl_k / (ms_k * 1e-3) / 1e12
-            kroof = {"bound": "tensor", "achieved": ach, "peak": peaks["bf16_tflops"],
-                     "unit": "TFLOP/s", "frac": ach / peaks["bf16_tflops"],
-                     "flops_per_launch": fl_k, "peak_source": f"{peak_src} bf16 dense (burst)"}
+            kroof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                     "frac": ach / peak, "frac_of_burst": ach / peaks["bf16_tflops"],
+                     "flops_per_launch": fl_k, "peak_source": src}
         else:
             ach = by_k / (ms_k * 1e-3) / 1e9
             kroof = {"bound": "hbm", "achieved": ach, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": ach / peaks["hbm_gbs"], "bytes_per_launch": by_k,
                      "peak_source": f"{peak_src} hbm copy"}
-        kroof.update({"traffic": ncu_traffic(f"{w.name}/{name}"), "kernel": f"{name}: {desc}",
+        kroof.update(traffic_entry(f"{w.name}/{name}"))
+        kroof.update({"kernel": f"{name}: {desc}",
                       "duration": "average launch duration, CUDA events on the launching stream "
                                   "around the layer's call inside a replayed graph",
-                      "launch_ms": ms_k, "step": roof})
+                      "launch_ms": ms_k, "loop_clocks": breakdown["clocks"], "step": roof})
         roof = kroof
-
-    breakdown = None
-    if kernels is not None:
-        def tfl(f, ms):
-            return f / (ms * 1e-3) / 1e12
-        breakdown = {
-            "column": {"ms": kernels["column"], "TFLOP/s": tfl(column_flops(w), kernels["column"]),
-                       "frac_bf16_peak": tfl(column_flops(w), kernels["column"]) / peaks["bf16_tflops"]},
-            "row": {"ms": kernels["row"], "TFLOP/s": tfl(row_flops(w), kernels["row"]),
-                    "frac_bf16_peak": tfl(row_flops(w), kernels["row"]) / peaks["bf16_tflops"]},
-            "reduce": {"ms": kernels["reduce"], "GB/s": reduce_bytes(w) / (kernels["reduce"] * 1e-3) / 1e9,
-                       "frac_hbm": reduce_bytes(w) / (kernels["reduce"] * 1e-3) / 1e9 / peaks["hbm_gbs"],
-                       "bytes": reduce_bytes(w)},
-            "step_ms": kernels["sum"],
-            "how": "the three C-ABI calls as one graph, external timing events between them",
-        }
 
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": a.steps,
@@ -742,14 +836,14 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
         "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "T": w.T, "d": w.d, "k": w.k, "p": w.p, "act": w.act,
                    "mode": a.mode, "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "launch": "eager" if g_block is None else "cuda-graph replay of tp_mlp_block",
+                   "launch": "eager" if B.g_block is None else "cuda-graph replay of tp_mlp_block",
                    "l2": "flushed before every step (256 MiB write, outside the timed events)"},
         "pct_bf16_peak": 100.0 * value / (peaks["bf16_tflops"] * world) if w.dtype == "bf16" else None,
         "reduce": None if breakdown is None else breakdown["reduce"],
         "unfused_breakdown": breakdown,
         "roofline": roof,
         "gpu_launches": int(launches),
-        "clocks": clocks.summary(),
+        "clocks": clocks,
         "e2e": e2e,
         "l2_resident": l2_resident,
         "wall_s_timed_region": t_wall,
@@ -770,11 +864,40 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
                 "sample": f"first {rows1} of {w.T} token rows, {reps1} reps, float64"}
         except Exception as exc:  # threadpoolctl missing or BLAS not controllable
             line["cpu_baseline"]["single_thread"] = {"unavailable": str(exc)[:120]}
+
+    # ---- the other MLP workloads, each measured the same way in this process
+    # (block step + three-call breakdown), for the per-workload table
+    if world == 1 and not a.no_configs and a.mode == "partials":
+        del B, inp
+        torch.cuda.empty_cache()
+        table = {}
+        for name in [n for n in CONFIG_ORDER if n != w.name]:
+            wc = WL.WORKLOADS[name]
+            Bc = MlpBench(a, torch, tp, wc, WL.make_inputs(wc), device, "partials", barrier, dist,
+                          world)
+            ms_c, _, clk_c, _ = Bc.time_block(local_rank)
+            kern_c, kclk_c = Bc.time_calls(local_rank)
+            lay = layer_figures(wc, kern_c, kclk_c, peaks, peak_src)
+            ent = {"T": wc.T, "d": wc.d, "k": wc.k, "p": wc.p, "act": wc.act, "dtype": wc.dtype,
+                   "ms_per_step": ms_c,
+                   "TFLOP/s": wc.gemm_flops() / (ms_c * 1e-3) / 1e12,
+                   "step_roofline": step_roofline(wc, ms_c, clk_c, peaks, peak_src),
+                   "clocks": clk_c,
+                   "column": lay["column"], "row": lay["row"], "reduce": lay["reduce"],
+                   "layer_loop_clocks": kclk_c, "layer_peak": lay["peak"]}
+            table[name] = ent
+            del Bc
+            torch.cuda.empty_cache()
+        line["configs"] = table
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+# The workloads of the per-workload table, smallest first.
+CONFIG_ORDER = ["toy", "gpt2", "decode", "wide", "llama"]
 
 
 def run_tp_attn(a, w: WL.AttnWorkload, rank: int, world: int, local_rank: int):
@@ -1287,13 +1410,15 @@ def main(argv=None):
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["tp", "reference"], default="tp")
     ap.add_argument("--workload", choices=sorted(WL.WORKLOADS) + sorted(WL.ATTN_WORKLOADS)
-                    + sorted(WL.BLOCK_WORKLOADS), default="gpt2")
+                    + sorted(WL.BLOCK_WORKLOADS), default="llama")
     ap.add_argument("--mode", choices=["partials", "fold", "splitk", "fused", "backward"],
                     default="partials")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch eagerly instead of graph replay")
     ap.add_argument("--no-breakdown", action="store_true", help="skip the per-kernel loop")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-workload table of the other MLP workloads")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")

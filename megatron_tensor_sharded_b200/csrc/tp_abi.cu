@@ -27,6 +27,8 @@ constexpr int kMaxDevices = 64;
 int g_num_sms[kMaxDevices] = {};
 int g_cc_major[kMaxDevices] = {};
 unsigned* g_status_addr[kMaxDevices] = {};
+unsigned long long g_ctx_id[kMaxDevices] = {};   // context the entries above belong to
+uint64_t g_epoch[kMaxDevices] = {};              // bumped whenever that context changes
 std::mutex g_dev_mu;
 
 tp_status fail(tp_status st, const char* fmt, ...) {
@@ -37,15 +39,52 @@ tp_status fail(tp_status st, const char* fmt, ...) {
   return st;
 }
 
+// Process-unique id of the calling thread's current CUDA context (0 if the
+// driver cannot tell).  A device reset, or a context lost after an error,
+// gives the device a new context with a new id, so per-device caches keyed
+// on it are refilled instead of reusing addresses, streams or attributes of
+// a context that no longer exists.
+unsigned long long current_context_id() {
+  using GetCurrent = CUresult (*)(CUcontext*);
+  using GetId = CUresult (*)(CUcontext, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(f);
+  });
+  if (get_current == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 // Per-device properties and the device address of the status word, looked
-// up once per device with that device current.
-tp_status device_state(int* dev_out, int* sms, int* cc_major, unsigned** status) {
+// up with that device current, once per context of the device.
+tp_status device_state(int* dev_out, int* sms, int* cc_major, unsigned** status,
+                       uint64_t* epoch) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return fail(TP_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
   if (dev < 0 || dev >= kMaxDevices) return fail(TP_ERR_UNSUPPORTED, "device index %d", dev);
+  // A thread on which the runtime has not yet made the device's context
+  // current reads id 0 here; the set-up below makes it current (looking up a
+  // device symbol does), and the id read after it decides whether the
+  // context really changed.  Where the driver cannot report ids at all, the
+  // set-up runs once per device.
+  unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lk(g_dev_mu);
-  if (g_status_addr[dev] == nullptr) {
+  if (g_status_addr[dev] == nullptr || g_ctx_id[dev] != ctx) {
     int n = 0, major = 0;
     e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
@@ -53,20 +92,24 @@ tp_status device_state(int* dev_out, int* sms, int* cc_major, unsigned** status)
     if (e == cudaSuccess) e = cudaGetSymbolAddress(&addr, g_tp_status_word);
     if (e != cudaSuccess)
       return fail(TP_ERR_CUDA, "device set-up: %s", cudaGetErrorString(e));
+    ctx = current_context_id();
+    if (g_status_addr[dev] == nullptr || g_ctx_id[dev] != ctx) ++g_epoch[dev];
     g_num_sms[dev] = n;
     g_cc_major[dev] = major;
     g_status_addr[dev] = static_cast<unsigned*>(addr);
+    g_ctx_id[dev] = ctx;
   }
   *dev_out = dev;
   *sms = g_num_sms[dev];
   *cc_major = g_cc_major[dev];
   *status = g_status_addr[dev];
+  if (epoch != nullptr) *epoch = g_epoch[dev];
   return TP_OK;
 }
 
 tp_status make_ctx(void* stream, bool tensor_core, LaunchCtx* c) {
   int cc = 0;
-  tp_status st = device_state(&c->device, &c->num_sms, &cc, &c->err_word);
+  tp_status st = device_state(&c->device, &c->num_sms, &cc, &c->err_word, &c->epoch);
   if (st != TP_OK) return st;
   if (tensor_core && cc != 10)
     return fail(TP_ERR_UNSUPPORTED, "bf16 path needs an sm_100 device (found sm_%d.x)", cc);
@@ -339,6 +382,12 @@ BlockLayout block_layout(int64_t T, int64_t d, int n_heads, int n_kv_heads, int 
 
 }  // namespace
 
+tp_status current_device(int* dev, uint64_t* epoch) {
+  int sms = 0, cc = 0;
+  unsigned* addr = nullptr;
+  return device_state(dev, &sms, &cc, &addr, epoch);
+}
+
 void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 void set_error_detail(const char* fmt, ...) {
@@ -420,13 +469,14 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
   float* P = (splitk || row_fold) ? nullptr : reinterpret_cast<float*>(ws + y_bytes);
   if (dtype == TP_BF16 && (flags & TP_FLAG_FUSED_LAUNCH)) {
     // Both GEMM layers in one persistent launch (its tile counters start at
-    // 0), then the fixed-order fold of the partials.
+    // 0), then the fixed-order fold of the partials.  The device check comes
+    // first, so that an unsupported device returns with nothing enqueued.
+    LaunchCtx c{};
+    TP_TRY(make_ctx(stream, true, &c));
     int* counters = reinterpret_cast<int*>(ws + need - block_counter_bytes(T, d));
     const cudaError_t e = cudaMemsetAsync(counters, 0, block_counter_bytes(T, d),
                                           static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(TP_ERR_CUDA, "counter reset: %s", cudaGetErrorString(e));
-    LaunchCtx c{};
-    TP_TRY(make_ctx(stream, true, &c));
     TP_TRY(launch_tc_block(c, X, W1, W_up, b1, W2, b2, Y, P, Z, counters, T, d, k, p, act, splitk));
     if (splitk) return TP_OK;
     return reduce_impl(P, b2, Z, T, d, p, stream);
@@ -686,7 +736,7 @@ tp_status tp_sync_status(void* stream) {
   g_detail[0] = 0;
   int dev = 0, sms = 0, cc = 0;
   unsigned* addr = nullptr;
-  TP_TRY(device_state(&dev, &sms, &cc, &addr));
+  TP_TRY(device_state(&dev, &sms, &cc, &addr, nullptr));
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(TP_ERR_CUDA, "stream: %s", cudaGetErrorString(e));
   unsigned word = 0;

@@ -512,18 +512,18 @@ tp_status launch_tc_attention(const LaunchCtx& c, const void* Q, const void* K, 
       !make_map_a(&mK, K, static_cast<int64_t>(hkv) * DH, T, p) ||
       !make_map_a(&mV, V, static_cast<int64_t>(hkv) * DH, T, p))
     return TP_ERR_CUDA;
-  static bool attr_done[64] = {};
+  static uint64_t attr_epoch[64] = {};   // context epoch the attribute was set under
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lk(mu);
     const int dev = c.device & 63;
-    if (!attr_done[dev]) {
+    if (attr_epoch[dev] != c.epoch) {
       if (cudaFuncSetAttribute(tc_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                SMEM_BYTES) != cudaSuccess) {
         set_error_detail("cudaFuncSetAttribute failed: %s", cudaGetErrorString(cudaGetLastError()));
         return TP_ERR_CUDA;
       }
-      attr_done[dev] = true;
+      attr_epoch[dev] = c.epoch;
     }
   }
   AttnParams prm{};

@@ -304,19 +304,19 @@ tp_status launch_cfg(const LaunchCtx& c, const CUtensorMap& mX, const CUtensorMa
                      BlockParams B) {
   constexpr int BNMAX = BNC > BNR ? BNC : BNR;
   using Cf = Cfg<BNMAX>;
-  static bool attr_done[64] = {};
+  static uint64_t attr_epoch[64] = {};   // context epoch the attribute was set under
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lk(mu);
     const int dev = c.device & 63;
-    if (!attr_done[dev]) {
+    if (attr_epoch[dev] != c.epoch) {
       if (cudaFuncSetAttribute(tc_block_kernel<SWIGLU, SPLITK, BNC, BNR>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cf::SMEM_BYTES) != cudaSuccess) {
         set_error_detail("cudaFuncSetAttribute failed: %s", cudaGetErrorString(cudaGetLastError()));
         return TP_ERR_CUDA;
       }
-      attr_done[dev] = true;
+      attr_epoch[dev] = c.epoch;
     }
   }
   const int grid = B.num_tiles < c.num_sms ? B.num_tiles : c.num_sms;

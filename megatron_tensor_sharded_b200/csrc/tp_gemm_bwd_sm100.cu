@@ -386,19 +386,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 template <int AMN, int BMN, int EPI, int BN>
 tp_status launch_g(const LaunchCtx& c, const CUtensorMap* maps, GParams prm) {
   using Cf = BCfg<EPI, BN>;
-  static bool attr_done[64] = {};
+  static uint64_t attr_epoch[64] = {};   // context epoch the attribute was set under
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lk(mu);
     const int dev = c.device & 63;
-    if (!attr_done[dev]) {
+    if (attr_epoch[dev] != c.epoch) {
       if (cudaFuncSetAttribute(tc_gemm_bwd_kernel<AMN, BMN, EPI, BN>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cf::SMEM_BYTES) != cudaSuccess) {
         set_error_detail("cudaFuncSetAttribute failed: %s", cudaGetErrorString(cudaGetLastError()));
         return TP_ERR_CUDA;
       }
-      attr_done[dev] = true;
+      attr_epoch[dev] = c.epoch;
     }
   }
   prm.n_tiles = ceil_div(prm.N, BN);

@@ -258,18 +258,18 @@ template <int BN>
 tp_status launch_fold(const LaunchCtx& c, const CUtensorMap& a, const CUtensorMap& b,
                       const CUtensorMap& z, TcParams prm) {
   using Cf = FCfg<BN>;
-  static bool attr_done[64] = {};
+  static uint64_t attr_epoch[64] = {};   // context epoch the attribute was set under
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lk(mu);
     const int dev = c.device & 63;
-    if (!attr_done[dev]) {
+    if (attr_epoch[dev] != c.epoch) {
       if (cudaFuncSetAttribute(tc_row_fold_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cf::SMEM_BYTES) != cudaSuccess) {
         set_error_detail("cudaFuncSetAttribute failed: %s", cudaGetErrorString(cudaGetLastError()));
         return TP_ERR_CUDA;
       }
-      attr_done[dev] = true;
+      attr_epoch[dev] = c.epoch;
     }
   }
   prm.n_tiles = ceil_div(prm.n_total, BN);

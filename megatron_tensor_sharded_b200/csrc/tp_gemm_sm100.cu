@@ -249,19 +249,19 @@ template <int MODE, int BN>
 tp_status launch_mode(const LaunchCtx& c, const CUtensorMap& a, const CUtensorMap& b0,
                       const CUtensorMap& b1, const CUtensorMap& cm, TcParams prm) {
   using Cf = KCfg<MODE, BN>;
-  static bool attr_done[64] = {};
+  static uint64_t attr_epoch[64] = {};   // context epoch the attribute was set under
   static std::mutex mu;
   {
     std::lock_guard<std::mutex> lk(mu);
     const int dev = c.device & 63;
-    if (!attr_done[dev]) {
+    if (attr_epoch[dev] != c.epoch) {
       if (cudaFuncSetAttribute(tc_gemm_kernel<MODE, BN>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
                                Cf::SMEM_BYTES) != cudaSuccess) {
         set_error_detail("cudaFuncSetAttribute failed: %s", cudaGetErrorString(cudaGetLastError()));
         return TP_ERR_CUDA;
       }
-      attr_done[dev] = true;
+      attr_epoch[dev] = c.epoch;
     }
   }
   prm.wait.err = c.err_word;

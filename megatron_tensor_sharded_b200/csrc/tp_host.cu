@@ -34,6 +34,7 @@ constexpr int64_t kRowAlign = 128;   // keeps every chunk's rows 256-byte aligne
 
 struct Pipe {
   bool ready = false;
+  uint64_t epoch = 0;   // context epoch the streams and events were created under
   cudaStream_t h2d = nullptr, d2h = nullptr;
   cudaEvent_t fork = nullptr, join = nullptr;
   cudaEvent_t in[kMaxChunks] = {}, out[kMaxChunks] = {};
@@ -79,9 +80,12 @@ tp_status cuda_fail(cudaError_t e, const char* what) {
   return TP_ERR_CUDA;
 }
 
-// The device's helper streams and events (created on first use).
-tp_status pipe_for(int dev, Pipe** out) {
+// The device's helper streams and events, created on first use and again
+// if the device has since been given a new CUDA context (the old handles died
+// with the old context and are dropped, not destroyed).
+tp_status pipe_for(int dev, uint64_t epoch, Pipe** out) {
   Pipe& P = g_pipe[dev];
+  if (P.ready && P.epoch != epoch) P = Pipe{};
   if (!P.ready) {
     cudaError_t e = cudaStreamCreateWithFlags(&P.h2d, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&P.d2h, cudaStreamNonBlocking);
@@ -93,6 +97,7 @@ tp_status pipe_for(int dev, Pipe** out) {
     }
     if (e != cudaSuccess) return cuda_fail(e, "helper streams / events");
     P.ready = true;
+    P.epoch = epoch;
   }
   *out = &P;
   return TP_OK;
@@ -166,12 +171,14 @@ tp_status tp_mlp_block_host(const void* X_host, const void* W1, const void* W_up
     return TP_ERR_ALIGNMENT;
   }
   int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) {
+  uint64_t epoch = 0;
+  const tp_status sd = tpk::current_device(&dev, &epoch);
+  if (sd != TP_OK) return sd;
+  if (dev >= kMaxDevices) {
     tpk::set_error_detail("device index %d", dev);
     return TP_ERR_UNSUPPORTED;
   }
+  cudaError_t e = cudaSuccess;
 
   const size_t esize = dtype == TP_BF16 ? 2 : 4;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -184,7 +191,7 @@ tp_status tp_mlp_block_host(const void* X_host, const void* W1, const void* W_up
 
   std::lock_guard<std::mutex> lk(g_pipe_mu[dev]);
   Pipe* P = nullptr;
-  const tp_status sp = pipe_for(dev, &P);
+  const tp_status sp = pipe_for(dev, epoch, &P);
   if (sp != TP_OK) return sp;
 
   // Fork: the copies start after the caller's earlier work on `s`.

@@ -18,7 +18,12 @@ struct LaunchCtx {
   unsigned* err_word;    // device address of the per-device status word
   uint64_t timeout_ns;   // limit of each bounded device wait
   int64_t debug_drop;    // fault injection: pipeline slot whose load is skipped (-1: none)
+  uint64_t epoch;        // changes whenever the device gets a new CUDA context: per-device
+                         // caches (function attributes, streams, symbol addresses) compare it
 };
+
+// The current device and its context epoch (see LaunchCtx::epoch).
+tp_status current_device(int* dev, uint64_t* epoch);
 
 // Counts one kernel launch (process-wide, thread-safe).
 void note_launch();

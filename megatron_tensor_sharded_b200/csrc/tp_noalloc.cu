@@ -37,31 +37,29 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 constexpr int kMaxDevices = 64;
 void* g_scratch_addr[kMaxDevices] = {};
+uint64_t g_scratch_epoch[kMaxDevices] = {};   // context epoch the address belongs to
 std::mutex g_scratch_mu;
 
-// Device address of the scratch array on the current device, looked up once
-// per device (the first call on a device does it; make that first call before
-// any stream capture begins).
+// Device address of the scratch array on the current device.  It is looked
+// up with cudaGetSymbolAddress once per device, at the first call on that
+// device (make that first call before any stream capture begins), and again
+// only if the device has since been given a new CUDA context (after a device
+// reset, say), whose copy of the array sits at a different address.
 tp_status scratch_address(void** out) {
   int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) {
-    tpk::set_error_detail("cudaGetDevice: %s", cudaGetErrorString(e));
-    return TP_ERR_CUDA;
-  }
-  if (dev < 0 || dev >= kMaxDevices) {
-    tpk::set_error_detail("device index %d", dev);
-    return TP_ERR_UNSUPPORTED;
-  }
+  uint64_t epoch = 0;
+  const tp_status st = tpk::current_device(&dev, &epoch);
+  if (st != TP_OK) return st;
   std::lock_guard<std::mutex> lk(g_scratch_mu);
-  if (g_scratch_addr[dev] == nullptr) {
+  if (g_scratch_addr[dev] == nullptr || g_scratch_epoch[dev] != epoch) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr) {
       tpk::set_error_detail("cudaGetSymbolAddress(scratch): %s", cudaGetErrorString(e));
       return TP_ERR_CUDA;
     }
     g_scratch_addr[dev] = p;
+    g_scratch_epoch[dev] = epoch;
   }
   *out = g_scratch_addr[dev];
   return TP_OK;

@@ -147,6 +147,22 @@ def test_valid_call_without_gpu_fails_loudly():
                             tp.TP_ACT_GELU_TANH, stream=0)
 
 
+def test_fused_launch_checks_the_device_before_enqueuing():
+    """TP_FLAG_FUSED_LAUNCH resets its tile counters with an asynchronous
+    memset; the device check runs before it, so a call that cannot run
+    returns with nothing enqueued.  Without a CUDA device the error comes from
+    the device query, not from the counter reset."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    st = tp.tp_mlp_block(FAKE, FAKE, None, None, FAKE, None, FAKE2, 0x40000, 1 << 30, 4, 64, 256,
+                         4, tp.TP_BF16, tp.TP_ACT_GELU_TANH, tp.TP_FLAG_FUSED_LAUNCH, stream=0,
+                         check=False)
+    assert st == 5
+    detail = tp.tp_last_error_detail()
+    assert "counter" not in detail, detail
+
+
 def test_bf16_bias_alignment_is_checked():
     """The bf16 column epilogue reads b1 as 16-byte vectors: a misaligned
     bias is refused before any launch."""

@@ -25,7 +25,7 @@ def test_reference_arm_prints_one_contract_line():
         assert key in d, key
     assert d["steps"] == 1 and d["warmup"] == 3 and d["n_gpus"] == 1
     assert d["value"] > 0 and d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
-    assert d["config"]["workload"] == "gpt2"
+    assert d["config"]["workload"] == "llama"   # the default: the largest workload
     cb = d["cpu_baseline"]
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"]
     assert cb["sample"]

@@ -6,9 +6,15 @@ workspace.
 
 Checked through the C ABI against the existing entry point, tp_mlp_block with
 a caller workspace, on two calls in a row (the second call reuses the scratch
-the first one left behind), within the tolerances the other parity tests use.
-This file is collected last so that a run stopping at its first failure has
-already run every other test; it also passes alone in a fresh process."""
+the first one left behind).  Both entry points run the same kernels on the
+same inputs, so the outputs must be identical bit for bit; that also catches
+a wrong offset or an overlap inside the scratch.  Every flag that changes the
+scratch layout is covered: the default (hidden shards then partials), split-K
+(hidden shards only), the single persistent launch (tile counters at the end
+of the scratch, which must start at zero on every call) and the fold in the
+row layer's epilogue.  This file is collected last so that a run stopping at
+its first failure has already run every other test; it also passes alone in
+a fresh process."""
 
 import numpy as np
 import pytest
@@ -16,16 +22,11 @@ import torch
 
 import megatron_tensor_sharded_b200 as tp
 import workloads as W
-from gpu_util import DeviceBlock, host_f32
+from gpu_util import DeviceBlock, bits, host_f32
 
 pytestmark = pytest.mark.gpu
 
 SCRATCH_BYTES = 16 << 20
-
-
-def _rel(a, b):
-    den = float(np.max(np.abs(b)))
-    return float(np.max(np.abs(a - b))) / den if den else float(np.max(np.abs(a - b)))
 
 
 def _noalloc(blk, flags=tp.TP_FLAG_NONE):
@@ -41,33 +42,37 @@ def _reference(blk, flags=tp.TP_FLAG_NONE):
     return Z
 
 
-@pytest.mark.parametrize("name,tol", [("gpt2", 1e-2), ("toy", 1e-5)])
-def test_matches_workspace_entry_point_two_calls_in_a_row(name, tol):
+def _same_bits(got, want):
+    g, w = host_f32(got), host_f32(want)
+    assert not np.isnan(g).any()
+    assert np.array_equal(bits(g), bits(w)), float(np.max(np.abs(g - w)))
+
+
+@pytest.mark.parametrize("name,flags", [
+    ("gpt2", tp.TP_FLAG_NONE),
+    ("toy", tp.TP_FLAG_NONE),
+    ("gpt2", tp.TP_FLAG_SPLITK_FUSED),
+    ("gpt2", tp.TP_FLAG_FUSED_LAUNCH),
+    ("gpt2", tp.TP_FLAG_ROW_FOLD),
+], ids=["gpt2", "toy", "gpt2-splitk", "gpt2-fused-launch", "gpt2-row-fold"])
+def test_bit_identical_to_workspace_entry_point_two_calls_in_a_row(name, flags):
     w = W.WORKLOADS[name]
     first = W.make_inputs(w, seed=42)
     second = W.make_inputs(w, seed=43)
     blocks = [DeviceBlock(x, w.T, w.d, w.k, w.p, w.act) for x in (first, second)]
-    need = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, w.p, blocks[0].dtype, blocks[0].act)
+    need = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, w.p, blocks[0].dtype, blocks[0].act,
+                                          flags)
     assert 0 < need <= SCRATCH_BYTES
-    outs = [_noalloc(b) for b in blocks]          # two calls in a row, same scratch
-    refs = [_reference(b) for b in blocks]
+    outs = [_noalloc(b, flags) for b in blocks]   # two calls in a row, same scratch
+    refs = [_reference(b, flags) for b in blocks]
     tp.tp_sync_status()
     for got, want in zip(outs, refs):
-        g, r = host_f32(got), host_f32(want)
-        assert not np.isnan(g).any()
-        assert _rel(g, r) <= tol
+        _same_bits(got, want)
     # the two inputs differ, so the second call really recomputed
-    assert _rel(host_f32(outs[0]), host_f32(outs[1])) > tol
-
-
-def test_split_k_flag_and_bias_passthrough():
-    w = W.WORKLOADS["gpt2"]
-    blk = DeviceBlock(W.make_inputs(w, seed=44), w.T, w.d, w.k, w.p, w.act)
-    for _ in range(2):
-        got = _noalloc(blk, tp.TP_FLAG_SPLITK_FUSED)
-        want = _reference(blk, tp.TP_FLAG_SPLITK_FUSED)
-        tp.tp_sync_status()
-        assert _rel(host_f32(got), host_f32(want)) <= 1e-2
+    assert not np.array_equal(host_f32(outs[0]), host_f32(outs[1]))
+    # and a third call on the first inputs, after the second call's leftovers
+    _same_bits(_noalloc(blocks[0], flags), refs[0])
+    tp.tp_sync_status()
 
 
 def test_rejects_problems_larger_than_the_scratch():
