@@ -427,6 +427,17 @@ void tp_set_wait_timeout_ns(uint64_t ns);
  * out.  -1 (default) disables it.  Applies to the next launch only. */
 void tp_debug_drop_load(int64_t stage_index);
 
+/* Test hook (not part of the method): y[i] = the attention softmax's
+ * fast 2^x for i < n, x and y fp32 device arrays of n elements (4-byte
+ * aligned, caller-owned).  The kernel computes part of the probabilities
+ * 2^(s - m) on the FMA pipe: round x to the nearest integer n0, a fitted
+ * degree-4 polynomial for 2^(x - n0) on [-1/2, 1/2], n0 added to the
+ * exponent; x is first clamped to >= -126.  On [-126, 0] its relative error
+ * against 2^x is at most 2.7e-6.  Asynchronous on `stream`; TP_ERR_INVALID_ARG
+ * for n < 0 or NULL arrays (n == 0 is a no-op), TP_ERR_ALIGNMENT, and
+ * TP_ERR_UNSUPPORTED off sm_100. */
+tp_status tp_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream);
+
 /* Human-readable name of a status code. */
 const char* tp_status_string(int status);
 

@@ -49,7 +49,8 @@ __all__ = [
     "tp_mlp_block_backward_workspace_size", "tp_mlp_block_backward_recompute",
     "tp_mlp_block_backward_recompute_workspace_size",
     # status, timeouts, introspection
-    "tp_sync_status", "tp_set_wait_timeout_ns", "tp_debug_drop_load", "tp_status_string",
+    "tp_sync_status", "tp_set_wait_timeout_ns", "tp_debug_drop_load", "tp_debug_exp2_poly",
+    "tp_status_string",
     "tp_last_error_detail", "tp_kernel_launch_count", "tp_abi_version",
 ]
 
@@ -121,6 +122,7 @@ def _load() -> ctypes.CDLL:
     lib.tp_set_wait_timeout_ns.restype = None
     lib.tp_debug_drop_load.argtypes = [i64]
     lib.tp_debug_drop_load.restype = None
+    lib.tp_debug_exp2_poly.argtypes = [vp, vp, i64, vp]
     lib.tp_status_string.argtypes = [i32]
     lib.tp_status_string.restype = ctypes.c_char_p
     lib.tp_last_error_detail.argtypes = []
@@ -131,7 +133,8 @@ def _load() -> ctypes.CDLL:
     for f in ("tp_column_linear", "tp_row_linear", "tp_reduce_partials", "tp_mlp_block",
               "tp_mlp_block_noalloc", "tp_mlp_block_host", "tp_attention_heads", "tp_attn_block", "tp_layer_norm",
               "tp_reduce_partials_residual", "tp_transformer_block", "tp_mlp_block_backward",
-              "tp_mlp_block_backward_recompute", "tp_sync_status", "tp_abi_version"):
+              "tp_mlp_block_backward_recompute", "tp_sync_status", "tp_abi_version",
+              "tp_debug_exp2_poly"):
         getattr(lib, f).restype = i32
     return lib
 
@@ -312,6 +315,11 @@ def tp_set_wait_timeout_ns(ns: int) -> None:
 
 def tp_debug_drop_load(stage_index: int) -> None:
     _lib.tp_debug_drop_load(stage_index)
+
+
+def tp_debug_exp2_poly(x, y, n, stream=None, check=True):
+    """Test hook: y[i] = the attention softmax's fast 2^x for i < n (fp32)."""
+    return _check(_lib.tp_debug_exp2_poly(_ptr(x), _ptr(y), n, _stream(stream)), check)
 
 
 def tp_status_string(status: int) -> str:

@@ -753,6 +753,17 @@ tp_status tp_sync_status(void* stream) {
 
 void tp_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns == 0 ? 2000000000ull : ns); }
 
+tp_status tp_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
+  g_detail[0] = 0;
+  if (n < 0 || n > (int64_t(1) << 40)) return fail(TP_ERR_INVALID_ARG, "n = %lld", (long long)n);
+  if (n == 0) return TP_OK;
+  if (x == nullptr || y == nullptr) return fail(TP_ERR_INVALID_ARG, "x or y is NULL");
+  if (!aligned4(x) || !aligned4(y)) return fail(TP_ERR_ALIGNMENT, "x and y must be 4-byte aligned");
+  LaunchCtx c{};
+  TP_TRY(make_ctx(stream, true, &c));
+  return cuda_status(launch_exp2_poly_probe(c, x, y, n), "exp2 probe launch");
+}
+
 void tp_debug_drop_load(int64_t stage_index) { g_debug_drop.store(stage_index < 0 ? -1 : stage_index); }
 
 const char* tp_status_string(int status) {

@@ -113,6 +113,9 @@ tp_status launch_bwd_dw2(const LaunchCtx& c, const void* Y, const void* dZ, floa
 tp_status launch_tc_attention(const LaunchCtx& c, const void* Q, const void* K, const void* V,
                               void* O, int64_t T, int p, int hq, int hkv, int causal);
 
+// Test hook: the attention softmax's 2^x polynomial applied to x[0..n).
+cudaError_t launch_exp2_poly_probe(const LaunchCtx& c, const float* x, float* y, int64_t n);
+
 // Records a human-readable detail for tp_last_error_detail().
 void set_error_detail(const char* fmt, ...);
 
