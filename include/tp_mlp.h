@@ -145,6 +145,66 @@ tp_status tp_reduce_partials(const float* partials, const float* b2, float* Z,
                              int64_t T, int64_t d, int p, void* stream);
 
 /*
+ * The all-reduce of the partials when the p shards live on p GPUs, one
+ * process per GPU ("Simulating row parallel linear": the sum of partials is
+ * the all-reduce over NVLink; "Building GPT from Scratch -- Part 9",
+ * "Implementation Sketch": RowParallelLinear.forward all-reduces the
+ * partial outputs, then adds the bias).  GPU r owns the token-row slab
+ * [row0, row0 + rows) of Z.  This call folds that slab of the p partials in
+ * shard order, exactly as tp_reduce_partials does (bit-identical on the same
+ * values: P_0 first, one fp32 round-to-nearest-even add per shard, b2
+ * last), and writes the folded slab to every destination in `outs` -- the
+ * caller's own Z and, through peer mappings, the other GPUs' Z, so one pass
+ * is both halves of the all-reduce (reduce-scatter and all-gather).
+ *
+ *   partials  HOST array of p device pointers, shard order; partials[j] is
+ *             P_j, a [T][d] fp32 row-major buffer on this GPU or a peer
+ *             mapping of another GPU's buffer (tp_ipc_import).  Only rows
+ *             [row0, row0 + rows) are read.
+ *   b2        [d] fp32 device pointer or NULL.
+ *   outs      HOST array of n_out device pointers, each a [T][d] fp32
+ *             buffer (local or peer-mapped); only the slab's rows are
+ *             written, the same values to each.
+ *   1 <= p <= TP_GATHER_MAX, 1 <= n_out <= TP_GATHER_MAX, 0 <= row0,
+ *   0 <= rows, d >= 1.  Pointers 4-byte aligned (16-byte aligned with
+ *   d % 4 == 0 takes 128-bit loads and stores).  No destination slab may
+ *   overlap a partial's slab.
+ * The kernel does not wait on other GPUs: order it after every GPU's P_j is
+ * complete and before any GPU reads its Z (for instance a one-element
+ * all-reduce on the stream before and after it).  Peer memory is read and
+ * written with plain loads and stores only.  Errors: TP_ERR_INVALID_ARG for
+ * bad counts, sizes, NULL or overlapping pointers, TP_ERR_ALIGNMENT,
+ * TP_ERR_CUDA.  rows == 0 is a no-op.
+ */
+#define TP_GATHER_MAX 16
+tp_status tp_reduce_partials_gather(const float* const* partials, int p, const float* b2,
+                                    float* const* outs, int n_out, int64_t row0, int64_t rows,
+                                    int64_t d, void* stream);
+
+/*
+ * Sharing device buffers between the processes of a p-GPU run (CUDA IPC),
+ * so that each rank can map its peers' partials and outputs.
+ *   tp_ipc_export   fills `handle` for the device buffer starting at `ptr`
+ *                   (which must lie in a cudaMalloc allocation: PyTorch's
+ *                   default allocator qualifies, its expandable segments do
+ *                   not).  TP_ERR_INVALID_ARG if `ptr` is not device memory,
+ *                   TP_ERR_CUDA if the allocation cannot be exported.
+ *   tp_ipc_import   maps the buffer of a handle exported by ANOTHER process
+ *                   and returns its address in this process (`*ptr`);
+ *                   importing the same allocation again reuses the mapping.
+ *   tp_ipc_release  drops one import; the mapping is closed with the last.
+ * A handle is plain bytes and may be sent through any channel.
+ */
+typedef struct {
+  unsigned char bytes[64];   /* cudaIpcMemHandle_t of the allocation        */
+  uint64_t offset;           /* ptr - allocation base                        */
+  uint64_t size;             /* allocation size in bytes                     */
+} tp_ipc_handle;
+tp_status tp_ipc_export(const void* ptr, tp_ipc_handle* handle);
+tp_status tp_ipc_import(const tp_ipc_handle* handle, void** ptr);
+tp_status tp_ipc_release(const tp_ipc_handle* handle);
+
+/*
  * The whole block, Z = sum_i act(X W1_i + b1_i) W2_i  [+ b2]
  * ("Pairing them: the Megatron-LM MLP"; "The MLP block: column then row,
  * one all-reduce").  Computes exactly what tp_column_linear ->

@@ -48,6 +48,9 @@ __all__ = [
     "tp_transformer_block_workspace_size", "tp_mlp_block_backward",
     "tp_mlp_block_backward_workspace_size", "tp_mlp_block_backward_recompute",
     "tp_mlp_block_backward_recompute_workspace_size",
+    # the all-reduce of partials held on p GPUs
+    "TP_GATHER_MAX", "IpcHandle", "tp_reduce_partials_gather", "tp_ipc_export", "tp_ipc_import",
+    "tp_ipc_release",
     # status, timeouts, introspection
     "tp_sync_status", "tp_set_wait_timeout_ns", "tp_debug_drop_load", "tp_debug_exp2_poly",
     "tp_status_string",
@@ -72,6 +75,24 @@ class TPError(RuntimeError):
         self.status = status
         self.name = STATUS.get(status, str(status))
         super().__init__(f"{self.name}: {detail}")
+
+
+TP_GATHER_MAX = 16
+
+
+class IpcHandle(ctypes.Structure):
+    """tp_ipc_handle: an exported device buffer (plain bytes, any channel)."""
+    _fields_ = [("bytes", ctypes.c_ubyte * 64), ("offset", ctypes.c_uint64),
+                ("size", ctypes.c_uint64)]
+
+    def to_bytes(self) -> bytes:
+        return ctypes.string_at(ctypes.addressof(self), ctypes.sizeof(self))
+
+    @classmethod
+    def from_bytes(cls, b: bytes) -> "IpcHandle":
+        h = cls()
+        ctypes.memmove(ctypes.addressof(h), b, ctypes.sizeof(h))
+        return h
 
 
 class BlockParams(ctypes.Structure):
@@ -123,6 +144,11 @@ def _load() -> ctypes.CDLL:
     lib.tp_debug_drop_load.argtypes = [i64]
     lib.tp_debug_drop_load.restype = None
     lib.tp_debug_exp2_poly.argtypes = [vp, vp, i64, vp]
+    lib.tp_reduce_partials_gather.argtypes = [ctypes.POINTER(vp), i32, vp, ctypes.POINTER(vp), i32,
+                                              i64, i64, i64, vp]
+    lib.tp_ipc_export.argtypes = [vp, ctypes.POINTER(IpcHandle)]
+    lib.tp_ipc_import.argtypes = [ctypes.POINTER(IpcHandle), ctypes.POINTER(vp)]
+    lib.tp_ipc_release.argtypes = [ctypes.POINTER(IpcHandle)]
     lib.tp_status_string.argtypes = [i32]
     lib.tp_status_string.restype = ctypes.c_char_p
     lib.tp_last_error_detail.argtypes = []
@@ -134,7 +160,8 @@ def _load() -> ctypes.CDLL:
               "tp_mlp_block_noalloc", "tp_mlp_block_host", "tp_attention_heads", "tp_attn_block", "tp_layer_norm",
               "tp_reduce_partials_residual", "tp_transformer_block", "tp_mlp_block_backward",
               "tp_mlp_block_backward_recompute", "tp_sync_status", "tp_abi_version",
-              "tp_debug_exp2_poly"):
+              "tp_debug_exp2_poly", "tp_reduce_partials_gather", "tp_ipc_export",
+              "tp_ipc_import", "tp_ipc_release"):
         getattr(lib, f).restype = i32
     return lib
 
@@ -315,6 +342,35 @@ def tp_set_wait_timeout_ns(ns: int) -> None:
 
 def tp_debug_drop_load(stage_index: int) -> None:
     _lib.tp_debug_drop_load(stage_index)
+
+
+def tp_reduce_partials_gather(partials, b2, outs, row0, rows, d, stream=None, check=True):
+    """Fold rows [row0, row0 + rows) of the p partials (a sequence of device
+    buffers or addresses, shard order, local or peer-mapped) in shard order
+    (+ b2) and write the slab to every buffer in `outs`."""
+    vp = ctypes.c_void_p
+    parts = (vp * len(partials))(*[_ptr(x) for x in partials])
+    dst = (vp * len(outs))(*[_ptr(x) for x in outs])
+    return _check(_lib.tp_reduce_partials_gather(parts, len(partials), _ptr(b2), dst, len(outs),
+                                                 row0, rows, d, _stream(stream)), check)
+
+
+def tp_ipc_export(buf) -> IpcHandle:
+    """Handle of the device buffer `buf` (tensor or address) for another process."""
+    h = IpcHandle()
+    _check(_lib.tp_ipc_export(_ptr(buf), ctypes.byref(h)), True)
+    return h
+
+
+def tp_ipc_import(handle: IpcHandle) -> int:
+    """Maps a buffer exported by another process; returns its address here."""
+    out = ctypes.c_void_p()
+    _check(_lib.tp_ipc_import(ctypes.byref(handle), ctypes.byref(out)), True)
+    return int(out.value)
+
+
+def tp_ipc_release(handle: IpcHandle) -> None:
+    _check(_lib.tp_ipc_release(ctypes.byref(handle)), True)
 
 
 def tp_debug_exp2_poly(x, y, n, stream=None, check=True):

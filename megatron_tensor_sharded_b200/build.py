@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
 
 SOURCES = ["tp_abi.cu", "tp_reduce.cu", "tp_simt_f32.cu", "tp_tmap.cu", "tp_gemm_sm100.cu",
            "tp_gemm2_sm100.cu", "tp_block_sm100.cu", "tp_attn_sm100.cu", "tp_rowops.cu", "tp_gemm_bwd_sm100.cu", "tp_gemm_fold_sm100.cu", "tp_noalloc.cu",
-           "tp_host.cu"]
+           "tp_host.cu", "tp_allreduce.cu"]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-cudart", "static",
                 f"-I{INCLUDE}", f"-I{CSRC}"]

@@ -753,6 +753,63 @@ tp_status tp_sync_status(void* stream) {
 
 void tp_set_wait_timeout_ns(uint64_t ns) { g_timeout_ns.store(ns == 0 ? 2000000000ull : ns); }
 
+tp_status tp_reduce_partials_gather(const float* const* partials, int p, const float* b2,
+                                    float* const* outs, int n_out, int64_t row0, int64_t rows,
+                                    int64_t d, void* stream) {
+  g_detail[0] = 0;
+  if (p < 1 || p > TP_GATHER_MAX) return fail(TP_ERR_INVALID_ARG, "p = %d (1..%d)", p, TP_GATHER_MAX);
+  if (n_out < 1 || n_out > TP_GATHER_MAX)
+    return fail(TP_ERR_INVALID_ARG, "n_out = %d (1..%d)", n_out, TP_GATHER_MAX);
+  if (row0 < 0 || rows < 0 || d < 1 || row0 > (int64_t(1) << 40) || rows > (int64_t(1) << 40) ||
+      d > (int64_t(1) << 30))
+    return fail(TP_ERR_INVALID_ARG, "row0=%lld rows=%lld d=%lld", (long long)row0,
+                (long long)rows, (long long)d);
+  if (partials == nullptr || outs == nullptr)
+    return fail(TP_ERR_INVALID_ARG, "pointer tables must not be NULL");
+  for (int j = 0; j < p; ++j) {
+    if (partials[j] == nullptr) return fail(TP_ERR_INVALID_ARG, "partials[%d] is NULL", j);
+    if (!aligned4(partials[j])) return fail(TP_ERR_ALIGNMENT, "partials[%d] not 4-byte aligned", j);
+  }
+  if (b2 != nullptr && !aligned4(b2)) return fail(TP_ERR_ALIGNMENT, "b2 not 4-byte aligned");
+  const uintptr_t lo = static_cast<uintptr_t>(row0 * d * 4);
+  const uintptr_t hi = static_cast<uintptr_t>((row0 + rows) * d * 4);
+  for (int q = 0; q < n_out; ++q) {
+    if (outs[q] == nullptr) return fail(TP_ERR_INVALID_ARG, "outs[%d] is NULL", q);
+    if (!aligned4(outs[q])) return fail(TP_ERR_ALIGNMENT, "outs[%d] not 4-byte aligned", q);
+    const uintptr_t o0 = reinterpret_cast<uintptr_t>(outs[q]) + lo;
+    const uintptr_t o1 = reinterpret_cast<uintptr_t>(outs[q]) + hi;
+    for (int j = 0; j < p && rows > 0; ++j) {
+      const uintptr_t p0 = reinterpret_cast<uintptr_t>(partials[j]) + lo;
+      const uintptr_t p1 = reinterpret_cast<uintptr_t>(partials[j]) + hi;
+      if (o0 < p1 && p0 < o1)
+        return fail(TP_ERR_INVALID_ARG, "outs[%d] overlaps partials[%d] on the slab", q, j);
+    }
+  }
+  if (rows == 0) return TP_OK;
+  LaunchCtx c{};
+  TP_TRY(make_ctx(stream, false, &c));
+  return cuda_status(launch_gather_fold(c, partials, p, b2, outs, n_out, row0, rows, d),
+                     "gather-fold launch");
+}
+
+tp_status tp_ipc_export(const void* ptr, tp_ipc_handle* handle) {
+  g_detail[0] = 0;
+  if (ptr == nullptr || handle == nullptr) return fail(TP_ERR_INVALID_ARG, "NULL argument");
+  return ipc_export(ptr, handle);
+}
+
+tp_status tp_ipc_import(const tp_ipc_handle* handle, void** ptr) {
+  g_detail[0] = 0;
+  if (ptr == nullptr || handle == nullptr) return fail(TP_ERR_INVALID_ARG, "NULL argument");
+  return ipc_import(handle, ptr);
+}
+
+tp_status tp_ipc_release(const tp_ipc_handle* handle) {
+  g_detail[0] = 0;
+  if (handle == nullptr) return fail(TP_ERR_INVALID_ARG, "NULL argument");
+  return ipc_release(handle);
+}
+
 tp_status tp_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
   g_detail[0] = 0;
   if (n < 0 || n > (int64_t(1) << 40)) return fail(TP_ERR_INVALID_ARG, "n = %lld", (long long)n);

@@ -113,6 +113,15 @@ tp_status launch_bwd_dw2(const LaunchCtx& c, const void* Y, const void* dZ, floa
 tp_status launch_tc_attention(const LaunchCtx& c, const void* Q, const void* K, const void* V,
                               void* O, int64_t T, int p, int hq, int hkv, int causal);
 
+// ---- the all-reduce of partials held on p GPUs (tp_allreduce.cu)
+// Z_q[rows of the slab] = fixed-order fold of parts[0..p) (+ b2), for q < n_out.
+cudaError_t launch_gather_fold(const LaunchCtx& c, const float* const* parts, int p,
+                               const float* b2, float* const* outs, int n_out, int64_t row0,
+                               int64_t rows, int64_t d);
+tp_status ipc_export(const void* ptr, tp_ipc_handle* h);
+tp_status ipc_import(const tp_ipc_handle* h, void** ptr);
+tp_status ipc_release(const tp_ipc_handle* h);
+
 // Test hook: the attention softmax's 2^x polynomial applied to x[0..n).
 cudaError_t launch_exp2_poly_probe(const LaunchCtx& c, const float* x, float* y, int64_t n);
 
