@@ -54,8 +54,7 @@ struct PCfg {
 
 // Loads of one slot for this CTA: A rows [m*256 + rank*128, +128), B columns
 // [n*256 + rank*128, +128) of the layer's weight (SwiGLU: the even CTA loads
-// the gate columns, the odd CTA the matching up columns).  P.l2_hints picks
-// the L2 eviction policy of each operand's copies.
+// the gate columns, the odd CTA the matching up columns).
 template <int MODE, int PBN>
 __device__ __forceinline__ void issue_slot_pair(const TcParams& P, const CUtensorMap* mA,
                                                 const CUtensorMap* mB0, const CUtensorMap* mB1,
@@ -63,43 +62,34 @@ __device__ __forceinline__ void issue_slot_pair(const TcParams& P, const CUtenso
                                                 uint32_t sa, uint32_t sb, uint32_t bar) {
   constexpr int PB_CHUNKS = PCfg<PBN>::B_CHUNKS;
   const int32_t row0 = tc.m * PBM + static_cast<int32_t>(rank) * BM;
-  const bool ha = (P.l2_hints & kL2ALast) != 0, hb = (P.l2_hints & kL2BFirst) != 0;
-  const uint64_t pa = ha ? l2_policy_evict_last() : 0, pb = hb ? l2_policy_evict_first() : 0;
-  auto load_a = [&](int32_t c0, int32_t c1, int32_t c2) {
-    if (ha) tma_load_3d_pair_hint(sa, mA, bar, c0, c1, c2, pa);
-    else tma_load_3d_pair(sa, mA, bar, c0, c1, c2);
-  };
-  auto load_b = [&](uint32_t dst, const CUtensorMap* m, int32_t c0, int32_t c1) {
-    if (hb) tma_load_2d_pair_hint(dst, m, bar, c0, c1, pb);
-    else tma_load_2d_pair(dst, m, bar, c0, c1);
-  };
   if constexpr (MODE == kModeColumn) {
-    load_a(kb * BK, row0, 0);
+    tma_load_3d_pair(sa, mA, bar, kb * BK, row0, 0);
     const int32_t col0 = tc.n * PBN + static_cast<int32_t>(rank) * (PBN / 2);
 #pragma unroll
     for (int c = 0; c < PB_CHUNKS; ++c)
-      load_b(sb + c * B_CHUNK_BYTES, mB0, col0 + c * B_BOX_COLS, kb * BK);
+      tma_load_2d_pair(sb + c * B_CHUNK_BYTES, mB0, bar, col0 + c * B_BOX_COLS, kb * BK);
   } else if constexpr (MODE == kModeColumnSwiglu) {
-    load_a(kb * BK, row0, 0);
+    tma_load_3d_pair(sa, mA, bar, kb * BK, row0, 0);
     const CUtensorMap* mB = rank == 0 ? mB0 : mB1;
     const int32_t col0 = tc.n * (PBN / 2);
 #pragma unroll
     for (int c = 0; c < PB_CHUNKS; ++c)
-      load_b(sb + c * B_CHUNK_BYTES, mB, col0 + c * B_BOX_COLS, kb * BK);
+      tma_load_2d_pair(sb + c * B_CHUNK_BYTES, mB, bar, col0 + c * B_BOX_COLS, kb * BK);
   } else if constexpr (MODE == kModeRowPartial) {
-    load_a(kb * BK, row0, tc.batch);
+    tma_load_3d_pair(sa, mA, bar, kb * BK, row0, tc.batch);
     const int32_t col0 = tc.n * PBN + static_cast<int32_t>(rank) * (PBN / 2);
 #pragma unroll
     for (int c = 0; c < PB_CHUNKS; ++c)
-      load_b(sb + c * B_CHUNK_BYTES, mB0, col0 + c * B_BOX_COLS, tc.batch * P.s + kb * BK);
+      tma_load_2d_pair(sb + c * B_CHUNK_BYTES, mB0, bar, col0 + c * B_BOX_COLS,
+                       tc.batch * P.s + kb * BK);
   } else {
     const int32_t shard = kb / P.kb_per_shard;
     const int32_t kin = kb - shard * P.kb_per_shard;
-    load_a(kin * BK, row0, shard);
+    tma_load_3d_pair(sa, mA, bar, kin * BK, row0, shard);
     const int32_t col0 = tc.n * PBN + static_cast<int32_t>(rank) * (PBN / 2);
 #pragma unroll
     for (int c = 0; c < PB_CHUNKS; ++c)
-      load_b(sb + c * B_CHUNK_BYTES, mB0, col0 + c * B_BOX_COLS, kb * BK);
+      tma_load_2d_pair(sb + c * B_CHUNK_BYTES, mB0, bar, col0 + c * B_BOX_COLS, kb * BK);
   }
 }
 
@@ -348,8 +338,6 @@ tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMa
   prm.m_tiles = ceil_div(prm.T, PBM);
   prm.n_tiles = ceil_div(prm.n_total, out_cols);
   prm.num_tiles = prm.m_tiles * prm.n_tiles * prm.batches;
-  prm.group_m = env_int("TP_GROUP_M", 0);
-  prm.l2_hints = env_int("TP_L2_HINTS", 0);
   if (pbn == 128) {
     switch (mode) {
       case kModeColumn: return launch_pair_mode<kModeColumn, 128>(c, a, b0, b1, cm, prm);

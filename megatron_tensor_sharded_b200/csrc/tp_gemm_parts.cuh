@@ -63,41 +63,21 @@ struct TcParams {
   const void* bias;      // b1 (bf16, column) or b2 (fp32, split-K row); may be null
   void* out;             // Y bf16 [p][T][s] | P fp32 [p][T][d] | Z fp32 [T][d]
   int32_t bulk_out;      // column layers: 1 = bulk tensor stores through shared memory
-  int32_t group_m;       // tile order: m-tiles per group (0: all m-tiles in one group)
-  int32_t l2_hints;      // kL2* bits: L2 eviction policies of the CTA-pair kernel's copies
   WaitCtl wait;
   int64_t debug_drop;    // slot (in issue order) whose load is skipped; -1 none
 };
-
-// l2_hints bits
-constexpr int32_t kL2ALast = 1;    // A operand (X or Y_i, read again by later tiles): evict_last
-constexpr int32_t kL2BFirst = 2;   // B operand (a weight panel): evict_first
-constexpr int32_t kL2OutFirst = 4; // bulk output stores: evict_first
 
 struct TileCoord {
   int32_t batch, m, n;
 };
 
-// Tile order inside a batch (shard): the m-tiles are cut into groups of
-// group_m (the last group takes the rest); a group is walked m fastest, one
-// n-tile column after another, before the next group starts.  Neighbouring
-// CTAs then share the weight panel, and a wave of CTAs covers group_m row
-// panels of A instead of all of them.  group_m = 0 (or >= m_tiles): one
-// group, plain m-fastest order.
 __device__ __forceinline__ TileCoord decode_tile(const TcParams& P, int32_t t) {
   const int32_t per_batch = P.m_tiles * P.n_tiles;
   TileCoord c;
   c.batch = t / per_batch;
   const int32_t r = t - c.batch * per_batch;
-  const int32_t G = (P.group_m <= 0 || P.group_m > P.m_tiles) ? P.m_tiles : P.group_m;
-  const int32_t full = P.m_tiles / G;           // groups of exactly G m-tiles
-  const int32_t per_group = G * P.n_tiles;
-  const int32_t g = r / per_group;
-  const int32_t m0 = g < full ? g * G : full * G;
-  const int32_t gm = g < full ? G : P.m_tiles - full * G;
-  const int32_t rr = r - (g < full ? g : full) * per_group;
-  c.n = rr / gm;
-  c.m = m0 + (rr - c.n * gm);
+  c.n = r / P.m_tiles;   // m fastest: neighbouring CTAs share the weight panel
+  c.m = r - c.n * P.m_tiles;
   return c;
 }
 
@@ -408,11 +388,7 @@ __device__ __forceinline__ void epilogue_tile_bulk(const TcParams& P, const Tile
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) {
-      if (P.l2_hints & kL2OutFirst)
-        tma_store_3d_hint(mapC, stage, j0, row0, MODE == kModeRowPartial ? tc.batch : 0,
-                          l2_policy_evict_first());
-      else
-        tma_store_3d(mapC, stage, j0, row0, MODE == kModeRowPartial ? tc.batch : 0);
+      tma_store_3d(mapC, stage, j0, row0, MODE == kModeRowPartial ? tc.batch : 0);
       bulk_commit();
     }
   }
@@ -463,10 +439,7 @@ __device__ __forceinline__ void epilogue_tile_bulk_col(const TcParams& P, const 
     __syncwarp();
     if (lane == 0) {
       const int32_t shard = j0 / P.s;
-      if (P.l2_hints & kL2OutFirst)
-        tma_store_3d_hint(mapY, buf, j0 - shard * P.s, row0, shard, l2_policy_evict_first());
-      else
-        tma_store_3d(mapY, buf, j0 - shard * P.s, row0, shard);
+      tma_store_3d(mapY, buf, j0 - shard * P.s, row0, shard);
       bulk_commit();
     }
     ++nchunk;
