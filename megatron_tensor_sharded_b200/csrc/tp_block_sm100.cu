@@ -8,8 +8,15 @@
 // needs the hidden rows of that m-tile from every column tile: column tiles
 // publish completion through a per-m-tile counter (release), and the
 // producer of a row tile waits on it (acquire, bounded) before its TMA reads
-// the hidden shards.  All CTAs are resident at once (one per SM, grid <= SM
-// count) and column tiles never wait, so the waits always end.  The row
+// the hidden shards.  The schedule cannot deadlock: column tiles never wait,
+// and every CTA runs all of its column tiles before any of its row tiles,
+// so each column tile a row tile waits for belongs to a CTA that is running
+// or has not started yet and needs nothing to make progress.  The grid is
+// at most one CTA per SM, so normally every CTA is resident from the start;
+// when other work holds SMs (other streams, processes, MPS), a CTA whose
+// column tiles have not been scheduled yet delays the row tiles waiting on
+// them, and under heavy contention that delay can run past the bounded wait
+// (TP_ERR_DEVICE_TIMEOUT, reported by the call's status word).  The row
 // layer thus starts without a kernel boundary, on SMs the column layer has
 // left idle.
 //
