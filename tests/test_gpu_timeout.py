@@ -102,3 +102,38 @@ def test_dropped_load_in_cta_pair_gemm_times_out(short_timeout):
                         "gelu_tanh")["Z"]
     assert O.rel_err(host_f32(blk.Z)[:64], ref) <= 1e-2
 
+
+
+def test_dropped_load_in_attention_times_out(short_timeout):
+    """The attention kernel: a K/V block the producer never loads makes the
+    MMA issuer's wait run out; the softmax warps (and, when a row's keys are
+    split over two threads, their pair exchanges) see the abort flag and
+    stop; the next launch is correct."""
+    rng = np.random.default_rng(2)
+    p, T, h, hkv = 2, 300, 4, 2
+    shape = lambda heads: (p, T, (heads // p) * 128)  # noqa: E731
+    Q = rng.standard_normal(shape(h), dtype=np.float32)
+    K = rng.standard_normal(shape(hkv), dtype=np.float32)
+    V = rng.standard_normal(shape(hkv), dtype=np.float32)
+    c = W.f32_to_bf16_bits
+    dv = lambda a: torch.from_numpy(c(a).view(np.int16)).view(torch.bfloat16).cuda()  # noqa: E731
+    Qd, Kd, Vd = dv(Q), dv(K), dv(V)
+    Od = torch.full(shape(h), float("nan"), dtype=torch.bfloat16, device="cuda")
+    tp.tp_debug_drop_load(2)
+    tp.tp_attention_heads(Qd, Kd, Vd, Od, T, p, h, hkv, 128, 1)
+    st = tp.tp_sync_status(check=False)
+    assert st == 6, tp.tp_status_string(st)
+    Od.fill_(float("nan"))
+    tp.tp_attention_heads(Qd, Kd, Vd, Od, T, p, h, hkv, 128, 1)
+    assert tp.tp_sync_status(check=False) == 0
+    got = host_f32(Od).astype(np.float64)
+    qv = W.bf16_bits_to_f32(c(Q)).astype(np.float64)
+    kv = W.bf16_bits_to_f32(c(K)).astype(np.float64)
+    vv = W.bf16_bits_to_f32(c(V)).astype(np.float64)
+    for s in range(p):
+        for hh in range(h // p):
+            g = hh // (h // hkv)   # the shard's K/V head of its query head hh
+            want = O.sdpa_head(qv[s, :, hh * 128:(hh + 1) * 128], kv[s, :, g * 128:(g + 1) * 128],
+                               vv[s, :, g * 128:(g + 1) * 128], True)
+            err = np.abs(got[s, :, hh * 128:(hh + 1) * 128] - want)
+            assert err.max() <= 2.0 ** -8 * (np.abs(vv).max() + 1.0)
