@@ -17,7 +17,10 @@
 //                  of the score buffer).  Issue order per block:
 //                  PV_0 -> S_0(next) -> PV_1 -> S_1(next), so the tensor core
 //                  runs one tile's products while the other tile's softmax
-//                  runs;
+//                  runs.  Only the Q K^T products read the Q tiles, so they
+//                  are handed back to the producer as soon as the unit's last
+//                  one completes: the next unit's Q load overlaps this unit's
+//                  last softmax and P V products;
 //   warp 2         TMEM allocation;
 //   warps 4..7     online softmax of tile 0, warps 8..11 of tile 1: thread =
 //                  query row (its TMEM lane), one round trip to TMEM per
@@ -369,6 +372,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int t = 0; t < NQT; ++t)
           if (x.nkb(t) > 0) issue_s(t, n0);
+        // Q is read only by the Q K^T products: once the unit's last one is
+        // issued, a commit hands the Q tiles back to the producer, which
+        // loads the next unit's while this unit's last softmax and P V run.
+        int s_pending = 0;   // tiles whose last Q K^T product is still to be issued
+#pragma unroll
+        for (int t = 0; t < NQT; ++t)
+          if (x.nkb(t) > 1) ++s_pending;
+        if (s_pending == 0) tc_commit(q_empty);
         for (int32_t j = 0; ok && j < x.nmax; ++j) {
           const uint32_t vst = (n0 + j) % NST;
 #pragma unroll
@@ -401,6 +412,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
               tc_fence_after();
               issue_s(t, n0 + j + 1);
+              if (j + 2 == x.nkb(t) && --s_pending == 0) tc_commit(q_empty);
             } else {
               tc_commit(o_full(t));
             }
@@ -411,7 +423,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int t = 0; t < NQT; ++t)
           if (x.nkb(t) > 0) ++ou[t];
         kv_n = n0 + x.nmax;
-        tc_commit(q_empty);
       }
       tc_commit(drain);
       wait_teardown(drain, 0, P.wait);
