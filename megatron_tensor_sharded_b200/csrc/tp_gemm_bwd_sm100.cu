@@ -383,6 +383,292 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// ------------------------------------------------------------------ CTA pairs
+// The same four GEMMs on CTA pairs (tcgen05 cta_group::2) for layers large
+// enough to fill the SMs with 256-row tiles: a cluster of two CTAs computes a
+// 256 x PBN tile; each CTA loads its own 128 rows of A and half (PBN/2
+// columns) of B, the even CTA's MMA thread issues M = 256 products that read
+// both CTAs' shared memory and write each CTA's 128 accumulator rows into its
+// own TMEM, and each CTA's epilogue stores its own rows.  Per SM the operand
+// bytes per MMA cycle drop from 96 to 64 at width 256.  Barriers as in the
+// forward pair kernel: the even CTA's full barrier counts both CTAs' bytes,
+// the MMA commits multicast to both CTAs, every epilogue warp of both CTAs
+// arrives on the even CTA's accumulator-empty barrier.  No load uses cluster
+// multicast.  Every wait is bounded.
+template <int PBN>
+struct PairB {
+  static constexpr int B_HALF_BYTES = (PBN / 2) * BK * 2;   // this CTA's half of B per slot
+};
+
+template <int AMN, int BMN, int PBN>
+__device__ __forceinline__ void issue_pair(const GParams& P, const CUtensorMap* mA0,
+                                           const CUtensorMap* mA1, const CUtensorMap* mB0,
+                                           const CUtensorMap* mB1, const GTile& g, int32_t kb,
+                                           uint32_t rank, uint32_t sa, uint32_t sb, uint32_t bar) {
+  bool second = false;
+  if (P.kb_half > 0 && kb >= P.kb_half) {
+    second = true;
+    kb -= P.kb_half;
+  }
+  const CUtensorMap* mA = second ? mA1 : mA0;
+  const CUtensorMap* mB = (second || g.half > 0) ? mB1 : mB0;
+  const int32_t za = P.a_batched ? g.shard : 0;
+  const int32_t zb = P.b_batched ? g.shard : 0;
+  const int32_t m0 = g.m * 2 * BM + static_cast<int32_t>(rank) * BM;
+  const int32_t n0 = g.n * PBN + static_cast<int32_t>(rank) * (PBN / 2);
+  const int32_t k0 = kb * BK;
+  if constexpr (AMN == 0) {
+    tma_load_3d_pair(sa, mA, bar, k0, m0, za);
+  } else {
+#pragma unroll
+    for (int c = 0; c < BM / 64; ++c)
+      tma_load_3d_pair(sa + c * A_CHUNK_BYTES, mA, bar, m0 + c * 64, k0, za);
+  }
+  if constexpr (BMN == 0) {
+    tma_load_3d_pair(sb, mB, bar, k0 + g.shard * P.b_koff, n0, zb);
+  } else {
+#pragma unroll
+    for (int c = 0; c < PBN / 2 / 64; ++c)
+      tma_load_3d_pair(sb + c * B_CHUNK_BYTES, mB, bar, n0 + c * 64, k0, zb);
+  }
+}
+
+template <int EPI, int PBN>
+struct PBCfg {
+  static constexpr int EPI_BYTES = EPI == kEpiF32 ? EPI_STAGE_BYTES : 0;
+  static constexpr int STAGE_BYTES = A_BYTES + PairB<PBN>::B_HALF_BYTES;
+  static constexpr int STAGES_FIT = (SMEM_LIMIT - 1024 - CTRL_BYTES - EPI_BYTES) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + EPI_BYTES + CTRL_BYTES;
+  static constexpr int TMEM_COLS = 2 * PBN <= 256 ? 256 : 512;
+  static_assert(PBN == 128 || PBN == 256, "pair tile width");
+  static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
+  static_assert(8 * (2 * STAGES + 5) + 16 <= CTRL_BYTES, "control block");
+};
+
+template <int AMN, int BMN, int EPI, int PBN>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    tc_gemm_bwd_pair_kernel(const __grid_constant__ CUtensorMap mapA0,
+                            const __grid_constant__ CUtensorMap mapA1,
+                            const __grid_constant__ CUtensorMap mapB0,
+                            const __grid_constant__ CUtensorMap mapB1,
+                            const __grid_constant__ CUtensorMap mapC0,
+                            const __grid_constant__ CUtensorMap mapC1, const GParams P) {
+  using C = PBCfg<EPI, PBN>;
+  constexpr int STAGES = C::STAGES;
+  constexpr uint32_t IDESC = idesc_bf16_f32(2 * BM, PBN, AMN, BMN);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  const uint32_t epi_stage = base + STAGES * C::STAGE_BYTES;
+  uint8_t* const ctrl = smem_raw + (base - raw) + STAGES * C::STAGE_BYTES + C::EPI_BYTES;
+  uint64_t* const bars = reinterpret_cast<uint64_t*>(ctrl);
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * (2 * STAGES + 5));
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto full_bar = [&](uint32_t s) { return smem_u32(&bars[s]); };
+  auto empty_bar = [&](uint32_t s) { return smem_u32(&bars[STAGES + s]); };
+  auto accf_bar = [&](uint32_t b) { return smem_u32(&bars[2 * STAGES + b]); };
+  auto acce_bar = [&](uint32_t b) { return smem_u32(&bars[2 * STAGES + 2 + b]); };
+  const uint32_t drain_bar = smem_u32(&bars[2 * STAGES + 4]);
+  auto slot_a = [&](uint32_t s) { return base + s * C::STAGE_BYTES; };
+  auto slot_b = [&](uint32_t s) { return base + s * C::STAGE_BYTES + A_BYTES; };
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const uint32_t rank = cluster_ctarank();
+  const int32_t cluster = blockIdx.x / 2;
+  const int32_t nclusters = gridDim.x / 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(accf_bar(b), 1);
+      mbar_init(acce_bar(b), 2 * NUM_EPI_WARPS);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&mapA0);
+    tma_prefetch_map(&mapB0);
+  }
+  if (warp == 2) {
+    tmem_alloc_pair(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
+  pdl_wait();
+  pdl_launch_dependents();
+
+  if (warp == 0) {
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      int64_t issued = 0;
+      bool ok = true;
+      for (int32_t t = cluster; ok && t < P.num_tiles; t += nclusters) {
+        const GTile g = decode(P, t);
+        for (int32_t kb = 0; kb < P.k_blocks; ++kb) {
+          if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, P.wait, kErrWaitEmpty)) {
+            ok = false;
+            break;
+          }
+          if (issued != P.debug_drop) {
+            if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
+            issue_pair<AMN, BMN, PBN>(P, &mapA0, &mapA1, &mapB0, &mapB1, g, kb, rank,
+                                      slot_a(stage), slot_b(stage),
+                                      mapa_shared(full_bar(stage), 0));
+          }
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      // our last loads must have landed before this CTA's shared memory is
+      // released: the even CTA sees that on its full barriers, the odd CTA
+      // on its empty barriers (the MMA consumed the slot)
+      const int64_t first = issued > STAGES ? issued - STAGES : 0;
+      for (int64_t q = first; q < issued; ++q) {
+        if (q == P.debug_drop) continue;
+        const uint32_t s = static_cast<uint32_t>(q % STAGES);
+        const uint32_t ph = static_cast<uint32_t>((q / STAGES) & 1);
+        wait_teardown(rank == 0 ? full_bar(s) : empty_bar(s), ph, P.wait);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      int32_t lt = 0;
+      for (int32_t t = cluster; ok && t < P.num_tiles; t += nclusters, ++lt) {
+        const uint32_t b = lt & 1, ap = (lt >> 1) & 1;
+        if (!wait_bounded(acce_bar(b), ap ^ 1u, abort_flag, P.wait, kErrWaitAccEmpty)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + b * PBN;
+        for (int32_t kb = 0; kb < P.k_blocks; ++kb) {
+          if (!wait_bounded(full_bar(stage), phase, abort_flag, P.wait, kErrWaitFull)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = slot_a(stage), sb = slot_b(stage);
+#pragma unroll
+          for (int kk = 0; kk < BK / UK; ++kk) {
+            const uint64_t adesc = AMN == 0 ? smem_desc_sw128(sa + kk * UK * 2, 16, 1024)
+                                            : smem_desc_sw128(sa + kk * UK * 128, A_CHUNK_BYTES, 1024);
+            const uint64_t bdesc = BMN == 0 ? smem_desc_sw128(sb + kk * UK * 2, 16, 1024)
+                                            : smem_desc_sw128(sb + kk * UK * 128, B_CHUNK_BYTES, 1024);
+            tc_mma_f16_pair(d_tmem, adesc, bdesc, IDESC, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          tc_commit_pair_mc(empty_bar(stage), 0x3);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit_pair_mc(accf_bar(b), 0x3);
+      }
+      tc_commit_pair_mc(drain_bar, 0x1);
+      wait_teardown(drain_bar, 0, P.wait);
+    }
+    __syncwarp();
+  } else if (warp >= 4) {
+    const int quad = warp & 3;
+    const int half = (warp - 4) >> 2;
+    int32_t lt = 0;
+    for (int32_t t = cluster; t < P.num_tiles; t += nclusters, ++lt) {
+      const uint32_t b = lt & 1, ap = (lt >> 1) & 1;
+      const GTile g = decode(P, t);
+      bool ok = wait_bounded(accf_bar(b), ap, abort_flag, P.wait, kErrWaitAccFull);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * PBN;
+      const int32_t row0 = g.m * 2 * BM + static_cast<int32_t>(rank) * BM + quad * 32;
+      if (EPI == kEpiF32 && P.bulk_out)
+        epilogue_f32_bulk<PBN>(P, g, tacc, row0, half,
+                               epi_stage + (warp - 4) * EPI_WARP_STAGE_BYTES,
+                               g.half > 0 ? &mapC1 : &mapC0, lane);
+      else
+        epilogue<EPI, PBN>(P, g, tacc, row0 + lane, half);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(b), 0));
+    }
+    if (lane == 0) bulk_wait_all0();   // staging read out before shared memory is released
+  }
+
+  tc_fence_before();
+  cluster_sync();  // the pair's MMAs, commits and arrivals are done with both CTAs
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+template <int AMN, int BMN, int EPI, int PBN>
+tp_status launch_gp(const LaunchCtx& c, const CUtensorMap* maps, GParams prm) {
+  using Cf = PBCfg<EPI, PBN>;
+  static uint64_t attr_epoch[64] = {};   // context epoch the attribute was set under
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    const int dev = c.device & 63;
+    if (attr_epoch[dev] != c.epoch) {
+      if (cudaFuncSetAttribute(tc_gemm_bwd_pair_kernel<AMN, BMN, EPI, PBN>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               Cf::SMEM_BYTES) != cudaSuccess) {
+        set_error_detail("cudaFuncSetAttribute failed: %s", cudaGetErrorString(cudaGetLastError()));
+        return TP_ERR_CUDA;
+      }
+      attr_epoch[dev] = c.epoch;
+    }
+  }
+  prm.m_tiles = ceil_div(prm.M, 2 * BM);
+  prm.n_tiles = ceil_div(prm.N, PBN);
+  prm.num_tiles = prm.m_tiles * prm.n_tiles * prm.p * prm.halves;
+  prm.wait.err = c.err_word;
+  prm.wait.timeout_ns = c.timeout_ns;
+  prm.debug_drop = c.debug_drop;
+  if (prm.num_tiles == 0) return TP_OK;
+  int clusters = c.num_sms / 2;
+  if (clusters > prm.num_tiles) clusters = prm.num_tiles;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = Cf::SMEM_BYTES;
+  cfg.stream = c.stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_allowed() ? 2 : 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_bwd_pair_kernel<AMN, BMN, EPI, PBN>,
+                                           maps[0], maps[1], maps[2], maps[3], maps[4], maps[5],
+                                           prm);
+  note_launch();
+  if (e != cudaSuccess) {
+    set_error_detail("paired backward GEMM launch failed: %s", cudaGetErrorString(e));
+    return TP_ERR_CUDA;
+  }
+  return TP_OK;
+}
+
 template <int AMN, int BMN, int EPI, int BN>
 tp_status launch_g(const LaunchCtx& c, const CUtensorMap* maps, GParams prm) {
   using Cf = BCfg<EPI, BN>;
@@ -419,18 +705,28 @@ tp_status launch_g(const LaunchCtx& c, const CUtensorMap* maps, GParams prm) {
   return TP_OK;
 }
 
-// Tile width for an (M x N) x batches problem with K / 64 slots: the
-// forward cost model, restricted to single-CTA tiles of 64, 128 or 256.
-int pick_bn(int64_t M, int64_t N, int64_t batches, int64_t k_blocks, int num_sms) {
-  const TileChoice t = pick_tile(M, N, batches, k_blocks, num_sms, false, false);
-  return t.bn == 192 ? 128 : t.bn;
+// Tile shape for an (M x N) x batches problem with K / 64 slots: the
+// forward's cost model (single-CTA widths 64, 128, 256; CTA-pair tiles of
+// 256 rows x 128 or 256 once single-CTA tiles take more than one wave).
+TileChoice choose_tile(int64_t M, int64_t N, int64_t batches, int64_t k_blocks, int num_sms) {
+  TileChoice t = pick_tile(M, N, batches, k_blocks, num_sms, false, pair_allowed());
+  if (!t.pair && t.bn == 192) t.bn = 128;
+  return t;
 }
 
+// Width of a K-major B operand's TMA box: the tile width, or its half on
+// CTA pairs (each CTA loads half of B's columns).
+uint32_t b_box(const TileChoice& t) { return static_cast<uint32_t>(t.pair ? t.bn / 2 : t.bn); }
+
 template <int AMN, int BMN, int EPI>
-tp_status launch_any(const LaunchCtx& c, const CUtensorMap* maps, GParams prm, int batches) {
-  const int bn = pick_bn(prm.M, prm.N, batches, prm.k_blocks, c.num_sms);
-  if (bn == 256) return launch_g<AMN, BMN, EPI, 256>(c, maps, prm);
-  if (bn == 128) return launch_g<AMN, BMN, EPI, 128>(c, maps, prm);
+tp_status dispatch(const LaunchCtx& c, const CUtensorMap* maps, const GParams& prm,
+                   const TileChoice& t) {
+  if (t.pair) {
+    if (t.bn == 256) return launch_gp<AMN, BMN, EPI, 256>(c, maps, prm);
+    return launch_gp<AMN, BMN, EPI, 128>(c, maps, prm);
+  }
+  if (t.bn == 256) return launch_g<AMN, BMN, EPI, 256>(c, maps, prm);
+  if (t.bn == 128) return launch_g<AMN, BMN, EPI, 128>(c, maps, prm);
   return launch_g<AMN, BMN, EPI, 64>(c, maps, prm);
 }
 
@@ -475,22 +771,16 @@ tp_status launch_bwd_act_grad(const LaunchCtx& c, const void* dZ, const void* W2
   prm.ldc = s;
   prm.aux0 = H;
   prm.aux1 = Hup;
-  const int bn = pick_bn(T, s, p, prm.k_blocks, c.num_sms);
+  const TileChoice tch = choose_tile(T, s, p, prm.k_blocks, c.num_sms);
   CUtensorMap maps[6];
   // A = dZ [T][d] K-major; B = W2 rows of shard i: [p][s][d] K-major (N rows)
-  if (!map3(&maps[0], dZ, d, T, 1, d, 0, BM) || !map3(&maps[2], W2, d, s, p, d, s * d, bn))
+  if (!map3(&maps[0], dZ, d, T, 1, d, 0, BM) || !map3(&maps[2], W2, d, s, p, d, s * d, b_box(tch)))
     return TP_ERR_CUDA;
   maps[1] = maps[0];
   maps[3] = maps[2];
   maps[4] = maps[5] = maps[0];   // bf16 outputs: per-thread stores
-  if (act == kActSwiglu) {
-    if (bn == 256) return launch_g<0, 0, kEpiSwigluGrad, 256>(c, maps, prm);
-    if (bn == 128) return launch_g<0, 0, kEpiSwigluGrad, 128>(c, maps, prm);
-    return launch_g<0, 0, kEpiSwigluGrad, 64>(c, maps, prm);
-  }
-  if (bn == 256) return launch_g<0, 0, kEpiActGrad, 256>(c, maps, prm);
-  if (bn == 128) return launch_g<0, 0, kEpiActGrad, 128>(c, maps, prm);
-  return launch_g<0, 0, kEpiActGrad, 64>(c, maps, prm);
+  if (act == kActSwiglu) return dispatch<0, 0, kEpiSwigluGrad>(c, maps, prm, tch);
+  return dispatch<0, 0, kEpiActGrad>(c, maps, prm, tch);
 }
 
 // G2: dX partials P_i = dH_i W1_i^T (+ dU_i Wup_i^T), fp32 [p][T][d]
@@ -511,14 +801,15 @@ tp_status launch_bwd_dx_partials(const LaunchCtx& c, const void* dH, const void*
   prm.out[1] = P;
   prm.out_shard_stride = T * d;
   prm.ldc = d;
-  const int bn = pick_bn(T, d, p, prm.k_blocks, c.num_sms);
+  const TileChoice tch = choose_tile(T, d, p, prm.k_blocks, c.num_sms);
   CUtensorMap maps[6];
   // A = dH [p][T][s] K-major; B = W1 [d][k] K-major (inner k, outer d = N
   // rows), shard i's block at K offset i s
-  if (!map3(&maps[0], dH, s, T, p, s, T * s, BM) || !map3(&maps[2], W1, k, d, 1, k, 0, bn))
+  if (!map3(&maps[0], dH, s, T, p, s, T * s, BM) || !map3(&maps[2], W1, k, d, 1, k, 0, b_box(tch)))
     return TP_ERR_CUDA;
   if (two) {
-    if (!map3(&maps[1], dU, s, T, p, s, T * s, BM) || !map3(&maps[3], Wup, k, d, 1, k, 0, bn))
+    if (!map3(&maps[1], dU, s, T, p, s, T * s, BM) ||
+        !map3(&maps[3], Wup, k, d, 1, k, 0, b_box(tch)))
       return TP_ERR_CUDA;
   } else {
     maps[1] = maps[0];
@@ -527,9 +818,7 @@ tp_status launch_bwd_dx_partials(const LaunchCtx& c, const void* dH, const void*
   if (!make_map_f32_out(&maps[4], P, d, T, p)) return TP_ERR_CUDA;
   maps[5] = maps[4];
   prm.bulk_out = 1;
-  if (bn == 256) return launch_g<0, 0, kEpiF32, 256>(c, maps, prm);
-  if (bn == 128) return launch_g<0, 0, kEpiF32, 128>(c, maps, prm);
-  return launch_g<0, 0, kEpiF32, 64>(c, maps, prm);
+  return dispatch<0, 0, kEpiF32>(c, maps, prm, tch);
 }
 
 // G3: dW1[:, i s:(i+1) s] = X^T dH_i  (SwiGLU: dW_up from dU as a second
@@ -545,7 +834,7 @@ tp_status launch_bwd_dw1(const LaunchCtx& c, const void* X, const void* dH, cons
   prm.out[1] = two ? dWup : dW1;
   prm.out_shard_stride = s;
   prm.ldc = k;
-  const int bn = pick_bn(d, s, p * prm.halves, prm.k_blocks, c.num_sms);
+  const TileChoice tch = choose_tile(d, s, p * prm.halves, prm.k_blocks, c.num_sms);
   CUtensorMap maps[6];
   // A = X^T: M-major view of X [T][d] (inner d = M, outer T = K);
   // B = dH [p][T][s] N-major (inner s = N, outer T = K)
@@ -564,9 +853,7 @@ tp_status launch_bwd_dw1(const LaunchCtx& c, const void* X, const void* dH, cons
   if (prm.bulk_out && two) prm.bulk_out = make_map_f32_strided(&maps[5], dWup, s, d, p, k, s) ? 1 : 0;
   if (!prm.bulk_out) maps[4] = maps[0];
   if (!two || !prm.bulk_out) maps[5] = maps[4];
-  if (bn == 256) return launch_g<1, 1, kEpiF32, 256>(c, maps, prm);
-  if (bn == 128) return launch_g<1, 1, kEpiF32, 128>(c, maps, prm);
-  return launch_g<1, 1, kEpiF32, 64>(c, maps, prm);
+  return dispatch<1, 1, kEpiF32>(c, maps, prm, tch);
 }
 
 // G4: dW2[i s:(i+1) s, :] = Y_i^T dZ, fp32 [k][d]
@@ -580,7 +867,7 @@ tp_status launch_bwd_dw2(const LaunchCtx& c, const void* Y, const void* dZ, floa
   prm.out[1] = dW2;
   prm.out_shard_stride = s * d;
   prm.ldc = d;
-  const int bn = pick_bn(s, d, p, prm.k_blocks, c.num_sms);
+  const TileChoice tch = choose_tile(s, d, p, prm.k_blocks, c.num_sms);
   CUtensorMap maps[6];
   // A = Y_i^T: M-major view of Y [p][T][s]; B = dZ [T][d] N-major
   if (!map3(&maps[0], Y, s, T, p, s, T * s, BK) || !map3(&maps[2], dZ, d, T, 1, d, 0, BK))
@@ -591,9 +878,7 @@ tp_status launch_bwd_dw2(const LaunchCtx& c, const void* Y, const void* dZ, floa
   if (!make_map_f32_out(&maps[4], dW2, d, s, p)) return TP_ERR_CUDA;
   maps[5] = maps[4];
   prm.bulk_out = 1;
-  if (bn == 256) return launch_g<1, 1, kEpiF32, 256>(c, maps, prm);
-  if (bn == 128) return launch_g<1, 1, kEpiF32, 128>(c, maps, prm);
-  return launch_g<1, 1, kEpiF32, 64>(c, maps, prm);
+  return dispatch<1, 1, kEpiF32>(c, maps, prm, tch);
 }
 
 }  // namespace tpk

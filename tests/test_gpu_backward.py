@@ -94,6 +94,10 @@ CASES = [
     (1, 256, 512, 2, "swiglu"),
     (200, 384, 768, 3, "identity"),
     (513, 1024, 4096, 8, "swiglu"),
+    # large enough for CTA-pair tiles (256-row tiles on two SMs) in all four
+    # GEMMs, one with a ragged last pair tile (2500 = 9 x 256 + 196 rows)
+    (2560, 2048, 4096, 2, "swiglu"),
+    (2500, 2048, 4096, 2, "gelu_tanh"),
 ]
 
 
