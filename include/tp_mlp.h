@@ -274,14 +274,18 @@ size_t tp_mlp_block_workspace_size(int64_t T, int64_t d, int64_t k, int p,
  *   Z_host     [T][d] fp32 host memory.
  *   workspace  device memory of at least tp_mlp_block_host_workspace_size()
  *              bytes, 256-byte aligned: device copies of X and Z, then the
- *              block's workspace for one chunk.
+ *              block's workspace for one chunk (for two when T spans more
+ *              than one chunk: consecutive chunks run on two streams).
  *   others     as for tp_mlp_block.
  *
- * Stream semantics: everything is ordered on `stream`.  The call forks two
- * library-owned helper streams (one per copy direction, created on the first
- * call on each device and kept for the process) from `stream` with an event
- * and joins them back before it returns, so Z_host is complete once `stream`
- * has reached the point of the call (cudaStreamSynchronize).  The call can be
+ * Stream semantics: everything is ordered on `stream`.  The call forks three
+ * library-owned helper streams (one per copy direction and a second compute
+ * stream, created on the first call on each device and kept for the
+ * process) from `stream` with an event and joins them back before it
+ * returns, so Z_host is complete once `stream` has reached the point of the
+ * call (cudaStreamSynchronize).  Even chunks run on `stream`, odd chunks on
+ * the second compute stream, so one chunk's kernels can fill the SMs the
+ * other's last wave of tiles leaves idle; Z has the same bits either way.  The call can be
  * captured into a CUDA graph from `stream` when both host buffers are pinned
  * and the device has had one uncaptured call first.  Calls on one device
  * enqueue under a lock (the helper events are shared).

@@ -10,9 +10,9 @@
 // kernels as tp_mlp_block on its rows, so Z has the same bits as copying X in,
 // calling tp_mlp_block on all T rows and copying Z out.
 //
-// Streams and events.  Each device gets two non-blocking helper streams (one
-// per copy direction) and a set of events, created by the first call and kept
-// for the process.  A call forks them from the caller's stream with an event
+// Streams and events.  Each device gets three non-blocking helper streams
+// (one per copy direction and a second compute stream for every other chunk)
+// and a set of events, created by the first call and kept for the process.  A call forks them from the caller's stream with an event
 // and joins them back before returning, so all of its work is ordered on the
 // caller's stream (and can be captured into a CUDA graph from it: the host
 // buffers must then be pinned).  The events are reused by every call, so the
@@ -23,6 +23,7 @@
 #include <mutex>
 
 #include "tp_internal.h"
+#include "tp_launch.cuh"
 #include "tp_mlp.h"
 
 namespace {
@@ -36,6 +37,7 @@ struct Pipe {
   bool ready = false;
   uint64_t epoch = 0;   // context epoch the streams and events were created under
   cudaStream_t h2d = nullptr, d2h = nullptr;
+  cudaStream_t cmp = nullptr;   // second compute stream: odd chunks run here
   cudaEvent_t fork = nullptr, join = nullptr;
   cudaEvent_t in[kMaxChunks] = {}, out[kMaxChunks] = {};
 };
@@ -56,11 +58,14 @@ int64_t chunk_rows(int64_t T) {
   return rc;
 }
 
-// Layout: X staging [T][d], Z staging [T][d] fp32, then one chunk's block
-// workspace, each at a 256-byte boundary.
+// Layout: X staging [T][d], Z staging [T][d] fp32, then the block workspace
+// of one chunk -- of two when there is more than one chunk (consecutive
+// chunks run on two streams, each with its own workspace) -- each at a
+// 256-byte boundary.
 struct HostLayout {
   size_t x_bytes = 0, z_bytes = 0, block_bytes = 0, total = 0;
   int64_t rc = 0;
+  int n_ws = 1;
 };
 
 bool host_layout(int64_t T, int64_t d, int64_t k, int p, tp_dtype dtype, tp_act act, int flags,
@@ -69,9 +74,11 @@ bool host_layout(int64_t T, int64_t d, int64_t k, int p, tp_dtype dtype, tp_act 
   L->rc = chunk_rows(T);
   L->block_bytes = tp_mlp_block_workspace_size(L->rc, d, k, p, dtype, act, flags);
   if (L->block_bytes == 0) return false;
+  L->block_bytes = align256(L->block_bytes);
   L->x_bytes = align256(static_cast<size_t>(T) * static_cast<size_t>(d) * esize);
   L->z_bytes = align256(static_cast<size_t>(T) * static_cast<size_t>(d) * 4);
-  L->total = L->x_bytes + L->z_bytes + L->block_bytes;
+  L->n_ws = T > L->rc ? 2 : 1;
+  L->total = L->x_bytes + L->z_bytes + L->n_ws * L->block_bytes;
   return true;
 }
 
@@ -89,6 +96,7 @@ tp_status pipe_for(int dev, uint64_t epoch, Pipe** out) {
   if (!P.ready) {
     cudaError_t e = cudaStreamCreateWithFlags(&P.h2d, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&P.d2h, cudaStreamNonBlocking);
+    if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&P.cmp, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&P.fork, cudaEventDisableTiming);
     if (e == cudaSuccess) e = cudaEventCreateWithFlags(&P.join, cudaEventDisableTiming);
     for (int c = 0; c < kMaxChunks && e == cudaSuccess; ++c) {
@@ -194,17 +202,21 @@ tp_status tp_mlp_block_host(const void* X_host, const void* W1, const void* W_up
   const tp_status sp = pipe_for(dev, epoch, &P);
   if (sp != TP_OK) return sp;
 
-  // Fork: the copies start after the caller's earlier work on `s`.
+  // Fork: the copies and the second compute stream start after the caller's
+  // earlier work on `s`.
+  const int n_streams = (L.n_ws == 2 && tpk::env_int("TP_HOST_STREAMS", 2) == 2) ? 2 : 1;
   if ((e = cudaEventRecord(P->fork, s)) != cudaSuccess) return cuda_fail(e, "fork record");
   if ((e = cudaStreamWaitEvent(P->h2d, P->fork, 0)) != cudaSuccess) return cuda_fail(e, "fork");
   if ((e = cudaStreamWaitEvent(P->d2h, P->fork, 0)) != cudaSuccess) return cuda_fail(e, "fork");
-  // From here on every exit joins both helper streams back into `s`, so the
-  // caller's stream never runs ahead of a copy this call has enqueued.
+  if ((e = cudaStreamWaitEvent(P->cmp, P->fork, 0)) != cudaSuccess) return cuda_fail(e, "fork");
+  // From here on every exit joins the helper streams back into `s`, so the
+  // caller's stream never runs ahead of work this call has enqueued.
   auto join = [&](tp_status st) {
-    cudaError_t j = cudaEventRecord(P->join, P->h2d);
-    if (j == cudaSuccess) j = cudaStreamWaitEvent(s, P->join, 0);
-    if (j == cudaSuccess) j = cudaEventRecord(P->join, P->d2h);
-    if (j == cudaSuccess) j = cudaStreamWaitEvent(s, P->join, 0);
+    cudaError_t j = cudaSuccess;
+    for (cudaStream_t h : {P->h2d, P->d2h, P->cmp}) {
+      if (j == cudaSuccess) j = cudaEventRecord(P->join, h);
+      if (j == cudaSuccess) j = cudaStreamWaitEvent(s, P->join, 0);
+    }
     if (st == TP_OK && j != cudaSuccess) return cuda_fail(j, "join");
     return st;
   };
@@ -219,19 +231,25 @@ tp_status tp_mlp_block_host(const void* X_host, const void* W1, const void* W_up
     if ((e = cudaEventRecord(P->in[c], P->h2d)) != cudaSuccess)
       return join(cuda_fail(e, "in record"));
   }
-  // Each chunk's block on the caller's stream once its rows have arrived;
-  // its Z rows leave on the other copy engine as soon as they are final.
+  // Each chunk's block once its rows have arrived, even chunks on the
+  // caller's stream and odd ones on the second compute stream, each stream
+  // with its own workspace: a chunk's kernels can then take the SMs the
+  // other chunk's last wave of tiles leaves idle.  Its Z rows leave on the
+  // other copy engine as soon as they are final.
   for (int64_t c = 0; c < n_chunks; ++c) {
     const int64_t r0 = c * L.rc;
     const int64_t rows = (T - r0) < L.rc ? (T - r0) : L.rc;
     const size_t xoff = static_cast<size_t>(r0) * static_cast<size_t>(d) * esize;
     const size_t zoff = static_cast<size_t>(r0) * static_cast<size_t>(d);
-    if ((e = cudaStreamWaitEvent(s, P->in[c], 0)) != cudaSuccess)
+    const int lane = n_streams == 2 ? static_cast<int>(c & 1) : 0;
+    const cudaStream_t cs = lane == 0 ? s : P->cmp;
+    uint8_t* const ws_c = static_cast<uint8_t*>(block_ws) + lane * L.block_bytes;
+    if ((e = cudaStreamWaitEvent(cs, P->in[c], 0)) != cudaSuccess)
       return join(cuda_fail(e, "in wait"));
-    const tp_status st = tp_mlp_block(Xd + xoff, W1, W_up, b1, W2, b2, Zd + zoff, block_ws,
-                                      L.block_bytes, rows, d, k, p, dtype, act, flags, stream);
+    const tp_status st = tp_mlp_block(Xd + xoff, W1, W_up, b1, W2, b2, Zd + zoff, ws_c,
+                                      L.block_bytes, rows, d, k, p, dtype, act, flags, cs);
     if (st != TP_OK) return join(st);
-    if ((e = cudaEventRecord(P->out[c], s)) != cudaSuccess)
+    if ((e = cudaEventRecord(P->out[c], cs)) != cudaSuccess)
       return join(cuda_fail(e, "out record"));
     if ((e = cudaStreamWaitEvent(P->d2h, P->out[c], 0)) != cudaSuccess)
       return join(cuda_fail(e, "out wait"));

@@ -172,30 +172,30 @@ def test_bf16_bias_alignment_is_checked():
 
 
 def test_host_entry_workspace_and_validation():
-    """tp_mlp_block_host: device copies of X and Z plus one chunk's block
-    workspace (chunks of >= 256 rows, multiples of 128, at most eight); every
-    argument error returns before anything is enqueued, and a valid call
+    """tp_mlp_block_host: device copies of X and Z plus the block workspace of
+    one chunk, or of two when there are several chunks (consecutive chunks run
+    on two streams); chunks of >= 256 rows, multiples of 128, at most eight.
+    Every argument error returns before anything is enqueued, and a valid call
     without a GPU fails loudly."""
     def r256(n):
         return -(-n // 256) * 256
 
+    def blk(rows):
+        return r256(tp.tp_mlp_block_workspace_size(rows, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH))
+
     T, d, k, p = 1024, 768, 3072, 2
     # 1024 rows -> four chunks of 256
-    want = r256(T * d * 2) + r256(T * d * 4) + tp.tp_mlp_block_workspace_size(
-        256, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH)
+    want = r256(T * d * 2) + r256(T * d * 4) + 2 * blk(256)
     assert tp.tp_mlp_block_host_workspace_size(T, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH) == want
     # 300 rows -> chunks of 256 and 44
     assert tp.tp_mlp_block_host_workspace_size(300, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH) == \
-        r256(300 * d * 2) + r256(300 * d * 4) + tp.tp_mlp_block_workspace_size(
-            256, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH)
+        r256(300 * d * 2) + r256(300 * d * 4) + 2 * blk(256)
     # 4096 rows -> eight chunks of 512
     assert tp.tp_mlp_block_host_workspace_size(4096, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH) == \
-        r256(4096 * d * 2) + r256(4096 * d * 4) + tp.tp_mlp_block_workspace_size(
-            512, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH)
-    # 100 rows -> one chunk (and 4096 above: eight of 512)
+        r256(4096 * d * 2) + r256(4096 * d * 4) + 2 * blk(512)
+    # 100 rows -> one chunk, one workspace
     assert tp.tp_mlp_block_host_workspace_size(100, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH) == \
-        r256(100 * d * 2) + r256(100 * d * 4) + tp.tp_mlp_block_workspace_size(
-            100, d, k, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH)
+        r256(100 * d * 2) + r256(100 * d * 4) + blk(100)
     assert tp.tp_mlp_block_host_workspace_size(T, d, 3071, p, tp.TP_BF16, tp.TP_ACT_GELU_TANH) == 0
 
     def call(**kw):
