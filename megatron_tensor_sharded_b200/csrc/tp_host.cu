@@ -23,7 +23,6 @@
 #include <mutex>
 
 #include "tp_internal.h"
-#include "tp_launch.cuh"
 #include "tp_mlp.h"
 
 namespace {
@@ -204,7 +203,7 @@ tp_status tp_mlp_block_host(const void* X_host, const void* W1, const void* W_up
 
   // Fork: the copies and the second compute stream start after the caller's
   // earlier work on `s`.
-  const int n_streams = (L.n_ws == 2 && tpk::env_int("TP_HOST_STREAMS", 2) == 2) ? 2 : 1;
+  const int n_streams = L.n_ws;
   if ((e = cudaEventRecord(P->fork, s)) != cudaSuccess) return cuda_fail(e, "fork record");
   if ((e = cudaStreamWaitEvent(P->h2d, P->fork, 0)) != cudaSuccess) return cuda_fail(e, "fork");
   if ((e = cudaStreamWaitEvent(P->d2h, P->fork, 0)) != cudaSuccess) return cuda_fail(e, "fork");

@@ -29,13 +29,6 @@ inline bool pair_allowed() {
   return on;
 }
 
-// Integer tuning knob from the environment (read at each launch).
-inline int env_int(const char* name, int fallback) {
-  const char* e = std::getenv(name);
-  if (e == nullptr || e[0] == 0) return fallback;
-  return std::atoi(e);
-}
-
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t stream, Args&&... args) {
