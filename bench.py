@@ -241,20 +241,21 @@ def oracle_sample_rows(w: WL.Workload, target_flops: float = 4e10) -> int:
     return int(max(1, min(w.T, target_flops // per_row)))
 
 
-def time_oracle(w: WL.Workload, inp: WL.Inputs, rows: int, min_seconds: float, max_reps: int):
+def time_oracle(w: WL.Workload, inp: WL.Inputs, rows: int, min_seconds: float, max_reps: int,
+                want_z: bool = False):
     """Time the oracle (as it stands) on the first `rows` token rows; returns
-    (seconds per rep, reps)."""
+    (seconds per rep, reps), plus the oracle's Z rows with `want_z`."""
     from oracle import tp_oracle as O
     X = inp.values("X")[:rows]
     args = (inp.values("W1"), inp.values("b1"), inp.values("W2"), inp.values("b2"))
     Wu = inp.values("W_up")
     reps, t0 = 0, time.perf_counter()
     while True:
-        O.mlp_sharded(X, args[0], args[1], args[2], args[3], w.p, w.act, W_up=Wu)
+        z = O.mlp_sharded(X, args[0], args[1], args[2], args[3], w.p, w.act, W_up=Wu)["Z"]
         reps += 1
         el = time.perf_counter() - t0
         if el >= min_seconds or reps >= max_reps:
-            return el / reps, reps
+            return (el / reps, reps, z) if want_z else (el / reps, reps)
 
 
 def run_reference(a, w: WL.Workload, rank: int, world: int):
@@ -850,10 +851,19 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
     }
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         rows = min(w.T, oracle_sample_rows(w))
-        sec, reps = time_oracle(w, inp, rows, min_seconds=10.0, max_reps=1000)
+        sec, reps, z_ref = time_oracle(w, inp, rows, min_seconds=10.0, max_reps=1000, want_z=True)
         line["cpu_baseline"] = {"value": w.gemm_flops() * rows / w.T / sec / 1e12, "unit": UNIT,
                                 "cores": blas_threads(), "kind": "oracle",
                                 "sample": f"first {rows} of {w.T} token rows, {reps} reps, float64"}
+        # the timed steps' own output on the same rows against the oracle
+        # (each output row depends only on its own input row)
+        from oracle import tp_oracle as O
+        tol = 1e-2 if w.dtype == "bf16" else 1e-5
+        err = O.rel_err(B.Z[:rows].cpu().numpy(), z_ref)
+        line["cpu_baseline"]["parity"] = {
+            "rows": rows, "measure": "max|gpu - oracle| / max|oracle|", "value": err,
+            "tolerance": tol, "ok": bool(err <= tol),
+            "of": "the device Z the timed calls wrote (each of them writes the same bits)"}
         try:   # the same oracle on one host thread
             from threadpoolctl import threadpool_limits
             with threadpool_limits(limits=1):
