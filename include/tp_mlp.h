@@ -19,8 +19,10 @@
  * (Y = X W), as on the day-41 post and "Tensor parallel math".
  *
  * Conventions shared by every call:
- *   - Every pointer is a DEVICE pointer owned by the caller.  The library
- *     never allocates device memory and never frees caller memory.
+ *   - Every pointer is a DEVICE pointer owned by the caller, unless a call
+ *     says otherwise (the host-buffer block, the pointer tables of the
+ *     p-GPU fold and the IPC handles are host memory).  The library never
+ *     allocates device memory and never frees caller memory.
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *     default stream).  Argument errors are returned synchronously before
  *     anything is launched; a CUDA launch error returns TP_ERR_CUDA.
@@ -511,10 +513,12 @@ const char* tp_last_error_detail(void);
 /* Number of GPU kernels this library has launched in this process. */
 uint64_t tp_kernel_launch_count(void);
 
-/* ABI version of this header (bumped on any signature change). */
+/* ABI version of this header (bumped on any signature change or added call;
+ * 2: the p-GPU fold and IPC calls, the exp2 test hook, and a host-buffer
+ * workspace sized for two chunks). */
 int tp_abi_version(void);
 
-#define TP_ABI_VERSION 1
+#define TP_ABI_VERSION 2
 
 #ifdef __cplusplus
 }
