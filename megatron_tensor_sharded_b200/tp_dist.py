@@ -139,13 +139,19 @@ class PeerAllReduce:
                 self.imported.append(handle)
 
     def _barrier(self):
-        """Stream-ordered barrier: a one-element all-reduce on the current
-        stream completes on a rank only once every rank has reached it."""
+        """Stream-ordered barrier: over NCCL a one-element all-reduce on the
+        current stream, which completes on a rank only once every rank has
+        reached it; over other backends (gloo: ranks sharing one GPU in the
+        tests) the stream is drained first and the barrier runs on the host."""
         import torch
         import torch.distributed as dist
 
-        flag = torch.zeros(1, dtype=torch.int32, device=self.P.device)
-        dist.all_reduce(flag, group=self.group)
+        if dist.get_backend(self.group) == "nccl":
+            flag = torch.zeros(1, dtype=torch.int32, device=self.P.device)
+            dist.all_reduce(flag, group=self.group)
+        else:
+            torch.cuda.current_stream(self.P.device).synchronize()
+            dist.barrier(group=self.group)
 
     def __call__(self, b2, T: int, d: int) -> None:
         parts, outs, row0, rows = peer_tables(self.rank, self.world, self.p_ptrs, self.z_ptrs, T)

@@ -225,3 +225,73 @@ def test_ipc_export_import_between_processes():
         proc.stdin.flush()
         proc.wait(timeout=60)
     assert proc.returncode == 0
+
+
+def _two_rank_worker(rank, world, port, out):
+    """One of two processes on the same GPU: gloo for the host-side
+    plumbing (handle exchange and the stream-ordered barriers, which for a
+    CUDA tensor wait for the stream's earlier kernels), CUDA IPC for the peer
+    mappings.  No kernel of one process waits on the other's."""
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    torch.cuda.set_device(0)
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=120))
+    try:
+        res = {}
+        # the block: each process runs its own shard, the peer exchange sums
+        w = W.WORKLOADS["gpt2"]
+        inp = W.make_inputs(w, seed=11)
+        X, W1, b1, W2, b2 = dev(inp.X), dev(inp.W1), dev(inp.b1), dev(inp.W2), dev(inp.b2)
+        w1, _, bb, w2 = tp_dist.shard_weights(W1, None, b1, W2, rank, world)
+        m = tp_dist.TensorParallelMLP(w1, None, bb, w2, b2, tp.TP_ACT_GELU_TANH, w.T,
+                                      exchange="peer")
+        Z = host_f32(m.forward(X)).copy()
+        torch.cuda.synchronize()
+        dist.barrier()          # both processes are done reading each other's buffers
+        m.close()
+        ws_n = tp.tp_mlp_block_workspace_size(w.T, w.d, w.k, world, tp.TP_BF16, tp.TP_ACT_GELU_TANH)
+        ws = torch.empty(ws_n, dtype=torch.uint8, device="cuda")
+        Z1 = torch.empty(w.T, w.d, device="cuda")
+        tp.tp_mlp_block(X, W1, None, b1, W2, b2, Z1, ws, ws_n, w.T, w.d, w.k, world, tp.TP_BF16,
+                        tp.TP_ACT_GELU_TANH)
+        tp.tp_sync_status()
+        res["block_same_bits"] = bool(np.array_equal(bits(Z), bits(host_f32(Z1))))
+        # the exchange alone on ragged sizes: rank r's partial drawn from seed r
+        T, d = 301, 1000
+        g = torch.Generator(device="cuda").manual_seed(100 + rank)
+        P = torch.randn(T, d, device="cuda", generator=g)
+        Zx = torch.full((T, d), float("nan"), device="cuda")
+        bx = torch.randn(d, device="cuda", generator=torch.Generator(device="cuda").manual_seed(7))
+        peer = tp_dist.PeerAllReduce(P, Zx)
+        peer(bx, T, d)
+        torch.cuda.synchronize()
+        dist.barrier()
+        peer.close()
+        Ps = [torch.randn(T, d, device="cuda",
+                          generator=torch.Generator(device="cuda").manual_seed(100 + r))
+              for r in range(world)]
+        want = _fold_ref(torch.stack(Ps), bx, T, d, world)
+        tp.tp_sync_status()
+        res["exchange_same_bits"] = bool(np.array_equal(bits(host_f32(Zx)), bits(host_f32(want))))
+        out[rank] = res
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_processes_on_one_gpu_peer_exchange():
+    """The "peer" exchange with world size 2, the two ranks being two
+    processes on the same GPU: every rank's output has the bits of the
+    single-GPU block with p = 2, and the exchange alone of the fixed-order
+    fold of both partials (+ b2)."""
+    import socket
+    import torch.multiprocessing as mp
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    mgr = mp.Manager()
+    out = mgr.dict()
+    mp.spawn(_two_rank_worker, args=(2, port, out), nprocs=2, join=True)
+    for r in range(2):
+        assert out[r] == {"block_same_bits": True, "exchange_same_bits": True}, (r, out[r])
