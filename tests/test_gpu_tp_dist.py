@@ -290,7 +290,7 @@ def test_two_processes_on_one_gpu_peer_exchange():
     with socket.socket() as s:
         s.bind(("127.0.0.1", 0))
         port = s.getsockname()[1]
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()   # never fork a process that has used CUDA
     out = mgr.dict()
     mp.spawn(_two_rank_worker, args=(2, port, out), nprocs=2, join=True)
     for r in range(2):
