@@ -1432,6 +1432,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the per-workload table of the other MLP workloads")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="MLP workloads: another token count T (same widths and shards)")
     a = ap.parse_args(argv)
     if a.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -1451,6 +1453,10 @@ def main(argv=None):
             return run_reference_attn(a, w, rank, world)
         return run_tp_attn(a, w, rank, world, local_rank)
     w = WL.WORKLOADS[a.workload]
+    if a.tokens is not None:
+        if a.tokens < 1:
+            ap.error("--tokens must be >= 1")
+        w = dataclasses.replace(w, T=a.tokens, name=f"{w.name}_T{a.tokens}")
     if a.mode == "backward":
         if a.impl == "reference":
             return run_reference_backward(a, w, rank, world)
