@@ -212,7 +212,11 @@ tp_status tp_ipc_release(const tp_ipc_handle* handle);
  * one all-reduce").  Computes exactly what tp_column_linear ->
  * tp_row_linear -> tp_reduce_partials compute (bit for bit), with the hidden
  * shards and the partials in the caller's workspace; the kernels are chained
- * with programmatic dependent launch.  With
+ * with programmatic dependent launch.  Where the row layer runs on CTA-pair
+ * tiles (bf16, b2 NULL or 16-byte aligned), the fold runs beside it: the
+ * row layer counts each 256-row region of the partials done once all p
+ * shard tiles of it are in memory, and the fold takes the regions in that
+ * order (same additions, same order, same bits).  With
  * TP_FLAG_SPLITK_FUSED the second layer accumulates over all shards and
  * writes Z directly (no partials).
  *
@@ -220,8 +224,11 @@ tp_status tp_ipc_release(const tp_ipc_handle* handle);
  *                    tp_mlp_block_workspace_size(...) bytes, 256-byte aligned;
  *                    contents on return: hidden shards [p][T][s] at offset 0,
  *                    then (default mode) the partials [p][T][d] fp32 at the
- *                    next 256-byte boundary, then tile counters (reset on
- *                    every call).
+ *                    next 256-byte boundary, then counters at the end (reset
+ *                    on every call that uses them): one int32 per 128-row
+ *                    m-tile for TP_FLAG_FUSED_LAUNCH, or one per region of
+ *                    the fold beside the row layer (regions in column-major
+ *                    order, each counted to 16 p).
  *   other arguments  as for the three calls above.
  */
 tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const void* b1,
@@ -335,13 +342,16 @@ tp_status tp_attention_heads(const void* Q, const void* K, const void* V, void* 
  * tp_attention_heads, row-parallel output projection (tp_row_linear) and the
  * fixed-order fold (tp_reduce_partials) -- one reduction per block ("Tensor
  * parallel math", "Attention: parallel across heads"; "Tensor Parallelism
- * Explained", section 2.A).
+ * Explained", section 2.A).  As in tp_mlp_block, the fold runs beside the
+ * output projection where that runs on CTA-pair tiles (bo NULL or 16-byte
+ * aligned); same bits.
  *
  *   X [T][d]; Wq [d][n_heads*head_dim]; Wk, Wv [d][n_kv_heads*head_dim];
  *   Wo [n_heads*head_dim][d]  (all bf16, [in, out]);  bo [d] fp32 nullable;
  *   Z [T][d] fp32.
  *   workspace: tp_attn_block_workspace_size(...) bytes, 256-byte aligned
- *   (Q, K, V, O shards, then the fp32 partials).
+ *   (Q, K, V, O shards, then the fp32 partials, then the fold's region
+ *   counters).
  */
 tp_status tp_attn_block(const void* X, const void* Wq, const void* Wk, const void* Wv,
                         const void* Wo, const float* bo, float* Z,
@@ -492,6 +502,10 @@ void tp_set_wait_timeout_ns(uint64_t ns);
  * slot (counted from 0 in issue order), so its consumer's wait must run
  * out.  -1 (default) disables it.  Applies to the next launch only. */
 void tp_debug_drop_load(int64_t stage_index);
+/* The same, for the tensor-core launch that follows `launches_to_skip`
+ * others (0: the next one), e.g. 1 for the row layer of a tp_mlp_block
+ * call. */
+void tp_debug_drop_load_after(int64_t stage_index, int launches_to_skip);
 
 /* Test hook (not part of the method): y[i] = the attention softmax's
  * fast 2^x for i < n, x and y fp32 device arrays of n elements (4-byte

@@ -143,6 +143,8 @@ def _load() -> ctypes.CDLL:
     lib.tp_set_wait_timeout_ns.restype = None
     lib.tp_debug_drop_load.argtypes = [i64]
     lib.tp_debug_drop_load.restype = None
+    lib.tp_debug_drop_load_after.argtypes = [i64, ctypes.c_int]
+    lib.tp_debug_drop_load_after.restype = None
     lib.tp_debug_exp2_poly.argtypes = [vp, vp, i64, vp]
     lib.tp_reduce_partials_gather.argtypes = [ctypes.POINTER(vp), i32, vp, ctypes.POINTER(vp), i32,
                                               i64, i64, i64, vp]
@@ -340,8 +342,10 @@ def tp_set_wait_timeout_ns(ns: int) -> None:
     _lib.tp_set_wait_timeout_ns(ns)
 
 
-def tp_debug_drop_load(stage_index: int) -> None:
-    _lib.tp_debug_drop_load(stage_index)
+def tp_debug_drop_load(stage_index: int, launches_to_skip: int = 0) -> None:
+    """Test hook: the tensor-core launch after `launches_to_skip` others
+    skips the load of pipeline slot `stage_index` (-1 disarms)."""
+    _lib.tp_debug_drop_load_after(stage_index, launches_to_skip)
 
 
 def tp_reduce_partials_gather(partials, b2, outs, row0, rows, d, stream=None, check=True):

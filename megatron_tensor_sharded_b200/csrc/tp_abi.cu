@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "tp_internal.h"
+#include "tp_launch.cuh"
 #include "tp_mlp.h"
 
 // Per-device status word written by the bounded device-side waits.
@@ -21,6 +22,7 @@ namespace {
 std::atomic<uint64_t> g_launches{0};
 std::atomic<uint64_t> g_timeout_ns{2000000000ull};
 std::atomic<int64_t> g_debug_drop{-1};
+std::atomic<int> g_debug_skip{0};   // tensor-core launches to pass before the drop applies
 thread_local char g_detail[512] = "";
 
 constexpr int kMaxDevices = 64;
@@ -115,7 +117,13 @@ tp_status make_ctx(void* stream, bool tensor_core, LaunchCtx* c) {
     return fail(TP_ERR_UNSUPPORTED, "bf16 path needs an sm_100 device (found sm_%d.x)", cc);
   c->stream = static_cast<cudaStream_t>(stream);
   c->timeout_ns = g_timeout_ns.load();
-  c->debug_drop = tensor_core ? g_debug_drop.exchange(-1) : -1;
+  c->debug_drop = -1;
+  if (tensor_core && g_debug_drop.load() >= 0) {
+    if (g_debug_skip.load() > 0)
+      g_debug_skip.fetch_sub(1);
+    else
+      c->debug_drop = g_debug_drop.exchange(-1);
+  }
   return TP_OK;
 }
 
@@ -168,14 +176,22 @@ tp_status cuda_status(cudaError_t e, const char* what) {
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
+// Counters at the end of the workspace: the single-launch block's per-m-tile
+// counters, or the row layer's per-region counters for the overlapped fold
+// (never both in one call).
+size_t counter_bytes(int64_t T, int64_t d) {
+  const size_t a = block_counter_bytes(T, d), b = region_counter_bytes(T, d);
+  return a > b ? a : b;
+}
+
 // Workspace layout: hidden shards Y, then (default mode) the fp32 partials,
-// then the fused kernel's tile counters, each at a 256-byte boundary.
+// then the counters, each at a 256-byte boundary.
 size_t workspace_bytes(int64_t T, int64_t d, int64_t k, int p, int dtype, int flags) {
   const size_t esize = dtype == TP_BF16 ? 2 : 4;
   size_t bytes = align256(static_cast<size_t>(T) * static_cast<size_t>(k) * esize);
   if (!(flags & (TP_FLAG_SPLITK_FUSED | TP_FLAG_ROW_FOLD)))
     bytes += align256(static_cast<size_t>(p) * static_cast<size_t>(T) * static_cast<size_t>(d) * 4);
-  return bytes + block_counter_bytes(T, d);
+  return bytes + counter_bytes(T, d);
 }
 
 tp_status column_impl(const void* X, const void* W1, const void* W_up, const void* b1, void* Y,
@@ -233,6 +249,43 @@ tp_status reduce_impl(const float* partials, const float* b2, float* Z, int64_t 
   LaunchCtx c{};
   TP_TRY(make_ctx(stream, false, &c));
   return cuda_status(launch_reduce(c, partials, b2, Z, T, d, p), "reduce launch");
+}
+
+// Zeroed counters at `at` for the fold beside the row layer, when that path
+// applies: bf16 row layer on CTA-pair tiles, b2 NULL or 16-byte aligned
+// (the fold reads it as vectors).  *out is NULL otherwise.  The reset is
+// enqueued here, before the caller's first launch, so that nothing sits
+// between the row layer and the layer before it.
+tp_status prepare_regions(void* at, int64_t T, int64_t k, int64_t d, int p, const float* b2,
+                          void* stream, int** out) {
+  *out = nullptr;
+  if (!region_fold_allowed() || (b2 != nullptr && !aligned16(b2))) return TP_OK;
+  LaunchCtx c{};
+  TP_TRY(make_ctx(stream, false, &c));
+  if (!row_on_pairs(c, T, k, d, p)) return TP_OK;
+  const cudaError_t e = cudaMemsetAsync(at, 0, region_counter_bytes(T, d),
+                                        static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(TP_ERR_CUDA, "counter reset: %s", cudaGetErrorString(e));
+  *out = static_cast<int*>(at);
+  return TP_OK;
+}
+
+// bf16 row layer to partials, then the fixed-order fold of the partials:
+// beside the row layer when `regions` came from prepare_regions, after it
+// otherwise.  Same bits either way.
+tp_status row_and_fold(const void* Y, const void* W2, float* P, const float* b2, float* Z,
+                       int64_t T, int64_t k, int64_t d, int p, int* regions, void* stream) {
+  if (regions == nullptr) {
+    TP_TRY(row_impl(Y, W2, P, T, k, d, p, TP_BF16, stream));
+    return reduce_impl(P, b2, Z, T, d, p, stream);
+  }
+  LaunchCtx c{};
+  TP_TRY(make_ctx(stream, true, &c));
+  RegionFold rf{};
+  TP_TRY(launch_tc_row(c, Y, W2, P, T, k, d, p, regions, &rf));
+  if (rf.cnt != nullptr)
+    return cuda_status(launch_fold_regions(c, P, b2, Z, T, d, p, rf), "fold launch");
+  return reduce_impl(P, b2, Z, T, d, p, stream);
 }
 
 tp_status check_heads(int p, int n_heads, int n_kv_heads, int head_dim) {
@@ -325,7 +378,7 @@ size_t attn_workspace_bytes(int64_t T, int64_t d, int n_heads, int n_kv_heads, i
   const size_t q = align256(static_cast<size_t>(T) * n_heads * head_dim * 2);
   const size_t kv = align256(static_cast<size_t>(T) * n_kv_heads * head_dim * 2);
   const size_t part = align256(static_cast<size_t>(p) * T * d * 4);
-  return 2 * q + 2 * kv + part;
+  return 2 * q + 2 * kv + part + region_counter_bytes(T, d);
 }
 
 struct BwdLayout {
@@ -473,7 +526,7 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
     // first, so that an unsupported device returns with nothing enqueued.
     LaunchCtx c{};
     TP_TRY(make_ctx(stream, true, &c));
-    int* counters = reinterpret_cast<int*>(ws + need - block_counter_bytes(T, d));
+    int* counters = reinterpret_cast<int*>(ws + need - counter_bytes(T, d));
     const cudaError_t e = cudaMemsetAsync(counters, 0, block_counter_bytes(T, d),
                                           static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return fail(TP_ERR_CUDA, "counter reset: %s", cudaGetErrorString(e));
@@ -481,7 +534,13 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
     if (splitk) return TP_OK;
     return reduce_impl(P, b2, Z, T, d, p, stream);
   }
+  // Default bf16 mode: the fold runs beside the row layer where that
+  // applies (prepare_regions).
+  int* regions = nullptr;
+  if (!splitk && !row_fold && dtype == TP_BF16)
+    TP_TRY(prepare_regions(ws + need - counter_bytes(T, d), T, k, d, p, b2, stream, &regions));
   TP_TRY(column_impl(X, W1, W_up, b1, Y, T, d, k, p, dtype, act, stream));
+  if (regions != nullptr) return row_and_fold(Y, W2, P, b2, Z, T, k, d, p, regions, stream);
   if (row_fold) {
     LaunchCtx c{};
     TP_TRY(make_ctx(stream, true, &c));
@@ -544,12 +603,14 @@ tp_status tp_attn_block(const void* X, const void* Wq, const void* Wk, const voi
   void* V = ws + qb + kvb;
   void* O = ws + qb + 2 * kvb;
   float* P = reinterpret_cast<float*>(ws + 2 * qb + 2 * kvb);
+  int* regions = nullptr;
+  TP_TRY(prepare_regions(ws + need - region_counter_bytes(T, d), T, kq, d, p, bo, stream,
+                         &regions));
   TP_TRY(column_impl(X, Wq, nullptr, nullptr, Q, T, d, kq, p, TP_BF16, TP_ACT_IDENTITY, stream));
   TP_TRY(column_impl(X, Wk, nullptr, nullptr, K, T, d, kkv, p, TP_BF16, TP_ACT_IDENTITY, stream));
   TP_TRY(column_impl(X, Wv, nullptr, nullptr, V, T, d, kkv, p, TP_BF16, TP_ACT_IDENTITY, stream));
   TP_TRY(attention_impl(Q, K, V, O, T, p, n_heads, n_kv_heads, head_dim, causal, stream));
-  TP_TRY(row_impl(O, Wo, P, T, kq, d, p, TP_BF16, stream));
-  return reduce_impl(P, bo, Z, T, d, p, stream);
+  return row_and_fold(O, Wo, P, bo, Z, T, kq, d, p, regions, stream);
 }
 
 tp_status tp_layer_norm(const float* X, const float* gamma, const float* beta, void* Y, int64_t T,
@@ -821,7 +882,12 @@ tp_status tp_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream) 
   return cuda_status(launch_exp2_poly_probe(c, x, y, n), "exp2 probe launch");
 }
 
-void tp_debug_drop_load(int64_t stage_index) { g_debug_drop.store(stage_index < 0 ? -1 : stage_index); }
+void tp_debug_drop_load(int64_t stage_index) { tp_debug_drop_load_after(stage_index, 0); }
+
+void tp_debug_drop_load_after(int64_t stage_index, int launches_to_skip) {
+  g_debug_skip.store(launches_to_skip < 0 ? 0 : launches_to_skip);
+  g_debug_drop.store(stage_index < 0 ? -1 : stage_index);
+}
 
 const char* tp_status_string(int status) {
   switch (status) {

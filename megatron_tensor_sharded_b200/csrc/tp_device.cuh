@@ -15,6 +15,7 @@ constexpr unsigned kErrWaitEmpty = 1u << 1;     // producer: slot never released
 constexpr unsigned kErrWaitAccFull = 1u << 2;   // epilogue: accumulator never committed
 constexpr unsigned kErrWaitAccEmpty = 1u << 3;  // mma: accumulator never drained
 constexpr unsigned kErrWaitDrain = 1u << 4;     // teardown: in-flight work never finished
+constexpr unsigned kErrWaitRegion = 1u << 7;    // fold: a region's partial tiles never completed
 
 struct WaitCtl {
   unsigned* err;        // per-device status word
@@ -124,6 +125,23 @@ __device__ __forceinline__ bool wait_teardown(uint32_t bar, uint32_t parity, con
       return false;
     }
   }
+}
+
+// ------------------------------------------------ counters between CTAs (global)
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void red_release_gpu_add(int* p, int v) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// Orders this thread's generic-proxy and async-proxy (TMA) accesses to
+// global memory with respect to each other.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
 }
 
 // ------------------------------------------------- programmatic dependent launch

@@ -267,6 +267,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(b), 0));
+      if constexpr (MODE == kModeRowPartial) {
+        if (P.region_cnt != nullptr) {
+          // Publish this warp's part of the tile to the overlapped fold: its
+          // bulk stores complete, are ordered for generic-proxy readers, and
+          // one release increment counts them (16 per tile and shard).  The
+          // accumulator was handed back above, so the wait delays no MMA.
+          if (lane == 0) {
+            bulk_wait_all0();
+            fence_proxy_async_global();
+            red_release_gpu_add(P.region_cnt + tc.n * P.m_tiles + tc.m, 1);
+          }
+          __syncwarp();
+        }
+      }
     }
     // the staging tiles must be read out before shared memory is released
     if (lane == 0) bulk_wait_all0();

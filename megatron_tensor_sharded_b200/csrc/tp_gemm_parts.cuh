@@ -63,6 +63,8 @@ struct TcParams {
   const void* bias;      // b1 (bf16, column) or b2 (fp32, split-K row); may be null
   void* out;             // Y bf16 [p][T][s] | P fp32 [p][T][d] | Z fp32 [T][d]
   int32_t bulk_out;      // column layers: 1 = bulk tensor stores through shared memory
+  int* region_cnt;       // row partials on CTA pairs: per-tile completion counters read by
+                         // the overlapped fold ([n_tiles][m_tiles], tile order); may be null
   WaitCtl wait;
   int64_t debug_drop;    // slot (in issue order) whose load is skipped; -1 none
 };

@@ -333,8 +333,17 @@ tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, co
   return launch_bn<kModeColumn>(c, tch.bn, mA, mB0, mB1, mY, prm);
 }
 
+size_t region_counter_bytes(int64_t T, int64_t d) {
+  const size_t n = static_cast<size_t>(ceil_div(T, 2 * BM)) * static_cast<size_t>(ceil_div(d, 128));
+  return (n * sizeof(int) + 255) & ~size_t(255);
+}
+
+bool row_on_pairs(const LaunchCtx& c, int64_t T, int64_t k, int64_t d, int p) {
+  return pick_tile(T, d, p, ceil_div(k / p, BK), c.num_sms, false, pair_allowed()).pair;
+}
+
 tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float* P, int64_t T,
-                        int64_t k, int64_t d, int p) {
+                        int64_t k, int64_t d, int p, int* region_cnt, RegionFold* rf) {
   const int64_t s = k / p;
   CUtensorMap mA, mB, mC;
   if (!make_map_a(&mA, Y, s, T, p) || !make_map_b(&mB, W2, d, k) ||
@@ -353,7 +362,17 @@ tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float
   prm.bias = nullptr;
   prm.out = P;
   const TileChoice tch = pick_tile(T, d, p, prm.k_blocks, c.num_sms, false, pair_allowed());
-  if (tch.pair) return launch_tc_pair(c, kModeRowPartial, tch.bn, mA, mB, mB, mC, prm);
+  if (rf != nullptr) *rf = RegionFold{};
+  if (tch.pair) {
+    if (region_cnt != nullptr && rf != nullptr) {
+      // regions = the pair tiles (256 rows x bn columns); 8 epilogue warps
+      // on each of the two CTAs count once per tile and shard
+      prm.region_cnt = region_cnt;
+      *rf = RegionFold{region_cnt, 2 * BM, tch.bn, ceil_div(T, 2 * BM), ceil_div(d, tch.bn),
+                       2 * NUM_EPI_WARPS * p};
+    }
+    return launch_tc_pair(c, kModeRowPartial, tch.bn, mA, mB, mB, mC, prm);
+  }
   return launch_bn<kModeRowPartial>(c, tch.bn, mA, mB, mB, mC, prm);
 }
 

@@ -46,8 +46,22 @@ cudaError_t launch_simt_row_splitk(const LaunchCtx& c, const float* Y, const flo
 tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, const void* Wup,
                            const void* b1, void* Y, int64_t T, int64_t d, int64_t k, int p,
                            int act);
+// Regions of the partials whose p shard tiles the row layer counts as done
+// (row layers on CTA-pair tiles only): region (m, n) covers rows
+// [m*rows, +rows) and columns [n*cols, +cols); counter n*m_regions + m
+// reaches `target` once every shard's tile of it is in memory.
+struct RegionFold {
+  int* cnt;   // null: the row layer publishes nothing, fold after it
+  int rows, cols, m_regions, n_regions, target;
+};
+// Row layer; with `region_cnt` (zeroed, region_counter_bytes()) it also
+// publishes per-tile completion when it runs on CTA pairs and says so in *rf.
 tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float* P, int64_t T,
-                        int64_t k, int64_t d, int p);
+                        int64_t k, int64_t d, int p, int* region_cnt = nullptr,
+                        RegionFold* rf = nullptr);
+size_t region_counter_bytes(int64_t T, int64_t d);
+// Whether launch_tc_row picks CTA-pair tiles for this layer.
+bool row_on_pairs(const LaunchCtx& c, int64_t T, int64_t k, int64_t d, int p);
 tp_status launch_tc_row_splitk(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
                                float* Z, int64_t T, int64_t k, int64_t d, int p);
 
@@ -88,6 +102,12 @@ tp_status launch_tc_block(const LaunchCtx& c, const void* X, const void* W1, con
 // ---- row layer with the fixed-order fold in its epilogue (tp_gemm_fold_sm100.cu)
 tp_status launch_tc_row_fold(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
                              float* Z, int64_t T, int64_t k, int64_t d, int p);
+
+// ---- fixed-order fold overlapped with the row layer (tp_reduce.cu): the
+// same additions as launch_reduce, region by region as the counters of `rf`
+// complete; launched right behind the row layer.
+cudaError_t launch_fold_regions(const LaunchCtx& c, const float* P, const float* b2, float* Z,
+                                int64_t T, int64_t d, int p, const RegionFold& rf);
 
 // ---- row-wise fold (+ bias, + residual) and LayerNorm (tp_rowops.cu)
 cudaError_t launch_row_fold_ln(const LaunchCtx& c, const float* P, int p, const float* bias,

@@ -29,6 +29,17 @@ inline bool pair_allowed() {
   return on;
 }
 
+// tp_mlp_block's fold overlapped with its row layer (CTA-pair row tiles);
+// TP_DISABLE_REGION_FOLD=1 folds after the row layer instead (for
+// comparisons; same bits).
+inline bool region_fold_allowed() {
+  static const bool on = [] {
+    const char* e = std::getenv("TP_DISABLE_REGION_FOLD");
+    return !(e != nullptr && e[0] == '1');
+  }();
+  return on;
+}
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t stream, Args&&... args) {

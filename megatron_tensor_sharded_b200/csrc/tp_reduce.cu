@@ -8,6 +8,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <mutex>
 
 #include "tp_device.cuh"
 #include "tp_internal.h"
@@ -72,7 +73,135 @@ __global__ void __launch_bounds__(256) reduce_scalar_kernel(const float* __restr
   }
 }
 
+// The same fold, region by region, while the row layer is still running:
+// launched right behind it (programmatic dependent launch, so its CTAs
+// become resident beside the row layer's as soon as those have started),
+// each CTA takes regions in the order the row layer finishes their tiles,
+// waits (bounded) until the region's counter shows every shard's tile in
+// memory, and folds it.  It has no griddepcontrol.wait: the counters, a
+// release per producer and an acquire here, order it after the stores it
+// reads, and the row layer itself ran after everything before it.  Vector
+// path only (d % 4 == 0, 16-byte aligned P, Z and b2).
+struct RegionArgs {
+  const float4* part;
+  const float* b2;
+  float4* Z;
+  const int* cnt;
+  int64_t T, d4, n4;   // rows, float4 per row, float4 per shard
+  int32_t rows, cols4, m_regions, n_regions, target;
+  WaitCtl wait;
+};
+
+__device__ __forceinline__ bool wait_region(const int* cnt, int target, const WaitCtl& w) {
+  if (ld_acquire_gpu(cnt) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (ld_acquire_gpu(cnt) < target) {
+    if (globaltimer_ns() - t0 > w.timeout_ns) {
+      atomicOr(w.err, kErrWaitRegion);
+      return false;
+    }
+    __nanosleep(500);
+  }
+  return true;
+}
+
+// 512 threads (16 warps of at most 64 registers: 32K registers) fit beside
+// a row-layer CTA (12 warps); 1024 would not.
+constexpr int kFoldThreads = 512;
+// Work unit: a quarter of a region's rows (64 of 256), so that the units
+// spread evenly over the CTAs and a region that completes is folded by
+// several CTAs at once.
+constexpr int kUnitsPerRegion = 4;
+
+template <int P>
+__global__ void __launch_bounds__(kFoldThreads, 2) fold_regions_kernel(const RegionArgs a, int p_runtime) {
+  pdl_launch_dependents();
+  __shared__ int s_ok;
+  const int32_t units = a.m_regions * a.n_regions * kUnitsPerRegion;
+  const int32_t sub = a.rows / kUnitsPerRegion;
+  for (int32_t u = blockIdx.x; u < units; u += gridDim.x) {
+    const int32_t r = u / kUnitsPerRegion, q = u - r * kUnitsPerRegion;
+    if (threadIdx.x == 0) s_ok = wait_region(a.cnt + r, a.target, a.wait) ? 1 : 0;
+    __syncthreads();
+    if (!s_ok) return;   // block-uniform
+    const int32_t n = r / a.m_regions, m = r - n * a.m_regions;
+    const int64_t r0 = static_cast<int64_t>(m) * a.rows + static_cast<int64_t>(q) * sub;
+    const int64_t nrows = a.T - r0 < sub ? a.T - r0 : sub;   // may be <= 0 at the ragged end
+    const int64_t c0 = static_cast<int64_t>(n) * a.cols4;
+    const int32_t w4 = static_cast<int32_t>(a.d4 - c0 < a.cols4 ? a.d4 - c0 : a.cols4);
+    const int64_t count = nrows > 0 ? nrows * w4 : 0;
+    for (int64_t e = threadIdx.x; e < count; e += blockDim.x) {
+      const int64_t row = r0 + e / w4;
+      const int64_t col = c0 + e % w4;
+      const int64_t i = row * a.d4 + col;
+      float4 acc;
+      if constexpr (P > 0) {
+        float4 v[P];
+#pragma unroll
+        for (int s = 0; s < P; ++s) v[s] = ld_stream(a.part + s * a.n4 + i);
+        acc = v[0];
+#pragma unroll
+        for (int s = 1; s < P; ++s) acc = add4(acc, v[s]);
+      } else {
+        acc = ld_stream(a.part + i);
+        for (int s = 1; s < p_runtime; ++s) acc = add4(acc, ld_stream(a.part + s * a.n4 + i));
+      }
+      if (a.b2 != nullptr) acc = add4(acc, __ldg(reinterpret_cast<const float4*>(a.b2) + col));
+      __stcs(a.Z + i, acc);
+    }
+    __syncthreads();   // s_ok is rewritten for the next unit
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_fold_regions(const LaunchCtx& c, const float* P, const float* b2, float* Z,
+                                int64_t T, int64_t d, int p, const RegionFold& rf) {
+  if (T == 0) return cudaSuccess;
+  RegionArgs a{};
+  a.part = reinterpret_cast<const float4*>(P);
+  a.b2 = b2;
+  a.Z = reinterpret_cast<float4*>(Z);
+  a.cnt = rf.cnt;
+  a.T = T;
+  a.d4 = d / 4;
+  a.n4 = T * d / 4;
+  a.rows = rf.rows;
+  a.cols4 = rf.cols / 4;
+  a.m_regions = rf.m_regions;
+  a.n_regions = rf.n_regions;
+  a.target = rf.target;
+  a.wait.err = c.err_word;
+  a.wait.timeout_ns = c.timeout_ns;
+  // One CTA per SM at most: beside a row-layer CTA only one more CTA fits
+  // (shared memory, registers), and the carve-out must match the row
+  // layer's for the two to share an SM.
+  int blocks = rf.m_regions * rf.n_regions * kUnitsPerRegion;
+  if (blocks > c.num_sms) blocks = c.num_sms;
+  static uint64_t attr_epoch[64] = {};
+  static std::mutex mu;
+  auto kern = p == 2 ? fold_regions_kernel<2>
+            : p == 4 ? fold_regions_kernel<4>
+            : p == 8 ? fold_regions_kernel<8>
+                     : fold_regions_kernel<0>;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    const int dev = c.device & 63;
+    if (attr_epoch[dev] != c.epoch) {
+      for (auto k : {fold_regions_kernel<0>, fold_regions_kernel<2>, fold_regions_kernel<4>,
+                     fold_regions_kernel<8>}) {
+        const cudaError_t e = cudaFuncSetAttribute(
+            k, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+        if (e != cudaSuccess) return e;
+      }
+      attr_epoch[dev] = c.epoch;
+    }
+  }
+  const cudaError_t e =
+      launch_pdl(kern, dim3(static_cast<unsigned>(blocks)), dim3(kFoldThreads), 0, c.stream, a, p);
+  note_launch();
+  return e;
+}
 
 cudaError_t launch_reduce(const LaunchCtx& c, const float* P, const float* b2, float* Z, int64_t T,
                           int64_t d, int p) {

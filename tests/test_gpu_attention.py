@@ -27,7 +27,7 @@ import torch
 
 import megatron_tensor_sharded_b200 as tp
 import workloads as W
-from gpu_util import dev, host_f32
+from gpu_util import bits, dev, host_f32
 from oracle import tp_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -205,3 +205,39 @@ def test_attention_dropped_load_times_out():
     got = _run_heads(Qb, Kb, Vb, p, T, h, hkv, True)
     Q, K, V = _bf16_vals(Qb), _bf16_vals(Kb), _bf16_vals(Vb)
     _check_head(got[1][:, :128], Q[1][:, :128], K[1][:, :128], V[1][:, :128], True)
+
+
+@pytest.mark.parametrize("bias", [True, False])
+def test_attention_block_is_bit_identical_to_separate_calls(bias):
+    """A shape whose output projection runs on CTA-pair tiles (T=1000,
+    d=2048, 16 query / 4 key-value heads on p=4): tp_attn_block, whose fold
+    runs beside that projection, gives the bits of the separate calls
+    (three column projections, tp_attention_heads, tp_row_linear,
+    tp_reduce_partials), call after call on one workspace."""
+    T, d, h, hkv, p = 1000, 2048, 16, 4, 4
+    inp = W.make_attn_inputs(T, d, h, hkv, 128, seed=7, with_bias=bias, w_std=0.03)
+    X, Wq, Wk, Wv, Wo = dev(inp.X), dev(inp.Wq), dev(inp.Wk), dev(inp.Wv), dev(inp.Wo)
+    bo = dev(inp.bo)
+    kq, kkv = h * 128, hkv * 128
+    Q = torch.empty((p, T, kq // p), dtype=torch.bfloat16, device="cuda")
+    K = torch.empty((p, T, kkv // p), dtype=torch.bfloat16, device="cuda")
+    V = torch.empty_like(K)
+    Oh = torch.empty_like(Q)
+    P = torch.empty((p, T, d), dtype=torch.float32, device="cuda")
+    Zs = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    ident = tp.TP_ACT_IDENTITY
+    tp.tp_column_linear(X, Wq, None, None, Q, T, d, kq, p, tp.TP_BF16, ident)
+    tp.tp_column_linear(X, Wk, None, None, K, T, d, kkv, p, tp.TP_BF16, ident)
+    tp.tp_column_linear(X, Wv, None, None, V, T, d, kkv, p, tp.TP_BF16, ident)
+    tp.tp_attention_heads(Q, K, V, Oh, T, p, h, hkv, 128, 1)
+    tp.tp_row_linear(Oh, Wo, P, T, kq, d, p, tp.TP_BF16)
+    tp.tp_reduce_partials(P, bo, Zs, T, d, p)
+    tp.tp_sync_status()
+    want = bits(host_f32(Zs))
+    n = tp.tp_attn_block_workspace_size(T, d, h, hkv, 128, p)
+    ws = torch.full((n,), 0x7F, dtype=torch.uint8, device="cuda")
+    for _ in range(2):
+        Z = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")
+        tp.tp_attn_block(X, Wq, Wk, Wv, Wo, bo, Z, ws, n, T, d, h, hkv, 128, p, 1)
+        tp.tp_sync_status()
+        assert np.array_equal(bits(host_f32(Z)), want)

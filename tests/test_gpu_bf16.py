@@ -302,3 +302,67 @@ def test_block_is_bit_identical_to_separate_calls(T, d, s, p, act, bias):
                         blk.dtype, blk.act, tp.TP_FLAG_NONE)
         blk.sync()
         assert np.array_equal(bits(host_f32(Zb)), want)
+
+
+def _counter_bytes(T, d):
+    r256 = lambda n: -(-n // 256) * 256  # noqa: E731
+    return max(r256(4 * -(-T // 128)), r256(4 * -(-T // 256) * -(-d // 128)))
+
+
+@pytest.mark.parametrize("T,d,s,p,act,bias", [(1000, 2176, 2048, 4, "gelu_tanh", True),
+                                              (777, 2048, 1536, 3, "relu", False),
+                                              (513, 1024, 3584, 8, "swiglu", True)])
+def test_block_fold_beside_row_layer(T, d, s, p, act, bias):
+    """Shapes whose row layer runs on CTA-pair tiles (256 rows x 256 or 128
+    columns; ragged T, a last region 128 columns wide, p = 3 on the generic
+    fold): tp_mlp_block folds each region of the partials beside the row
+    layer once all p shard tiles of it are in memory.  Z has the bits of the
+    three separate calls, call after call on one workspace, and the
+    workspace's region counters show every region counted to 16 p (eight
+    epilogue warps on each CTA of a pair, once per shard)."""
+    k = s * p
+    inp = _random_bf16(T, d, k, act, with_bias=bias, seed=T + d + p + 1)
+    blk = DeviceBlock(inp, T, d, k, p, act)
+    blk.column()
+    blk.row()
+    blk.reduce()
+    blk.sync()
+    want = bits(host_f32(blk.Z))
+    n = tp.tp_mlp_block_workspace_size(T, d, k, p, blk.dtype, blk.act)
+    ws = torch.full((n,), 0x7F, dtype=torch.uint8, device="cuda")
+    m_regions = -(-T // 256)
+    for _ in range(3):
+        Zb = torch.full_like(blk.Z, float("nan"))
+        tp.tp_mlp_block(blk.X, blk.W1, blk.Wu, blk.b1, blk.W2, blk.b2, Zb, ws, n, T, d, k, p,
+                        blk.dtype, blk.act, tp.TP_FLAG_NONE)
+        blk.sync()
+        assert np.array_equal(bits(host_f32(Zb)), want)
+        cnt = ws[n - _counter_bytes(T, d):].cpu().numpy().view(np.int32)
+        assert cnt[0] == 16 * p
+        assert set(np.unique(cnt).tolist()) <= {0, 16 * p}
+        assert int((cnt == 16 * p).sum()) in (m_regions * -(-d // 256), m_regions * -(-d // 128))
+    if T <= 1024:
+        assert O.rel_err(host_f32(blk.Z), _oracle(inp, p, act)["Z"]) <= TOL_BF16
+
+
+def test_block_fold_after_row_layer_with_unaligned_b2():
+    """A b2 that is only 4-byte aligned keeps the fold after the row layer
+    (the overlapped fold reads b2 as 16-byte vectors): same bits."""
+    T, d, s, p, act = 1000, 2048, 512, 4, "gelu_tanh"
+    k = s * p
+    inp = _random_bf16(T, d, k, act, with_bias=True, seed=5)
+    blk = DeviceBlock(inp, T, d, k, p, act)
+    blk.column()
+    blk.row()
+    blk.reduce()
+    blk.sync()
+    want = bits(host_f32(blk.Z))
+    b2u = torch.empty(d + 1, dtype=torch.float32, device="cuda")[1:]
+    b2u.copy_(blk.b2)
+    n = tp.tp_mlp_block_workspace_size(T, d, k, p, blk.dtype, blk.act)
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
+    Zb = torch.full_like(blk.Z, float("nan"))
+    tp.tp_mlp_block(blk.X, blk.W1, blk.Wu, blk.b1, blk.W2, b2u, Zb, ws, n, T, d, k, p,
+                    blk.dtype, blk.act, tp.TP_FLAG_NONE)
+    blk.sync()
+    assert np.array_equal(bits(host_f32(Zb)), want)

@@ -4,6 +4,8 @@ the CTA, frees its TMEM and returns, and the context stays usable.  The fault
 is injected on the host (tp_debug_drop_load: the next tensor-core launch skips
 one pipeline slot) -- nothing traps or faults."""
 
+import re
+
 import numpy as np
 import pytest
 import torch
@@ -106,9 +108,8 @@ def test_dropped_load_in_cta_pair_gemm_times_out(short_timeout):
 
 def test_dropped_load_in_attention_times_out(short_timeout):
     """The attention kernel: a K/V block the producer never loads makes the
-    MMA issuer's wait run out; the softmax warps (and, when a row's keys are
-    split over two threads, their pair exchanges) see the abort flag and
-    stop; the next launch is correct."""
+    MMA issuer's wait run out; the softmax warps see the abort flag and stop;
+    the next launch is correct."""
     rng = np.random.default_rng(2)
     p, T, h, hkv = 2, 300, 4, 2
     shape = lambda heads: (p, T, (heads // p) * 128)  # noqa: E731
@@ -137,3 +138,31 @@ def test_dropped_load_in_attention_times_out(short_timeout):
                                vv[s, :, g * 128:(g + 1) * 128], True)
             err = np.abs(got[s, :, hh * 128:(hh + 1) * 128] - want)
             assert err.max() <= 2.0 ** -8 * (np.abs(vv).max() + 1.0)
+
+
+def test_dropped_load_in_block_row_layer_times_out(short_timeout):
+    """tp_mlp_block on a shape whose row layer runs on CTA pairs, with the
+    fold running beside it: a load the row layer (the call's second
+    tensor-core launch) never issues makes its MMA wait run out, the layer
+    stops without counting its remaining tiles, and the fold's waits on those
+    regions run out as well (status bit 0x80); the next call is correct."""
+    rng = np.random.default_rng(3)
+    c = W.f32_to_bf16_bits
+    T, d, k, p = 1000, 2048, 2048, 4
+    inp = W.Inputs(c(rng.standard_normal((T, d), dtype=np.float32)),
+                   c(rng.standard_normal((d, k), dtype=np.float32) * 0.02), None, None,
+                   c(rng.standard_normal((k, d), dtype=np.float32) * 0.02), None, "bf16")
+    blk = DeviceBlock(inp, T, d, k, p, "gelu_tanh")
+    assert tp.tp_sync_status(check=False) == 0
+    tp.tp_debug_drop_load(3, 1)
+    blk.block()
+    st = tp.tp_sync_status(check=False)
+    assert st == 6, tp.tp_status_string(st)
+    word = int(re.search(r"status bits 0x([0-9a-f]+)", tp.tp_last_error_detail()).group(1), 16)
+    assert word & 0x80 and word & 0x1, hex(word)
+    blk.Z.fill_(float("nan"))
+    blk.block()
+    assert tp.tp_sync_status(check=False) == 0
+    ref = O.mlp_sharded(inp.values("X")[:64], inp.values("W1"), None, inp.values("W2"), None, p,
+                        "gelu_tanh")["Z"]
+    assert O.rel_err(host_f32(blk.Z)[:64], ref) <= 1e-2
