@@ -787,7 +787,8 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
     e2e = None if a.no_e2e else measure_e2e(a, torch, tp, B, w, world, barrier)
 
     value = whole_job_value(w.gemm_flops(), world, ms_step) / 1e12
-    kernel_name = {"partials": "tp_mlp_block: column GEMM -> row GEMM -> fixed-order fold (PDL-chained)",
+    kernel_name = {"partials": "tp_mlp_block: column GEMM -> row GEMM -> fixed-order fold (PDL-chained; "
+                               "on CTA-pair row tiles the fold runs beside the row GEMM)",
                    "fold": "tp_mlp_block row-fold: column GEMM -> row GEMM folding the p partials "
                            "in its epilogue (bit-identical to partials + fold)",
                    "splitk": "tp_mlp_block split-K: column GEMM -> row GEMM accumulating all shards",

@@ -64,7 +64,9 @@ struct TcParams {
   void* out;             // Y bf16 [p][T][s] | P fp32 [p][T][d] | Z fp32 [T][d]
   int32_t bulk_out;      // column layers: 1 = bulk tensor stores through shared memory
   int* region_cnt;       // row partials on CTA pairs: per-tile completion counters read by
-                         // the overlapped fold ([n_tiles][m_tiles], tile order); may be null
+                         // the overlapped fold ([n_tiles][m_tiles]); may be null
+  int32_t m_group;       // > 0: tiles walk groups of this many m-tiles, group slowest (all
+                         // shards of one group before the next); 0: one group
   WaitCtl wait;
   int64_t debug_drop;    // slot (in issue order) whose load is skipped; -1 none
 };
@@ -74,12 +76,19 @@ struct TileCoord {
 };
 
 __device__ __forceinline__ TileCoord decode_tile(const TcParams& P, int32_t t) {
-  const int32_t per_batch = P.m_tiles * P.n_tiles;
+  // Within a group of m-tiles: shard slowest, then n, m fastest (neighbouring
+  // CTAs share the weight panel).  Every group but the last is full.
+  const int32_t mg_full = P.m_group > 0 ? P.m_group : P.m_tiles;
+  const int32_t group_tiles = mg_full * P.n_tiles * P.batches;
+  const int32_t g = t / group_tiles;
+  const int32_t m0 = g * mg_full;
+  const int32_t mg = P.m_tiles - m0 < mg_full ? P.m_tiles - m0 : mg_full;
+  int32_t r = t - g * group_tiles;
   TileCoord c;
-  c.batch = t / per_batch;
-  const int32_t r = t - c.batch * per_batch;
-  c.n = r / P.m_tiles;   // m fastest: neighbouring CTAs share the weight panel
-  c.m = r - c.n * P.m_tiles;
+  c.batch = r / (mg * P.n_tiles);
+  r -= c.batch * mg * P.n_tiles;
+  c.n = r / mg;
+  c.m = m0 + r - c.n * mg;
   return c;
 }
 

@@ -40,7 +40,6 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -368,8 +367,14 @@ tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float
       // regions = the pair tiles (256 rows x bn columns); 8 epilogue warps
       // on each of the two CTAs count once per tile and shard
       prm.region_cnt = region_cnt;
-      *rf = RegionFold{region_cnt, 2 * BM, tch.bn, ceil_div(T, 2 * BM), ceil_div(d, tch.bn),
-                       2 * NUM_EPI_WARPS * p};
+      // Two halves of the m-tiles, all shards of the first half before the
+      // second: the first half's regions complete mid-layer and are folded
+      // while the tensor cores work on the second (each W2 panel is then
+      // read once per half).
+      const int32_t m_tiles = ceil_div(T, 2 * BM);
+      prm.m_group = m_tiles >= 4 ? ceil_div(m_tiles, 2) : 0;
+      *rf = RegionFold{region_cnt, 2 * BM, tch.bn, m_tiles, ceil_div(d, tch.bn),
+                       2 * NUM_EPI_WARPS * p, prm.m_group};
     }
     return launch_tc_pair(c, kModeRowPartial, tch.bn, mA, mB, mB, mC, prm);
   }

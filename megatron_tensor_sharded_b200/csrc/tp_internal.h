@@ -53,6 +53,7 @@ tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, co
 struct RegionFold {
   int* cnt;   // null: the row layer publishes nothing, fold after it
   int rows, cols, m_regions, n_regions, target;
+  int m_group;   // regions complete group by group of this many m (0: one group)
 };
 // Row layer; with `region_cnt` (zeroed, region_counter_bytes()) it also
 // publishes per-tile completion when it runs on CTA pairs and says so in *rf.

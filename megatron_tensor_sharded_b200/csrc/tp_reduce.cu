@@ -88,9 +88,24 @@ struct RegionArgs {
   float4* Z;
   const int* cnt;
   int64_t T, d4, n4;   // rows, float4 per row, float4 per shard
-  int32_t rows, cols4, m_regions, n_regions, target;
+  int32_t rows, cols4, m_regions, n_regions, target, m_group;
   WaitCtl wait;
 };
+
+// The r-th region in the order the row layer completes them: group by
+// group of m_group m-regions, within a group n slowest, m fastest.  Returns
+// the region's counter index n * m_regions + m.
+__device__ __forceinline__ int32_t region_in_order(const RegionArgs& a, int32_t r, int32_t& m,
+                                                   int32_t& n) {
+  const int32_t mg_full = a.m_group > 0 ? a.m_group : a.m_regions;
+  const int32_t g = r / (mg_full * a.n_regions);
+  const int32_t m0 = g * mg_full;
+  const int32_t mg = a.m_regions - m0 < mg_full ? a.m_regions - m0 : mg_full;
+  const int32_t q = r - g * mg_full * a.n_regions;
+  n = q / mg;
+  m = m0 + q - n * mg;
+  return n * a.m_regions + m;
+}
 
 __device__ __forceinline__ bool wait_region(const int* cnt, int target, const WaitCtl& w) {
   if (ld_acquire_gpu(cnt) >= target) return true;
@@ -121,10 +136,11 @@ __global__ void __launch_bounds__(kFoldThreads, 2) fold_regions_kernel(const Reg
   const int32_t sub = a.rows / kUnitsPerRegion;
   for (int32_t u = blockIdx.x; u < units; u += gridDim.x) {
     const int32_t r = u / kUnitsPerRegion, q = u - r * kUnitsPerRegion;
-    if (threadIdx.x == 0) s_ok = wait_region(a.cnt + r, a.target, a.wait) ? 1 : 0;
+    int32_t m, n;
+    const int32_t ci = region_in_order(a, r, m, n);
+    if (threadIdx.x == 0) s_ok = wait_region(a.cnt + ci, a.target, a.wait) ? 1 : 0;
     __syncthreads();
     if (!s_ok) return;   // block-uniform
-    const int32_t n = r / a.m_regions, m = r - n * a.m_regions;
     const int64_t r0 = static_cast<int64_t>(m) * a.rows + static_cast<int64_t>(q) * sub;
     const int64_t nrows = a.T - r0 < sub ? a.T - r0 : sub;   // may be <= 0 at the ragged end
     const int64_t c0 = static_cast<int64_t>(n) * a.cols4;
@@ -171,6 +187,7 @@ cudaError_t launch_fold_regions(const LaunchCtx& c, const float* P, const float*
   a.m_regions = rf.m_regions;
   a.n_regions = rf.n_regions;
   a.target = rf.target;
+  a.m_group = rf.m_group;
   a.wait.err = c.err_word;
   a.wait.timeout_ns = c.timeout_ns;
   // One CTA per SM at most: beside a row-layer CTA only one more CTA fits
