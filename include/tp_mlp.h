@@ -421,6 +421,11 @@ typedef struct tp_block_params {
  *   H   = X + tp_attn_block(LayerNorm(X; ln1))        (reduction #1 + residual)
  *   out = H + tp_mlp_block(LayerNorm(H; ln2))          (reduction #2 + residual)
  *
+ * Each reduction adds, per element, the p partials in shard order, then the
+ * bias, then the residual.  Reduction #2 runs beside the MLP's row layer
+ * where that runs on CTA-pair tiles (b2 NULL or 16-byte aligned), as in
+ * tp_mlp_block; same bits.
+ *
  * X, out [T][d] fp32 (out may equal X); every GEMM reads bf16 and
  * accumulates fp32; head_dim 128; d % 8 == 0 and d <= 16384.  workspace:
  * tp_transformer_block_workspace_size(...) bytes, 256-byte aligned.

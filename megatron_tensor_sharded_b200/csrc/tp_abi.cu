@@ -257,9 +257,11 @@ tp_status reduce_impl(const float* partials, const float* b2, float* Z, int64_t 
 // enqueued here, before the caller's first launch, so that nothing sits
 // between the row layer and the layer before it.
 tp_status prepare_regions(void* at, int64_t T, int64_t k, int64_t d, int p, const float* b2,
-                          void* stream, int** out) {
+                          void* stream, int** out, const float* R = nullptr) {
   *out = nullptr;
-  if (!region_fold_allowed() || (b2 != nullptr && !aligned16(b2))) return TP_OK;
+  if (!region_fold_allowed() || (b2 != nullptr && !aligned16(b2)) ||
+      (R != nullptr && !aligned16(R)))
+    return TP_OK;
   LaunchCtx c{};
   TP_TRY(make_ctx(stream, false, &c));
   if (!row_on_pairs(c, T, k, d, p)) return TP_OK;
@@ -270,22 +272,32 @@ tp_status prepare_regions(void* at, int64_t T, int64_t k, int64_t d, int p, cons
   return TP_OK;
 }
 
-// bf16 row layer to partials, then the fixed-order fold of the partials:
-// beside the row layer when `regions` came from prepare_regions, after it
-// otherwise.  Same bits either way.
+tp_status fold_residual_impl(const float* partials, const float* bias, const float* R, float* H,
+                             int64_t T, int64_t d, int p, const float* gamma, const float* beta,
+                             void* Y, float eps, void* stream);
+
+// bf16 row layer to partials, then the fixed-order fold of the partials
+// (+ b2, + the residual R if given): beside the row layer when `regions`
+// came from prepare_regions, after it otherwise.  Same bits either way.
 tp_status row_and_fold(const void* Y, const void* W2, float* P, const float* b2, float* Z,
-                       int64_t T, int64_t k, int64_t d, int p, int* regions, void* stream) {
+                       int64_t T, int64_t k, int64_t d, int p, int* regions, void* stream,
+                       const float* R = nullptr) {
+  auto fold_after = [&]() {
+    return R == nullptr ? reduce_impl(P, b2, Z, T, d, p, stream)
+                        : fold_residual_impl(P, b2, R, Z, T, d, p, nullptr, nullptr, nullptr, 1e-5f,
+                                             stream);
+  };
   if (regions == nullptr) {
     TP_TRY(row_impl(Y, W2, P, T, k, d, p, TP_BF16, stream));
-    return reduce_impl(P, b2, Z, T, d, p, stream);
+    return fold_after();
   }
   LaunchCtx c{};
   TP_TRY(make_ctx(stream, true, &c));
   RegionFold rf{};
   TP_TRY(launch_tc_row(c, Y, W2, P, T, k, d, p, regions, &rf));
   if (rf.cnt != nullptr)
-    return cuda_status(launch_fold_regions(c, P, b2, Z, T, d, p, rf), "fold launch");
-  return reduce_impl(P, b2, Z, T, d, p, stream);
+    return cuda_status(launch_fold_regions(c, P, b2, Z, T, d, p, rf, R), "fold launch");
+  return fold_after();
 }
 
 tp_status check_heads(int p, int n_heads, int n_kv_heads, int head_dim) {
@@ -407,7 +419,7 @@ BwdLayout bwd_layout(int64_t T, int64_t d, int64_t k, int p, bool swiglu) {
 }
 
 struct BlockLayout {
-  size_t a, h, q, k, v, o, y, p, total;
+  size_t a, h, q, k, v, o, y, p, cnt, total;
 };
 
 BlockLayout block_layout(int64_t T, int64_t d, int n_heads, int n_kv_heads, int head_dim,
@@ -428,6 +440,7 @@ BlockLayout block_layout(int64_t T, int64_t d, int n_heads, int n_kv_heads, int 
   L.o = take(t * n_heads * head_dim * 2);
   L.y = take(t * k * 2);
   L.p = take(static_cast<size_t>(p) * t * d * 4);
+  L.cnt = take(region_counter_bytes(T, d));
   L.total = off;
   return L;
 }
@@ -672,6 +685,10 @@ tp_status tp_transformer_block(const float* X, const tp_block_params* prm, float
   const int64_t kq = static_cast<int64_t>(n_heads) * head_dim;
   const int64_t kkv = static_cast<int64_t>(n_kv_heads) * head_dim;
   const int ident = TP_ACT_IDENTITY;
+  // The MLP's fold (+ b2 + the residual H) runs beside its row layer where
+  // that applies; its counters are reset before the first launch.
+  int* regions = nullptr;
+  TP_TRY(prepare_regions(ws + L.cnt, T, k, d, p, prm->b2, stream, &regions, H));
   // LayerNorm -> attention (column Q, K, V by heads; local attention; row Wo)
   TP_TRY(layer_norm_impl(X, prm->ln1_gamma, prm->ln1_beta, A, T, d, eps, stream));
   TP_TRY(column_impl(A, prm->Wq, nullptr, nullptr, Q, T, d, kq, p, TP_BF16, ident, stream));
@@ -684,9 +701,8 @@ tp_status tp_transformer_block(const float* X, const tp_block_params* prm, float
                             stream));
   // MLP: column W1 (+ activation), row W2
   TP_TRY(column_impl(A, prm->W1, prm->W_up, prm->b1, Yh, T, d, k, p, TP_BF16, act, stream));
-  TP_TRY(row_impl(Yh, prm->W2, P, T, k, d, p, TP_BF16, stream));
-  // reduction #2 with the residual: out = H + fold + b2
-  return fold_residual_impl(P, prm->b2, H, out, T, d, p, nullptr, nullptr, nullptr, eps, stream);
+  // row W2, then reduction #2 with the residual: out = fold + b2 + H
+  return row_and_fold(Yh, prm->W2, P, prm->b2, out, T, k, d, p, regions, stream, H);
 }
 
 size_t tp_mlp_block_backward_workspace_size(int64_t T, int64_t d, int64_t k, int p, int act) {

@@ -105,10 +105,12 @@ tp_status launch_tc_row_fold(const LaunchCtx& c, const void* Y, const void* W2, 
                              float* Z, int64_t T, int64_t k, int64_t d, int p);
 
 // ---- fixed-order fold overlapped with the row layer (tp_reduce.cu): the
-// same additions as launch_reduce, region by region as the counters of `rf`
-// complete; launched right behind the row layer.
+// same additions as launch_reduce (then + R, as the row-wise fold with
+// residual adds it), region by region as the counters of `rf` complete;
+// launched right behind the row layer.
 cudaError_t launch_fold_regions(const LaunchCtx& c, const float* P, const float* b2, float* Z,
-                                int64_t T, int64_t d, int p, const RegionFold& rf);
+                                int64_t T, int64_t d, int p, const RegionFold& rf,
+                                const float* R = nullptr);
 
 // ---- row-wise fold (+ bias, + residual) and LayerNorm (tp_rowops.cu)
 cudaError_t launch_row_fold_ln(const LaunchCtx& c, const float* P, int p, const float* bias,

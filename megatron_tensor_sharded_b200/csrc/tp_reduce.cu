@@ -78,13 +78,15 @@ __global__ void __launch_bounds__(256) reduce_scalar_kernel(const float* __restr
 // become resident beside the row layer's as soon as those have started),
 // each CTA takes regions in the order the row layer finishes their tiles,
 // waits (bounded) until the region's counter shows every shard's tile in
-// memory, and folds it.  It has no griddepcontrol.wait: the counters, a
-// release per producer and an acquire here, order it after the stores it
-// reads, and the row layer itself ran after everything before it.  Vector
-// path only (d % 4 == 0, 16-byte aligned P, Z and b2).
+// memory, and folds it (then b2, then the residual R if given: the order of
+// the row-wise fold with residual).  It has no griddepcontrol.wait: the
+// counters, a release per producer and an acquire here, order it after the
+// stores it reads, and the row layer itself ran after everything before it
+// (R included).  Vector path only (d % 4 == 0, 16-byte aligned P, Z, b2, R).
 struct RegionArgs {
   const float4* part;
   const float* b2;
+  const float4* R;     // residual added last, or null
   float4* Z;
   const int* cnt;
   int64_t T, d4, n4;   // rows, float4 per row, float4 per shard
@@ -163,6 +165,7 @@ __global__ void __launch_bounds__(kFoldThreads, 2) fold_regions_kernel(const Reg
         for (int s = 1; s < p_runtime; ++s) acc = add4(acc, ld_stream(a.part + s * a.n4 + i));
       }
       if (a.b2 != nullptr) acc = add4(acc, __ldg(reinterpret_cast<const float4*>(a.b2) + col));
+      if (a.R != nullptr) acc = add4(acc, ld_stream(a.R + i));
       __stcs(a.Z + i, acc);
     }
     __syncthreads();   // s_ok is rewritten for the next unit
@@ -172,11 +175,12 @@ __global__ void __launch_bounds__(kFoldThreads, 2) fold_regions_kernel(const Reg
 }  // namespace
 
 cudaError_t launch_fold_regions(const LaunchCtx& c, const float* P, const float* b2, float* Z,
-                                int64_t T, int64_t d, int p, const RegionFold& rf) {
+                                int64_t T, int64_t d, int p, const RegionFold& rf, const float* R) {
   if (T == 0) return cudaSuccess;
   RegionArgs a{};
   a.part = reinterpret_cast<const float4*>(P);
   a.b2 = b2;
+  a.R = reinterpret_cast<const float4*>(R);
   a.Z = reinterpret_cast<float4*>(Z);
   a.cnt = rf.cnt;
   a.T = T;

@@ -154,3 +154,44 @@ def test_transformer_block_full_size_prefix(name, n):
     ref = O.transformer_block_sharded(inp.X[:n], inp.value_dict(), w.p, w.n_heads, w.n_kv_heads,
                                       w.head_dim, w.act, True, hidden_round="bf16")["out"]
     assert O.rel_err(got[:n] - inp.X[:n], ref - inp.X[:n]) <= 1e-2
+
+
+@pytest.mark.parametrize("act", ["gelu_tanh", "swiglu"])
+def test_transformer_block_is_bit_identical_to_separate_calls(act):
+    """A shape whose MLP row layer runs on CTA-pair tiles (T=1000, d=2048,
+    k=2048 on p=4), so reduction #2 runs beside that layer: the block gives
+    the bits of its steps called one by one (LayerNorm, the three
+    projections, attention, W_O, fold + bo + X, LayerNorm, the MLP layers,
+    fold + b2 + H), call after call on one workspace."""
+    T, d, h, hkv, k, p = 1000, 2048, 16, 4, 2048, 4
+    inp = W.make_block_inputs(T, d, h, hkv, 128, k, act, seed=11, w_std=0.03)
+    blk = DeviceTransformerBlock(inp, T, d, h, hkv, 128, k, p, act)
+    t, X = blk.t, blk.X
+    kq, kkv, s = h * 128, hkv * 128, k // p
+    bf = torch.bfloat16
+    A = torch.empty((T, d), dtype=bf, device="cuda")
+    Q = torch.empty((p, T, kq // p), dtype=bf, device="cuda")
+    K = torch.empty((p, T, kkv // p), dtype=bf, device="cuda")
+    V = torch.empty_like(K)
+    Oh = torch.empty_like(Q)
+    P = torch.empty((p, T, d), dtype=torch.float32, device="cuda")
+    H = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    Yh = torch.empty((p, T, s), dtype=bf, device="cuda")
+    out = torch.empty((T, d), dtype=torch.float32, device="cuda")
+    ident, a = tp.TP_ACT_IDENTITY, tp.ACT[act]
+    tp.tp_layer_norm(X, t["ln1_gamma"], t["ln1_beta"], A, T, d)
+    tp.tp_column_linear(A, t["Wq"], None, None, Q, T, d, kq, p, tp.TP_BF16, ident)
+    tp.tp_column_linear(A, t["Wk"], None, None, K, T, d, kkv, p, tp.TP_BF16, ident)
+    tp.tp_column_linear(A, t["Wv"], None, None, V, T, d, kkv, p, tp.TP_BF16, ident)
+    tp.tp_attention_heads(Q, K, V, Oh, T, p, h, hkv, 128, 1)
+    tp.tp_row_linear(Oh, t["Wo"], P, T, kq, d, p, tp.TP_BF16)
+    tp.tp_reduce_partials_residual(P, t["bo"], X, H, T, d, p)
+    tp.tp_layer_norm(H, t["ln2_gamma"], t["ln2_beta"], A, T, d)
+    tp.tp_column_linear(A, t["W1"], t.get("W_up"), t["b1"], Yh, T, d, k, p, tp.TP_BF16, a)
+    tp.tp_row_linear(Yh, t["W2"], P, T, k, d, p, tp.TP_BF16)
+    tp.tp_reduce_partials_residual(P, t["b2"], H, out, T, d, p)
+    tp.tp_sync_status()
+    want = bits(host_f32(out))
+    for _ in range(2):
+        got = blk.run(True)
+        assert np.array_equal(bits(got), want)
