@@ -251,20 +251,28 @@ tp_status reduce_impl(const float* partials, const float* b2, float* Z, int64_t 
   return cuda_status(launch_reduce(c, partials, b2, Z, T, d, p), "reduce launch");
 }
 
-// Zeroed counters at `at` for the fold beside the row layer, when that path
-// applies: bf16 row layer on CTA-pair tiles, b2 NULL or 16-byte aligned
-// (the fold reads it as vectors).  *out is NULL otherwise.  The reset is
+// Zeroed counters at `at` for the fold beside the row layer (or beside the
+// backward's dX partials: `on_pairs`), when that path applies: the layer on
+// CTA-pair tiles, b2 and R NULL or 16-byte aligned (the fold reads them as
+// vectors).  *out is NULL otherwise.  The reset is
 // enqueued here, before the caller's first launch, so that nothing sits
 // between the row layer and the layer before it.
+using PairTest = bool (*)(const LaunchCtx&, int64_t T, int64_t k, int64_t d, int p);
+
 tp_status prepare_regions(void* at, int64_t T, int64_t k, int64_t d, int p, const float* b2,
-                          void* stream, int** out, const float* R = nullptr) {
+                          void* stream, int** out, const float* R = nullptr,
+                          PairTest on_pairs = row_on_pairs) {
   *out = nullptr;
   if (!region_fold_allowed() || (b2 != nullptr && !aligned16(b2)) ||
       (R != nullptr && !aligned16(R)))
     return TP_OK;
+  // No debug drop is taken here (the next tensor-core launch keeps it), and
+  // on a device without the tensor-core path nothing is enqueued: the
+  // caller's first launch then fails before any work is on the stream.
   LaunchCtx c{};
-  TP_TRY(make_ctx(stream, false, &c));
-  if (!row_on_pairs(c, T, k, d, p)) return TP_OK;
+  int cc = 0;
+  TP_TRY(device_state(&c.device, &c.num_sms, &cc, &c.err_word, &c.epoch));
+  if (cc != 10 || !on_pairs(c, T, k, d, p)) return TP_OK;
   const cudaError_t e = cudaMemsetAsync(at, 0, region_counter_bytes(T, d),
                                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(TP_ERR_CUDA, "counter reset: %s", cudaGetErrorString(e));
@@ -394,7 +402,7 @@ size_t attn_workspace_bytes(int64_t T, int64_t d, int n_heads, int n_kv_heads, i
 }
 
 struct BwdLayout {
-  size_t dh, du, part, scratch, total;
+  size_t dh, du, part, scratch, cnt, total;
 };
 
 BwdLayout bwd_layout(int64_t T, int64_t d, int64_t k, int p, bool swiglu) {
@@ -414,6 +422,7 @@ BwdLayout bwd_layout(int64_t T, int64_t d, int64_t k, int p, bool swiglu) {
   const size_t sc = chunks * (static_cast<size_t>(p) * s > static_cast<size_t>(d)
                                   ? static_cast<size_t>(p) * s : static_cast<size_t>(d));
   L.scratch = take(sc * 4);
+  L.cnt = take(region_counter_bytes(T, d));
   L.total = off;
   return L;
 }
@@ -745,6 +754,12 @@ tp_status tp_mlp_block_backward(const void* X, const void* W1, const void* W_up,
   float* part = reinterpret_cast<float*>(ws + L.part);
   float* scratch = reinterpret_cast<float*>(ws + L.scratch);
   const int64_t s = k / p;
+  // The dX fold runs beside the dX partials' GEMM where that runs on
+  // CTA-pair tiles; its counters are reset before the first launch.
+  int* regions = nullptr;
+  if (dX != nullptr)
+    TP_TRY(prepare_regions(ws + L.cnt, T, swiglu ? 2 * k : k, d, p, nullptr, stream, &regions,
+                           nullptr, bwd_dx_on_pairs));
   LaunchCtx c{};
   TP_TRY(make_ctx(stream, true, &c));
   // g backward (identity): every shard uses the whole dZ
@@ -760,8 +775,12 @@ tp_status tp_mlp_block_backward(const void* X, const void* W1, const void* W_up,
     TP_TRY(cuda_status(launch_colsum(c, dZ, db2, scratch, 1, T, d, d), "bias gradient launch"));
   if (dX != nullptr) {
     // f backward (all-reduce): p input-gradient partials, folded in shard order
-    TP_TRY(launch_bwd_dx_partials(c, dH, dU, W1, W_up, part, T, d, k, p));
-    TP_TRY(cuda_status(launch_reduce(c, part, nullptr, dX, T, d, p), "fold launch"));
+    RegionFold rf{};
+    TP_TRY(launch_bwd_dx_partials(c, dH, dU, W1, W_up, part, T, d, k, p, regions, &rf));
+    if (rf.cnt != nullptr)
+      TP_TRY(cuda_status(launch_fold_regions(c, part, nullptr, dX, T, d, p, rf), "fold launch"));
+    else
+      TP_TRY(cuda_status(launch_reduce(c, part, nullptr, dX, T, d, p), "fold launch"));
   }
   return TP_OK;
 }

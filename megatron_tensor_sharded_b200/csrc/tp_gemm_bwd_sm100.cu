@@ -63,6 +63,9 @@ struct GParams {
   int32_t b_koff;               // K-major B: K coordinate offset per shard (W1's column blocks)
   int32_t act;
   int32_t bulk_out;             // fp32 epilogue through shared memory + TMA tensor stores
+  int* region_cnt;              // fp32 partials on CTA pairs (bulk_out): per-tile completion
+                                // counters [n_tiles][m_tiles] for the fold beside it; or null
+  int32_t m_group;              // > 0: tiles walk groups of this many m-tiles, group slowest
   // epilogue
   void* out[2];                 // per half
   int64_t out_shard_stride;     // elements
@@ -78,12 +81,20 @@ struct GTile {
 };
 
 __device__ __forceinline__ GTile decode(const GParams& P, int32_t t) {
-  const int32_t per = P.m_tiles * P.n_tiles;
+  // Within a group of m-tiles (all of them when m_group == 0): batch
+  // slowest, then n, m fastest.  Every group but the last is full.
+  const int32_t mg_full = P.m_group > 0 ? P.m_group : P.m_tiles;
+  const int32_t batches = P.p * P.halves;
+  const int32_t group_tiles = mg_full * P.n_tiles * batches;
+  const int32_t grp = t / group_tiles;
+  const int32_t m0 = grp * mg_full;
+  const int32_t mg = P.m_tiles - m0 < mg_full ? P.m_tiles - m0 : mg_full;
+  int32_t r = t - grp * group_tiles;
   GTile g;
-  g.b = t / per;
-  const int32_t r = t - g.b * per;
-  g.n = r / P.m_tiles;
-  g.m = r - g.n * P.m_tiles;
+  g.b = r / (mg * P.n_tiles);
+  r -= g.b * mg * P.n_tiles;
+  g.n = r / mg;
+  g.m = m0 + r - g.n * mg;
   g.shard = g.b % P.p;
   g.half = g.b / P.p;
   return g;
@@ -605,6 +616,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(b), 0));
+      if constexpr (EPI == kEpiF32) {
+        if (P.region_cnt != nullptr) {
+          // Publish this warp's part of the tile to the fold beside this
+          // layer (as the forward row layer does): bulk stores complete,
+          // ordered for generic-proxy readers, one release increment.
+          if (lane == 0) {
+            bulk_wait_all0();
+            fence_proxy_async_global();
+            red_release_gpu_add(P.region_cnt + g.n * P.m_tiles + g.m, 1);
+          }
+          __syncwarp();
+        }
+      }
     }
     if (lane == 0) bulk_wait_all0();   // staging read out before shared memory is released
   }
@@ -784,9 +808,13 @@ tp_status launch_bwd_act_grad(const LaunchCtx& c, const void* dZ, const void* W2
 }
 
 // G2: dX partials P_i = dH_i W1_i^T (+ dU_i Wup_i^T), fp32 [p][T][d]
+bool bwd_dx_on_pairs(const LaunchCtx& c, int64_t T, int64_t k_eff, int64_t d, int p) {
+  return choose_tile(T, d, p, ceil_div(k_eff / p, BK), c.num_sms).pair;
+}
+
 tp_status launch_bwd_dx_partials(const LaunchCtx& c, const void* dH, const void* dU,
                                  const void* W1, const void* Wup, float* P, int64_t T, int64_t d,
-                                 int64_t k, int p) {
+                                 int64_t k, int p, int* region_cnt, RegionFold* rf) {
   const int64_t s = k / p;
   const bool two = dU != nullptr;
   GParams prm = base_params(T, d, two ? 2 * s : s, p, 1);
@@ -818,6 +846,16 @@ tp_status launch_bwd_dx_partials(const LaunchCtx& c, const void* dH, const void*
   if (!make_map_f32_out(&maps[4], P, d, T, p)) return TP_ERR_CUDA;
   maps[5] = maps[4];
   prm.bulk_out = 1;
+  if (rf != nullptr) *rf = RegionFold{};
+  if (tch.pair && region_cnt != nullptr && rf != nullptr) {
+    // regions = the pair tiles, taken in two halves of the m-tiles as in the
+    // forward row layer; 16 epilogue warps count once per tile and shard
+    const int32_t m_tiles = ceil_div(T, 2 * BM);
+    prm.region_cnt = region_cnt;
+    prm.m_group = m_tiles >= 4 ? ceil_div(m_tiles, 2) : 0;
+    *rf = RegionFold{region_cnt, 2 * BM, tch.bn, m_tiles, ceil_div(d, tch.bn),
+                     2 * NUM_EPI_WARPS * p, prm.m_group};
+  }
   return dispatch<0, 0, kEpiF32>(c, maps, prm, tch);
 }
 

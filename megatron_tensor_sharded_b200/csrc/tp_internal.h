@@ -124,9 +124,14 @@ cudaError_t launch_colsum(const LaunchCtx& c, const void* A, float* out, float* 
 tp_status launch_bwd_act_grad(const LaunchCtx& c, const void* dZ, const void* W2, const void* H,
                               const void* Hup, void* dH, void* dU, int64_t T, int64_t d, int64_t k,
                               int p, int act);
+// dX partials; with `region_cnt` (zeroed, region_counter_bytes()) it also
+// publishes per-tile completion when it runs on CTA pairs and says so in *rf.
 tp_status launch_bwd_dx_partials(const LaunchCtx& c, const void* dH, const void* dU,
                                  const void* W1, const void* Wup, float* P, int64_t T, int64_t d,
-                                 int64_t k, int p);
+                                 int64_t k, int p, int* region_cnt = nullptr,
+                                 RegionFold* rf = nullptr);
+// Whether the dX partials run on CTA-pair tiles (k_eff: k, or 2k for SwiGLU).
+bool bwd_dx_on_pairs(const LaunchCtx& c, int64_t T, int64_t k_eff, int64_t d, int p);
 tp_status launch_bwd_dw1(const LaunchCtx& c, const void* X, const void* dH, const void* dU,
                          float* dW1, float* dWup, int64_t T, int64_t d, int64_t k, int p);
 tp_status launch_bwd_dw2(const LaunchCtx& c, const void* Y, const void* dZ, float* dW2, int64_t T,

@@ -95,9 +95,10 @@ CASES = [
     (200, 384, 768, 3, "identity"),
     (513, 1024, 4096, 8, "swiglu"),
     # large enough for CTA-pair tiles (256-row tiles on two SMs) in all four
-    # GEMMs, one with a ragged last pair tile (2500 = 9 x 256 + 196 rows)
-    (2560, 2048, 4096, 2, "swiglu"),
-    (2500, 2048, 4096, 2, "gelu_tanh"),
+    # GEMMs (so the dX fold runs beside its GEMM), one with a ragged last
+    # pair tile (1800 = 7 x 256 + 8 rows)
+    (2048, 2048, 4096, 4, "swiglu"),
+    (1800, 2048, 4096, 4, "gelu_tanh"),
 ]
 
 
@@ -216,3 +217,33 @@ def test_backward_recompute_matches_explicit(T, d, k, p, act):
     for name, v in out.items():
         got = host_f32(v)
         assert np.array_equal(got.view(np.uint32), want[name].view(np.uint32)), name
+
+
+def _r256(n):
+    return -(-n // 256) * 256
+
+
+@pytest.mark.parametrize("T,d,k,p,act", [(2048, 2048, 4096, 4, "swiglu"),
+                                         (1800, 2048, 4096, 4, "gelu_tanh")])
+def test_dx_fold_beside_its_gemm_is_the_fixed_order_fold(T, d, k, p, act):
+    """On shapes whose dX partials run on CTA-pair tiles the dX fold runs
+    beside that GEMM: dX must have the bits of tp_reduce_partials applied to
+    the partials the call left in its workspace, and the workspace's region
+    counters must read 16 p (the layout: dH, dU for SwiGLU, the partials,
+    the bias-gradient scratch, the counters)."""
+    inp = _inputs(T, d, k, act, seed=5)
+    blk = DeviceBackward(inp, T, d, k, p, act)
+    blk.ws.fill_(0x7F)
+    blk.run()
+    off = _r256(T * k * 2) * (2 if act == "swiglu" else 1)
+    part = blk.ws[off:off + p * T * d * 4].view(torch.float32).view(p, T, d)
+    Z = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")
+    tp.tp_reduce_partials(part, None, Z, T, d, p)
+    tp.tp_sync_status()
+    assert np.array_equal(host_f32(Z).view(np.uint32), host_f32(blk.dX).view(np.uint32))
+    scratch = _r256(-(-T // 128) * max(k, d) * 4)
+    cnt_off = off + _r256(p * T * d * 4) + scratch
+    m_regions = -(-T // 256)
+    cnt = blk.ws[cnt_off:cnt_off + 4 * m_regions * -(-d // 128)].cpu().numpy().view(np.int32)
+    assert cnt[0] == 16 * p
+    assert set(np.unique(cnt).tolist()) <= {0, 16 * p}
