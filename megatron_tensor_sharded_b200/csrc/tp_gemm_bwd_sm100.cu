@@ -733,9 +733,8 @@ tp_status launch_g(const LaunchCtx& c, const CUtensorMap* maps, GParams prm) {
 // forward's cost model (single-CTA widths 64, 128, 256; CTA-pair tiles of
 // 256 rows x 128 or 256 once single-CTA tiles take more than one wave).
 TileChoice choose_tile(int64_t M, int64_t N, int64_t batches, int64_t k_blocks, int num_sms) {
-  TileChoice t = pick_tile(M, N, batches, k_blocks, num_sms, false, pair_allowed());
-  if (!t.pair && t.bn == 192) t.bn = 128;
-  return t;
+  // the backward kernels have no 192-wide single-CTA tile
+  return pick_tile(M, N, batches, k_blocks, num_sms, false, pair_allowed(), false);
 }
 
 // Width of a K-major B operand's TMA box: the tile width, or its half on

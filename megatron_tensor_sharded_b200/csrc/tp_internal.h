@@ -87,7 +87,7 @@ struct TileChoice {
   bool pair;
 };
 TileChoice pick_tile(int64_t T, int64_t n_total, int64_t batches, int64_t k_blocks, int num_sms,
-                     bool swiglu, bool allow_pair);
+                     bool swiglu, bool allow_pair, bool allow_192 = true);
 
 inline int32_t ceil_div(int64_t a, int64_t b) { return static_cast<int32_t>((a + b - 1) / b); }
 

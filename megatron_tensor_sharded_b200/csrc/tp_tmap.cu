@@ -179,7 +179,7 @@ bool make_map_b(CUtensorMap* m, const void* g, int64_t cols, int64_t rows) {
 // 256 rows and are considered only when single-CTA tiles need more than one
 // wave.  Ties keep the earlier (wider, single-CTA) choice.
 TileChoice pick_tile(int64_t T, int64_t n_total, int64_t batches, int64_t k_blocks, int num_sms,
-                     bool swiglu, bool allow_pair) {
+                     bool swiglu, bool allow_pair, bool allow_192) {
   constexpr double kIngest = 80.0, kFixed = 2000.0;
   TileChoice best{256, false};
   double best_cost = 1e300;
@@ -200,7 +200,7 @@ TileChoice pick_tile(int64_t T, int64_t n_total, int64_t batches, int64_t k_bloc
     }
   };
   consider(256, false);
-  if (!swiglu) consider(192, false);
+  if (!swiglu && allow_192) consider(192, false);
   consider(128, false);
   if (!swiglu) consider(64, false);
   // Pair tiles only pay once the layer takes more than one wave of
