@@ -227,8 +227,9 @@ tp_status tp_ipc_release(const tp_ipc_handle* handle);
  *                    next 256-byte boundary, then counters at the end (reset
  *                    on every call that uses them): one int32 per 128-row
  *                    m-tile for TP_FLAG_FUSED_LAUNCH, or one per region of
- *                    the fold beside the row layer (regions in column-major
- *                    order, each counted to 16 p).
+ *                    the fold beside the row layer (256-row regions in
+ *                    column-major order, each counted to 16 p; the area
+ *                    has room for ceil(T/128) * ceil(d/64) of them).
  *   other arguments  as for the three calls above.
  */
 tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const void* b1,

@@ -195,7 +195,8 @@ size_t workspace_bytes(int64_t T, int64_t d, int64_t k, int p, int dtype, int fl
 }
 
 tp_status column_impl(const void* X, const void* W1, const void* W_up, const void* b1, void* Y,
-                      int64_t T, int64_t d, int64_t k, int p, int dtype, int act, void* stream) {
+                      int64_t T, int64_t d, int64_t k, int p, int dtype, int act, void* stream,
+                      int* zero_cnt = nullptr, int zero_n = 0) {
   TP_TRY(check_shape(T, d, k, p, dtype));
   TP_TRY(check_act(act, W_up));
   if (T == 0) return TP_OK;
@@ -206,7 +207,8 @@ tp_status column_impl(const void* X, const void* W1, const void* W_up, const voi
   if (b1 != nullptr) TP_TRY(check_ptr(b1, "b1", dtype, dtype == TP_BF16));
   LaunchCtx c{};
   TP_TRY(make_ctx(stream, dtype == TP_BF16, &c));
-  if (dtype == TP_BF16) return launch_tc_column(c, X, W1, W_up, b1, Y, T, d, k, p, act);
+  if (dtype == TP_BF16)
+    return launch_tc_column(c, X, W1, W_up, b1, Y, T, d, k, p, act, zero_cnt, zero_n);
   return cuda_status(launch_simt_column(c, static_cast<const float*>(X),
                                         static_cast<const float*>(W1),
                                         static_cast<const float*>(W_up),
@@ -251,32 +253,36 @@ tp_status reduce_impl(const float* partials, const float* b2, float* Z, int64_t 
   return cuda_status(launch_reduce(c, partials, b2, Z, T, d, p), "reduce launch");
 }
 
-// Zeroed counters at `at` for the fold beside the row layer (or beside the
-// backward's dX partials: `on_pairs`), when that path applies: the layer on
-// CTA-pair tiles, b2 and R NULL or 16-byte aligned (the fold reads them as
-// vectors).  *out is NULL otherwise.  The reset is
-// enqueued here, before the caller's first launch, so that nothing sits
-// between the row layer and the layer before it.
-using PairTest = bool (*)(const LaunchCtx&, int64_t T, int64_t k, int64_t d, int p);
-
-tp_status prepare_regions(void* at, int64_t T, int64_t k, int64_t d, int p, const float* b2,
-                          void* stream, int** out, const float* R = nullptr,
-                          PairTest on_pairs = row_on_pairs) {
+// Counters at `at` for the fold beside the row layer, when that path
+// applies: the bf16 path on an sm_100 device, b2 and R NULL or 16-byte
+// aligned (the fold reads them as vectors).  *out is NULL otherwise, and
+// *n the number of counters.  Nothing is enqueued here: the column layer
+// launched before the row layer zeroes them (launch_tc_column's zero_cnt),
+// or, where no column layer of this library comes first, regions_reset().
+tp_status region_counters(void* at, int64_t T, int64_t d, const float* b2, const float* R,
+                          int** out, int* n) {
   *out = nullptr;
+  *n = 0;
   if (!region_fold_allowed() || (b2 != nullptr && !aligned16(b2)) ||
       (R != nullptr && !aligned16(R)))
     return TP_OK;
-  // No debug drop is taken here (the next tensor-core launch keeps it), and
-  // on a device without the tensor-core path nothing is enqueued: the
-  // caller's first launch then fails before any work is on the stream.
   LaunchCtx c{};
   int cc = 0;
   TP_TRY(device_state(&c.device, &c.num_sms, &cc, &c.err_word, &c.epoch));
-  if (cc != 10 || !on_pairs(c, T, k, d, p)) return TP_OK;
-  const cudaError_t e = cudaMemsetAsync(at, 0, region_counter_bytes(T, d),
+  if (cc != 10) return TP_OK;
+  *out = static_cast<int*>(at);
+  *n = static_cast<int>(region_counter_bytes(T, d) / sizeof(int));
+  return TP_OK;
+}
+
+// Zeroes the counters with a memset enqueued before the caller's first
+// launch (so that nothing sits between the counting layer and the one
+// before it).
+tp_status regions_reset(int* cnt, int n, void* stream) {
+  if (cnt == nullptr) return TP_OK;
+  const cudaError_t e = cudaMemsetAsync(cnt, 0, static_cast<size_t>(n) * sizeof(int),
                                         static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return fail(TP_ERR_CUDA, "counter reset: %s", cudaGetErrorString(e));
-  *out = static_cast<int*>(at);
   return TP_OK;
 }
 
@@ -286,7 +292,8 @@ tp_status fold_residual_impl(const float* partials, const float* bias, const flo
 
 // bf16 row layer to partials, then the fixed-order fold of the partials
 // (+ b2, + the residual R if given): beside the row layer when `regions`
-// came from prepare_regions, after it otherwise.  Same bits either way.
+// came from region_counters (and were zeroed), after it otherwise.  Same
+// bits either way.
 tp_status row_and_fold(const void* Y, const void* W2, float* P, const float* b2, float* Z,
                        int64_t T, int64_t k, int64_t d, int p, int* regions, void* stream,
                        const float* R = nullptr) {
@@ -557,11 +564,13 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
     return reduce_impl(P, b2, Z, T, d, p, stream);
   }
   // Default bf16 mode: the fold runs beside the row layer where that
-  // applies (prepare_regions).
+  // applies (region_counters); the column layer zeroes the counters.
   int* regions = nullptr;
+  int n_regions = 0;
   if (!splitk && !row_fold && dtype == TP_BF16)
-    TP_TRY(prepare_regions(ws + need - counter_bytes(T, d), T, k, d, p, b2, stream, &regions));
-  TP_TRY(column_impl(X, W1, W_up, b1, Y, T, d, k, p, dtype, act, stream));
+    TP_TRY(region_counters(ws + need - counter_bytes(T, d), T, d, b2, nullptr, &regions,
+                           &n_regions));
+  TP_TRY(column_impl(X, W1, W_up, b1, Y, T, d, k, p, dtype, act, stream, regions, n_regions));
   if (regions != nullptr) return row_and_fold(Y, W2, P, b2, Z, T, k, d, p, regions, stream);
   if (row_fold) {
     LaunchCtx c{};
@@ -626,9 +635,11 @@ tp_status tp_attn_block(const void* X, const void* Wq, const void* Wk, const voi
   void* O = ws + qb + 2 * kvb;
   float* P = reinterpret_cast<float*>(ws + 2 * qb + 2 * kvb);
   int* regions = nullptr;
-  TP_TRY(prepare_regions(ws + need - region_counter_bytes(T, d), T, kq, d, p, bo, stream,
-                         &regions));
-  TP_TRY(column_impl(X, Wq, nullptr, nullptr, Q, T, d, kq, p, TP_BF16, TP_ACT_IDENTITY, stream));
+  int n_regions = 0;
+  TP_TRY(region_counters(ws + need - region_counter_bytes(T, d), T, d, bo, nullptr, &regions,
+                         &n_regions));
+  TP_TRY(column_impl(X, Wq, nullptr, nullptr, Q, T, d, kq, p, TP_BF16, TP_ACT_IDENTITY, stream,
+                     regions, n_regions));
   TP_TRY(column_impl(X, Wk, nullptr, nullptr, K, T, d, kkv, p, TP_BF16, TP_ACT_IDENTITY, stream));
   TP_TRY(column_impl(X, Wv, nullptr, nullptr, V, T, d, kkv, p, TP_BF16, TP_ACT_IDENTITY, stream));
   TP_TRY(attention_impl(Q, K, V, O, T, p, n_heads, n_kv_heads, head_dim, causal, stream));
@@ -697,7 +708,8 @@ tp_status tp_transformer_block(const float* X, const tp_block_params* prm, float
   // The MLP's fold (+ b2 + the residual H) runs beside its row layer where
   // that applies; its counters are reset before the first launch.
   int* regions = nullptr;
-  TP_TRY(prepare_regions(ws + L.cnt, T, k, d, p, prm->b2, stream, &regions, H));
+  int n_regions = 0;
+  TP_TRY(region_counters(ws + L.cnt, T, d, prm->b2, H, &regions, &n_regions));
   // LayerNorm -> attention (column Q, K, V by heads; local attention; row Wo)
   TP_TRY(layer_norm_impl(X, prm->ln1_gamma, prm->ln1_beta, A, T, d, eps, stream));
   TP_TRY(column_impl(A, prm->Wq, nullptr, nullptr, Q, T, d, kq, p, TP_BF16, ident, stream));
@@ -709,7 +721,8 @@ tp_status tp_transformer_block(const float* X, const tp_block_params* prm, float
   TP_TRY(fold_residual_impl(P, prm->bo, X, H, T, d, p, prm->ln2_gamma, prm->ln2_beta, A, eps,
                             stream));
   // MLP: column W1 (+ activation), row W2
-  TP_TRY(column_impl(A, prm->W1, prm->W_up, prm->b1, Yh, T, d, k, p, TP_BF16, act, stream));
+  TP_TRY(column_impl(A, prm->W1, prm->W_up, prm->b1, Yh, T, d, k, p, TP_BF16, act, stream,
+                     regions, n_regions));
   // row W2, then reduction #2 with the residual: out = fold + b2 + H
   return row_and_fold(Yh, prm->W2, P, prm->b2, out, T, k, d, p, regions, stream, H);
 }
@@ -757,9 +770,18 @@ tp_status tp_mlp_block_backward(const void* X, const void* W1, const void* W_up,
   // The dX fold runs beside the dX partials' GEMM where that runs on
   // CTA-pair tiles; its counters are reset before the first launch.
   int* regions = nullptr;
-  if (dX != nullptr)
-    TP_TRY(prepare_regions(ws + L.cnt, T, swiglu ? 2 * k : k, d, p, nullptr, stream, &regions,
-                           nullptr, bwd_dx_on_pairs));
+  int n_regions = 0;
+  if (dX != nullptr) {
+    TP_TRY(region_counters(ws + L.cnt, T, d, nullptr, nullptr, &regions, &n_regions));
+    if (regions != nullptr) {
+      LaunchCtx q{};
+      TP_TRY(make_ctx(stream, false, &q));
+      if (bwd_dx_on_pairs(q, T, swiglu ? 2 * k : k, d, p))
+        TP_TRY(regions_reset(regions, n_regions, stream));
+      else
+        regions = nullptr;
+    }
+  }
   LaunchCtx c{};
   TP_TRY(make_ctx(stream, true, &c));
   // g backward (identity): every shard uses the whole dZ

@@ -158,6 +158,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *reinterpret_cast<volatile uint32_t*>(tmem_slot);
   pdl_wait();
+  zero_counters(P, warp, lane);
   pdl_launch_dependents();
 
   if (warp == 0) {

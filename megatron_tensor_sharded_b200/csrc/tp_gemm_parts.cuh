@@ -63,8 +63,10 @@ struct TcParams {
   const void* bias;      // b1 (bf16, column) or b2 (fp32, split-K row); may be null
   void* out;             // Y bf16 [p][T][s] | P fp32 [p][T][d] | Z fp32 [T][d]
   int32_t bulk_out;      // column layers: 1 = bulk tensor stores through shared memory
-  int* region_cnt;       // row partials on CTA pairs: per-tile completion counters read by
-                         // the overlapped fold ([n_tiles][m_tiles]); may be null
+  int* region_cnt;       // row partials: per-tile completion counters read by the fold
+                         // beside the layer ([n_tiles][m_tiles]); may be null
+  int* zero_cnt;         // column layers: counters this launch zeroes (after its wait for
+  int32_t zero_n;        // the previous kernel) for the row layer that follows; may be null
   int32_t m_group;       // > 0: tiles walk groups of this many m-tiles, group slowest (all
                          // shards of one group before the next); 0: one group
   WaitCtl wait;
@@ -74,6 +76,14 @@ struct TcParams {
 struct TileCoord {
   int32_t batch, m, n;
 };
+
+// Zeroes the counters the next row layer will count into: one warp of CTA 0,
+// after griddepcontrol.wait (so no kernel before this one still reads them);
+// the row layer waits for this grid to complete before it counts.
+__device__ __forceinline__ void zero_counters(const TcParams& P, int warp, int lane) {
+  if (P.zero_cnt != nullptr && blockIdx.x == 0 && warp == 3)
+    for (int32_t i = lane; i < P.zero_n; i += 32) P.zero_cnt[i] = 0;
+}
 
 __device__ __forceinline__ TileCoord decode_tile(const TcParams& P, int32_t t) {
   // Within a group of m-tiles: shard slowest, then n, m fastest (neighbouring

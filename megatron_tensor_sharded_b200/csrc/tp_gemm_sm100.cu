@@ -118,6 +118,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   // Everything above overlaps the previous kernel; from here on global
   // memory is read and written.
   pdl_wait();
+  zero_counters(P, warp, lane);
   pdl_launch_dependents();
 
   if (warp == 0) {
@@ -300,7 +301,7 @@ tp_status launch_bn(const LaunchCtx& c, int bn, const CUtensorMap& a, const CUte
 
 tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, const void* Wup,
                            const void* b1, void* Y, int64_t T, int64_t d, int64_t k, int p,
-                           int act) {
+                           int act, int* zero_cnt, int zero_n) {
   CUtensorMap mA, mB0, mB1, mY;
   if (!make_map_a(&mA, X, d, T, 1) || !make_map_b(&mB0, W1, k, d)) return TP_ERR_CUDA;
   const bool bulk = (k / p) % 32 == 0;
@@ -325,6 +326,8 @@ tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, co
   prm.bias = b1;
   prm.out = Y;
   prm.bulk_out = bulk ? 1 : 0;
+  prm.zero_cnt = zero_cnt;
+  prm.zero_n = zero_n;
   const TileChoice tch = pick_tile(T, k, 1, prm.k_blocks, c.num_sms, swiglu, pair_allowed());
   const int mode = swiglu ? kModeColumnSwiglu : kModeColumn;
   if (tch.pair) return launch_tc_pair(c, mode, tch.bn, mA, mB0, mB1, mY, prm);
@@ -332,13 +335,11 @@ tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, co
   return launch_bn<kModeColumn>(c, tch.bn, mA, mB0, mB1, mY, prm);
 }
 
+// One int per region at most: regions are row tiles of 128 or 256 rows and
+// 64 to 256 columns.
 size_t region_counter_bytes(int64_t T, int64_t d) {
-  const size_t n = static_cast<size_t>(ceil_div(T, 2 * BM)) * static_cast<size_t>(ceil_div(d, 128));
+  const size_t n = static_cast<size_t>(ceil_div(T, BM)) * static_cast<size_t>(ceil_div(d, 64));
   return (n * sizeof(int) + 255) & ~size_t(255);
-}
-
-bool row_on_pairs(const LaunchCtx& c, int64_t T, int64_t k, int64_t d, int p) {
-  return pick_tile(T, d, p, ceil_div(k / p, BK), c.num_sms, false, pair_allowed()).pair;
 }
 
 tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float* P, int64_t T,
@@ -378,6 +379,9 @@ tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float
     }
     return launch_tc_pair(c, kModeRowPartial, tch.bn, mA, mB, mB, mC, prm);
   }
+  // Single-CTA row tiles (one wave on GPT-2, weight streaming on decode)
+  // publish nothing: the fold beside them measured slower than the fold
+  // after them.
   return launch_bn<kModeRowPartial>(c, tch.bn, mA, mB, mB, mC, prm);
 }
 

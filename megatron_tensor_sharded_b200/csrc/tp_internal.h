@@ -43,9 +43,11 @@ cudaError_t launch_simt_row_splitk(const LaunchCtx& c, const float* Y, const flo
                                    int p);
 
 // ---- bf16 tensor-core path, tcgen05 + TMEM + TMA (tp_gemm_sm100.cu)
+// Column layer; with `zero_cnt` it also zeroes zero_n counters for the row
+// layer that follows (region_counter_bytes()).
 tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, const void* Wup,
                            const void* b1, void* Y, int64_t T, int64_t d, int64_t k, int p,
-                           int act);
+                           int act, int* zero_cnt = nullptr, int zero_n = 0);
 // Regions of the partials whose p shard tiles the row layer counts as done
 // (row layers on CTA-pair tiles only): region (m, n) covers rows
 // [m*rows, +rows) and columns [n*cols, +cols); counter n*m_regions + m
@@ -56,13 +58,12 @@ struct RegionFold {
   int m_group;   // regions complete group by group of this many m (0: one group)
 };
 // Row layer; with `region_cnt` (zeroed, region_counter_bytes()) it also
-// publishes per-tile completion when it runs on CTA pairs and says so in *rf.
+// publishes per-tile completion when it runs on CTA-pair tiles and
+// describes the regions in *rf (rf->cnt stays null otherwise).
 tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float* P, int64_t T,
                         int64_t k, int64_t d, int p, int* region_cnt = nullptr,
                         RegionFold* rf = nullptr);
 size_t region_counter_bytes(int64_t T, int64_t d);
-// Whether launch_tc_row picks CTA-pair tiles for this layer.
-bool row_on_pairs(const LaunchCtx& c, int64_t T, int64_t k, int64_t d, int p);
 tp_status launch_tc_row_splitk(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
                                float* Z, int64_t T, int64_t k, int64_t d, int p);
 

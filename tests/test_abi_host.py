@@ -95,13 +95,13 @@ def test_row_and_reduce_validation():
 def test_workspace_size_formula():
     # bf16: hidden shards T*k*2 bytes, then p*T*d*4 bytes of partials, each
     # rounded up to 256 bytes, then the counters: one int per 128-row m-tile
-    # (single-launch block) or per 256-row x 128-column region (fold beside
-    # the row layer), whichever is larger
+    # (single-launch block) or per 128-row x 64-column region at most (fold
+    # beside the row layer), whichever is larger
     def r256(n):
         return -(-n // 256) * 256
 
     def counters(T, d):
-        return max(r256(4 * (-(-T // 128))), r256(4 * (-(-T // 256)) * (-(-d // 128))))
+        return max(r256(4 * (-(-T // 128))), r256(4 * (-(-T // 128)) * (-(-d // 64))))
 
     T, d, k, p = 1000, 768, 3072, 2
     ys = r256(T * k * 2)
@@ -113,10 +113,10 @@ def test_workspace_size_formula():
     assert tp.tp_mlp_block_workspace_size(4, 512, 2048, 4, tp.TP_F32, tp.TP_ACT_GELU_TANH) == \
         r256(4 * 2048 * 4) + r256(4 * 4 * 512 * 4) + counters(4, 512)
     assert tp.tp_mlp_block_workspace_size(4, 512, 2047, 4, tp.TP_F32, tp.TP_ACT_GELU_TANH) == 0
-    # Llama-shaped prefill: 16 x 64 regions outgrow the 32 m-tile counters
+    # Llama-shaped prefill: room for 32 x 128 regions
     T, d, k, p = 4096, 8192, 28672, 8
     assert tp.tp_mlp_block_workspace_size(T, d, k, p, tp.TP_BF16, tp.TP_ACT_SWIGLU) == \
-        r256(T * k * 2) + r256(p * T * d * 4) + 4096
+        r256(T * k * 2) + r256(p * T * d * 4) + 16384
 
 
 def test_block_validation():

@@ -306,7 +306,7 @@ def test_block_is_bit_identical_to_separate_calls(T, d, s, p, act, bias):
 
 def _counter_bytes(T, d):
     r256 = lambda n: -(-n // 256) * 256  # noqa: E731
-    return max(r256(4 * -(-T // 128)), r256(4 * -(-T // 256) * -(-d // 128)))
+    return max(r256(4 * -(-T // 128)), r256(4 * -(-T // 128) * -(-d // 64)))
 
 
 @pytest.mark.parametrize("T,d,s,p,act,bias", [(1000, 2176, 2048, 4, "gelu_tanh", True),
