@@ -315,6 +315,27 @@ tp_status row_and_fold(const void* Y, const void* W2, float* P, const float* b2,
   return fold_after();
 }
 
+// The attention block's Q, K, V projections (identity column layers of the
+// same input): one launch of CTA-pair tiles where the shapes suit it, else
+// three.  The first launch zeroes `zero_cnt` (the row layer's counters).
+tp_status qkv_impl(const void* X, const void* Wq, const void* Wk, const void* Wv, void* Q,
+                   void* K, void* V, int64_t T, int64_t d, int64_t kq, int64_t kkv, int p,
+                   void* stream, int* zero_cnt, int zero_n) {
+  LaunchCtx c{};
+  TP_TRY(make_ctx(stream, true, &c));
+  const void* W[3] = {Wq, Wk, Wv};
+  void* Y[3] = {Q, K, V};
+  const int64_t k[3] = {kq, kkv, kkv};
+  bool done = false;
+  TP_TRY(launch_tc_column_multi(c, X, W, Y, k, 3, T, d, p, zero_cnt, zero_n, &done));
+  if (done) return TP_OK;
+  const int ident = TP_ACT_IDENTITY;
+  TP_TRY(launch_tc_column(c, X, Wq, nullptr, nullptr, Q, T, d, kq, p, ident, zero_cnt, zero_n));
+  c.debug_drop = -1;   // an armed fault injection applies to the first launch only
+  TP_TRY(launch_tc_column(c, X, Wk, nullptr, nullptr, K, T, d, kkv, p, ident));
+  return launch_tc_column(c, X, Wv, nullptr, nullptr, V, T, d, kkv, p, ident);
+}
+
 tp_status check_heads(int p, int n_heads, int n_kv_heads, int head_dim) {
   if (p < 1) return fail(TP_ERR_INVALID_ARG, "p = %d, must be >= 1", p);
   if (n_heads < 1 || n_kv_heads < 1 || head_dim < 1)
@@ -638,10 +659,7 @@ tp_status tp_attn_block(const void* X, const void* Wq, const void* Wk, const voi
   int n_regions = 0;
   TP_TRY(region_counters(ws + need - region_counter_bytes(T, d), T, d, bo, nullptr, &regions,
                          &n_regions));
-  TP_TRY(column_impl(X, Wq, nullptr, nullptr, Q, T, d, kq, p, TP_BF16, TP_ACT_IDENTITY, stream,
-                     regions, n_regions));
-  TP_TRY(column_impl(X, Wk, nullptr, nullptr, K, T, d, kkv, p, TP_BF16, TP_ACT_IDENTITY, stream));
-  TP_TRY(column_impl(X, Wv, nullptr, nullptr, V, T, d, kkv, p, TP_BF16, TP_ACT_IDENTITY, stream));
+  TP_TRY(qkv_impl(X, Wq, Wk, Wv, Q, K, V, T, d, kq, kkv, p, stream, regions, n_regions));
   TP_TRY(attention_impl(Q, K, V, O, T, p, n_heads, n_kv_heads, head_dim, causal, stream));
   return row_and_fold(O, Wo, P, bo, Z, T, kq, d, p, regions, stream);
 }
@@ -712,9 +730,7 @@ tp_status tp_transformer_block(const float* X, const tp_block_params* prm, float
   TP_TRY(region_counters(ws + L.cnt, T, d, prm->b2, H, &regions, &n_regions));
   // LayerNorm -> attention (column Q, K, V by heads; local attention; row Wo)
   TP_TRY(layer_norm_impl(X, prm->ln1_gamma, prm->ln1_beta, A, T, d, eps, stream));
-  TP_TRY(column_impl(A, prm->Wq, nullptr, nullptr, Q, T, d, kq, p, TP_BF16, ident, stream));
-  TP_TRY(column_impl(A, prm->Wk, nullptr, nullptr, K, T, d, kkv, p, TP_BF16, ident, stream));
-  TP_TRY(column_impl(A, prm->Wv, nullptr, nullptr, V, T, d, kkv, p, TP_BF16, ident, stream));
+  TP_TRY(qkv_impl(A, prm->Wq, prm->Wk, prm->Wv, Q, K, V, T, d, kq, kkv, p, stream, nullptr, 0));
   TP_TRY(attention_impl(Q, K, V, O, T, p, n_heads, n_kv_heads, head_dim, causal, stream));
   TP_TRY(row_impl(O, prm->Wo, P, T, kq, d, p, TP_BF16, stream));
   // reduction #1 with the residual: H = X + fold + bo; then LayerNorm of H

@@ -96,6 +96,20 @@ __device__ __forceinline__ void issue_slot_pair(const TcParams& P, const CUtenso
 template <int MODE>
 constexpr bool kPairBulkOut = (MODE == kModeRowPartial || MODE == kModeRowSplitK);
 
+// Tile t of the launch and its segment (0 unless several column layers share
+// the launch; within a segment m fastest, as decode_tile walks one layer).
+__device__ __forceinline__ TileCoord decode_pair_tile(const TcParams& P, int32_t t, int& seg) {
+  seg = 0;
+  if (P.nseg <= 1) return decode_tile(P, t);
+  while (seg + 1 < P.nseg && t >= P.seg_start[seg + 1]) ++seg;
+  const int32_t r = t - P.seg_start[seg];
+  TileCoord c;
+  c.batch = 0;
+  c.n = r / P.m_tiles;
+  c.m = r - c.n * P.m_tiles;
+  return c;
+}
+
 template <int MODE, int PBN>
 using PKCfg = PCfg<PBN, EPI_STAGE_BYTES>;
 
@@ -104,7 +118,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     tc_gemm_pair_kernel(const __grid_constant__ CUtensorMap mapA,
                         const __grid_constant__ CUtensorMap mapB0,
                         const __grid_constant__ CUtensorMap mapB1,
-                        const __grid_constant__ CUtensorMap mapC, const TcParams P) {
+                        const __grid_constant__ CUtensorMap mapC, const TcParams P,
+                        const __grid_constant__ CUtensorMap mapB2,
+                        const __grid_constant__ CUtensorMap mapC1,
+                        const __grid_constant__ CUtensorMap mapC2) {
   using C = PKCfg<MODE, PBN>;
   constexpr int PSTAGES = C::STAGES;
   constexpr int PSTAGE_BYTES = C::STAGE_BYTES;
@@ -168,7 +185,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int64_t issued = 0;
       bool ok = true;
       for (int32_t t = cluster; ok && t < P.num_tiles; t += nclusters) {
-        const TileCoord tc = decode_tile(P, t);
+        int seg;
+        const TileCoord tc = decode_pair_tile(P, t, seg);
+        // several column layers in one launch: segment seg's weight
+        const CUtensorMap* mB0 = seg == 0 ? &mapB0 : (seg == 1 ? &mapB1 : &mapB2);
         for (int32_t kb = 0; kb < P.k_blocks; ++kb) {
           if (!wait_bounded(empty_bar(stage), phase ^ 1u, abort_flag, P.wait, kErrWaitEmpty)) {
             ok = false;
@@ -176,7 +196,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           if (issued != P.debug_drop) {
             if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * PSTAGE_BYTES);
-            issue_slot_pair<MODE, PBN>(P, &mapA, &mapB0, &mapB1, tc, kb, rank, slot_a(stage),
+            issue_slot_pair<MODE, PBN>(P, &mapA, mB0, &mapB1, tc, kb, rank, slot_a(stage),
                                   slot_b(stage), mapa_shared(full_bar(stage), 0));
           }
           ++issued;
@@ -246,9 +266,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int32_t lt = 0;
     for (int32_t t = cluster; t < P.num_tiles; t += nclusters, ++lt) {
       const uint32_t b = lt & 1, ap = (lt >> 1) & 1;
-      const TileCoord tc = decode_tile(P, t);
+      int seg;
+      const TileCoord tc = decode_pair_tile(P, t, seg);
+      TcParams SP = P;   // the segment's width and shard width
+      if (P.nseg > 1) {
+        SP.n_total = P.seg_n[seg];
+        SP.s = P.seg_s[seg];
+      }
+      const CUtensorMap* mC = seg == 0 ? &mapC : (seg == 1 ? &mapC1 : &mapC2);
       EpiBias<MODE, PBN> eb;
-      load_epi_bias<MODE, PBN>(P, tc, half, eb);
+      load_epi_bias<MODE, PBN>(SP, tc, half, eb);
       bool ok = wait_bounded(accf_bar(b), ap, abort_flag, P.wait, kErrWaitAccFull);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
@@ -260,10 +287,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         epilogue_tile_bulk<MODE, PBN>(P, tc, tacc, row0, half, stage_w, &mapC, lane);
       } else {
         if (P.bulk_out)
-          epilogue_tile_bulk_col<MODE, PBN>(P, tc, tacc, row0, half, eb, stage_w, &mapC, lane,
+          epilogue_tile_bulk_col<MODE, PBN>(SP, tc, tacc, row0, half, eb, stage_w, mC, lane,
                                             nchunk);
         else
-          epilogue_tile<MODE, PBN>(P, tc, tacc, row0 + lane, half, eb);
+          epilogue_tile<MODE, PBN>(SP, tc, tacc, row0 + lane, half, eb);
       }
       tc_fence_before();
       __syncwarp();
@@ -299,7 +326,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 template <int MODE, int PBN>
 tp_status launch_pair_mode(const LaunchCtx& c, const CUtensorMap& a, const CUtensorMap& b0,
-                           const CUtensorMap& b1, const CUtensorMap& cm, TcParams prm) {
+                           const CUtensorMap& b1, const CUtensorMap& cm, TcParams prm,
+                           const CUtensorMap* b2 = nullptr, const CUtensorMap* c1 = nullptr,
+                           const CUtensorMap* c2 = nullptr) {
   constexpr int PSMEM_BYTES = PKCfg<MODE, PBN>::SMEM_BYTES;
   static uint64_t attr_epoch[64] = {};   // context epoch the attribute was set under
   static std::mutex mu;
@@ -335,7 +364,9 @@ tp_status launch_pair_mode(const LaunchCtx& c, const CUtensorMap& a, const CUten
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = pdl_allowed() ? 2 : 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<MODE, PBN>, a, b0, b1, cm, prm);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<MODE, PBN>, a, b0, b1, cm, prm,
+                                           b2 != nullptr ? *b2 : b0, c1 != nullptr ? *c1 : cm,
+                                           c2 != nullptr ? *c2 : cm);
   note_launch();
   if (e != cudaSuccess) {
     set_error_detail("paired GEMM launch failed: %s", cudaGetErrorString(e));
@@ -367,6 +398,29 @@ tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMa
     case kModeRowPartial: return launch_pair_mode<kModeRowPartial, 256>(c, a, b0, b1, cm, prm);
     default: return launch_pair_mode<kModeRowSplitK, 256>(c, a, b0, b1, cm, prm);
   }
+}
+
+// Several column layers (identity activation, no bias) of one input in one
+// launch of 256 x 256 pair tiles: weight maps b[i], output maps cm[i], k[i]
+// output columns on prm.p shards; the segments' tiles follow each other.
+tp_status launch_tc_pair_column_multi(const LaunchCtx& c, const CUtensorMap& a,
+                                      const CUtensorMap* b, const CUtensorMap* cm,
+                                      const int64_t* k, int nseg, TcParams prm) {
+  prm.m_tiles = ceil_div(prm.T, PBM);
+  int32_t start = 0;
+  for (int i = 0; i < nseg; ++i) {
+    prm.seg_start[i] = start;
+    prm.seg_n[i] = static_cast<int32_t>(k[i]);
+    prm.seg_s[i] = static_cast<int32_t>(k[i] / prm.p);
+    start += prm.m_tiles * ceil_div(k[i], 256);
+  }
+  prm.seg_start[nseg] = start;
+  prm.nseg = nseg;
+  prm.n_tiles = 0;   // per segment: (seg_start[i+1] - seg_start[i]) / m_tiles
+  prm.num_tiles = start;
+  return launch_pair_mode<kModeColumn, 256>(c, a, b[0], nseg > 1 ? b[1] : b[0], cm[0], prm,
+                                            nseg > 2 ? &b[2] : &b[0], nseg > 1 ? &cm[1] : &cm[0],
+                                            nseg > 2 ? &cm[2] : &cm[0]);
 }
 
 }  // namespace tpk

@@ -69,6 +69,14 @@ struct TcParams {
   int32_t zero_n;        // the previous kernel) for the row layer that follows; may be null
   int32_t m_group;       // > 0: tiles walk groups of this many m-tiles, group slowest (all
                          // shards of one group before the next); 0: one group
+  // Column layer on CTA pairs with several weights and outputs in one launch
+  // (the Q, K, V projections): nseg > 1 segments, segment i owning tiles
+  // [seg_start[i], seg_start[i + 1]), k = seg_n[i] output columns, shard
+  // width seg_s[i]; weight i and output i come as the kernel's i-th B and C
+  // tensor maps.
+  int32_t nseg;
+  int32_t seg_start[4];
+  int32_t seg_n[3], seg_s[3];
   WaitCtl wait;
   int64_t debug_drop;    // slot (in issue order) whose load is skipped; -1 none
 };
@@ -474,5 +482,10 @@ __device__ __forceinline__ void epilogue_tile_bulk_col(const TcParams& P, const 
 tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMap& a,
                          const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& cm,
                          gemm::TcParams prm);
+// Up to three identity column layers of one input in one launch of 256 x 256
+// pair tiles (tp_gemm2_sm100.cu).
+tp_status launch_tc_pair_column_multi(const LaunchCtx& c, const CUtensorMap& a,
+                                      const CUtensorMap* b, const CUtensorMap* cm,
+                                      const int64_t* k, int nseg, gemm::TcParams prm);
 
 }  // namespace tpk

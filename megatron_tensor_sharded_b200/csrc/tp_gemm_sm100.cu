@@ -335,6 +335,40 @@ tp_status launch_tc_column(const LaunchCtx& c, const void* X, const void* W1, co
   return launch_bn<kModeColumn>(c, tch.bn, mA, mB0, mB1, mY, prm);
 }
 
+tp_status launch_tc_column_multi(const LaunchCtx& c, const void* X, const void* const* W,
+                                 void* const* Y, const int64_t* k, int nseg, int64_t T, int64_t d,
+                                 int p, int* zero_cnt, int zero_n, bool* done) {
+  *done = false;
+  if (nseg < 1 || nseg > 3 || !pair_allowed()) return TP_OK;
+  int64_t ktot = 0;
+  for (int i = 0; i < nseg; ++i) {
+    if (k[i] % p != 0 || (k[i] / p) % 32 != 0) return TP_OK;   // bulk stores per shard
+    ktot += k[i];
+  }
+  const TileChoice tch = pick_tile(T, ktot, 1, ceil_div(d, BK), c.num_sms, false, true);
+  if (!tch.pair || tch.bn != 256) return TP_OK;
+  CUtensorMap mA, mB[3], mC[3];
+  if (!make_map_a(&mA, X, d, T, 1)) return TP_ERR_CUDA;
+  for (int i = 0; i < nseg; ++i)
+    if (!make_map_b(&mB[i], W[i], k[i], d) || !make_map_bf16_out(&mC[i], Y[i], k[i] / p, T, p))
+      return TP_ERR_CUDA;
+  TcParams prm{};
+  prm.T = static_cast<int32_t>(T);
+  prm.n_total = static_cast<int32_t>(k[0]);
+  prm.s = static_cast<int32_t>(k[0] / p);
+  prm.p = p;
+  prm.batches = 1;
+  prm.k_blocks = ceil_div(d, BK);
+  prm.act = kActIdentity;
+  prm.bias = nullptr;
+  prm.out = Y[0];
+  prm.bulk_out = 1;
+  prm.zero_cnt = zero_cnt;
+  prm.zero_n = zero_n;
+  *done = true;
+  return launch_tc_pair_column_multi(c, mA, mB, mC, k, nseg, prm);
+}
+
 // One int per region at most: regions are row tiles of 128 or 256 rows and
 // 64 to 256 columns.
 size_t region_counter_bytes(int64_t T, int64_t d) {

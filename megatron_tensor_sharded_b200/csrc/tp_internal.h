@@ -57,6 +57,13 @@ struct RegionFold {
   int rows, cols, m_regions, n_regions, target;
   int m_group;   // regions complete group by group of this many m (0: one group)
 };
+// Up to three identity column layers of the same X in one launch (the
+// attention block's Q, K, V projections): *done = false (nothing launched)
+// when the shapes do not suit one launch of CTA-pair tiles, and the caller
+// launches them one by one.
+tp_status launch_tc_column_multi(const LaunchCtx& c, const void* X, const void* const* W,
+                                 void* const* Y, const int64_t* k, int nseg, int64_t T, int64_t d,
+                                 int p, int* zero_cnt, int zero_n, bool* done);
 // Row layer; with `region_cnt` (zeroed, region_counter_bytes()) it also
 // publishes per-tile completion when it runs on CTA-pair tiles and
 // describes the regions in *rf (rf->cnt stays null otherwise).

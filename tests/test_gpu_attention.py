@@ -207,14 +207,15 @@ def test_attention_dropped_load_times_out():
     _check_head(got[1][:, :128], Q[1][:, :128], K[1][:, :128], V[1][:, :128], True)
 
 
-@pytest.mark.parametrize("bias", [True, False])
-def test_attention_block_is_bit_identical_to_separate_calls(bias):
-    """A shape whose output projection runs on CTA-pair tiles (T=1000,
-    d=2048, 16 query / 4 key-value heads on p=4): tp_attn_block, whose fold
-    runs beside that projection, gives the bits of the separate calls
-    (three column projections, tp_attention_heads, tp_row_linear,
+@pytest.mark.parametrize("T,bias", [(1000, True), (1000, False), (2048, True)])
+def test_attention_block_is_bit_identical_to_separate_calls(T, bias):
+    """Shapes whose output projection runs on CTA-pair tiles (d=2048, 16
+    query / 4 key-value heads on p=4; at T=2048 the Q, K, V projections also
+    run as one launch of pair tiles): tp_attn_block, whose fold runs beside
+    the output projection, gives the bits of the separate calls (three
+    column projections, tp_attention_heads, tp_row_linear,
     tp_reduce_partials), call after call on one workspace."""
-    T, d, h, hkv, p = 1000, 2048, 16, 4, 4
+    d, h, hkv, p = 2048, 16, 4, 4
     inp = W.make_attn_inputs(T, d, h, hkv, 128, seed=7, with_bias=bias, w_std=0.03)
     X, Wq, Wk, Wv, Wo = dev(inp.X), dev(inp.Wq), dev(inp.Wk), dev(inp.Wv), dev(inp.Wo)
     bo = dev(inp.bo)

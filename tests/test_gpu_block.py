@@ -156,14 +156,15 @@ def test_transformer_block_full_size_prefix(name, n):
     assert O.rel_err(got[:n] - inp.X[:n], ref - inp.X[:n]) <= 1e-2
 
 
-@pytest.mark.parametrize("act", ["gelu_tanh", "swiglu"])
-def test_transformer_block_is_bit_identical_to_separate_calls(act):
-    """A shape whose MLP row layer runs on CTA-pair tiles (T=1000, d=2048,
-    k=2048 on p=4), so reduction #2 runs beside that layer: the block gives
-    the bits of its steps called one by one (LayerNorm, the three
-    projections, attention, W_O, fold + bo + X, LayerNorm, the MLP layers,
-    fold + b2 + H), call after call on one workspace."""
-    T, d, h, hkv, k, p = 1000, 2048, 16, 4, 2048, 4
+@pytest.mark.parametrize("T,act", [(1000, "gelu_tanh"), (1000, "swiglu"), (2048, "gelu_tanh")])
+def test_transformer_block_is_bit_identical_to_separate_calls(T, act):
+    """Shapes whose MLP row layer runs on CTA-pair tiles (d=2048, k=2048 on
+    p=4), so reduction #2 runs beside that layer (at T=2048 the Q, K, V
+    projections also run as one launch): the block gives the bits of its
+    steps called one by one (LayerNorm, the three projections, attention,
+    W_O, fold + bo + X, LayerNorm, the MLP layers, fold + b2 + H), call
+    after call on one workspace."""
+    d, h, hkv, k, p = 2048, 16, 4, 2048, 4
     inp = W.make_block_inputs(T, d, h, hkv, 128, k, act, seed=11, w_std=0.03)
     blk = DeviceTransformerBlock(inp, T, d, h, hkv, 128, k, p, act)
     t, X = blk.t, blk.X
