@@ -403,7 +403,7 @@ tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMa
 // Several column layers (identity activation, no bias) of one input in one
 // launch of 256 x 256 pair tiles: weight maps b[i], output maps cm[i], k[i]
 // output columns on prm.p shards; the segments' tiles follow each other.
-tp_status launch_tc_pair_column_multi(const LaunchCtx& c, const CUtensorMap& a,
+tp_status launch_tc_pair_column_multi(const LaunchCtx& c, int pbn, const CUtensorMap& a,
                                       const CUtensorMap* b, const CUtensorMap* cm,
                                       const int64_t* k, int nseg, TcParams prm) {
   prm.m_tiles = ceil_div(prm.T, PBM);
@@ -412,15 +412,18 @@ tp_status launch_tc_pair_column_multi(const LaunchCtx& c, const CUtensorMap& a,
     prm.seg_start[i] = start;
     prm.seg_n[i] = static_cast<int32_t>(k[i]);
     prm.seg_s[i] = static_cast<int32_t>(k[i] / prm.p);
-    start += prm.m_tiles * ceil_div(k[i], 256);
+    start += prm.m_tiles * ceil_div(k[i], pbn);
   }
   prm.seg_start[nseg] = start;
   prm.nseg = nseg;
   prm.n_tiles = 0;   // per segment: (seg_start[i+1] - seg_start[i]) / m_tiles
   prm.num_tiles = start;
-  return launch_pair_mode<kModeColumn, 256>(c, a, b[0], nseg > 1 ? b[1] : b[0], cm[0], prm,
-                                            nseg > 2 ? &b[2] : &b[0], nseg > 1 ? &cm[1] : &cm[0],
-                                            nseg > 2 ? &cm[2] : &cm[0]);
+  const CUtensorMap& b1 = nseg > 1 ? b[1] : b[0];
+  const CUtensorMap* b2 = nseg > 2 ? &b[2] : &b[0];
+  const CUtensorMap* c1 = nseg > 1 ? &cm[1] : &cm[0];
+  const CUtensorMap* c2 = nseg > 2 ? &cm[2] : &cm[0];
+  if (pbn == 128) return launch_pair_mode<kModeColumn, 128>(c, a, b[0], b1, cm[0], prm, b2, c1, c2);
+  return launch_pair_mode<kModeColumn, 256>(c, a, b[0], b1, cm[0], prm, b2, c1, c2);
 }
 
 }  // namespace tpk

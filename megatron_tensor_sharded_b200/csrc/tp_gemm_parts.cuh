@@ -482,9 +482,9 @@ __device__ __forceinline__ void epilogue_tile_bulk_col(const TcParams& P, const 
 tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMap& a,
                          const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& cm,
                          gemm::TcParams prm);
-// Up to three identity column layers of one input in one launch of 256 x 256
-// pair tiles (tp_gemm2_sm100.cu).
-tp_status launch_tc_pair_column_multi(const LaunchCtx& c, const CUtensorMap& a,
+// Up to three identity column layers of one input in one launch of 256 x pbn
+// pair tiles, pbn 128 or 256 (tp_gemm2_sm100.cu).
+tp_status launch_tc_pair_column_multi(const LaunchCtx& c, int pbn, const CUtensorMap& a,
                                       const CUtensorMap* b, const CUtensorMap* cm,
                                       const int64_t* k, int nseg, gemm::TcParams prm);
 

@@ -346,7 +346,7 @@ tp_status launch_tc_column_multi(const LaunchCtx& c, const void* X, const void* 
     ktot += k[i];
   }
   const TileChoice tch = pick_tile(T, ktot, 1, ceil_div(d, BK), c.num_sms, false, true);
-  if (!tch.pair || tch.bn != 256) return TP_OK;
+  if (!tch.pair) return TP_OK;
   CUtensorMap mA, mB[3], mC[3];
   if (!make_map_a(&mA, X, d, T, 1)) return TP_ERR_CUDA;
   for (int i = 0; i < nseg; ++i)
@@ -366,7 +366,7 @@ tp_status launch_tc_column_multi(const LaunchCtx& c, const void* X, const void* 
   prm.zero_cnt = zero_cnt;
   prm.zero_n = zero_n;
   *done = true;
-  return launch_tc_pair_column_multi(c, mA, mB, mC, k, nseg, prm);
+  return launch_tc_pair_column_multi(c, tch.bn, mA, mB, mC, k, nseg, prm);
 }
 
 // One int per region at most: regions are row tiles of 128 or 256 rows and

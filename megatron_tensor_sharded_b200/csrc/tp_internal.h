@@ -57,10 +57,11 @@ struct RegionFold {
   int rows, cols, m_regions, n_regions, target;
   int m_group;   // regions complete group by group of this many m (0: one group)
 };
-// Up to three identity column layers of the same X in one launch (the
-// attention block's Q, K, V projections): *done = false (nothing launched)
-// when the shapes do not suit one launch of CTA-pair tiles, and the caller
-// launches them one by one.
+// Up to three identity column layers of the same X in one launch of
+// CTA-pair tiles (the attention block's Q, K, V projections): *done = false
+// (nothing launched) when the combined layer would not take pair tiles or a
+// shard width is not a multiple of 32, and the caller launches them one by
+// one.
 tp_status launch_tc_column_multi(const LaunchCtx& c, const void* X, const void* const* W,
                                  void* const* Y, const int64_t* k, int nseg, int64_t T, int64_t d,
                                  int p, int* zero_cnt, int zero_n, bool* done);

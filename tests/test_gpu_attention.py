@@ -207,15 +207,19 @@ def test_attention_dropped_load_times_out():
     _check_head(got[1][:, :128], Q[1][:, :128], K[1][:, :128], V[1][:, :128], True)
 
 
-@pytest.mark.parametrize("T,bias", [(1000, True), (1000, False), (2048, True)])
-def test_attention_block_is_bit_identical_to_separate_calls(T, bias):
-    """Shapes whose output projection runs on CTA-pair tiles (d=2048, 16
-    query / 4 key-value heads on p=4; at T=2048 the Q, K, V projections also
-    run as one launch of pair tiles): tp_attn_block, whose fold runs beside
-    the output projection, gives the bits of the separate calls (three
-    column projections, tp_attention_heads, tp_row_linear,
-    tp_reduce_partials), call after call on one workspace."""
-    d, h, hkv, p = 2048, 16, 4, 4
+@pytest.mark.parametrize("T,h,hkv,bias", [(1000, 16, 4, True), (1000, 16, 4, False),
+                                          (2048, 16, 4, True), (2000, 12, 4, False),
+                                          (2048, 32, 8, False)])
+def test_attention_block_is_bit_identical_to_separate_calls(T, h, hkv, bias):
+    """Shapes whose output projection runs on CTA-pair tiles (d=2048, p=4).
+    At T >= 2000 the Q, K, V projections also run as one launch of pair
+    tiles: 256 x 128 tiles at 16 and 12 query heads (T=2000: a ragged last
+    row tile and 384-column Q shards that start inside a tile), 256 x 256
+    tiles at 32 / 8 heads.  tp_attn_block, whose fold runs beside the output
+    projection, gives the bits of the separate calls (three column
+    projections, tp_attention_heads, tp_row_linear, tp_reduce_partials),
+    call after call on one workspace."""
+    d, p = 2048, 4
     inp = W.make_attn_inputs(T, d, h, hkv, 128, seed=7, with_bias=bias, w_std=0.03)
     X, Wq, Wk, Wv, Wo = dev(inp.X), dev(inp.Wq), dev(inp.Wk), dev(inp.Wv), dev(inp.Wo)
     bo = dev(inp.bo)
@@ -239,6 +243,11 @@ def test_attention_block_is_bit_identical_to_separate_calls(T, bias):
     ws = torch.full((n,), 0x7F, dtype=torch.uint8, device="cuda")
     for _ in range(2):
         Z = torch.full((T, d), float("nan"), dtype=torch.float32, device="cuda")
+        before = tp.tp_kernel_launch_count()
         tp.tp_attn_block(X, Wq, Wk, Wv, Wo, bo, Z, ws, n, T, d, h, hkv, 128, p, 1)
+        launches = tp.tp_kernel_launch_count() - before
         tp.tp_sync_status()
         assert np.array_equal(bits(host_f32(Z)), want)
+        # Q, K, V in one launch at T >= 2000, three below; then attention,
+        # W_O and the fold
+        assert launches == (4 if T >= 2000 else 6)

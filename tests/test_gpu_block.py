@@ -194,5 +194,10 @@ def test_transformer_block_is_bit_identical_to_separate_calls(T, act):
     tp.tp_sync_status()
     want = bits(host_f32(out))
     for _ in range(2):
+        before = tp.tp_kernel_launch_count()
         got = blk.run(True)
+        launches = tp.tp_kernel_launch_count() - before
         assert np.array_equal(bits(got), want)
+        # LN, Q K V (one launch at T=2048, three at T=1000), attention, W_O,
+        # fold + LN, the two MLP layers, fold
+        assert launches == (8 if T >= 2000 else 10)
