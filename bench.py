@@ -140,15 +140,20 @@ def blas_threads() -> int:
 
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed
+    region: sampling starts (and its first line is waited for) before the
+    region, every sample carries nvidia-smi's timestamp, and the summary keeps
+    the samples taken between entering and leaving the context."""
 
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    PERIOD_MS = 20
 
     def __init__(self, gpu_index: int):
         self.gpu_index = gpu_index
         self.proc = None
+        self.t0 = self.t1 = None
         # raw samples: $TP_BENCH_CLOCK_DIR if set (kept for inspection), else a
         # temporary directory
         out_dir = os.environ.get("TP_BENCH_CLOCK_DIR") or tempfile.gettempdir()
@@ -160,16 +165,25 @@ class ClockSampler:
             self.f = open(self.path, "w")
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.QUERY}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", str(self.PERIOD_MS)],
                 stdout=self.f, stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
-        time.sleep(0.3)
+        # nvidia-smi takes a moment to start: wait (up to 3 s) for its first
+        # line, so that the timed region is sampled from its start
+        deadline = time.time() + 3.0
+        while self.proc is not None and time.time() < deadline:
+            self.f.flush()
+            if os.path.getsize(self.path) > 0 or self.proc.poll() is not None:
+                break
+            time.sleep(0.01)
+        self.t0 = time.time()
         return self
 
     def __exit__(self, *exc):
+        self.t1 = time.time()
         if self.proc is not None:
-            time.sleep(0.2)
+            time.sleep(2.5 * self.PERIOD_MS / 1000.0)   # the sample in flight at t1
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
@@ -177,25 +191,58 @@ class ClockSampler:
                 self.proc.kill()
             self.f.close()
 
+    @staticmethod
+    def parse(lines):
+        """(unix time or None, sm MHz, max sm MHz, power W, [4 reason flags])
+        per well-formed line of the query above."""
+        import datetime
+        rows = []
+        for line in lines:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                ts = None
+            try:
+                rows.append((ts, float(parts[2]), float(parts[3]),
+                             float(parts[4]) if parts[4] not in ("[N/A]", "N/A") else 0.0,
+                             parts[6:10]))
+            except ValueError:
+                continue
+        return rows
+
+    @staticmethod
+    def summarise(rows, t0=None, t1=None):
+        """Median SM clock of the loaded samples inside [t0, t1] (all samples
+        when none falls inside), the maximum clock, and every throttle reason
+        seen in that window."""
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        window = "timed region"
+        if t0 is not None and t1 is not None:
+            slack = 0.03
+            inside = [r for r in rows if r[0] is not None and t0 - slack <= r[0] <= t1 + slack]
+            if inside:
+                rows_w = inside
+            else:
+                rows_w, window = rows, "whole sampling (no sample inside the timed region)"
+        else:
+            rows_w = rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows_w for i, v in enumerate(r[4]) if v.lower() == "active"})
+        loaded = [r for r in rows_w if r[3] > 0.5 * max(x[3] for x in rows_w)] or rows_w
+        return {"sm_mhz": statistics.median(r[1] for r in loaded),
+                "sm_max_mhz": max(r[2] for r in rows), "reasons": reasons,
+                "samples": len(rows_w), "window": window}
+
     def summary(self):
         if self.proc is None or not os.path.exists(self.path):
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        rows = []
-        for line in open(self.path):
-            parts = [x.strip() for x in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                rows.append((float(parts[1]), float(parts[2]), float(parts[3]) if parts[3] not in ("[N/A]", "N/A") else 0.0, parts[5:9]))
-            except ValueError:
-                continue
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[3]) if v.lower() == "active"})
-        loaded = [r for r in rows if r[2] > 0.5 * max(x[2] for x in rows)] or rows
-        return {"sm_mhz": statistics.median(r[0] for r in loaded), "sm_max_mhz": max(r[1] for r in rows),
-                "reasons": reasons, "samples": len(rows)}
+        with open(self.path) as f:
+            rows = self.parse(f)
+        return self.summarise(rows, self.t0, self.t1)
 
 
 def source_digest(files) -> str:

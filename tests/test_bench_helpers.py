@@ -72,3 +72,32 @@ def test_whole_job_value_and_tokens_override():
     import dataclasses
     w = dataclasses.replace(WL.WORKLOADS["llama"], T=1024, name="llama_T1024")
     assert w.gemm_flops() * 4 == WL.WORKLOADS["llama"].gemm_flops()
+
+
+def test_clock_samples_are_taken_from_the_timed_region():
+    """ClockSampler keeps the nvidia-smi samples whose timestamps fall inside
+    the timed region: an idle sample before it (low clock, no load) and a
+    throttled one after it do not count; the loaded samples' median does."""
+    import datetime
+    t0 = datetime.datetime(2026, 1, 2, 3, 4, 5).timestamp()
+
+    def line(dt, mhz, watts, power_cap="Not Active", thermal="Not Active"):
+        ts = datetime.datetime.fromtimestamp(t0 + dt).strftime("%Y/%m/%d %H:%M:%S.%f")[:-3]
+        return (f"{ts}, 0, {mhz}, 1965, {watts}, 0x0, Not Active, Not Active, {thermal}, "
+                f"{power_cap}\n")
+
+    lines = [line(-0.2, 345, 90.0),                       # idle, before the region
+             line(0.01, 1965, 900.0), line(0.03, 1950, 950.0, power_cap="Active"),
+             line(0.05, 1965, 910.0), line(0.07, 120, 100.0),   # a dip in load inside
+             line(0.5, 1200, 950.0, thermal="Active")]    # after the region
+    rows = bench.ClockSampler.parse(lines)
+    assert len(rows) == 6
+    s = bench.ClockSampler.summarise(rows, t0, t0 + 0.08)
+    assert s["samples"] == 4 and s["window"] == "timed region"
+    assert s["sm_mhz"] == 1965.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
+    # no sample inside the window: all samples, said so
+    s = bench.ClockSampler.summarise(rows, t0 + 10, t0 + 11)
+    assert s["samples"] == 6 and s["window"].startswith("whole sampling")
+    assert "sw_thermal_slowdown" in s["reasons"]
+    assert bench.ClockSampler.summarise([], t0, t0 + 1)["reasons"] == ["no samples"]
