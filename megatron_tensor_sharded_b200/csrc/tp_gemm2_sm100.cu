@@ -19,6 +19,12 @@
 // No load uses cluster multicast: every CTA reads its own tiles.  Epilogues
 // store through shared memory with TMA tensor stores, as in the single-CTA
 // kernel.
+//
+// Two launch-level options: a row layer of partials can publish per-tile
+// completion counters for the fold that runs beside it (region_cnt, tiles
+// taken in two halves of the m-tiles), and a column layer can carry up to
+// three weight/output segments of the same input (the attention block's
+// Q, K and V in one launch; nseg).
 #include <cuda.h>
 #include <cuda_runtime.h>
 

@@ -26,6 +26,21 @@ def bits(a):
     return np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
 
 
+def pairs_enabled():
+    """CTA-pair tiles are in use (the library's TP_DISABLE_PAIR=1 turns them
+    off, and with them the one-launch Q, K, V and the fold beside the row
+    layer)."""
+    import os
+    return os.environ.get("TP_DISABLE_PAIR", "") != "1"
+
+
+def region_fold_enabled():
+    """The fold beside the row layer is in use (TP_DISABLE_REGION_FOLD=1 and
+    single-CTA tiles turn it off)."""
+    import os
+    return pairs_enabled() and os.environ.get("TP_DISABLE_REGION_FOLD", "") != "1"
+
+
 class DeviceBlock:
     """Device copies of one workload instance plus output buffers."""
 

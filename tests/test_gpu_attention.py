@@ -27,7 +27,7 @@ import torch
 
 import megatron_tensor_sharded_b200 as tp
 import workloads as W
-from gpu_util import bits, dev, host_f32
+from gpu_util import bits, dev, host_f32, pairs_enabled
 from oracle import tp_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -250,4 +250,4 @@ def test_attention_block_is_bit_identical_to_separate_calls(T, h, hkv, bias):
         assert np.array_equal(bits(host_f32(Z)), want)
         # Q, K, V in one launch at T >= 2000, three below; then attention,
         # W_O and the fold
-        assert launches == (4 if T >= 2000 else 6)
+        assert launches == (4 if T >= 2000 and pairs_enabled() else 6)

@@ -16,7 +16,7 @@ import torch
 
 import megatron_tensor_sharded_b200 as tp
 import workloads as W
-from gpu_util import dev, host_f32
+from gpu_util import dev, host_f32, region_fold_enabled
 from oracle import tp_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -241,6 +241,8 @@ def test_dx_fold_beside_its_gemm_is_the_fixed_order_fold(T, d, k, p, act):
     tp.tp_reduce_partials(part, None, Z, T, d, p)
     tp.tp_sync_status()
     assert np.array_equal(host_f32(Z).view(np.uint32), host_f32(blk.dX).view(np.uint32))
+    if not region_fold_enabled():
+        return
     scratch = _r256(-(-T // 128) * max(k, d) * 4)
     cnt_off = off + _r256(p * T * d * 4) + scratch
     m_regions = -(-T // 256)
