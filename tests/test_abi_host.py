@@ -229,3 +229,29 @@ def test_host_entry_workspace_and_validation():
     import torch
     if not torch.cuda.is_available():
         assert call() == 5
+
+
+def test_block_workspace_layouts_hold_the_region_counters():
+    """The attention block, transformer block and backward workspaces: their
+    buffers, each at a 256-byte boundary, then room for one int32 counter per
+    128-row x 64-column region (the fold beside the row layer)."""
+    def r256(n):
+        return -(-n // 256) * 256
+
+    def regions(T, d):
+        return r256(4 * (-(-T // 128)) * (-(-d // 64)))
+
+    T, d, h, hkv, dh, p = 1000, 2048, 16, 4, 128, 4
+    q, kv = r256(T * h * dh * 2), r256(T * hkv * dh * 2)
+    assert tp.tp_attn_block_workspace_size(T, d, h, hkv, dh, p) == \
+        2 * q + 2 * kv + r256(p * T * d * 4) + regions(T, d)
+    k = 2048
+    want = (r256(T * d * 2) + r256(T * d * 4) + q + 2 * kv + q + r256(T * k * 2)
+            + r256(p * T * d * 4) + regions(T, d))
+    assert tp.tp_transformer_block_workspace_size(T, d, h, hkv, dh, k, p) == want
+    # backward: dH (and dU for SwiGLU), the dX partials, the bias-gradient
+    # scratch (one row per 128 tokens of max(k, d) fp32), the counters
+    for act, halves in ((tp.TP_ACT_GELU_TANH, 1), (tp.TP_ACT_SWIGLU, 2)):
+        want = (halves * r256(T * k * 2) + r256(p * T * d * 4)
+                + r256(-(-T // 128) * max(k, d) * 4) + regions(T, d))
+        assert tp.tp_mlp_block_backward_workspace_size(T, d, k, p, act) == want
