@@ -506,7 +506,10 @@ void tp_set_wait_timeout_ns(uint64_t ns);
 /* Fault injection for tests of the bounded waits: when `stage_index` >= 0,
  * the next tensor-core launch's producer skips the load of that pipeline
  * slot (counted from 0 in issue order), so its consumer's wait must run
- * out.  -1 (default) disables it.  Applies to the next launch only. */
+ * out.  In a launch of CTA-pair tiles only the first pair skips it (the
+ * other pairs' waits on that pair's tiles then run out too); in other
+ * launches every CTA does.  -1 (default) disables it.  Applies to the next
+ * launch only. */
 void tp_debug_drop_load(int64_t stage_index);
 /* The same, for the tensor-core launch that follows `launches_to_skip`
  * others (0: the next one), e.g. 1 for the row layer of a tp_mlp_block

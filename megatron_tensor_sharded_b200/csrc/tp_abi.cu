@@ -291,9 +291,11 @@ tp_status fold_residual_impl(const float* partials, const float* bias, const flo
                              void* Y, float eps, void* stream);
 
 // bf16 row layer to partials, then the fixed-order fold of the partials
-// (+ b2, + the residual R if given): beside the row layer when `regions`
-// came from region_counters (and were zeroed), after it otherwise.  Same
-// bits either way.
+// (+ b2, + the residual R if given).  When `regions` came from
+// region_counters (and were zeroed) and the layer runs on CTA pairs: without
+// R, inside the row layer (each shard's tile adds its partial to the running
+// sum in Z, no partials written); with R, beside the row layer.  After it
+// otherwise.  Same bits every way.
 tp_status row_and_fold(const void* Y, const void* W2, float* P, const float* b2, float* Z,
                        int64_t T, int64_t k, int64_t d, int p, int* regions, void* stream,
                        const float* R = nullptr) {
@@ -308,6 +310,11 @@ tp_status row_and_fold(const void* Y, const void* W2, float* P, const float* b2,
   }
   LaunchCtx c{};
   TP_TRY(make_ctx(stream, true, &c));
+  if (R == nullptr && row_chain_allowed()) {
+    bool done = false;
+    TP_TRY(launch_tc_row_chain(c, Y, W2, b2, Z, T, k, d, p, regions, &done));
+    if (done) return TP_OK;
+  }
   RegionFold rf{};
   TP_TRY(launch_tc_row(c, Y, W2, P, T, k, d, p, regions, &rf));
   if (rf.cnt != nullptr)

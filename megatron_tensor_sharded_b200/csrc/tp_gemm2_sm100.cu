@@ -55,7 +55,8 @@ struct PCfg {
   static constexpr uint32_t IDESC = idesc_bf16_f32(PBM, PBN, /*a_mn=*/0, /*b_mn=*/1);
   static_assert(PBN == 128 || PBN == 256, "pair tile width");
   static_assert(SMEM_BYTES <= SMEM_LIMIT, "shared memory budget");
-  static_assert(8 * (2 * STAGES + 5) + 16 <= CTRL_BYTES, "control block");
+  // barriers, TMEM slot + abort flag, then one barrier per epilogue warp (chain loads)
+  static_assert(8 * (2 * STAGES + 5) + 16 + 8 * NUM_EPI_WARPS <= CTRL_BYTES, "control block");
 };
 
 // Loads of one slot for this CTA: A rows [m*256 + rank*128, +128), B columns
@@ -81,7 +82,7 @@ __device__ __forceinline__ void issue_slot_pair(const TcParams& P, const CUtenso
 #pragma unroll
     for (int c = 0; c < PB_CHUNKS; ++c)
       tma_load_2d_pair(sb + c * B_CHUNK_BYTES, mB, bar, col0 + c * B_BOX_COLS, kb * BK);
-  } else if constexpr (MODE == kModeRowPartial) {
+  } else if constexpr (MODE == kModeRowPartial || MODE == kModeRowChain) {
     tma_load_3d_pair(sa, mA, bar, kb * BK, row0, tc.batch);
     const int32_t col0 = tc.n * PBN + static_cast<int32_t>(rank) * (PBN / 2);
 #pragma unroll
@@ -101,6 +102,109 @@ __device__ __forceinline__ void issue_slot_pair(const TcParams& P, const CUtenso
 
 template <int MODE>
 constexpr bool kPairBulkOut = (MODE == kModeRowPartial || MODE == kModeRowSplitK);
+
+// One lane waits until *cnt reaches target (acquire at GPU scope), bounded;
+// false, with the CTA's abort flag and kErrWaitRegion set, when it does not.
+__device__ __forceinline__ bool wait_count(const int* cnt, int target, volatile int* abort,
+                                           const WaitCtl& w) {
+  if (ld_acquire_gpu(cnt) >= target) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    __nanosleep(200);
+    if (ld_acquire_gpu(cnt) >= target) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > w.timeout_ns) {
+      *abort = 1;
+      atomicOr(w.err, kErrWaitRegion);
+      return false;
+    }
+  }
+}
+
+// Chain fold of a row layer (kModeRowChain): the tile of shard s adds its partial
+// to the running sum that shard s-1's tile of the same rows and columns left
+// in Z, and the last shard adds b2, so Z = ((P_0 + P_1) + ... + P_{p-1}) + b2
+// with one fp32 RNE addition per element in shard order -- the fixed-order
+// fold -- and no partials reach memory.  The warp waits (once per tile) for
+// the region counter to show all earlier shards' tiles stored; then per
+// 32 x 32 chunk the previous sum comes into the warp's staging tile by a
+// TMA load (128-byte swizzle, the store's layout), each lane adds its row
+// of the accumulator to its row of the chunk, and a TMA store writes the new
+// sum back.  False if a wait gave up.
+template <int PBN>
+__device__ __forceinline__ bool epilogue_tile_chain(const TcParams& P, const TileCoord& tc,
+                                                    uint32_t tacc, int32_t row0, int half,
+                                                    uint32_t stage, uint32_t bar, uint32_t& ph,
+                                                    const CUtensorMap* mapZ, volatile int* abort,
+                                                    int lane) {
+  const float* __restrict__ b2 = static_cast<const float*>(P.bias);
+  const bool first = tc.batch == 0;
+  const bool last = tc.batch == P.p - 1;
+  if (!first) {
+    bool ok = true;
+    if (lane == 0) {
+      ok = wait_count(P.region_cnt + tc.n * P.m_tiles + tc.m, 2 * NUM_EPI_WARPS * tc.batch, abort,
+                      P.wait);
+      // the TMA loads below read, in the async proxy, what the acquire made visible
+      fence_proxy_async_global();
+    }
+    if (!__shfl_sync(0xffffffffu, ok ? 1 : 0, 0)) return false;
+  }
+#pragma unroll 1
+  for (int q = 0; q < PBN / 64; ++q) {
+    const int c0 = half * (PBN / 2) + q * 32;
+    const int32_t j0 = tc.n * PBN + c0;
+    uint32_t v[32];
+    tmem_ld_32x32b_x32(tacc + c0, v);
+    tmem_ld_wait();
+    if (j0 >= P.n_total) continue;   // warp-uniform
+    // the staging tile is free once the previous store has read it
+    if (lane == 0) bulk_wait_read0();
+    __syncwarp();
+    if (!first) {
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar, 32 * 32 * 4);
+        tma_load_3d(stage, mapZ, bar, j0, row0, 0);
+      }
+      // not abortable: the load must land before the staging tile is reused
+      if (!wait_teardown(bar, ph, P.wait)) return false;
+      ph ^= 1u;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t addr = stage + lane * 128 + ((c ^ (lane & 7)) << 4);
+        uint32_t z0, z1, z2, z3;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(z0), "=r"(z1), "=r"(z2), "=r"(z3)
+                     : "r"(addr)
+                     : "memory");
+        v[4 * c + 0] = __float_as_uint(__fadd_rn(__uint_as_float(z0), __uint_as_float(v[4 * c + 0])));
+        v[4 * c + 1] = __float_as_uint(__fadd_rn(__uint_as_float(z1), __uint_as_float(v[4 * c + 1])));
+        v[4 * c + 2] = __float_as_uint(__fadd_rn(__uint_as_float(z2), __uint_as_float(v[4 * c + 2])));
+        v[4 * c + 3] = __float_as_uint(__fadd_rn(__uint_as_float(z3), __uint_as_float(v[4 * c + 3])));
+      }
+    }
+    if (last && b2 != nullptr) {
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        v[e] = __float_as_uint(
+            __fadd_rn(__uint_as_float(v[e]), j0 + e < P.n_total ? __ldg(b2 + j0 + e) : 0.0f));
+    }
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint32_t addr = stage + lane * 128 + ((c ^ (lane & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v[4 * c]),
+                   "r"(v[4 * c + 1]), "r"(v[4 * c + 2]), "r"(v[4 * c + 3])
+                   : "memory");
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_3d(mapZ, stage, j0, row0, 0);
+      bulk_commit();
+    }
+  }
+  return true;
+}
 
 // Tile t of the launch and its segment (0 unless several column layers share
 // the launch; within a segment m fastest, as decode_tile walks one layer).
@@ -139,6 +243,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* const bars = reinterpret_cast<uint64_t*>(ctrl);
   uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(ctrl + 8 * (2 * PSTAGES + 5));
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  uint64_t* const chain_bars = reinterpret_cast<uint64_t*>(ctrl + 8 * (2 * PSTAGES + 5) + 16);
 
   auto full_bar = [&](uint32_t s) { return smem_u32(&bars[s]); };
   auto empty_bar = [&](uint32_t s) { return smem_u32(&bars[PSTAGES + s]); };
@@ -164,6 +269,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(acce_bar(b), 2 * NUM_EPI_WARPS);
     }
     mbar_init(drain_bar, 1);
+    for (int w = 0; w < NUM_EPI_WARPS; ++w) mbar_init(smem_u32(&chain_bars[w]), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -200,7 +306,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          if (issued != P.debug_drop) {
+          // fault injection (tests of the bounded waits): the first pair only
+          if (issued != P.debug_drop || cluster != 0) {
             if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * PSTAGE_BYTES);
             issue_slot_pair<MODE, PBN>(P, &mapA, mB0, &mapB1, tc, kb, rank, slot_a(stage),
                                   slot_b(stage), mapa_shared(full_bar(stage), 0));
@@ -217,7 +324,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // odd CTA on its empty barriers (the MMA consumed the slot).
       const int64_t first = issued > PSTAGES ? issued - PSTAGES : 0;
       for (int64_t q = first; q < issued; ++q) {
-        if (q == P.debug_drop) continue;
+        if (q == P.debug_drop && cluster == 0) continue;
         const uint32_t s = static_cast<uint32_t>(q % PSTAGES);
         const uint32_t ph = static_cast<uint32_t>((q / PSTAGES) & 1);
         wait_teardown(rank == 0 ? full_bar(s) : empty_bar(s), ph, P.wait);
@@ -269,6 +376,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quad = warp & 3;
     const int half = (warp - 4) >> 2;
     uint32_t nchunk = 0;   // bf16 chunks this warp has staged (alternating halves)
+    uint32_t chain_ph = 0;   // phase of this warp's chain-load barrier
+    const uint32_t chain_bar = smem_u32(&chain_bars[warp - 4]);
     int32_t lt = 0;
     for (int32_t t = cluster; t < P.num_tiles; t += nclusters, ++lt) {
       const uint32_t b = lt & 1, ap = (lt >> 1) & 1;
@@ -289,7 +398,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t tacc = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + b * PBN;
       const int row0 = tc.m * PBM + static_cast<int>(rank) * BM + quad * 32;
       const uint32_t stage_w = epi_stage + (warp - 4) * EPI_WARP_STAGE_BYTES;
-      if constexpr (kPairBulkOut<MODE>) {
+      if constexpr (MODE == kModeRowChain) {
+        if (!epilogue_tile_chain<PBN>(P, tc, tacc, row0, half, stage_w, chain_bar, chain_ph,
+                                      &mapC, abort_flag, lane))
+          break;   // a wait gave up (error bit set); the MMA's waits end on the abort flag
+      } else if constexpr (kPairBulkOut<MODE>) {
         epilogue_tile_bulk<MODE, PBN>(P, tc, tacc, row0, half, stage_w, &mapC, lane);
       } else {
         if (P.bulk_out)
@@ -301,7 +414,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(mapa_shared(acce_bar(b), 0));
-      if constexpr (MODE == kModeRowPartial) {
+      if constexpr (MODE == kModeRowPartial || MODE == kModeRowChain) {
         if (P.region_cnt != nullptr) {
           // Publish this warp's part of the tile to the overlapped fold: its
           // bulk stores complete, are ordered for generic-proxy readers, and
@@ -395,6 +508,7 @@ tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMa
       case kModeColumn: return launch_pair_mode<kModeColumn, 128>(c, a, b0, b1, cm, prm);
       case kModeColumnSwiglu: return launch_pair_mode<kModeColumnSwiglu, 128>(c, a, b0, b1, cm, prm);
       case kModeRowPartial: return launch_pair_mode<kModeRowPartial, 128>(c, a, b0, b1, cm, prm);
+      case kModeRowChain: return launch_pair_mode<kModeRowChain, 128>(c, a, b0, b1, cm, prm);
       default: return launch_pair_mode<kModeRowSplitK, 128>(c, a, b0, b1, cm, prm);
     }
   }
@@ -402,6 +516,7 @@ tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMa
     case kModeColumn: return launch_pair_mode<kModeColumn, 256>(c, a, b0, b1, cm, prm);
     case kModeColumnSwiglu: return launch_pair_mode<kModeColumnSwiglu, 256>(c, a, b0, b1, cm, prm);
     case kModeRowPartial: return launch_pair_mode<kModeRowPartial, 256>(c, a, b0, b1, cm, prm);
+    case kModeRowChain: return launch_pair_mode<kModeRowChain, 256>(c, a, b0, b1, cm, prm);
     default: return launch_pair_mode<kModeRowSplitK, 256>(c, a, b0, b1, cm, prm);
   }
 }

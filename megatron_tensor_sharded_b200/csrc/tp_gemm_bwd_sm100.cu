@@ -528,7 +528,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ok = false;
             break;
           }
-          if (issued != P.debug_drop) {
+          // fault injection (tests of the bounded waits): the first pair only
+          if (issued != P.debug_drop || cluster != 0) {
             if (rank == 0) mbar_arrive_expect_tx(full_bar(stage), 2 * C::STAGE_BYTES);
             issue_pair<AMN, BMN, PBN>(P, &mapA0, &mapA1, &mapB0, &mapB1, g, kb, rank,
                                       slot_a(stage), slot_b(stage),
@@ -546,7 +547,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // on its empty barriers (the MMA consumed the slot)
       const int64_t first = issued > STAGES ? issued - STAGES : 0;
       for (int64_t q = first; q < issued; ++q) {
-        if (q == P.debug_drop) continue;
+        if (q == P.debug_drop && cluster == 0) continue;
         const uint32_t s = static_cast<uint32_t>(q % STAGES);
         const uint32_t ph = static_cast<uint32_t>((q / STAGES) & 1);
         wait_teardown(rank == 0 ? full_bar(s) : empty_bar(s), ph, P.wait);

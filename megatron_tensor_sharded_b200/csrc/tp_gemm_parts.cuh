@@ -49,7 +49,15 @@ struct Cfg {
   static_assert(8 * (2 * STAGES + 5) + 16 <= CTRL_BYTES, "control block");
 };
 
-enum Mode : int { kModeColumn = 0, kModeColumnSwiglu = 1, kModeRowPartial = 2, kModeRowSplitK = 3 };
+// kModeRowChain (CTA pairs only): the row layer's tiles fold shard by shard
+// into Z in the epilogue instead of writing partials.
+enum Mode : int {
+  kModeColumn = 0,
+  kModeColumnSwiglu = 1,
+  kModeRowPartial = 2,
+  kModeRowSplitK = 3,
+  kModeRowChain = 4
+};
 
 struct TcParams {
   int32_t T;             // tokens
@@ -60,11 +68,12 @@ struct TcParams {
   int32_t k_blocks;      // pipeline slots per tile
   int32_t kb_per_shard;  // split-K: slots per shard (s / 64)
   int32_t act;
-  const void* bias;      // b1 (bf16, column) or b2 (fp32, split-K row); may be null
+  const void* bias;      // b1 (bf16, column) or b2 (fp32, split-K and chain row); may be null
   void* out;             // Y bf16 [p][T][s] | P fp32 [p][T][d] | Z fp32 [T][d]
   int32_t bulk_out;      // column layers: 1 = bulk tensor stores through shared memory
   int* region_cnt;       // row partials: per-tile completion counters read by the fold
-                         // beside the layer ([n_tiles][m_tiles]); may be null
+                         // beside the layer ([n_tiles][m_tiles]); may be null.  Chain
+                         // row layer: the same counters order the shards' tiles
   int* zero_cnt;         // column layers: counters this launch zeroes (after its wait for
   int32_t zero_n;        // the previous kernel) for the row layer that follows; may be null
   int32_t m_group;       // > 0: tiles walk groups of this many m-tiles, group slowest (all

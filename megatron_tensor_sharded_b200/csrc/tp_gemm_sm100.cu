@@ -419,6 +419,39 @@ tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float
   return launch_bn<kModeRowPartial>(c, tch.bn, mA, mB, mB, mC, prm);
 }
 
+tp_status launch_tc_row_chain(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
+                              float* Z, int64_t T, int64_t k, int64_t d, int p, int* region_cnt,
+                              bool* done) {
+  *done = false;
+  const int64_t s = k / p;
+  TcParams prm{};
+  prm.T = static_cast<int32_t>(T);
+  prm.n_total = static_cast<int32_t>(d);
+  prm.s = static_cast<int32_t>(s);
+  prm.p = p;
+  prm.m_tiles = ceil_div(T, BM);
+  prm.batches = p;
+  prm.k_blocks = ceil_div(s, BK);
+  prm.kb_per_shard = prm.k_blocks;
+  prm.act = kActIdentity;
+  const TileChoice tch = pick_tile(T, d, p, prm.k_blocks, c.num_sms, false, pair_allowed());
+  if (!tch.pair || region_cnt == nullptr) return TP_OK;   // the caller folds the partials
+  CUtensorMap mA, mB, mZ;
+  if (!make_map_a(&mA, Y, s, T, p) || !make_map_b(&mB, W2, d, k) ||
+      !make_map_f32_out(&mZ, Z, d, T, 1))
+    return TP_ERR_CUDA;
+  prm.bias = b2;
+  prm.out = Z;
+  prm.region_cnt = region_cnt;
+  // Shards in order within each half of the m-tiles (as for the fold beside
+  // the layer): a half's running sums, 128 T d bytes, are read and written
+  // once per shard, so a half keeps them within reach of L2.
+  const int32_t m_tiles = ceil_div(T, 2 * BM);
+  prm.m_group = m_tiles >= 4 ? ceil_div(m_tiles, 2) : 0;
+  *done = true;
+  return launch_tc_pair(c, kModeRowChain, tch.bn, mA, mB, mB, mZ, prm);
+}
+
 tp_status launch_tc_row_splitk(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
                                float* Z, int64_t T, int64_t k, int64_t d, int p) {
   const int64_t s = k / p;

@@ -40,6 +40,16 @@ inline bool region_fold_allowed() {
   return on;
 }
 
+// TP_DISABLE_ROW_CHAIN=1 keeps the partials and the fold beside the row layer
+// where the chain fold would run (for comparisons; same bits).
+inline bool row_chain_allowed() {
+  static const bool on = [] {
+    const char* e = std::getenv("TP_DISABLE_ROW_CHAIN");
+    return !(e != nullptr && e[0] == '1');
+  }();
+  return on;
+}
+
 template <typename... KArgs, typename... Args>
 cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
                        cudaStream_t stream, Args&&... args) {

@@ -41,6 +41,13 @@ def region_fold_enabled():
     return pairs_enabled() and os.environ.get("TP_DISABLE_REGION_FOLD", "") != "1"
 
 
+def row_chain_enabled():
+    """The row layer folds the partials in its own epilogue where the fold
+    beside it would run (TP_DISABLE_ROW_CHAIN=1 keeps the fold beside it)."""
+    import os
+    return region_fold_enabled() and os.environ.get("TP_DISABLE_ROW_CHAIN", "") != "1"
+
+
 class DeviceBlock:
     """Device copies of one workload instance plus output buffers."""
 

@@ -27,7 +27,7 @@ import torch
 
 import megatron_tensor_sharded_b200 as tp
 import workloads as W
-from gpu_util import bits, dev, host_f32, pairs_enabled
+from gpu_util import bits, dev, host_f32, pairs_enabled, row_chain_enabled
 from oracle import tp_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -215,8 +215,8 @@ def test_attention_block_is_bit_identical_to_separate_calls(T, h, hkv, bias):
     At T >= 2000 the Q, K, V projections also run as one launch of pair
     tiles: 256 x 128 tiles at 16 and 12 query heads (T=2000: a ragged last
     row tile and 384-column Q shards that start inside a tile), 256 x 256
-    tiles at 32 / 8 heads.  tp_attn_block, whose fold runs beside the output
-    projection, gives the bits of the separate calls (three column
+    tiles at 32 / 8 heads.  tp_attn_block, whose fold runs in the output
+    projection's epilogue, gives the bits of the separate calls (three column
     projections, tp_attention_heads, tp_row_linear, tp_reduce_partials),
     call after call on one workspace."""
     d, p = 2048, 4
@@ -249,5 +249,6 @@ def test_attention_block_is_bit_identical_to_separate_calls(T, h, hkv, bias):
         tp.tp_sync_status()
         assert np.array_equal(bits(host_f32(Z)), want)
         # Q, K, V in one launch at T >= 2000, three below; then attention,
-        # W_O and the fold
-        assert launches == (4 if T >= 2000 and pairs_enabled() else 6)
+        # and W_O with the fold in its epilogue, or W_O and the fold
+        qkv = 1 if T >= 2000 and pairs_enabled() else 3
+        assert launches == qkv + (2 if row_chain_enabled() else 3)

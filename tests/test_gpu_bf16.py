@@ -11,7 +11,7 @@ import torch
 import megatron_tensor_sharded_b200 as tp
 from oracle import tp_oracle as O
 import workloads as W
-from gpu_util import DeviceBlock, bits, host_f32, region_fold_enabled
+from gpu_util import DeviceBlock, bits, host_f32, region_fold_enabled, row_chain_enabled
 
 pytestmark = pytest.mark.gpu
 
@@ -311,15 +311,21 @@ def _counter_bytes(T, d):
 
 @pytest.mark.parametrize("T,d,s,p,act,bias", [(1000, 2176, 2048, 4, "gelu_tanh", True),
                                               (777, 2048, 1536, 3, "relu", False),
-                                              (513, 1024, 3584, 8, "swiglu", True)])
+                                              (513, 1024, 3584, 8, "swiglu", True),
+                                              (2048, 4096, 1024, 1, "relu", True),
+                                              (1800, 2048, 2048, 2, "gelu_tanh", False)])
 def test_block_fold_beside_row_layer(T, d, s, p, act, bias):
     """Shapes whose row layer runs on CTA-pair tiles (256 rows x 256 or 128
     columns; ragged T, a last region 128 columns wide, p = 3 on the generic
-    fold): tp_mlp_block folds each region of the partials beside the row
-    layer once all p shard tiles of it are in memory.  Z has the bits of the
-    three separate calls, call after call on one workspace, and the
-    workspace's region counters show every region counted to 16 p (eight
-    epilogue warps on each CTA of a pair, once per shard)."""
+    fold, one shard, two): tp_mlp_block folds the partials in the row
+    layer's epilogue (each shard's tile adds its partial to the sum the
+    previous shard's tile left in Z, the last adds b2), or, with
+    TP_DISABLE_ROW_CHAIN=1, beside the row layer once all p shard tiles of a
+    region are in memory.  Z has the bits of the three separate calls, call
+    after call on one workspace, the workspace's region counters show every
+    region counted to 16 p (eight epilogue warps on each CTA of a pair, once
+    per shard), and the chain leaves the partials area of the workspace
+    unwritten."""
     k = s * p
     inp = _random_bf16(T, d, k, act, with_bias=bias, seed=T + d + p + 1)
     blk = DeviceBlock(inp, T, d, k, p, act)
@@ -343,6 +349,10 @@ def test_block_fold_beside_row_layer(T, d, s, p, act, bias):
         assert cnt[0] == 16 * p
         assert set(np.unique(cnt).tolist()) <= {0, 16 * p}
         assert int((cnt == 16 * p).sum()) in (m_regions * -(-d // 256), m_regions * -(-d // 128))
+        y_bytes = -(-T * k * 2 // 256) * 256
+        partials = ws[y_bytes:y_bytes + p * T * d * 4]
+        untouched = bool((partials == 0x7F).all().item())
+        assert untouched == row_chain_enabled()
     if T <= 1024:
         assert O.rel_err(host_f32(blk.Z), _oracle(inp, p, act)["Z"]) <= TOL_BF16
 

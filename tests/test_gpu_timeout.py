@@ -84,8 +84,8 @@ def test_drop_applies_to_one_launch_only(short_timeout):
 
 def test_dropped_load_in_cta_pair_gemm_times_out(short_timeout):
     """A shape whose column layer runs on CTA pairs (256 x 256 tiles): the
-    even CTA's MMA wait runs out, both CTAs of every pair stop, meet at the
-    cluster barrier and free their TMEM."""
+    first pair's even CTA's MMA wait runs out, both CTAs of that pair stop,
+    meet at the cluster barrier and free their TMEM; the other pairs finish."""
     rng = np.random.default_rng(1)
     c = W.f32_to_bf16_bits
     T, d, k, p = 1000, 2048, 8192, 4
@@ -142,10 +142,11 @@ def test_dropped_load_in_attention_times_out(short_timeout):
 
 def test_dropped_load_in_block_row_layer_times_out(short_timeout):
     """tp_mlp_block on a shape whose row layer runs on CTA pairs, with the
-    fold running beside it: a load the row layer (the call's second
-    tensor-core launch) never issues makes its MMA wait run out, the layer
-    stops without counting its remaining tiles, and the fold's waits on those
-    regions run out as well (status bit 0x80); the next call is correct."""
+    fold in its epilogue (or beside it): a load the row layer (the call's
+    second tensor-core launch) never issues makes its MMA wait run out, the
+    layer stops without counting its remaining tiles, and the later shards'
+    waits for those regions (or the fold's) run out as well (status bit
+    0x80); the next call is correct."""
     rng = np.random.default_rng(3)
     c = W.f32_to_bf16_bits
     T, d, k, p = 1000, 2048, 2048, 4
