@@ -292,10 +292,10 @@ tp_status fold_residual_impl(const float* partials, const float* bias, const flo
 
 // bf16 row layer to partials, then the fixed-order fold of the partials
 // (+ b2, + the residual R if given).  When `regions` came from
-// region_counters (and were zeroed) and the layer runs on CTA pairs: without
-// R, inside the row layer (each shard's tile adds its partial to the running
-// sum in Z, no partials written); with R, beside the row layer.  After it
-// otherwise.  Same bits every way.
+// region_counters (and were zeroed) and the layer runs on CTA pairs: inside
+// the row layer (each shard's tile adds its partial to the running sum in Z,
+// the last adds b2 and R; no partials written), or beside it with
+// TP_DISABLE_ROW_CHAIN=1.  After it otherwise.  Same bits every way.
 tp_status row_and_fold(const void* Y, const void* W2, float* P, const float* b2, float* Z,
                        int64_t T, int64_t k, int64_t d, int p, int* regions, void* stream,
                        const float* R = nullptr) {
@@ -310,9 +310,9 @@ tp_status row_and_fold(const void* Y, const void* W2, float* P, const float* b2,
   }
   LaunchCtx c{};
   TP_TRY(make_ctx(stream, true, &c));
-  if (R == nullptr && row_chain_allowed()) {
+  if (row_chain_allowed()) {
     bool done = false;
-    TP_TRY(launch_tc_row_chain(c, Y, W2, b2, Z, T, k, d, p, regions, &done));
+    TP_TRY(launch_tc_row_chain(c, Y, W2, b2, R, Z, T, k, d, p, regions, &done));
     if (done) return TP_OK;
   }
   RegionFold rf{};
@@ -730,8 +730,8 @@ tp_status tp_transformer_block(const float* X, const tp_block_params* prm, float
   const int64_t kq = static_cast<int64_t>(n_heads) * head_dim;
   const int64_t kkv = static_cast<int64_t>(n_kv_heads) * head_dim;
   const int ident = TP_ACT_IDENTITY;
-  // The MLP's fold (+ b2 + the residual H) runs beside its row layer where
-  // that applies; its counters are reset before the first launch.
+  // The MLP's fold (+ b2 + the residual H) runs in its row layer's epilogue
+  // where that applies; the counters are zeroed by the MLP's column layer.
   int* regions = nullptr;
   int n_regions = 0;
   TP_TRY(region_counters(ws + L.cnt, T, d, prm->b2, H, &regions, &n_regions));

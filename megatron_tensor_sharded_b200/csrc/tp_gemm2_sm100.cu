@@ -123,9 +123,9 @@ __device__ __forceinline__ bool wait_count(const int* cnt, int target, volatile 
 
 // Chain fold of a row layer (kModeRowChain): the tile of shard s adds its partial
 // to the running sum that shard s-1's tile of the same rows and columns left
-// in Z, and the last shard adds b2, so Z = ((P_0 + P_1) + ... + P_{p-1}) + b2
-// with one fp32 RNE addition per element in shard order -- the fixed-order
-// fold -- and no partials reach memory.  The warp waits (once per tile) for
+// in Z, and the last shard adds b2 (then R with P.resid), so Z = (((P_0 +
+// P_1) + ... + P_{p-1}) + b2) + R with one fp32 RNE addition per element in
+// that order -- the fixed-order fold -- and no partials reach memory.  The warp waits (once per tile) for
 // the region counter to show all earlier shards' tiles stored; then per
 // 32 x 32 chunk the previous sum comes into the warp's staging tile by a
 // TMA load (128-byte swizzle, the store's layout), each lane adds its row
@@ -135,8 +135,8 @@ template <int PBN>
 __device__ __forceinline__ bool epilogue_tile_chain(const TcParams& P, const TileCoord& tc,
                                                     uint32_t tacc, int32_t row0, int half,
                                                     uint32_t stage, uint32_t bar, uint32_t& ph,
-                                                    const CUtensorMap* mapZ, volatile int* abort,
-                                                    int lane) {
+                                                    const CUtensorMap* mapZ, const CUtensorMap* mapR,
+                                                    volatile int* abort, int lane) {
   const float* __restrict__ b2 = static_cast<const float*>(P.bias);
   const bool first = tc.batch == 0;
   const bool last = tc.batch == P.p - 1;
@@ -188,6 +188,28 @@ __device__ __forceinline__ bool epilogue_tile_chain(const TcParams& P, const Til
       for (int e = 0; e < 32; ++e)
         v[e] = __float_as_uint(
             __fadd_rn(__uint_as_float(v[e]), j0 + e < P.n_total ? __ldg(b2 + j0 + e) : 0.0f));
+    }
+    if (last && P.resid) {
+      __syncwarp();   // every lane has read the previous sum out of the staging tile
+      if (lane == 0) {
+        mbar_arrive_expect_tx(bar, 32 * 32 * 4);
+        tma_load_3d(stage, mapR, bar, j0, row0, 0);
+      }
+      if (!wait_teardown(bar, ph, P.wait)) return false;
+      ph ^= 1u;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t addr = stage + lane * 128 + ((c ^ (lane & 7)) << 4);
+        uint32_t r0, r1, r2, r3;
+        asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                     : "r"(addr)
+                     : "memory");
+        v[4 * c + 0] = __float_as_uint(__fadd_rn(__uint_as_float(v[4 * c + 0]), __uint_as_float(r0)));
+        v[4 * c + 1] = __float_as_uint(__fadd_rn(__uint_as_float(v[4 * c + 1]), __uint_as_float(r1)));
+        v[4 * c + 2] = __float_as_uint(__fadd_rn(__uint_as_float(v[4 * c + 2]), __uint_as_float(r2)));
+        v[4 * c + 3] = __float_as_uint(__fadd_rn(__uint_as_float(v[4 * c + 3]), __uint_as_float(r3)));
+      }
     }
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -400,7 +422,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t stage_w = epi_stage + (warp - 4) * EPI_WARP_STAGE_BYTES;
       if constexpr (MODE == kModeRowChain) {
         if (!epilogue_tile_chain<PBN>(P, tc, tacc, row0, half, stage_w, chain_bar, chain_ph,
-                                      &mapC, abort_flag, lane))
+                                      &mapC, &mapC1, abort_flag, lane))
           break;   // a wait gave up (error bit set); the MMA's waits end on the abort flag
       } else if constexpr (kPairBulkOut<MODE>) {
         epilogue_tile_bulk<MODE, PBN>(P, tc, tacc, row0, half, stage_w, &mapC, lane);
@@ -498,7 +520,7 @@ tp_status launch_pair_mode(const LaunchCtx& c, const CUtensorMap& a, const CUten
 // (SwiGLU: pbn/2 output columns) n-tiles.
 tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMap& a,
                          const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& cm,
-                         TcParams prm) {
+                         TcParams prm, const CUtensorMap* c1) {
   const int out_cols = mode == kModeColumnSwiglu ? pbn / 2 : pbn;
   prm.m_tiles = ceil_div(prm.T, PBM);
   prm.n_tiles = ceil_div(prm.n_total, out_cols);
@@ -508,7 +530,8 @@ tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMa
       case kModeColumn: return launch_pair_mode<kModeColumn, 128>(c, a, b0, b1, cm, prm);
       case kModeColumnSwiglu: return launch_pair_mode<kModeColumnSwiglu, 128>(c, a, b0, b1, cm, prm);
       case kModeRowPartial: return launch_pair_mode<kModeRowPartial, 128>(c, a, b0, b1, cm, prm);
-      case kModeRowChain: return launch_pair_mode<kModeRowChain, 128>(c, a, b0, b1, cm, prm);
+      case kModeRowChain:
+        return launch_pair_mode<kModeRowChain, 128>(c, a, b0, b1, cm, prm, nullptr, c1);
       default: return launch_pair_mode<kModeRowSplitK, 128>(c, a, b0, b1, cm, prm);
     }
   }
@@ -516,7 +539,8 @@ tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMa
     case kModeColumn: return launch_pair_mode<kModeColumn, 256>(c, a, b0, b1, cm, prm);
     case kModeColumnSwiglu: return launch_pair_mode<kModeColumnSwiglu, 256>(c, a, b0, b1, cm, prm);
     case kModeRowPartial: return launch_pair_mode<kModeRowPartial, 256>(c, a, b0, b1, cm, prm);
-    case kModeRowChain: return launch_pair_mode<kModeRowChain, 256>(c, a, b0, b1, cm, prm);
+    case kModeRowChain:
+      return launch_pair_mode<kModeRowChain, 256>(c, a, b0, b1, cm, prm, nullptr, c1);
     default: return launch_pair_mode<kModeRowSplitK, 256>(c, a, b0, b1, cm, prm);
   }
 }

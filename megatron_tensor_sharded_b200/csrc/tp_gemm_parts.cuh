@@ -78,6 +78,8 @@ struct TcParams {
   int32_t zero_n;        // the previous kernel) for the row layer that follows; may be null
   int32_t m_group;       // > 0: tiles walk groups of this many m-tiles, group slowest (all
                          // shards of one group before the next); 0: one group
+  int32_t resid;         // chain row layer: 1 = the last shard also adds R (fp32 [T][d],
+                         // the kernel's second output tensor map) after b2
   // Column layer on CTA pairs with several weights and outputs in one launch
   // (the Q, K, V projections): nseg > 1 segments, segment i owning tiles
   // [seg_start[i], seg_start[i + 1]), k = seg_n[i] output columns, shard
@@ -488,9 +490,10 @@ __device__ __forceinline__ void epilogue_tile_bulk_col(const TcParams& P, const 
 
 // Per-layer GEMM on CTA pairs (tp_gemm2_sm100.cu): 256 x pbn tiles (pbn 128
 // or 256); `mode` is a gemm::Mode; prm's tile space is recomputed.
+// (chain row layer: `c1` is the map of R when prm.resid is set)
 tp_status launch_tc_pair(const LaunchCtx& c, int mode, int pbn, const CUtensorMap& a,
                          const CUtensorMap& b0, const CUtensorMap& b1, const CUtensorMap& cm,
-                         gemm::TcParams prm);
+                         gemm::TcParams prm, const CUtensorMap* c1 = nullptr);
 // Up to three identity column layers of one input in one launch of 256 x pbn
 // pair tiles, pbn 128 or 256 (tp_gemm2_sm100.cu).
 tp_status launch_tc_pair_column_multi(const LaunchCtx& c, int pbn, const CUtensorMap& a,

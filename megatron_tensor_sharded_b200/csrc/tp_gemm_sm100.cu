@@ -420,8 +420,8 @@ tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float
 }
 
 tp_status launch_tc_row_chain(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
-                              float* Z, int64_t T, int64_t k, int64_t d, int p, int* region_cnt,
-                              bool* done) {
+                              const float* R, float* Z, int64_t T, int64_t k, int64_t d, int p,
+                              int* region_cnt, bool* done) {
   *done = false;
   const int64_t s = k / p;
   TcParams prm{};
@@ -436,12 +436,14 @@ tp_status launch_tc_row_chain(const LaunchCtx& c, const void* Y, const void* W2,
   prm.act = kActIdentity;
   const TileChoice tch = pick_tile(T, d, p, prm.k_blocks, c.num_sms, false, pair_allowed());
   if (!tch.pair || region_cnt == nullptr) return TP_OK;   // the caller folds the partials
-  CUtensorMap mA, mB, mZ;
+  CUtensorMap mA, mB, mZ, mR;
   if (!make_map_a(&mA, Y, s, T, p) || !make_map_b(&mB, W2, d, k) ||
-      !make_map_f32_out(&mZ, Z, d, T, 1))
+      !make_map_f32_out(&mZ, Z, d, T, 1) ||
+      (R != nullptr && !make_map_f32_out(&mR, const_cast<float*>(R), d, T, 1)))
     return TP_ERR_CUDA;
   prm.bias = b2;
   prm.out = Z;
+  prm.resid = R != nullptr ? 1 : 0;
   prm.region_cnt = region_cnt;
   // Shards in order within each half of the m-tiles (as for the fold beside
   // the layer): a half's running sums, 128 T d bytes, are read and written
@@ -449,7 +451,8 @@ tp_status launch_tc_row_chain(const LaunchCtx& c, const void* Y, const void* W2,
   const int32_t m_tiles = ceil_div(T, 2 * BM);
   prm.m_group = m_tiles >= 4 ? ceil_div(m_tiles, 2) : 0;
   *done = true;
-  return launch_tc_pair(c, kModeRowChain, tch.bn, mA, mB, mB, mZ, prm);
+  return launch_tc_pair(c, kModeRowChain, tch.bn, mA, mB, mB, mZ, prm,
+                        R != nullptr ? &mR : nullptr);
 }
 
 tp_status launch_tc_row_splitk(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,

@@ -74,12 +74,13 @@ tp_status launch_tc_row(const LaunchCtx& c, const void* Y, const void* W2, float
 size_t region_counter_bytes(int64_t T, int64_t d);
 // Row layer and the fixed-order fold in one launch, where it runs on CTA-pair
 // tiles: shard by shard each tile adds its partial to the running sum in Z,
-// the last shard adds b2; region_cnt (zeroed, region_counter_bytes()) orders
-// the shards.  *done = false (nothing launched) where the layer would not run
-// on pairs: the caller then folds the partials itself.
+// the last shard adds b2, then R (fp32 [T][d], 16-byte aligned; may be null);
+// region_cnt (zeroed, region_counter_bytes()) orders the shards.  *done =
+// false (nothing launched) where the layer would not run on pairs: the
+// caller then folds the partials itself.
 tp_status launch_tc_row_chain(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
-                              float* Z, int64_t T, int64_t k, int64_t d, int p, int* region_cnt,
-                              bool* done);
+                              const float* R, float* Z, int64_t T, int64_t k, int64_t d, int p,
+                              int* region_cnt, bool* done);
 tp_status launch_tc_row_splitk(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,
                                float* Z, int64_t T, int64_t k, int64_t d, int p);
 

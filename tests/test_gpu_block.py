@@ -18,7 +18,7 @@ import torch
 
 import megatron_tensor_sharded_b200 as tp
 import workloads as W
-from gpu_util import bits, dev, host_f32, pairs_enabled
+from gpu_util import bits, dev, host_f32, pairs_enabled, row_chain_enabled
 from oracle import tp_oracle as O
 
 pytestmark = pytest.mark.gpu
@@ -159,8 +159,9 @@ def test_transformer_block_full_size_prefix(name, n):
 @pytest.mark.parametrize("T,act", [(1000, "gelu_tanh"), (1000, "swiglu"), (2048, "gelu_tanh")])
 def test_transformer_block_is_bit_identical_to_separate_calls(T, act):
     """Shapes whose MLP row layer runs on CTA-pair tiles (d=2048, k=2048 on
-    p=4), so reduction #2 runs beside that layer (at T=2048 the Q, K, V
-    projections also run as one launch): the block gives the bits of its
+    p=4), so reduction #2 (+ b2 + H) runs in that layer's epilogue, or beside
+    it with TP_DISABLE_ROW_CHAIN=1 (at T=2048 the Q, K, V projections also
+    run as one launch): the block gives the bits of its
     steps called one by one (LayerNorm, the three projections, attention,
     W_O, fold + bo + X, LayerNorm, the MLP layers, fold + b2 + H), call
     after call on one workspace."""
@@ -199,5 +200,7 @@ def test_transformer_block_is_bit_identical_to_separate_calls(T, act):
         launches = tp.tp_kernel_launch_count() - before
         assert np.array_equal(bits(got), want)
         # LN, Q K V (one launch at T=2048, three at T=1000), attention, W_O,
-        # fold + LN, the two MLP layers, fold
-        assert launches == (8 if T >= 2000 and pairs_enabled() else 10)
+        # fold + LN, the two MLP layers, and the fold unless the row layer
+        # does it
+        qkv = 1 if T >= 2000 and pairs_enabled() else 3
+        assert launches == qkv + (6 if row_chain_enabled() else 7)
