@@ -835,8 +835,9 @@ def run_tp(a, w: WL.Workload, rank: int, world: int, local_rank: int):
     e2e = None if a.no_e2e else measure_e2e(a, torch, tp, B, w, world, barrier)
 
     value = whole_job_value(w.gemm_flops(), world, ms_step) / 1e12
-    kernel_name = {"partials": "tp_mlp_block: column GEMM -> row GEMM -> fixed-order fold (PDL-chained; "
-                               "on CTA-pair row tiles the fold runs beside the row GEMM)",
+    kernel_name = {"partials": "tp_mlp_block: column GEMM -> row GEMM with the fixed-order fold "
+                               "(PDL-chained; on CTA-pair row tiles the row GEMM's epilogue folds "
+                               "shard by shard into Z, else a fold kernel follows)",
                    "fold": "tp_mlp_block row-fold: column GEMM -> row GEMM folding the p partials "
                            "in its epilogue (bit-identical to partials + fold)",
                    "splitk": "tp_mlp_block split-K: column GEMM -> row GEMM accumulating all shards",
@@ -1070,7 +1071,8 @@ def run_tp_attn(a, w: WL.AttnWorkload, rank: int, world: int, local_rank: int):
     roof = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"],
             "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
             "traffic": ncu_traffic(f"{w.name}/block"),
-            "kernel": "tp_attn_block: QKV column GEMMs -> tc_attn_kernel -> row GEMM -> fold",
+            "kernel": "tp_attn_block: QKV column GEMMs -> tc_attn_kernel -> row GEMM with the "
+                      "fixed-order fold in its epilogue (CTA-pair tiles; else -> fold)",
             "duration": "block step time (graph replay, CUDA events on the launching stream)",
             "peak_source": f"{peak_src} bf16 dense (burst)",
             "flops_per_step": fl}
@@ -1247,7 +1249,8 @@ def run_tp_block(a, w: WL.BlockWorkload, rank: int, world: int, local_rank: int)
             "unit": "TFLOP/s", "frac": achieved / peaks["bf16_tflops"],
             "traffic": ncu_traffic(f"{w.name}/block"),
             "kernel": "tp_transformer_block: LN -> QKV GEMMs -> tc_attn_kernel -> Wo GEMM -> "
-                      "fold+residual+LN -> MLP GEMMs -> fold+residual",
+                      "fold+residual+LN -> MLP GEMMs, the row GEMM folding + b2 + residual in "
+                      "its epilogue (CTA-pair tiles; else -> fold+residual)",
             "duration": "block step time (graph replay, CUDA events on the launching stream)",
             "peak_source": f"{peak_src} bf16 dense (burst)", "flops_per_step": fl}
     if breakdown is not None:

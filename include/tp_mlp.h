@@ -213,23 +213,26 @@ tp_status tp_ipc_release(const tp_ipc_handle* handle);
  * tp_row_linear -> tp_reduce_partials compute (bit for bit), with the hidden
  * shards and the partials in the caller's workspace; the kernels are chained
  * with programmatic dependent launch.  Where the row layer runs on CTA-pair
- * tiles (bf16, b2 NULL or 16-byte aligned), the fold runs beside it: the
- * row layer counts each 256-row region of the partials done once all p
- * shard tiles of it are in memory, and the fold takes the regions in that
- * order (same additions, same order, same bits).  With
- * TP_FLAG_SPLITK_FUSED the second layer accumulates over all shards and
- * writes Z directly (no partials).
+ * tiles (bf16, b2 NULL or 16-byte aligned), it does the fold itself: shard
+ * by shard, each tile adds its partial to the running sum that the previous
+ * shard's tile left in Z, and the last shard adds b2 (same additions, same
+ * order, same bits; no partials are written).  That layer is a cooperative
+ * launch, so all its CTAs are resident together.  Z must not overlap the
+ * workspace.  With TP_FLAG_SPLITK_FUSED the second layer accumulates over
+ * all shards and writes Z directly (no partials).
  *
  *   workspace        device memory of at least
  *                    tp_mlp_block_workspace_size(...) bytes, 256-byte aligned;
  *                    contents on return: hidden shards [p][T][s] at offset 0,
- *                    then (default mode) the partials [p][T][d] fp32 at the
- *                    next 256-byte boundary, then counters at the end (reset
- *                    on every call that uses them): one int32 per 128-row
- *                    m-tile for TP_FLAG_FUSED_LAUNCH, or one per region of
- *                    the fold beside the row layer (256-row regions in
- *                    column-major order, each counted to 16 p; the area
- *                    has room for ceil(T/128) * ceil(d/64) of them).
+ *                    then (default mode) room for the partials [p][T][d]
+ *                    fp32 at the next 256-byte boundary (written only where
+ *                    the row layer does not fold itself), then counters at
+ *                    the end (reset on every call that uses them): one int32
+ *                    per 128-row m-tile for TP_FLAG_FUSED_LAUNCH, or one per
+ *                    256-row region of the row layer (column-major order,
+ *                    each counted to 16 p, which orders the shards of the
+ *                    fold; the area has room for ceil(T/128) * ceil(d/64) of
+ *                    them).
  *   other arguments  as for the three calls above.
  */
 tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const void* b1,
@@ -343,15 +346,15 @@ tp_status tp_attention_heads(const void* Q, const void* K, const void* V, void* 
  * tp_attention_heads, row-parallel output projection (tp_row_linear) and the
  * fixed-order fold (tp_reduce_partials) -- one reduction per block ("Tensor
  * parallel math", "Attention: parallel across heads"; "Tensor Parallelism
- * Explained", section 2.A).  As in tp_mlp_block, the fold runs beside the
- * output projection where that runs on CTA-pair tiles (bo NULL or 16-byte
- * aligned); same bits.
+ * Explained", section 2.A).  As in tp_mlp_block, the output projection
+ * folds the shards itself where it runs on CTA-pair tiles (bo NULL or
+ * 16-byte aligned); same bits.  Z must not overlap the workspace.
  *
  *   X [T][d]; Wq [d][n_heads*head_dim]; Wk, Wv [d][n_kv_heads*head_dim];
  *   Wo [n_heads*head_dim][d]  (all bf16, [in, out]);  bo [d] fp32 nullable;
  *   Z [T][d] fp32.
  *   workspace: tp_attn_block_workspace_size(...) bytes, 256-byte aligned
- *   (Q, K, V, O shards, then the fp32 partials, then the fold's region
+ *   (Q, K, V, O shards, then room for the fp32 partials, then the region
  *   counters).
  */
 tp_status tp_attn_block(const void* X, const void* Wq, const void* Wk, const void* Wv,
@@ -423,9 +426,10 @@ typedef struct tp_block_params {
  *   out = H + tp_mlp_block(LayerNorm(H; ln2))          (reduction #2 + residual)
  *
  * Each reduction adds, per element, the p partials in shard order, then the
- * bias, then the residual.  Reduction #2 runs beside the MLP's row layer
- * where that runs on CTA-pair tiles (b2 NULL or 16-byte aligned), as in
- * tp_mlp_block; same bits.
+ * bias, then the residual.  Reduction #2 runs in the MLP's row layer, which
+ * adds b2 and then the residual after the last shard, where that layer runs
+ * on CTA-pair tiles (b2 NULL or 16-byte aligned), as in tp_mlp_block; same
+ * bits.  out must not overlap the workspace.
  *
  * X, out [T][d] fp32 (out may equal X); every GEMM reads bf16 and
  * accumulates fp32; head_dim 128; d % 8 == 0 and d <= 16384.  workspace:

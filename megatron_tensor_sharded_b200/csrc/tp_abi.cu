@@ -253,6 +253,12 @@ tp_status reduce_impl(const float* partials, const float* b2, float* Z, int64_t 
   return cuda_status(launch_reduce(c, partials, b2, Z, T, d, p), "reduce launch");
 }
 
+// True when [a, a + an) and [b, b + bn) share a byte.
+bool ranges_overlap(const void* a, size_t an, const void* b, size_t bn) {
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+  return a0 < b0 + bn && b0 < a0 + an;
+}
+
 // Counters at `at` for the fold beside the row layer, when that path
 // applies: the bf16 path on an sm_100 device, b2 and R NULL or 16-byte
 // aligned (the fold reads them as vectors).  *out is NULL otherwise, and
@@ -571,6 +577,10 @@ tp_status tp_mlp_block(const void* X, const void* W1, const void* W_up, const vo
                 workspace == nullptr ? size_t(0) : workspace_size);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(TP_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  // Z is written while the row layer still reads the workspace (running sums
+  // of the fold in its epilogue; partials read by the fold)
+  if (ranges_overlap(Z, static_cast<size_t>(T) * d * 4, workspace, need))
+    return fail(TP_ERR_INVALID_ARG, "Z overlaps the workspace");
 
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* Y = ws;
@@ -654,6 +664,8 @@ tp_status tp_attn_block(const void* X, const void* Wq, const void* Wk, const voi
                 workspace == nullptr ? size_t(0) : workspace_size);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(TP_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  if (ranges_overlap(Z, static_cast<size_t>(T) * d * 4, workspace, need))
+    return fail(TP_ERR_INVALID_ARG, "Z overlaps the workspace");
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const size_t qb = align256(static_cast<size_t>(T) * kq * 2);
   const size_t kvb = align256(static_cast<size_t>(T) * kkv * 2);
@@ -718,6 +730,8 @@ tp_status tp_transformer_block(const float* X, const tp_block_params* prm, float
                 workspace == nullptr ? size_t(0) : workspace_bytes);
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     return fail(TP_ERR_ALIGNMENT, "workspace must be 256-byte aligned");
+  if (ranges_overlap(out, static_cast<size_t>(T) * d * 4, workspace, L.total))
+    return fail(TP_ERR_INVALID_ARG, "out overlaps the workspace");
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   void* A = ws + L.a;                       // LN1(X), later LN2(H): bf16 [T][d]
   float* H = reinterpret_cast<float*>(ws + L.h);

@@ -20,11 +20,14 @@
 // store through shared memory with TMA tensor stores, as in the single-CTA
 // kernel.
 //
-// Two launch-level options: a row layer of partials can publish per-tile
+// Launch-level options: a row layer of partials can publish per-tile
 // completion counters for the fold that runs beside it (region_cnt, tiles
-// taken in two halves of the m-tiles), and a column layer can carry up to
-// three weight/output segments of the same input (the attention block's
-// Q, K and V in one launch; nseg).
+// taken in two halves of the m-tiles); a row layer can instead fold the
+// shards itself (kModeRowChain: each shard's tile adds its partial to the
+// running sum in Z once the counters show the previous shard's tile
+// stored; a cooperative launch, so every pair it waits for is running);
+// and a column layer can carry up to three weight/output segments of the
+// same input (the attention block's Q, K and V in one launch; nseg).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -471,24 +474,14 @@ tp_status launch_pair_mode(const LaunchCtx& c, const CUtensorMap& a, const CUten
                            const CUtensorMap* b2 = nullptr, const CUtensorMap* c1 = nullptr,
                            const CUtensorMap* c2 = nullptr) {
   constexpr int PSMEM_BYTES = PKCfg<MODE, PBN>::SMEM_BYTES;
+  // The chain row layer's tiles wait for other tiles of the same grid, so it
+  // is launched cooperatively: all its CTAs are then resident together and
+  // every such wait ends, whatever else runs on the GPU.  (Without
+  // programmatic serialization: it starts after the layer before it ends.)
+  constexpr bool kCoop = (MODE == kModeRowChain);
   static uint64_t attr_epoch[64] = {};   // context epoch the attribute was set under
+  static int max_coop_clusters[64] = {};  // co-resident clusters of a cooperative launch
   static std::mutex mu;
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    const int dev = c.device & 63;
-    if (attr_epoch[dev] != c.epoch) {
-      if (cudaFuncSetAttribute(tc_gemm_pair_kernel<MODE, PBN>,
-                               cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               PSMEM_BYTES) != cudaSuccess) {
-        set_error_detail("cudaFuncSetAttribute failed: %s", cudaGetErrorString(cudaGetLastError()));
-        return TP_ERR_CUDA;
-      }
-      attr_epoch[dev] = c.epoch;
-    }
-  }
-  prm.wait.err = c.err_word;
-  prm.wait.timeout_ns = c.timeout_ns;
-  prm.debug_drop = c.debug_drop;
   int clusters = c.num_sms / 2;
   if (clusters > prm.num_tiles) clusters = prm.num_tiles;
   cudaLaunchConfig_t cfg = {};
@@ -501,10 +494,50 @@ tp_status launch_pair_mode(const LaunchCtx& c, const CUtensorMap& a, const CUten
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = pdl_allowed() ? 2 : 1;
+  cfg.numAttrs = 1;
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    const int dev = c.device & 63;
+    if (attr_epoch[dev] != c.epoch) {
+      if (cudaFuncSetAttribute(tc_gemm_pair_kernel<MODE, PBN>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               PSMEM_BYTES) != cudaSuccess) {
+        set_error_detail("cudaFuncSetAttribute failed: %s", cudaGetErrorString(cudaGetLastError()));
+        return TP_ERR_CUDA;
+      }
+      max_coop_clusters[dev] = 0;
+      if (kCoop) {
+        int coop = 0, n = 0;
+        if (cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, c.device) == cudaSuccess &&
+            coop != 0 &&
+            cudaOccupancyMaxActiveClusters(&n, tc_gemm_pair_kernel<MODE, PBN>, &cfg) == cudaSuccess)
+          max_coop_clusters[dev] = n;
+        (void)cudaGetLastError();
+      }
+      attr_epoch[dev] = c.epoch;
+    }
+    if (kCoop) {
+      // as many clusters as can be resident together (the tiles are taken
+      // round-robin by however many there are); none: nothing is enqueued
+      // and the caller folds another way
+      if (max_coop_clusters[dev] < 1) return TP_ERR_UNSUPPORTED;
+      if (clusters > max_coop_clusters[dev]) clusters = max_coop_clusters[dev];
+      cfg.gridDim = dim3(2 * clusters);
+    }
+  }
+  prm.wait.err = c.err_word;
+  prm.wait.timeout_ns = c.timeout_ns;
+  prm.debug_drop = c.debug_drop;
+  if (kCoop) {
+    attr[1].id = cudaLaunchAttributeCooperative;
+    attr[1].val.cooperative = 1;
+    cfg.numAttrs = 2;
+  } else if (pdl_allowed()) {
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.numAttrs = 2;
+  }
   const cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<MODE, PBN>, a, b0, b1, cm, prm,
                                            b2 != nullptr ? *b2 : b0, c1 != nullptr ? *c1 : cm,
                                            c2 != nullptr ? *c2 : cm);

@@ -450,9 +450,11 @@ tp_status launch_tc_row_chain(const LaunchCtx& c, const void* Y, const void* W2,
   // once per shard, so a half keeps them within reach of L2.
   const int32_t m_tiles = ceil_div(T, 2 * BM);
   prm.m_group = m_tiles >= 4 ? ceil_div(m_tiles, 2) : 0;
-  *done = true;
-  return launch_tc_pair(c, kModeRowChain, tch.bn, mA, mB, mB, mZ, prm,
-                        R != nullptr ? &mR : nullptr);
+  const tp_status st = launch_tc_pair(c, kModeRowChain, tch.bn, mA, mB, mB, mZ, prm,
+                                      R != nullptr ? &mR : nullptr);
+  if (st == TP_ERR_UNSUPPORTED) return TP_OK;   // no cooperative launch of this grid here
+  *done = st == TP_OK;
+  return st;
 }
 
 tp_status launch_tc_row_splitk(const LaunchCtx& c, const void* Y, const void* W2, const float* b2,

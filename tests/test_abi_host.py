@@ -138,6 +138,8 @@ def test_block_validation():
     assert blk(k=4 * 72, flags=tp.TP_FLAG_ROW_FOLD) == 4      # s = 72, not a multiple of 64
     assert blk(k=4 * 72, flags=tp.TP_FLAG_SPLITK_FUSED) == 4   # s = 72, not a multiple of 64
     assert blk(Z=None) == 1
+    assert blk(Z=0x40000 + 256) == 1                           # Z inside the workspace
+    assert blk(ws=0x40000, Z=0x40000 - 256) == 1               # Z runs into the workspace
 
 
 def test_valid_call_without_gpu_fails_loudly():
