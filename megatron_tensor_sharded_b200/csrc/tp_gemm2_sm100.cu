@@ -478,7 +478,7 @@ tp_status launch_pair_mode(const LaunchCtx& c, const CUtensorMap& a, const CUten
   // is launched cooperatively: all its CTAs are then resident together and
   // every such wait ends, whatever else runs on the GPU.  (Without
   // programmatic serialization: it starts after the layer before it ends.)
-  constexpr bool kCoop = (MODE == kModeRowChain);
+  const bool kCoop = (MODE == kModeRowChain) && coop_allowed();
   static uint64_t attr_epoch[64] = {};   // context epoch the attribute was set under
   static int max_coop_clusters[64] = {};  // co-resident clusters of a cooperative launch
   static std::mutex mu;
@@ -541,6 +541,14 @@ tp_status launch_pair_mode(const LaunchCtx& c, const CUtensorMap& a, const CUten
   const cudaError_t e = cudaLaunchKernelEx(&cfg, tc_gemm_pair_kernel<MODE, PBN>, a, b0, b1, cm, prm,
                                            b2 != nullptr ? *b2 : b0, c1 != nullptr ? *c1 : cm,
                                            c2 != nullptr ? *c2 : cm);
+  if (kCoop && (e == cudaErrorCooperativeLaunchTooLarge || e == cudaErrorNotSupported)) {
+    // refused before anything ran: no cooperative launches of this grid on
+    // this context; the caller folds another way
+    (void)cudaGetLastError();
+    std::lock_guard<std::mutex> lk(mu);
+    max_coop_clusters[c.device & 63] = 0;
+    return TP_ERR_UNSUPPORTED;
+  }
   note_launch();
   if (e != cudaSuccess) {
     set_error_detail("paired GEMM launch failed: %s", cudaGetErrorString(e));

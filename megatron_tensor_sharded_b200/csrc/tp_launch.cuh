@@ -40,6 +40,17 @@ inline bool region_fold_allowed() {
   return on;
 }
 
+// TP_DISABLE_COOP=1 launches the folding row layer like the other layers
+// (programmatic serialization, no co-residency guarantee): for profilers
+// that cannot launch a cooperative cluster grid, and for comparisons.
+inline bool coop_allowed() {
+  static const bool on = [] {
+    const char* e = std::getenv("TP_DISABLE_COOP");
+    return !(e != nullptr && e[0] == '1');
+  }();
+  return on;
+}
+
 // TP_DISABLE_ROW_CHAIN=1 keeps the partials and the fold beside the row layer
 // where the chain fold would run (for comparisons; same bits).
 inline bool row_chain_allowed() {
