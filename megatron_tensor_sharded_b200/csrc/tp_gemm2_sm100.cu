@@ -124,16 +124,17 @@ __device__ __forceinline__ bool wait_count(const int* cnt, int target, volatile 
   }
 }
 
-// Chain fold of a row layer (kModeRowChain): the tile of shard s adds its partial
-// to the running sum that shard s-1's tile of the same rows and columns left
-// in Z, and the last shard adds b2 (then R with P.resid), so Z = (((P_0 +
-// P_1) + ... + P_{p-1}) + b2) + R with one fp32 RNE addition per element in
-// that order -- the fixed-order fold -- and no partials reach memory.  The warp waits (once per tile) for
-// the region counter to show all earlier shards' tiles stored; then per
-// 32 x 32 chunk the previous sum comes into the warp's staging tile by a
-// TMA load (128-byte swizzle, the store's layout), each lane adds its row
-// of the accumulator to its row of the chunk, and a TMA store writes the new
-// sum back.  False if a wait gave up.
+// Chain fold of a row layer (kModeRowChain): the tile of shard s adds its
+// partial to the running sum that shard s-1's tile of the same rows and
+// columns left in Z, and the last shard adds b2 (then R with P.resid), so
+// Z = (((P_0 + P_1) + ... + P_{p-1}) + b2) + R with one fp32 RNE addition
+// per element in that order -- the fixed-order fold -- and no partials reach
+// memory.  The warp waits (once per tile) for the region counter to show
+// all earlier shards' tiles stored; then per 32 x 32 chunk the previous sum
+// comes into the warp's staging tile by a TMA load (128-byte swizzle, the
+// store's layout), each lane adds its row of the accumulator to its row of
+// the chunk, and a TMA store writes the new sum back.  False if a wait gave
+// up.
 template <int PBN>
 __device__ __forceinline__ bool epilogue_tile_chain(const TcParams& P, const TileCoord& tc,
                                                     uint32_t tacc, int32_t row0, int half,
