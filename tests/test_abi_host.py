@@ -139,7 +139,31 @@ def test_block_validation():
     assert blk(k=4 * 72, flags=tp.TP_FLAG_SPLITK_FUSED) == 4   # s = 72, not a multiple of 64
     assert blk(Z=None) == 1
     assert blk(Z=0x40000 + 256) == 1                           # Z inside the workspace
+    assert "Z overlaps the workspace" in tp.tp_last_error_detail()
     assert blk(ws=0x40000, Z=0x40000 - 256) == 1               # Z runs into the workspace
+
+
+def test_block_outputs_must_not_overlap_the_workspace():
+    """The attention and transformer blocks write their output while their
+    row layers still read the workspace (the running sums of the fold in the
+    row layer's epilogue), so an output inside the workspace is rejected
+    before anything is launched."""
+    T, d, h, hkv, dh, p, k = 4, 256, 2, 2, 128, 2, 512
+    ws = 0x100000
+    n0 = tp.tp_kernel_launch_count()
+    na = tp.tp_attn_block_workspace_size(T, d, h, hkv, dh, p)
+    assert tp.tp_attn_block(FAKE, FAKE, FAKE, FAKE, FAKE, None, ws + 256, ws, na, T, d, h, hkv,
+                            dh, p, True, stream=0, check=False) == 1
+    assert tp.tp_attn_block(FAKE, FAKE, FAKE, FAKE, FAKE, None, ws - 256, ws, na, T, d, h, hkv,
+                            dh, p, True, stream=0, check=False) == 1
+    assert "Z overlaps the workspace" in tp.tp_last_error_detail()
+    nt = tp.tp_transformer_block_workspace_size(T, d, h, hkv, dh, k, p)
+    prm = tp.block_params(**{name: FAKE for name, _ in tp.BlockParams._fields_
+                             if name not in ("W_up", "bo", "b2")})
+    assert tp.tp_transformer_block(FAKE2, prm, ws + 512, ws, nt, T, d, h, hkv, dh, k, p,
+                                   tp.TP_ACT_GELU_TANH, stream=0, check=False) == 1
+    assert "out overlaps the workspace" in tp.tp_last_error_detail()
+    assert tp.tp_kernel_launch_count() == n0
 
 
 def test_valid_call_without_gpu_fails_loudly():
